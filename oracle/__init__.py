@@ -1,0 +1,171 @@
+"""CPU oracle for the indirect expert matmul - TEST INFRASTRUCTURE ONLY.
+
+Only the test suite, ``__graft_entry__.smoke()`` and the benchmark's CPU
+baseline leg may import this package.  The library never does.  It wraps
+``moe_oracle.c`` (plain C, fp64, no code shared with the GPU library) with
+numpy-in / numpy-out helpers.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "moe_oracle.c")
+_LIB = os.path.join(_HERE, "_oracle.so")
+
+BROADCAST, PER_SLOT = 0, 1
+DTYPES = {"bf16": 0, "f16": 1, "f32": 2}
+OK, ERR_INVALID, ERR_RANGE, ERR_BAD_ID = 0, -1, -2, -3
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (-O2, OpenMP; no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fno-fast-math", "-shared", "-fPIC",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def _L():
+    global _lib
+    if _lib is None:
+        _lib = ctypes.CDLL(build())
+        vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+        _lib.oracle_check_args.argtypes = [i64, i32, i32]
+        _lib.oracle_row_ids.argtypes = [vp, i64, i32, i32, i32, vp, vp, vp]
+        for f in (_lib.oracle_mul_mat_id_brute, _lib.oracle_mul_mat_id_grouped):
+            f.argtypes = [vp, i32, i32, i32, vp, i32, vp, i64, i32, i32, vp, vp]
+        _lib.oracle_mul_mat_id_rows.argtypes = [vp, i32, i32, i32, vp, i32, vp, i64, i32, i32, vp, i64, vp, vp]
+        _lib.oracle_ffn_rows.argtypes = [vp, vp, vp, i32, i32, i32, vp, i32, vp, i64, i32, vp, i64, vp, vp]
+        _lib.oracle_shared_rows.argtypes = [vp, vp, vp, i32, i32, vp, i32, vp, i64, vp, vp]
+        _lib.oracle_ffn_hidden.argtypes = [vp, vp, i32, i32, i32, vp, i32, vp, i64, i32, vp, i64, vp, vp, vp]
+        _lib.oracle_dequant.argtypes = [vp, i32, i32, i32, vp]
+        _lib.oracle_dequant.restype = None
+    return _lib
+
+
+def _p(a):
+    if a is None:
+        return None
+    assert isinstance(a, np.ndarray) and a.flags["C_CONTIGUOUS"], "need a C-contiguous numpy array"
+    return ctypes.c_void_p(a.ctypes.data)
+
+
+def _mode(mode):
+    return {"broadcast": BROADCAST, "per_slot": PER_SLOT}.get(mode, mode)
+
+
+class OracleError(RuntimeError):
+    def __init__(self, code):
+        super().__init__(f"oracle error {code}")
+        self.code = code
+
+
+def _chk(rc):
+    if rc != OK:
+        raise OracleError(rc)
+
+
+def check_args(n_tokens, k, n_experts) -> int:
+    return _L().oracle_check_args(n_tokens, k, n_experts)
+
+
+def row_ids(ids: np.ndarray, n_experts: int, mode="broadcast"):
+    """(ids_src1, ids_dst, expert_bounds) of the stable counting sort."""
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    T, k = ids.shape
+    S = T * k
+    src1 = np.zeros(max(S, 1), np.int32)
+    dst = np.zeros(max(S, 1), np.int32)
+    bounds = np.zeros(n_experts + 1, np.int32)
+    _chk(_L().oracle_row_ids(_p(ids), T, k, n_experts, _mode(mode), _p(src1), _p(dst), _p(bounds)))
+    return src1[:S], dst[:S], bounds
+
+
+def dequant(W: np.ndarray, e: int) -> np.ndarray:
+    """fp64 weights of expert e, [n_out][n_in], from Q8_0 blocks."""
+    E, n_out, nb, _ = W.shape
+    out = np.empty((n_out, nb * 32), np.float64)
+    _L().oracle_dequant(_p(W), n_out, nb * 32, e, _p(out))
+    return out
+
+
+def mul_mat_id(W, x, x_type, ids, mode="broadcast", grouped=False):
+    """dst [T][k][n_out] (fp64) and its per-element tolerance."""
+    E, n_out, nb, _ = W.shape
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    T, k = ids.shape
+    dst = np.zeros((T, k, n_out), np.float64)
+    tol = np.zeros((T, k, n_out), np.float64)
+    f = _L().oracle_mul_mat_id_grouped if grouped else _L().oracle_mul_mat_id_brute
+    _chk(f(_p(W), E, n_out, nb * 32, _p(x), DTYPES[x_type], _p(ids), T, k, _mode(mode), _p(dst), _p(tol)))
+    return dst, tol
+
+
+def mul_mat_id_rows(W, x, x_type, ids, slots, mode="broadcast"):
+    """Rows of dst for flat slots t*k+s only: ([n][n_out], tol)."""
+    E, n_out, nb, _ = W.shape
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    T, k = ids.shape
+    slots = np.ascontiguousarray(slots, dtype=np.int64)
+    out = np.zeros((len(slots), n_out), np.float64)
+    tol = np.zeros_like(out)
+    _chk(_L().oracle_mul_mat_id_rows(_p(W), E, n_out, nb * 32, _p(x), DTYPES[x_type], _p(ids), T, k,
+                                     _mode(mode), _p(slots), len(slots), _p(out), _p(tol)))
+    return out, tol
+
+
+def ffn(Wg, Wu, Wd, x, x_type, ids, slots=None):
+    """Routed expert FFN rows ([n][n_embd] fp64, tol) for flat slots (all when None)."""
+    E, n_ff, nb, _ = Wg.shape
+    n_embd = nb * 32
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    T, k = ids.shape
+    if slots is None:
+        n = T * k
+        sp = None
+    else:
+        slots = np.ascontiguousarray(slots, dtype=np.int64)
+        n = len(slots)
+        sp = _p(slots)
+    y = np.zeros((n, n_embd), np.float64)
+    tol = np.zeros_like(y)
+    _chk(_L().oracle_ffn_rows(_p(Wg), _p(Wu), _p(Wd), E, n_embd, n_ff, _p(x), DTYPES[x_type], _p(ids), T, k,
+                              sp, n, _p(y), _p(tol)))
+    return y, tol
+
+
+def shared_ffn(Sg, Su, Sd, x, x_type, tokens=None):
+    """Shared-expert FFN rows for the listed tokens (all when None)."""
+    _, n_ff, nb, _ = Sg.shape
+    n_embd = nb * 32
+    T = x.shape[0]
+    tokens = np.arange(T, dtype=np.int64) if tokens is None else np.ascontiguousarray(tokens, dtype=np.int64)
+    y = np.zeros((len(tokens), n_embd), np.float64)
+    tol = np.zeros_like(y)
+    _chk(_L().oracle_shared_rows(_p(Sg), _p(Su), _p(Sd), n_embd, n_ff, _p(x), DTYPES[x_type], _p(tokens),
+                                 len(tokens), _p(y), _p(tol)))
+    return y, tol
+
+
+def ffn_hidden(Wg, Wu, x, x_type, ids, slots):
+    """(h, g, u) fp64 [n][n_ff] for flat slots."""
+    E, n_ff, nb, _ = Wg.shape
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    T, k = ids.shape
+    slots = np.ascontiguousarray(slots, dtype=np.int64)
+    h = np.zeros((len(slots), n_ff), np.float64)
+    g = np.zeros_like(h)
+    u = np.zeros_like(h)
+    _chk(_L().oracle_ffn_hidden(_p(Wg), _p(Wu), E, nb * 32, n_ff, _p(x), DTYPES[x_type], _p(ids), T, k,
+                                _p(slots), len(slots), _p(h), _p(g), _p(u)))
+    return h, g, u

@@ -1,0 +1,302 @@
+"""Pins of the CPU oracle to facts other than itself (no GPU).
+
+Each check ties the oracle to something independent: a hand-worked example,
+invariants of a stable counting sort, brute force over every tiny input,
+dense special cases checked with numpy's float64 matmul, symmetries that must
+hold exactly, and SwiGLU special values.  A dropped term, a wrong sign or
+index, or a transposed operand in the oracle fails at least one of them.
+"""
+import itertools
+
+import numpy as np
+import pytest
+
+import oracle
+import workloads
+from tests.fixtures import hand_example, pack_q8_0, unpack_q8_0
+
+
+def rand_q8(rng, E, n_out, n_in):
+    q = rng.integers(-127, 128, size=(E, n_out, n_in), dtype=np.int64).astype(np.int8)
+    d = rng.uniform(0.001, 0.01, size=(E, n_out, n_in // 32))
+    return pack_q8_0(d, q)
+
+
+def rand_ids_distinct(rng, T, E, k):
+    return np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32).reshape(T, k)
+
+
+# ------------------------------------------------------------- hand example
+@pytest.mark.parametrize("grouped", [False, True])
+def test_hand_example_broadcast(grouped):
+    g, W, xb, xs, ids = hand_example()
+    dst, tol = oracle.mul_mat_id(W, xb, "f32", ids, "broadcast", grouped=grouped)
+    assert np.array_equal(dst, np.array(g["dst_broadcast"], np.float64))
+    assert np.all(tol > 0)
+
+
+@pytest.mark.parametrize("grouped", [False, True])
+def test_hand_example_per_slot(grouped):
+    g, W, xb, xs, ids = hand_example()
+    dst, _ = oracle.mul_mat_id(W, xs, "f32", ids, "per_slot", grouped=grouped)
+    assert np.array_equal(dst, np.array(g["dst_per_slot"], np.float64))
+
+
+def test_hand_example_tables():
+    g, W, xb, xs, ids = hand_example()
+    s1, dr, b = oracle.row_ids(ids, 2, "broadcast")
+    assert b.tolist() == g["expert_bounds"]
+    assert dr.tolist() == g["ids_dst"]
+    assert s1.tolist() == g["ids_src1_broadcast"]
+    s1, dr, b = oracle.row_ids(ids, 2, "per_slot")
+    assert s1.tolist() == g["ids_src1_per_slot"]
+
+
+# --------------------------------------------------------- row-id invariants
+def check_invariants(ids, E, mode, src1, dst, bounds):
+    T, k = ids.shape
+    S = T * k
+    flat = ids.reshape(-1)
+    assert bounds[0] == 0 and bounds[E] == S
+    assert np.all(np.diff(bounds) >= 0)
+    assert np.array_equal(np.diff(bounds), np.bincount(flat, minlength=E)[:E])
+    assert np.array_equal(np.sort(dst), np.arange(S))
+    for e in range(E):
+        seg = dst[bounds[e]:bounds[e + 1]]
+        assert np.all(np.diff(seg) > 0)            # stable: ascending (t, s)
+        assert np.all(flat[seg] == e)
+    if mode == "per_slot":
+        assert np.array_equal(src1, dst)
+    else:
+        assert np.array_equal(src1, dst // k)
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_row_ids_invariants_fuzz(seed):
+    rng = np.random.default_rng(seed)
+    E = int(rng.integers(1, 300))
+    k = int(rng.integers(1, min(E, 33) + 1))
+    T = int(rng.integers(0, 700))
+    ids = rng.integers(0, E, size=(T, k)).astype(np.int32)  # duplicates allowed
+    for mode in ("broadcast", "per_slot"):
+        src1, dst, bounds = oracle.row_ids(ids, E, mode)
+        check_invariants(ids, E, mode, src1, dst, bounds)
+
+
+def test_row_ids_brute_force_all_tiny():
+    """Every id matrix with E <= 3, k <= 2, T <= 4 against numpy's stable sort."""
+    for E in (1, 2, 3):
+        for k in (1, 2):
+            if k > E:
+                continue
+            for T in range(0, 5):
+                for flat in itertools.product(range(E), repeat=T * k):
+                    ids = np.array(flat, np.int32).reshape(T, k)
+                    src1, dst, bounds = oracle.row_ids(ids, E, "broadcast")
+                    order = np.argsort(ids.reshape(-1), kind="stable")
+                    assert np.array_equal(dst, order)
+                    assert np.array_equal(src1, order // k)
+                    assert np.array_equal(bounds, np.searchsorted(np.sort(ids.reshape(-1)), np.arange(E + 1)))
+
+
+def test_row_ids_limits():
+    assert oracle.check_args((1 << 22) - 1, 1, 1) == oracle.OK
+    assert oracle.check_args(1 << 22, 1, 1) == oracle.ERR_RANGE
+    assert oracle.check_args(1, 1023, 1023) == oracle.OK
+    assert oracle.check_args(1, 1024, 2000) == oracle.ERR_RANGE
+    assert oracle.check_args(4, 3, 2) == oracle.ERR_RANGE
+    assert oracle.check_args(4, 0, 2) == oracle.ERR_INVALID
+    assert oracle.check_args((1 << 22) - 1, 1000, 1000) == oracle.ERR_RANGE  # T*k >= 2^31
+    with pytest.raises(oracle.OracleError) as ei:
+        oracle.row_ids(np.array([[0, 5]], np.int32), 3)
+    assert ei.value.code == oracle.ERR_BAD_ID
+    with pytest.raises(oracle.OracleError) as ei:
+        oracle.row_ids(np.array([[-1]], np.int32), 3)
+    assert ei.value.code == oracle.ERR_BAD_ID
+
+
+# ----------------------------------------------------- grouped == brute force
+@pytest.mark.parametrize("mode", ["broadcast", "per_slot"])
+@pytest.mark.parametrize("x_type", ["f32", "bf16"])
+def test_grouped_equals_brute(mode, x_type):
+    rng = np.random.default_rng(7)
+    E, k, T, n_in, n_out = 5, 3, 23, 64, 48
+    W = rand_q8(rng, E, n_out, n_in)
+    ids = rand_ids_distinct(rng, T, E, k)
+    rows = T if mode == "broadcast" else T * k
+    x = workloads.activations(rows, n_in, x_type, seed=3, tensor=9)
+    a, ta = oracle.mul_mat_id(W, x, x_type, ids, mode, grouped=False)
+    b, tb = oracle.mul_mat_id(W, x, x_type, ids, mode, grouped=True)
+    assert np.array_equal(a, b) and np.array_equal(ta, tb)
+    slots = np.array([0, 5, T * k - 1])
+    r, tr = oracle.mul_mat_id_rows(W, x, x_type, ids, slots, mode)
+    assert np.array_equal(r, a.reshape(T * k, n_out)[slots])
+
+
+# ---------------------------------------------------------- dense reductions
+def test_single_expert_is_plain_gemm():
+    rng = np.random.default_rng(11)
+    n_in, n_out, T = 96, 40, 17
+    W = rand_q8(rng, 1, n_out, n_in)
+    x = rng.standard_normal((T, n_in)).astype(np.float32)
+    ids = np.zeros((T, 1), np.int32)
+    dst, tol = oracle.mul_mat_id(W, x, "f32", ids)
+    w = unpack_q8_0(W)[0]                              # numpy's own decode
+    ref = x.astype(np.float64) @ w.T                   # float64 library matmul
+    assert np.allclose(dst[:, 0, :], ref, rtol=1e-12, atol=1e-12)
+    mag = np.abs(x.astype(np.float64)) @ np.abs(w).T
+    assert np.allclose(tol[:, 0, :], 2e-3 * mag + 1e-5, rtol=1e-12)
+
+
+def test_oracle_dequant_matches_numpy_decode():
+    rng = np.random.default_rng(2)
+    W = rand_q8(rng, 3, 5, 64)
+    for e in range(3):
+        assert np.array_equal(oracle.dequant(W, e), unpack_q8_0(W)[e])
+
+
+def test_all_ids_equal_is_dense_gemm_of_that_expert():
+    rng = np.random.default_rng(12)
+    E, n_in, n_out, T, k = 4, 64, 24, 9, 1
+    W = rand_q8(rng, E, n_out, n_in)
+    x = rng.standard_normal((T, n_in)).astype(np.float32)
+    ids = np.full((T, k), 2, np.int32)
+    dst, _ = oracle.mul_mat_id(W, x, "f32", ids)
+    ref = x.astype(np.float64) @ unpack_q8_0(W)[2].T
+    assert np.allclose(dst[:, 0], ref, rtol=1e-12, atol=1e-12)
+
+
+def test_identical_experts_make_ids_irrelevant():
+    rng = np.random.default_rng(13)
+    n_in, n_out, T, k = 64, 16, 11, 3
+    W1 = rand_q8(rng, 1, n_out, n_in)
+    W = np.repeat(W1, 5, axis=0)
+    x = rng.standard_normal((T, n_in)).astype(np.float32)
+    a, _ = oracle.mul_mat_id(W, x, "f32", rand_ids_distinct(rng, T, 5, k))
+    b, _ = oracle.mul_mat_id(W, x, "f32", rand_ids_distinct(rng, T, 5, k))
+    assert np.array_equal(a, b)
+
+
+def test_relabelling_experts_is_exact():
+    rng = np.random.default_rng(14)
+    E, n_in, n_out, T, k = 6, 64, 16, 10, 2
+    W = rand_q8(rng, E, n_out, n_in)
+    x = rng.standard_normal((T, n_in)).astype(np.float32)
+    ids = rand_ids_distinct(rng, T, E, k)
+    perm = rng.permutation(E)           # expert e becomes perm[e]
+    Wp = np.empty_like(W)
+    Wp[perm] = W
+    a, _ = oracle.mul_mat_id(W, x, "f32", ids)
+    b, _ = oracle.mul_mat_id(Wp, x, "f32", perm[ids].astype(np.int32))
+    assert np.array_equal(a, b)
+
+
+def test_transposed_operand_would_fail():
+    """n_out != n_in and a non-symmetric W: out[n] must use row n of W."""
+    rng = np.random.default_rng(15)
+    W = rand_q8(rng, 1, 32, 64)
+    x = np.zeros((1, 64), np.float32)
+    x[0, 5] = 1.0
+    dst, _ = oracle.mul_mat_id(W, x, "f32", np.zeros((1, 1), np.int32))
+    assert np.array_equal(dst[0, 0], unpack_q8_0(W)[0][:, 5])
+
+
+# ------------------------------------------------------------------- FFN
+def silu(z):
+    return z / (1.0 + np.exp(-z))
+
+
+def test_ffn_single_expert_matches_numpy():
+    rng = np.random.default_rng(21)
+    n_embd, n_ff, T = 64, 96, 7
+    Wg, Wu, Wd = rand_q8(rng, 1, n_ff, n_embd), rand_q8(rng, 1, n_ff, n_embd), rand_q8(rng, 1, n_embd, n_ff)
+    x = rng.standard_normal((T, n_embd)).astype(np.float32)
+    ids = np.zeros((T, 1), np.int32)
+    y, tol = oracle.ffn(Wg, Wu, Wd, x, "f32", ids)
+    xg = x.astype(np.float64)
+    h = silu(xg @ unpack_q8_0(Wg)[0].T) * (xg @ unpack_q8_0(Wu)[0].T)
+    ref = h @ unpack_q8_0(Wd)[0].T
+    assert np.allclose(y, ref, rtol=1e-11, atol=1e-9)
+    assert np.all(tol > 2e-3 * (np.abs(h) @ np.abs(unpack_q8_0(Wd)[0]).T))
+
+
+def test_ffn_routed_matches_composition_of_mul_mat_id():
+    """FFN = down(per_slot) o SwiGLU o gate/up(broadcast), composed from the
+    oracle's mul_mat_id and numpy's SwiGLU."""
+    rng = np.random.default_rng(22)
+    E, k, T, n_embd, n_ff = 4, 2, 6, 64, 64
+    Wg, Wu, Wd = rand_q8(rng, E, n_ff, n_embd), rand_q8(rng, E, n_ff, n_embd), rand_q8(rng, E, n_embd, n_ff)
+    x = rng.standard_normal((T, n_embd)).astype(np.float32)
+    ids = rand_ids_distinct(rng, T, E, k)
+    y, _ = oracle.ffn(Wg, Wu, Wd, x, "f32", ids)
+    g, _ = oracle.mul_mat_id(Wg, x, "f32", ids, "broadcast")
+    u, _ = oracle.mul_mat_id(Wu, x, "f32", ids, "broadcast")
+    h = (silu(g) * u).reshape(T * k, n_ff)
+    wd = unpack_q8_0(Wd)
+    ref = np.stack([wd[ids.reshape(-1)[i]] @ h[i] for i in range(T * k)])
+    assert np.allclose(y, ref, rtol=1e-11, atol=1e-9)
+
+
+def test_swiglu_special_values():
+    rng = np.random.default_rng(23)
+    n_embd, n_ff = 32, 32
+    zero_gate = pack_q8_0(np.full((1, n_ff, 1), 0.01), np.zeros((1, n_ff, n_embd), np.int8))
+    Wu = rand_q8(rng, 1, n_ff, n_embd)
+    Wd = rand_q8(rng, 1, n_embd, n_ff)
+    x = rng.standard_normal((3, n_embd)).astype(np.float32)
+    ids = np.zeros((3, 1), np.int32)
+    y, _ = oracle.ffn(zero_gate, Wu, Wd, x, "f32", ids)
+    assert np.all(y == 0.0)                        # silu(0) = 0
+    # large gate: silu(g) -> g (relative gap e^-g)
+    big_gate = pack_q8_0(np.full((1, n_ff, 1), 2.0), np.full((1, n_ff, n_embd), 100, np.int8))
+    xo = np.ones((1, n_embd), np.float32)
+    h, g, u = oracle.ffn_hidden(big_gate, Wu, xo, "f32", np.zeros((1, 1), np.int32), np.array([0]))
+    assert np.all(g == 6400.0)
+    assert np.array_equal(h, g * u)
+    # negative gate: silu(-40) ~ -40 e^-40 ~ 0
+    neg_gate = pack_q8_0(np.full((1, n_ff, 1), 2.0 ** -6), np.full((1, n_ff, n_embd), -80, np.int8))
+    h, g, u = oracle.ffn_hidden(neg_gate, Wu, xo, "f32", np.zeros((1, 1), np.int32), np.array([0]))
+    assert np.all(g == -40.0)
+    assert np.all(np.abs(h) <= np.abs(u) * 40 * np.exp(-40) * 1.0000001)
+
+
+def test_shared_expert_equals_single_expert_routed_ffn():
+    rng = np.random.default_rng(24)
+    n_embd, n_ff, T = 64, 64, 5
+    Sg, Su, Sd = rand_q8(rng, 1, n_ff, n_embd), rand_q8(rng, 1, n_ff, n_embd), rand_q8(rng, 1, n_embd, n_ff)
+    x = workloads.activations(T, n_embd, "bf16", seed=1, tensor=5)
+    a, ta = oracle.shared_ffn(Sg, Su, Sd, x, "bf16")
+    b, tb = oracle.ffn(Sg, Su, Sd, x, "bf16", np.zeros((T, 1), np.int32))
+    assert np.array_equal(a, b) and np.array_equal(ta, tb)
+
+
+def test_ffn_tolerance_covers_bf16_h_rounding():
+    """Rounding h to bfloat16 before the down projection stays inside tol."""
+    rng = np.random.default_rng(25)
+    E, k, T, n_embd, n_ff = 3, 2, 8, 64, 64
+    Wg, Wu, Wd = rand_q8(rng, E, n_ff, n_embd), rand_q8(rng, E, n_ff, n_embd), rand_q8(rng, E, n_embd, n_ff)
+    x = rng.standard_normal((T, n_embd)).astype(np.float32)
+    ids = rand_ids_distinct(rng, T, E, k)
+    y, tol = oracle.ffn(Wg, Wu, Wd, x, "f32", ids)
+    h, _, _ = oracle.ffn_hidden(Wg, Wu, x, "f32", ids, np.arange(T * k))
+    from tests.fixtures import bf16_bits_to_f64, f32_to_bf16_bits
+    hb = bf16_bits_to_f64(f32_to_bf16_bits(h.astype(np.float32)))
+    wd = unpack_q8_0(Wd)
+    yb = np.stack([wd[ids.reshape(-1)[i]] @ hb[i] for i in range(T * k)])
+    assert np.all(np.abs(yb - y) <= tol)
+
+
+# ------------------------------------------------------- input generator
+def test_workload_inputs_are_deterministic_and_shardable():
+    wl = workloads.WORKLOADS["v3"]
+    a = wl.ids(64)
+    b = np.concatenate([wl.ids(32, t0=0), wl.ids(32, t0=32)])
+    assert np.array_equal(a, b)
+    for row in a:
+        assert len(set(row.tolist())) == wl.k
+    xa = wl.x(8)
+    xb = np.concatenate([wl.x(4), wl.x(4, t0=4)])
+    assert np.array_equal(xa, xb)
+    sk = workloads.WORKLOADS["skew"]
+    c = np.bincount(sk.ids(2048).reshape(-1), minlength=sk.n_experts)
+    assert (c == 0).sum() >= sk.n_zero
