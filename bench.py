@@ -1,0 +1,435 @@
+#!/usr/bin/env python
+"""Benchmark of the MoE indirect expert matmul on B200.
+
+Workload (one step): a DeepSeek-V3-shaped routed expert layer, moe_ffn =
+row-id pass + gate/up grouped GEMM with SwiGLU + down grouped GEMM with the
+scatter to dst; 256 experts, top-8, n_embd 7168, expert ffn 2048, Q8_0
+weights (~12 GB), 4096 bf16 tokens per GPU, routing = top-8 of N(0,1) logits
+plus a per-expert N(0, 0.5) bias.  Synthetic, seeded inputs (workloads/).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun every rank runs its own 4096-token batch with replicated
+weights (weak scaling, no data-path collective); the step time is the max
+over ranks.  Rank 0 prints one JSON line.  Also reported: the decode step
+(T = 1, 4, 8 tokens, 256 experts top-8 + a shared expert, n_embd 2048, ffn
+512) as HBM bandwidth, an end-to-end number through host buffers, the
+roofline of the dominant kernel, and the CPU oracle on a bounded sample.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "mul_mat_id tokens/s at pp4096 (V3 shape)"
+WL = workloads.WORKLOADS["v3"]
+DEC = workloads.WORKLOADS["decode"]
+Q8_BYTES_PER_W = 34.0 / 32.0
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained", d["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        load = [s for s in sm if smax and s > 0.3 * smax] or sm
+        return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------ CPU baseline
+def cpu_baseline(budget_s: float = 12.0, t0: int = 0):
+    """The oracle as it stands on a bounded sample of the V3 layer: routed FFN
+    rows of sampled slots (one expert's weights regenerated per sampled slot)."""
+    import oracle
+
+    T = WL.n_tokens[0]
+    ids = WL.ids(T, t0=t0)
+    x = WL.x(T, t0=t0)
+    flat = ids.reshape(-1)
+    rng = np.random.default_rng(1)
+    order = rng.permutation(len(flat))
+    cores = len(os.sched_getaffinity(0))
+    done, elapsed, i = 0, 0.0, 0
+    while elapsed < budget_s and i < len(order):
+        batch = order[i:i + cores]
+        i += len(batch)
+        es = sorted(set(int(flat[s]) for s in batch))
+        remap = {e: j for j, e in enumerate(es)}
+        Wg = np.concatenate([workloads.q8_0_weights_experts(e, 1, WL.n_out, WL.n_in, WL.seed, workloads.T_WG)
+                             for e in es])
+        Wu = np.concatenate([workloads.q8_0_weights_experts(e, 1, WL.n_out, WL.n_in, WL.seed, workloads.T_WU)
+                             for e in es])
+        Wd = np.concatenate([workloads.q8_0_weights_experts(e, 1, WL.n_in, WL.n_out, WL.seed, workloads.T_WD)
+                             for e in es])
+        sub_ids = np.vectorize(lambda e: remap.get(int(e), 0))(ids).astype(np.int32)
+        t = time.perf_counter()
+        oracle.ffn(Wg, Wu, Wd, x, "bf16", sub_ids, slots=np.asarray(batch, np.int64))
+        elapsed += time.perf_counter() - t
+        done += len(batch)
+    tok_s = (done / WL.k) / elapsed
+    return {"value": tok_s, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{done} of {T * WL.k} (token, slot) rows of the V3 moe_ffn (fp64 oracle, "
+                      f"{elapsed:.1f} s), scaled to tokens/s at k={WL.k}"}
+
+
+# ------------------------------------------------------------------ GPU arm
+def upload_prepared(moe, torch, n_experts, n_out, n_in, tensor, seed=0, chunk=16):
+    """Generate a stacked Q8_0 matrix in expert chunks and repack it on the GPU."""
+    per_expert = moe.weights_prepared_size(1, n_out, n_in)
+    out = torch.empty(per_expert * n_experts, dtype=torch.uint8, device="cuda")
+    for e0 in range(0, n_experts, chunk):
+        n_e = min(chunk, n_experts - e0)
+        q = workloads.q8_0_weights_experts(e0, n_e, n_out, n_in, seed, tensor)
+        raw = torch.from_numpy(q).cuda()
+        moe.weights_prepare(raw, n_e, n_out, n_in, out=out[e0 * per_expert:(e0 + n_e) * per_expert])
+        del raw
+    return out
+
+
+def bf16_dev(torch, a):
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def touched_ffn_bytes(ids, n_experts, n_embd, n_ff):
+    used = np.unique(ids.reshape(-1)).size
+    return used, used * 3 * n_embd * n_ff * Q8_BYTES_PER_W
+
+
+def run_ours(args):
+    import torch
+
+    import indirect_expert_matmul_b200 as moe
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    hbm_peak, tc_peak, tc_sust, peak_src = load_peaks()
+
+    E, k, n_embd, n_ff, T = WL.n_experts, WL.k, WL.n_in, WL.n_out, WL.n_tokens[0]
+    S = T * k
+    t0 = rank * T  # each rank its own batch of tokens
+    Wg = upload_prepared(moe, torch, E, n_ff, n_embd, workloads.T_WG)
+    Wu = upload_prepared(moe, torch, E, n_ff, n_embd, workloads.T_WU)
+    Wd = upload_prepared(moe, torch, E, n_embd, n_ff, workloads.T_WD)
+    ids_np = WL.ids(T, t0=t0)
+    x_np = WL.x(T, t0=t0)
+    x = bf16_dev(torch, x_np)
+    ids = torch.from_numpy(ids_np).cuda()
+    ws = moe.workspace(T, k, E, n_embd, n_ff, 0, torch.bfloat16)
+    dst = torch.empty((T, k, n_embd), dtype=torch.float32, device="cuda")
+
+    def step():
+        moe.ffn(Wg, Wu, Wd, E, n_embd, n_ff, x, ids, ws=ws, out=dst)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = moe.get_status(ws)
+    if st != moe.OK:
+        raise RuntimeError(f"device status after warm-up: {moe.status_string(st)}")
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    # ---- timed region (device, resident inputs)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        moe.profile_enable(True)
+        ev0.record()
+        for _ in range(args.steps):
+            step()
+        ev1.record()
+        torch.cuda.synchronize()
+        moe.profile_enable(False)
+    barrier()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    stages = moe.profile_read()
+    st = moe.get_status(ws)
+    if st != moe.OK:
+        raise RuntimeError(f"device status after timed run: {moe.status_string(st)}")
+    if dist is not None:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # algorithmic work of one step
+    used, w_bytes = touched_ffn_bytes(ids_np, E, n_embd, n_ff)
+    x_bytes = T * n_embd * 2
+    h_bytes = S * n_ff * 2
+    dst_bytes = S * n_embd * 4
+    step_bytes = w_bytes + x_bytes + 2 * h_bytes + dst_bytes
+    step_flops = 2.0 * S * n_embd * n_ff * 3
+    gu_bytes = w_bytes * 2 / 3 + x_bytes + h_bytes
+    gu_flops = 2.0 * S * n_embd * n_ff * 2
+    n_gu, ms_gu = stages.get("gemm_gate_up", (0, float("nan")))
+    t_gu = ms_gu / max(n_gu, 1) * 1e-3
+    gu_gbs = gu_bytes / t_gu / 1e9
+    gu_tflops = gu_flops / t_gu / 1e12
+    bound = "hbm" if gu_bytes / (hbm_peak * 1e9) >= gu_flops / (tc_peak * 1e12) else "tensor"
+    if bound == "hbm":
+        roof = {"bound": "hbm", "achieved": round(gu_gbs, 1), "peak": hbm_peak, "unit": "GB/s",
+                "frac": round(gu_gbs / hbm_peak, 4)}
+    else:
+        roof = {"bound": "tensor", "achieved": round(gu_tflops, 1), "peak": tc_peak, "unit": "TFLOP/s",
+                "frac": round(gu_tflops / tc_peak, 4)}
+    roof.update({"traffic": args.traffic, "kernel": "grouped_gemm_kernel<1> (gate/up + SwiGLU)",
+                 "peak_source": peak_src, "ms_per_launch": round(t_gu * 1e3, 4),
+                 "tensor_tflops": round(gu_tflops, 1), "tensor_frac": round(gu_tflops / tc_peak, 4),
+                 "algorithmic_bytes": int(gu_bytes), "flops": gu_flops})
+    step_roof_ms = max(step_bytes / (hbm_peak * 1e9), step_flops / (tc_peak * 1e12)) * 1e3
+    launches_per_step = sum(n for n, _ in stages.values()) / args.steps
+
+    result = {
+        "metric": METRIC, "value": round(T * world / (ms * 1e-3), 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "v3 moe_ffn: 256 experts top-8, n_embd 7168, expert ffn 2048, Q8_0 gate/up/down, "
+                               "bf16 x, 4096 tokens per GPU, biased top-8 routing",
+                   "tokens_per_gpu": T, "experts_touched": int(used),
+                   "l2": "inputs larger than L2 (12 GB of weights per step)", "parallelism": f"dp{world}"},
+        "tflops": round(step_flops * world / (ms * 1e-3) / 1e12, 1),
+        "step_roofline": {"ms": round(step_roof_ms, 4), "frac": round(step_roof_ms / ms, 4),
+                          "bytes": int(step_bytes), "flops": step_flops},
+        "stages_ms_per_step": {k_: round(v[1] / args.steps, 4) for k_, v in stages.items()},
+        "roofline": roof,
+        "gpu_launches": int(round(launches_per_step * args.steps)),
+    }
+    result["clocks"] = clk.summary()
+
+    # ---- end to end through host buffers (pinned), same metric
+    if not args.no_e2e:
+        x_pin = torch.from_numpy(np.ascontiguousarray(x_np).view(np.int16)).view(torch.bfloat16).pin_memory()
+        ids_pin = torch.from_numpy(ids_np).pin_memory()
+        dst_pin = torch.empty((T, k, n_embd), dtype=torch.float32).pin_memory()
+
+        def e2e_step():
+            x.copy_(x_pin, non_blocking=True)
+            ids.copy_(ids_pin, non_blocking=True)
+            moe.ffn(Wg, Wu, Wd, E, n_embd, n_ff, x, ids, ws=ws, out=dst)
+            dst_pin.copy_(dst, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        ev0.record()
+        n_e2e = max(2, min(args.steps, 5))
+        for _ in range(n_e2e):
+            e2e_step()
+        ev1.record()
+        torch.cuda.synchronize()
+        barrier()
+        ms_e2e = ev0.elapsed_time(ev1) / n_e2e
+        if dist is not None:
+            t = torch.tensor([ms_e2e], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms_e2e = float(t.item())
+        result["e2e"] = {"value": round(T * world / (ms_e2e * 1e-3), 1), "unit": "tokens/s",
+                         "h2d_bytes_per_step": int(x_bytes + ids_np.nbytes), "d2h_bytes_per_step": int(dst_bytes),
+                         "ms_per_step": round(ms_e2e, 3)}
+        del x_pin, dst_pin
+
+    del Wg, Wu, Wd
+    torch.cuda.empty_cache()
+    if not args.no_decode:
+        result["decode"] = run_decode(moe, torch, args, hbm_peak)
+
+    if rank == 0 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+def run_decode(moe, torch, args, hbm_peak):
+    """Decode step: n_layers distinct layer copies (beyond L2), fresh routing per
+    layer, replayed as one CUDA graph per token count."""
+    E, k, n_embd, n_ff, n_sh = DEC.n_experts, DEC.k, DEC.n_in, DEC.n_out, DEC.n_ff_shared
+    L = args.decode_layers
+    base_g = upload_prepared(moe, torch, E, n_ff, n_embd, workloads.T_WG)
+    base_u = upload_prepared(moe, torch, E, n_ff, n_embd, workloads.T_WU)
+    base_d = upload_prepared(moe, torch, E, n_embd, n_ff, workloads.T_WD)
+    sh = [upload_prepared(moe, torch, 1, n_sh, n_embd, workloads.T_SG),
+          upload_prepared(moe, torch, 1, n_sh, n_embd, workloads.T_SU),
+          upload_prepared(moe, torch, 1, n_embd, n_sh, workloads.T_SD)]
+    layers = [(base_g, base_u, base_d)] + [(base_g.clone(), base_u.clone(), base_d.clone()) for _ in range(L - 1)]
+    shared = [[t.clone() for t in sh] for _ in range(L)]
+    per_expert = 3 * n_embd * n_ff * Q8_BYTES_PER_W
+    per_shared = 3 * n_embd * n_sh * Q8_BYTES_PER_W
+    out = {}
+    for T in DEC.n_tokens:
+        x = bf16_dev(torch, DEC.x(T))
+        ids = [torch.from_numpy(DEC.ids(T, layer=l)).cuda() for l in range(L)]
+        touched = sum(np.unique(i.cpu().numpy()).size for i in ids)
+        ws = [moe.workspace(T, k, E, n_embd, n_ff, n_sh, torch.bfloat16) for _ in range(L)]
+        dst = [torch.empty((T, k, n_embd), dtype=torch.float32, device="cuda") for _ in range(L)]
+        dsh = [torch.empty((T, n_embd), dtype=torch.float32, device="cuda") for _ in range(L)]
+
+        def all_layers():
+            for l in range(L):
+                g, u, d = layers[l]
+                moe.ffn(g, u, d, E, n_embd, n_ff, x, ids[l], shared=(*shared[l], n_sh), ws=ws[l], out=dst[l],
+                        out_shared=dsh[l])
+
+        all_layers()
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            with torch.cuda.graph(graph, stream=s):
+                all_layers()
+        torch.cuda.current_stream().wait_stream(s)
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 20
+        ev0.record()
+        for _ in range(reps):
+            graph.replay()
+        ev1.record()
+        torch.cuda.synchronize()
+        ms = ev0.elapsed_time(ev1) / reps
+        for w in ws:
+            st = moe.get_status(w)
+            if st != moe.OK:
+                raise RuntimeError(f"decode T={T}: {moe.status_string(st)}")
+        bytes_step = touched * per_expert + L * per_shared
+        gbs = bytes_step / (ms * 1e-3) / 1e9
+        out[f"T={T}"] = {"us_per_layer": round(ms * 1e3 / L, 2), "GB/s": round(gbs, 1),
+                         "frac_of_hbm": round(gbs / hbm_peak, 4), "layers": L,
+                         "experts_touched_per_layer": round(touched / L, 2)}
+        del graph
+    del layers, shared, base_g, base_u, base_d
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_reference(args):
+    """The oracle timed on the host cores on a bounded sample of the same workload."""
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    per_step = []
+    cb = None
+    for _ in range(args.warmup + args.steps):
+        cb = cpu_baseline(args.cpu_seconds / 4)
+        per_step.append(cb["value"])
+    vals = per_step[args.warmup:]
+    v = statistics.median(vals)
+    ms = WL.n_tokens[0] / v * 1e3
+    line = {"impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 1), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "v3 moe_ffn: 256 experts top-8, n_embd 7168, expert ffn 2048, Q8_0 gate/up/down, "
+                                   "bf16 x, 4096 tokens per GPU, biased top-8 routing", "parallelism": "host"},
+            "cpu_baseline": {"value": round(v, 3), "unit": "tokens/s", "cores": cb["cores"], "kind": "oracle",
+                             "sample": cb["sample"]},
+            "e2e": {"value": round(v, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--decode-layers", type=int, default=16)
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="dram bytes per launch of the dominant kernel from an ncu capture (null if stale)")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

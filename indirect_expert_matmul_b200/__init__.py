@@ -1,0 +1,229 @@
+"""B200-native MoE indirect matrix multiplication (GGML_OP_MUL_MAT_ID).
+
+Thin ctypes binding of ``libmoe_b200.so`` (C ABI in ``include/moe.h``).
+Every function here only marshals arguments: it takes torch CUDA tensors for
+device memory and the current torch stream, and calls the library.  All
+arithmetic runs in the library's sm_100a kernels; there is no CPU or PyTorch
+fallback, and importing fails loudly if the library has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
+
+OK, ERR_INVALID, ERR_RANGE, ERR_BAD_ID, ERR_CUDA, ERR_TIMEOUT, ERR_UNSUPPORTED = 0, -1, -2, -3, -4, -5, -6
+BROADCAST, PER_SLOT = 0, 1
+BF16, F16, F32 = 0, 1, 2
+
+# every symbol declared in include/moe.h
+ABI_SYMBOLS = (
+    "moe_status_string", "moe_workspace_size", "moe_workspace_init", "moe_get_status",
+    "moe_weights_prepared_size", "moe_weights_prepare", "moe_row_ids", "moe_mul_mat_id", "moe_ffn",
+    "moe_set_gemv_threshold", "moe_get_gemv_threshold", "moe_set_path", "moe_profile_enable", "moe_profile_read",
+)
+
+_lib = None
+_vp, _i32, _i64, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+
+
+def _L() -> ctypes.CDLL:
+    """The loaded library; raises ImportError when it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing; build it with `python -m indirect_expert_matmul_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    L.moe_status_string.argtypes = [_i32]
+    L.moe_status_string.restype = ctypes.c_char_p
+    L.moe_workspace_size.argtypes = [_i64, _i32, _i32, _i32, _i32, _i32, _i32]
+    L.moe_workspace_size.restype = _sz
+    L.moe_workspace_init.argtypes = [_vp, _vp]
+    L.moe_get_status.argtypes = [_vp, _vp]
+    L.moe_weights_prepared_size.argtypes = [_i32, _i32, _i32]
+    L.moe_weights_prepared_size.restype = _sz
+    L.moe_weights_prepare.argtypes = [_vp, _i32, _i32, _i32, _vp, _vp]
+    L.moe_row_ids.argtypes = [_vp, _i64, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp]
+    L.moe_mul_mat_id.argtypes = [_vp, _i32, _i32, _i32, _vp, _i32, _vp, _i64, _i32, _i32, _vp, _vp, _vp]
+    L.moe_ffn.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _i32, _vp, _i64, _i32,
+                          _vp, _vp, _vp, _vp]
+    L.moe_set_gemv_threshold.argtypes = [_i32]
+    L.moe_set_gemv_threshold.restype = None
+    L.moe_get_gemv_threshold.argtypes = []
+    L.moe_set_path.argtypes = [_i32]
+    L.moe_set_path.restype = None
+    L.moe_profile_enable.argtypes = [_i32]
+    L.moe_profile_enable.restype = None
+    L.moe_profile_read.argtypes = [ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(_i32),
+                                   ctypes.POINTER(ctypes.c_double), _i32]
+    _lib = L
+    return L
+
+
+class MoeError(RuntimeError):
+    def __init__(self, code: int, what: str = ""):
+        self.code = code
+        super().__init__(f"{what}: {status_string(code)} ({code})")
+
+
+def status_string(code: int) -> str:
+    return _L().moe_status_string(code).decode()
+
+
+def lib() -> ctypes.CDLL:
+    return _L()
+
+
+def _chk(rc: int, what: str):
+    if rc != OK:
+        raise MoeError(rc, what)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device=None):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+_XTYPE = {torch.bfloat16: BF16, torch.float16: F16, torch.float32: F32}
+_MODE = {"broadcast": BROADCAST, "per_slot": PER_SLOT, BROADCAST: BROADCAST, PER_SLOT: PER_SLOT}
+
+
+def _cuda(t, name, dtype=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}")
+    return t
+
+
+# ----------------------------------------------------------------- memory
+def workspace_size(n_tokens, k, n_experts, n_in, n_hidden=0, n_hidden_shared=0, x_dtype=torch.bfloat16) -> int:
+    return _L().moe_workspace_size(n_tokens, k, n_experts, n_in, n_hidden, n_hidden_shared, _XTYPE[x_dtype])
+
+
+def workspace(n_tokens, k, n_experts, n_in, n_hidden=0, n_hidden_shared=0, x_dtype=torch.bfloat16, device="cuda"):
+    """A zero-status workspace tensor (uint8) for calls of these sizes."""
+    n = workspace_size(n_tokens, k, n_experts, n_in, n_hidden, n_hidden_shared, x_dtype)
+    ws = torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+    _chk(_L().moe_workspace_init(_ptr(ws), _stream(ws.device)), "moe_workspace_init")
+    return ws
+
+
+def get_status(ws) -> int:
+    """Synchronise the current stream, return and clear the device status."""
+    return _L().moe_get_status(_ptr(ws), _stream(ws.device))
+
+
+# ---------------------------------------------------------------- weights
+def weights_prepared_size(n_experts, n_out, n_in) -> int:
+    return _L().moe_weights_prepared_size(n_experts, n_out, n_in)
+
+
+def weights_prepare(q8_0, n_experts, n_out, n_in, out=None):
+    """Repack Q8_0 blocks (uint8 [E][n_out][n_in/32][34], on the GPU)."""
+    _cuda(q8_0, "q8_0", torch.uint8)
+    n = weights_prepared_size(n_experts, n_out, n_in)
+    if out is None:
+        out = torch.empty(n, dtype=torch.uint8, device=q8_0.device)
+    _chk(_L().moe_weights_prepare(_ptr(q8_0), n_experts, n_out, n_in, _ptr(out), _stream(q8_0.device)),
+         "moe_weights_prepare")
+    return out
+
+
+# ----------------------------------------------------------------- row ids
+def row_ids(ids, n_experts, mode="broadcast", ws=None):
+    """(ids_src1, ids_dst, expert_bounds) int32 tensors of the stable counting sort."""
+    _cuda(ids, "ids", torch.int32)
+    T, k = ids.shape
+    S = T * k
+    dev = ids.device
+    src1 = torch.empty(max(S, 1), dtype=torch.int32, device=dev)
+    dst = torch.empty(max(S, 1), dtype=torch.int32, device=dev)
+    bounds = torch.empty(n_experts + 1, dtype=torch.int32, device=dev)
+    if ws is None:
+        ws = workspace(T, k, n_experts, 0, device=dev)
+    _chk(_L().moe_row_ids(_ptr(ids), T, k, n_experts, _MODE[mode], _ptr(src1), _ptr(dst), _ptr(bounds), _ptr(ws),
+                          _stream(dev)), "moe_row_ids")
+    return src1[:S], dst[:S], bounds
+
+
+# --------------------------------------------------------------- operators
+def mul_mat_id(W, n_experts, n_out, n_in, x, ids, mode="broadcast", ws=None, out=None):
+    """dst float32 [T][k][n_out] = W[ids[t][s]] . x[t or (t, s)]."""
+    _cuda(W, "W", torch.uint8)
+    _cuda(x, "x")
+    _cuda(ids, "ids", torch.int32)
+    T, k = ids.shape
+    if ws is None:
+        ws = workspace(T, k, n_experts, n_in, x_dtype=x.dtype, device=x.device)
+    if out is None:
+        out = torch.empty((T, k, n_out), dtype=torch.float32, device=x.device)
+    _chk(_L().moe_mul_mat_id(_ptr(W), n_experts, n_out, n_in, _ptr(x), _XTYPE[x.dtype], _ptr(ids), T, k,
+                             _MODE[mode], _ptr(out), _ptr(ws), _stream(x.device)), "moe_mul_mat_id")
+    return out
+
+
+def ffn(Wg, Wu, Wd, n_experts, n_embd, n_ff, x, ids, shared=None, ws=None, out=None, out_shared=None):
+    """Routed SwiGLU expert FFN (+ optional shared expert (Sg, Su, Sd, n_ff_shared)).
+
+    Returns (dst [T][k][n_embd], dst_shared [T][n_embd] or None), float32."""
+    for name, t in (("Wg", Wg), ("Wu", Wu), ("Wd", Wd)):
+        _cuda(t, name, torch.uint8)
+    _cuda(x, "x")
+    _cuda(ids, "ids", torch.int32)
+    T, k = ids.shape
+    Sg = Su = Sd = None
+    n_ff_sh = 0
+    if shared is not None:
+        Sg, Su, Sd, n_ff_sh = shared
+    if ws is None:
+        ws = workspace(T, k, n_experts, n_embd, n_ff, n_ff_sh, x.dtype, device=x.device)
+    if out is None:
+        out = torch.empty((T, k, n_embd), dtype=torch.float32, device=x.device)
+    if shared is not None and out_shared is None:
+        out_shared = torch.empty((T, n_embd), dtype=torch.float32, device=x.device)
+    _chk(_L().moe_ffn(_ptr(Wg), _ptr(Wu), _ptr(Wd), n_experts, n_embd, n_ff, _ptr(Sg), _ptr(Su), _ptr(Sd), n_ff_sh,
+                      _ptr(x), _XTYPE[x.dtype], _ptr(ids), T, k, _ptr(out), _ptr(out_shared), _ptr(ws),
+                      _stream(x.device)), "moe_ffn")
+    return out, out_shared
+
+
+# ------------------------------------------------------------------ tuning
+def set_gemv_threshold(n: int):
+    _L().moe_set_gemv_threshold(n)
+
+
+def get_gemv_threshold() -> int:
+    return _L().moe_get_gemv_threshold()
+
+
+def set_path(path: int):
+    """0 = by threshold, 1 = mat-vec kernel, 2 = grouped tensor-core GEMM."""
+    _L().moe_set_path(path)
+
+
+# --------------------------------------------------------------- profiling
+def profile_enable(on: bool = True):
+    """Record CUDA events between the library's kernels (see moe_profile_enable)."""
+    _L().moe_profile_enable(1 if on else 0)
+
+
+def profile_read(max_stages: int = 32) -> dict:
+    """{stage name: (launches, total device ms)} of the calls recorded so far."""
+    names = (ctypes.c_char_p * max_stages)()
+    launches = (_i32 * max_stages)()
+    ms = (ctypes.c_double * max_stages)()
+    n = _L().moe_profile_read(names, launches, ms, max_stages)
+    if n < 0:
+        raise MoeError(n, "moe_profile_read")
+    return {names[i].decode(): (launches[i], ms[i]) for i in range(n)}

@@ -1,0 +1,96 @@
+// Shared definitions of the sm_100a MoE indirect-matmul library: status
+// handling, workspace and repacked-weight layouts, and thin PTX wrappers.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "moe.h"
+
+namespace moe {
+
+// ----------------------------------------------------------------- limits
+constexpr int kMaxExperts = 16384;
+constexpr int64_t kMaxTokens = (int64_t)1 << 22;  // exclusive
+constexpr int kMaxK = 1 << 10;                      // exclusive
+
+// ------------------------------------------------------- device status word
+// The first error sticks (compare-and-swap from MOE_OK).
+__device__ __forceinline__ void set_status(int* status, int code) { atomicCAS(status, 0, code); }
+__device__ __forceinline__ int read_status(const int* status) { return *(volatile const int*)status; }
+
+// ------------------------------------------------------------ repacked weights
+// Tile-major form: per expert, per 128-row tile mt, per 64-column tile kt, one
+// block of rows(mt) rows: rows*64 bytes of u = q + 128, then rows*4 bytes of
+// scales (two fp16 per row: columns [0,32) and [32,64) of the tile).
+// rows(mt) = min(128, n_out_pad - 128*mt), n_out_pad = round_up(n_out, 16).
+constexpr int kTileM = 128;
+constexpr int kTileK = 64;
+constexpr int kRowBytes = kTileK + 4;  // 64 q bytes + 2 fp16 scales
+
+struct WLayout {
+    int n_out, n_in, n_out_pad, kt_count, mt_count;
+    int64_t expert_bytes;
+    __host__ __device__ WLayout() {}
+    __host__ __device__ WLayout(int n_out_, int n_in_) : n_out(n_out_), n_in(n_in_) {
+        n_out_pad = (n_out + 15) / 16 * 16;
+        kt_count = (n_in + kTileK - 1) / kTileK;
+        mt_count = (n_out_pad + kTileM - 1) / kTileM;
+        expert_bytes = (int64_t)n_out_pad * kt_count * kRowBytes;
+    }
+    __host__ __device__ int rows(int mt) const {
+        int r = n_out_pad - mt * kTileM;
+        return r < kTileM ? r : kTileM;
+    }
+    // byte offset of block (e, mt, kt)
+    __host__ __device__ int64_t block(int e, int mt, int kt) const {
+        return e * expert_bytes + (int64_t)mt * kTileM * kt_count * kRowBytes + (int64_t)rows(mt) * kt * kRowBytes;
+    }
+};
+
+// ------------------------------------------------------------------ workspace
+struct WsLayout {
+    int64_t S;
+    size_t hdr, src1, dst, bounds, active, tiles, h, h_sh, x16, total;
+    static size_t up(size_t v) { return (v + 255) / 256 * 256; }
+    WsLayout(int64_t n_tokens, int k, int n_experts, int n_in, int n_hidden, int n_hidden_sh, int x_type) {
+        S = n_tokens * k;
+        size_t o = 0;
+        hdr = o; o += 256;
+        src1 = o; o += up(S * 4);
+        dst = o; o += up(S * 4);
+        bounds = o; o += up((size_t)(n_experts + 1) * 4);
+        active = o; o += up((size_t)(n_experts + 1) * 4);
+        tiles = o; o += up((size_t)(n_experts + 1) * 4);
+        h = o; o += up((size_t)S * n_hidden * 2);
+        h_sh = o; o += up((size_t)n_tokens * n_hidden_sh * 2);
+        x16 = o; o += (x_type == MOE_F32) ? up((size_t)S * n_in * 2) : 0;
+        total = o;
+    }
+};
+// header words
+constexpr int kHdrStatus = 0;
+constexpr int kHdrActive = 1;
+constexpr int kHdrTiles = 2;   // total column tiles of the grouped GEMM
+constexpr int kGemmBN = 256;   // column (token) tile of the grouped GEMM
+
+// ---------------------------------------------------------------- profiling
+void prof_begin(cudaStream_t s);                     // start of an operator call
+void prof_mark(cudaStream_t s, const char* stage);   // after the launch of `stage`
+
+// ------------------------------------------------------------------ dequant
+// u = q + 128 as a byte; f = as_float(0x47000000 | u << 8) = 32768 + u exactly.
+// fma(f, d, -32896*d) = (u - 128) * d = q * d, exact in fp32: q*d needs at most
+// 7 + 11 significant bits and 32896*d at most 9 + 11, so neither the constant
+// nor the single rounding of the fma loses anything.
+__device__ __forceinline__ float magic_byte(uint32_t word, int byte) {
+    uint32_t f;
+    // select byte `byte` of word into bits 8..15 of 0x47000000
+    const uint32_t sel = 0x7404u | ((uint32_t)byte << 4);
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(f) : "r"(word), "r"(0x47000000u), "r"(sel));
+    return __uint_as_float(f);
+}
+
+}  // namespace moe

@@ -1,0 +1,605 @@
+// Grouped per-expert GEMM on the sm_100a tensor cores with the Q8_0
+// dequantisation fused into the tile pipeline - the prompt-size path of
+// GGML_OP_MUL_MAT_ID (the PR #283 article "ik_llama.cpp 的 CUDA 更优 MoE 实现",
+// sections 2.1 and 6: gather src1 rows by ids_src1, multiply per expert, write
+// dst rows by ids_dst), restated for Blackwell.
+//
+// Tile = (expert e, column tile j of up to 256 of the expert's sorted slots,
+// row tile mt of 128 output rows).  One persistent CTA per SM walks tiles in
+// (e, j, mt) order, so CTAs running together share the gathered activations
+// (and an expert's later column tiles find its weights in L2).  Every output
+// element is produced by exactly one CTA with one fixed reduction order: the
+// result is bit-identical from run to run.
+//
+// Warp roles (512 threads):
+//   warp 0      producer: 1-D bulk copies of the repacked int8+scale weight
+//               blocks, and TMA tile::gather4 loads of the activation rows
+//               named by the row table (4 rows per instruction, 32 lanes
+//               issuing in parallel).
+//   warp 1      TMEM allocation and the single thread issuing tcgen05.mma
+//               (M=128, N=16..256, K=16 per instruction, fp32 accumulators).
+//   warps 4-7   epilogue: tcgen05.ld of the accumulators; scatter fp32 rows to
+//               dst by ids_dst, or SwiGLU of the gate/up pair to bf16 h.
+//   warps 8-15  dequantisation: int8 q + fp16 d in shared memory -> exact fp32
+//               q*d -> bf16 or fp16, written in the 128-byte-swizzled K-major
+//               layout the tensor core reads.
+// All waits are bounded; an expired wait sets MOE_ERR_TIMEOUT in the status
+// word and every role leaves its loop.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "gemm_api.cuh"
+#include "ptx.cuh"
+
+namespace moe {
+
+constexpr int kGemmThreads = 512;
+constexpr int kWarpProducer = 0;
+constexpr int kWarpMma = 1;
+constexpr int kEpiWarp0 = 4;
+constexpr int kDeqWarp0 = 8;
+constexpr int kDeqWarps = 8;
+constexpr uint32_t kATileBytes = kTileM * kTileK * 2;  // 16 KB
+constexpr uint32_t kBTileBytes = kGemmBN * kTileK * 2; // 32 KB
+constexpr uint32_t kRawBytes = kTileM * kRowBytes;     // 8704
+constexpr int kSmemGroups = 1024;                      // schedule tables kept in shared memory up to this
+constexpr long long kWaitLimitCycles = 1ll << 32;      // ~2 s
+
+template <int DUAL>
+struct Cfg {
+    static constexpr int NMAT = DUAL + 1;
+    static constexpr int MS = DUAL ? 2 : 3;  // operand stages (A bf16 + B)
+    static constexpr int RS = 4;             // raw weight stages
+    static constexpr uint32_t a_off = 0;
+    static constexpr uint32_t b_off = a_off + MS * NMAT * kATileBytes;
+    static constexpr uint32_t raw_off = b_off + MS * kBTileBytes;
+    static constexpr uint32_t bar_off = raw_off + RS * NMAT * kRawBytes;
+    static constexpr int n_bars = 2 * RS + 3 * MS + 4;
+    static constexpr uint32_t misc_off = bar_off + n_bars * 8;
+    static constexpr uint32_t smem_bytes = misc_off + 64 + 1024;  // + alignment slack
+};
+
+struct GemmParams {
+    const uint8_t* A0;
+    const uint8_t* A1;
+    WLayout L;
+    int n_groups;               // > 0: grouped by bounds / ntile_prefix; 0: one group of n_rows
+    const int32_t* bounds;      // [n_groups + 1]
+    const int32_t* ntile_prefix;// [n_groups + 1]
+    int n_rows;
+    const int32_t* src_rows;    // B row of sorted position p (null: p)
+    const int32_t* dst_rows;    // output row of sorted position p (null: p)
+    float* out;                 // single-matrix output
+    __nv_bfloat16* h;           // dual output (SwiGLU)
+    int out_ld;
+    int* hdr;
+    int bf16;                   // operand type: 1 bf16, 0 fp16
+    int grid_tiles_hint;
+};
+
+struct Tile {
+    int e, mt, p0, n;
+};
+
+__device__ __forceinline__ Tile decode_tile(int t, int mt_count, const GemmParams& p, const int* s_prefix,
+                                            const int* s_bounds) {
+    Tile r;
+    const int q = t / mt_count;
+    r.mt = t - q * mt_count;
+    if (p.n_groups == 0) {
+        r.e = 0;
+        r.p0 = q * kGemmBN;
+        r.n = min(kGemmBN, p.n_rows - r.p0);
+        return r;
+    }
+    const int* pre = p.n_groups <= kSmemGroups ? s_prefix : p.ntile_prefix;
+    const int* bnd = p.n_groups <= kSmemGroups ? s_bounds : p.bounds;
+    // largest e with pre[e] <= q (empty experts share their successor's prefix)
+    int lo = 0, hi = p.n_groups;  // invariant: pre[lo] <= q < pre[hi]
+    while (hi - lo > 1) {
+        int mid = (lo + hi) >> 1;
+        if (pre[mid] <= q) lo = mid; else hi = mid;
+    }
+    r.e = lo;
+    const int j = q - pre[lo];
+    r.p0 = bnd[lo] + j * kGemmBN;
+    r.n = min(kGemmBN, bnd[lo + 1] - r.p0);
+    return r;
+}
+
+// Bounded wait by one lane; false when the kernel is aborting.
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (true) {
+        if (ptx::mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (clock64() - t0 > kWaitLimitCycles) {
+            *abort_flag = 1;
+            set_status(status, MOE_ERR_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+// lane 0 waits, the warp learns the outcome
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status) {
+    int ok = 1;
+    if ((threadIdx.x & 31) == 0) ok = wait_bar(bar, parity, abort_flag, status);
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+__device__ __forceinline__ uint32_t pack2(float lo, float hi, int bf16) {
+    if (bf16) {
+        __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+        return *(uint32_t*)&v;
+    }
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *(uint32_t*)&v;
+}
+
+template <int DUAL>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmB, const GemmParams p) {
+    using C = Cfg<DUAL>;
+    extern __shared__ uint8_t smem_dyn[];
+    __shared__ int s_prefix[kSmemGroups + 1];
+    __shared__ int s_bounds[kSmemGroups + 1];
+
+    if (read_status(p.hdr + kHdrStatus) != 0) return;
+
+    uint8_t* smem = (uint8_t*)(((uintptr_t)smem_dyn + 1023) & ~(uintptr_t)1023);
+    uint8_t* sA = smem + C::a_off;
+    uint8_t* sB = smem + C::b_off;
+    uint8_t* sRaw = smem + C::raw_off;
+    uint64_t* bars = (uint64_t*)(smem + C::bar_off);
+    uint64_t* raw_full = bars;
+    uint64_t* raw_empty = raw_full + C::RS;
+    uint64_t* a_full = raw_empty + C::RS;
+    uint64_t* b_full = a_full + C::MS;
+    uint64_t* mma_empty = b_full + C::MS;
+    uint64_t* tmem_full = mma_empty + C::MS;
+    uint64_t* tmem_empty = tmem_full + 2;
+    uint32_t* tmem_base_sh = (uint32_t*)(smem + C::misc_off);
+    volatile int* abort_flag = (volatile int*)(smem + C::misc_off + 4);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const WLayout L = p.L;
+    const int MT = L.mt_count, KT = L.kt_count;
+
+    if (tid == 0) {
+        for (int i = 0; i < C::RS; ++i) {
+            ptx::mbar_init(&raw_full[i], 1);
+            ptx::mbar_init(&raw_empty[i], kDeqWarps);
+        }
+        for (int i = 0; i < C::MS; ++i) {
+            ptx::mbar_init(&a_full[i], kDeqWarps);
+            ptx::mbar_init(&b_full[i], 1);
+            ptx::mbar_init(&mma_empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            ptx::mbar_init(&tmem_full[i], 1);
+            ptx::mbar_init(&tmem_empty[i], 4);
+        }
+        *abort_flag = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == kWarpMma) {
+        ptx::tmem_alloc(tmem_base_sh, 512);
+        ptx::tmem_relinquish();
+    }
+    if (p.n_groups > 0 && p.n_groups <= kSmemGroups) {
+        for (int i = tid; i <= p.n_groups; i += kGemmThreads) {
+            s_prefix[i] = p.ntile_prefix[i];
+            s_bounds[i] = p.bounds[i];
+        }
+    }
+    const int n_coltiles = p.n_groups > 0 ? p.hdr[kHdrTiles] : (p.n_rows + kGemmBN - 1) / kGemmBN;
+    const int total = n_coltiles * MT;
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem_base = *tmem_base_sh;
+
+    if (warp == kWarpProducer) {
+        // ------------------------------------------------------------ producer
+        int rs = 0, ms = 0;
+        uint32_t rph = 0, mph = 0;
+        uint32_t raw_used = 0, raw_par = 0, b_used = 0, b_par = 0;  // per-stage issue record, for draining
+        bool ok = true;
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            const Tile tl = decode_tile(t, MT, p, s_prefix, s_bounds);
+            const int n16 = (tl.n + 15) & ~15;
+            int rows4[2][4];
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const int g = lane + 32 * i;
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    const int pos = tl.p0 + min(4 * g + r, tl.n - 1);
+                    rows4[i][r] = p.src_rows ? __ldg(p.src_rows + pos) : pos;
+                }
+            }
+            const int rows = L.rows(tl.mt);
+            const uint32_t raw_bytes = (uint32_t)rows * kRowBytes;
+            const uint8_t* a0 = p.A0 + L.block(tl.e, tl.mt, 0);
+            const uint8_t* a1 = DUAL ? p.A1 + L.block(tl.e, tl.mt, 0) : nullptr;
+            for (int kt = 0; kt < KT; ++kt) {
+                // weights: raw int8 + scales of both matrices
+                if (lane == 0) {
+                    ok = wait_bar(&raw_empty[rs], rph ^ 1, abort_flag, p.hdr + kHdrStatus);
+                    if (ok) {
+                        ptx::mbar_arrive_expect_tx(&raw_full[rs], raw_bytes * C::NMAT);
+                        ptx::bulk_g2s(sRaw + (rs * C::NMAT) * kRawBytes, a0 + (size_t)kt * raw_bytes, raw_bytes,
+                                      &raw_full[rs]);
+                        if (DUAL)
+                            ptx::bulk_g2s(sRaw + (rs * C::NMAT + 1) * kRawBytes, a1 + (size_t)kt * raw_bytes,
+                                          raw_bytes, &raw_full[rs]);
+                        raw_used |= 1u << rs;
+                        raw_par = (raw_par & ~(1u << rs)) | (rph << rs);
+                    }
+                }
+                ok = __shfl_sync(0xffffffffu, (int)ok, 0) != 0;
+                if (!ok) break;
+                if (++rs == C::RS) { rs = 0; rph ^= 1; }
+                // activations: gathered rows of this column tile
+                if (lane == 0) {
+                    ok = wait_bar(&mma_empty[ms], mph ^ 1, abort_flag, p.hdr + kHdrStatus);
+                    if (ok) {
+                        ptx::mbar_arrive_expect_tx(&b_full[ms], (uint32_t)n16 * 128u);
+                        b_used |= 1u << ms;
+                        b_par = (b_par & ~(1u << ms)) | (mph << ms);
+                    }
+                }
+                ok = __shfl_sync(0xffffffffu, (int)ok, 0) != 0;
+                if (!ok) break;
+                uint8_t* bdst = sB + ms * kBTileBytes;
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const int g = lane + 32 * i;
+                    if (4 * g < n16)
+                        ptx::tma_gather4(bdst + g * 512, &tmB, kt * kTileK, rows4[i][0], rows4[i][1], rows4[i][2],
+                                         rows4[i][3], &b_full[ms]);
+                }
+                if (++ms == C::MS) { ms = 0; mph ^= 1; }
+            }
+        }
+        // before leaving, let every copy this warp issued land (bounded)
+        if (lane == 0) {
+            volatile int never = 0;
+            for (int s = 0; s < C::RS; ++s)
+                if (raw_used >> s & 1) wait_bar(&raw_full[s], (raw_par >> s) & 1, &never, p.hdr + kHdrStatus);
+            for (int s = 0; s < C::MS; ++s)
+                if (b_used >> s & 1) wait_bar(&b_full[s], (b_par >> s) & 1, &never, p.hdr + kHdrStatus);
+        }
+    } else if (warp == kWarpMma) {
+        // ----------------------------------------------------------------- MMA
+        if (lane == 0) {
+            int ms = 0;
+            uint32_t mph = 0;
+            uint32_t use[2] = {0, 0};
+            int it = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
+                const Tile tl = decode_tile(t, MT, p, s_prefix, s_bounds);
+                const int n16 = (tl.n + 15) & ~15;
+                const int buf = DUAL ? 0 : (it & 1);
+                ok = wait_bar(&tmem_empty[buf], (use[buf] & 1) ^ 1, abort_flag, p.hdr + kHdrStatus);
+                if (!ok) break;
+                ptx::tc_fence_after();
+                const uint32_t d0 = tmem_base + (DUAL ? 0u : (uint32_t)buf * 256u);
+                const uint32_t d1 = tmem_base + 256u;
+                const uint32_t idesc = ptx::idesc_f16(p.bf16, n16, 128);
+                for (int kt = 0; kt < KT; ++kt) {
+                    ok = wait_bar(&a_full[ms], mph, abort_flag, p.hdr + kHdrStatus) &&
+                         wait_bar(&b_full[ms], mph, abort_flag, p.hdr + kHdrStatus);
+                    if (!ok) break;
+                    ptx::tc_fence_after();
+                    const uint32_t a0 = ptx::smem_u32(sA + (ms * C::NMAT) * kATileBytes);
+                    const uint32_t a1 = a0 + kATileBytes;
+                    const uint32_t b = ptx::smem_u32(sB + ms * kBTileBytes);
+#pragma unroll
+                    for (int kk = 0; kk < kTileK / 16; ++kk) {
+                        const uint32_t acc = (kt | kk) != 0;
+                        ptx::mma_f16_ss(d0, ptx::desc_k_sw128(a0 + kk * 32), ptx::desc_k_sw128(b + kk * 32), idesc,
+                                        acc);
+                        if (DUAL)
+                            ptx::mma_f16_ss(d1, ptx::desc_k_sw128(a1 + kk * 32), ptx::desc_k_sw128(b + kk * 32),
+                                            idesc, acc);
+                    }
+                    ptx::mma_commit(&mma_empty[ms]);
+                    if (++ms == C::MS) { ms = 0; mph ^= 1; }
+                }
+                if (!ok) break;
+                ptx::mma_commit(&tmem_full[buf]);
+                use[buf] += 1;
+            }
+        }
+        __syncwarp();
+    } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
+        // ------------------------------------------------------------ epilogue
+        const int ew = warp - kEpiWarp0;
+        uint32_t use[2] = {0, 0};
+        int it = 0;
+        for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
+            const Tile tl = decode_tile(t, MT, p, s_prefix, s_bounds);
+            const int buf = DUAL ? 0 : (it & 1);
+            if (!warp_wait(&tmem_full[buf], use[buf] & 1, abort_flag, p.hdr + kHdrStatus)) break;
+            use[buf] += 1;
+            ptx::tc_fence_after();
+            const int m = tl.mt * kTileM + 32 * ew + lane;
+            const bool m_ok = m < L.n_out;
+            const uint32_t tbase = tmem_base + ((uint32_t)(32 * ew) << 16) + (DUAL ? 0u : (uint32_t)buf * 256u);
+            for (int c0 = 0; c0 < tl.n; c0 += 32) {
+                uint32_t v[32];
+                ptx::tmem_ld_32x32b_x32(tbase + c0, v);
+                if (DUAL) {
+                    uint32_t u[32];
+                    ptx::tmem_ld_32x32b_x32(tbase + 256 + c0, u);
+                    ptx::tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        if (c0 + i < tl.n && m_ok) {
+                            const float g = __uint_as_float(v[i]), up = __uint_as_float(u[i]);
+                            const float hv = g / (1.0f + expf(-g)) * up;
+                            p.h[(int64_t)(tl.p0 + c0 + i) * p.out_ld + m] = __float2bfloat16_rn(hv);
+                        }
+                    }
+                } else {
+                    ptx::tmem_ld_wait();
+                    const int col = c0 + lane;
+                    int orow = -1;
+                    if (col < tl.n) orow = p.dst_rows ? __ldg(p.dst_rows + tl.p0 + col) : tl.p0 + col;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int r = __shfl_sync(0xffffffffu, orow, i);
+                        if (r >= 0 && m_ok) p.out[(int64_t)r * p.out_ld + m] = __uint_as_float(v[i]);
+                    }
+                }
+            }
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&tmem_empty[buf]);
+        }
+    } else if (warp >= kDeqWarp0) {
+        // ------------------------------------------------------- dequantisation
+        const int d = tid - kDeqWarp0 * 32;  // 0..255
+        const int r = d >> 1, hlf = d & 1;
+        const int first = (d >> 2) & 1;      // alternate read order: conflict-free 16-byte loads
+        int rs = 0, ms = 0;
+        uint32_t rph = 0, mph = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            const Tile tl = decode_tile(t, MT, p, s_prefix, s_bounds);
+            const int rows = L.rows(tl.mt);
+            for (int kt = 0; kt < KT; ++kt) {
+                ok = warp_wait(&raw_full[rs], rph, abort_flag, p.hdr + kHdrStatus) &&
+                     warp_wait(&mma_empty[ms], mph ^ 1, abort_flag, p.hdr + kHdrStatus);
+                if (!ok) break;
+#pragma unroll
+                for (int mat = 0; mat < C::NMAT; ++mat) {
+                    const uint8_t* raw = sRaw + (rs * C::NMAT + mat) * kRawBytes;
+                    uint8_t* dstA = sA + (ms * C::NMAT + mat) * kATileBytes + r * 128;
+                    uint32_t pk[16];
+                    if (r < rows) {
+                        const uint8_t* qrow = raw + r * kTileK + hlf * 32;
+                        const uint4 qa = *(const uint4*)(qrow + first * 16);
+                        const uint4 qb = *(const uint4*)(qrow + (first ^ 1) * 16);
+                        const uint4 q0 = first ? qb : qa, q1 = first ? qa : qb;
+                        const float dsc = __half2float(*(const __half*)(raw + rows * kTileK + r * 4 + hlf * 2));
+                        const float nd = -32896.0f * dsc;
+                        const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const float v0 = fmaf(magic_byte(w[j], 0), dsc, nd);
+                            const float v1 = fmaf(magic_byte(w[j], 1), dsc, nd);
+                            const float v2 = fmaf(magic_byte(w[j], 2), dsc, nd);
+                            const float v3 = fmaf(magic_byte(w[j], 3), dsc, nd);
+                            pk[2 * j] = pack2(v0, v1, p.bf16);
+                            pk[2 * j + 1] = pack2(v2, v3, p.bf16);
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) pk[j] = 0u;
+                    }
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int phys = (hlf * 4 + i) ^ (r & 7);
+                        *(uint4*)(dstA + phys * 16) = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                    }
+                }
+                ptx::fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    ptx::mbar_arrive(&raw_empty[rs]);
+                    ptx::mbar_arrive(&a_full[ms]);
+                }
+                if (++rs == C::RS) { rs = 0; rph ^= 1; }
+                if (++ms == C::MS) { ms = 0; mph ^= 1; }
+            }
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == kWarpMma) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem_base, 512);
+    }
+}
+
+// fp32 activations -> fp16 copy (the tensor core reads fp16 operands)
+__global__ void f32_to_f16_kernel(const float* __restrict__ x, __half* __restrict__ y, int64_t n) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+        y[i] = __float2half_rn(x[i]);
+}
+
+// ------------------------------------------------------------------- host
+static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void* f = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = (PFN_cuTensorMapEncodeTiled_v12000)f;
+    }
+    return fn;
+}
+
+// 2-D map over rows x n_in 16-bit elements, box = 64 columns x 1 row, 128-byte swizzle
+static bool make_gather_map(CUtensorMap* m, const void* base, int64_t rows, int n_in, int bf16) {
+    auto enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)n_in, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)n_in * 2};
+    cuuint32_t box[2] = {(cuuint32_t)kTileK, 1};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                     const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+static int sm_count() {
+    static int dev_cached = -1, n = 0;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev != dev_cached) {
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        dev_cached = dev;
+    }
+    return n > 0 ? n : 148;
+}
+
+template <int DUAL>
+static moe_status run_gemm(const GemmParams& p, const void* B, int64_t b_rows, int b_cols, int64_t max_coltiles,
+                           cudaStream_t stream) {
+    static int attr_dev = -1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (attr_dev != dev) {
+        if (cudaFuncSetAttribute(grouped_gemm_kernel<DUAL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)Cfg<DUAL>::smem_bytes) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        attr_dev = dev;
+    }
+    CUtensorMap map;
+    if (!make_gather_map(&map, B, b_rows, b_cols, p.bf16)) return MOE_ERR_CUDA;
+    int64_t tiles = max_coltiles * p.L.mt_count;
+    if (tiles <= 0) return MOE_OK;
+    int grid = (int)(tiles < sm_count() ? tiles : sm_count());
+    grouped_gemm_kernel<DUAL><<<grid, kGemmThreads, Cfg<DUAL>::smem_bytes, stream>>>(map, p);
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+static int64_t coltile_bound(int64_t S, int E) { return (S + kGemmBN - 1) / kGemmBN + (S < E ? S : E); }
+
+static moe_status to_f16(const void* x, void* x16, int64_t n, cudaStream_t s) {
+    int64_t blocks = (n + 255) / 256;
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    if (blocks < 1) blocks = 1;
+    f32_to_f16_kernel<<<(unsigned)blocks, 256, 0, s>>>((const float*)x, (__half*)x16, n);
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status launch_gemm_mul_mat_id(const GemmMulMatId& g, cudaStream_t stream) {
+    const void* B = g.x;
+    int bf16 = g.x_type == MOE_BF16;
+    if (g.x_type == MOE_F32) {
+        moe_status st = to_f16(g.x, g.x16, g.x_rows * g.n_in, stream);
+        if (st) return st;
+        prof_mark(stream, "x_to_f16");
+        B = g.x16;
+    }
+    GemmParams p = {};
+    p.A0 = g.W;
+    p.L = WLayout(g.n_out, g.n_in);
+    p.n_groups = g.E;
+    p.bounds = g.bounds;
+    p.ntile_prefix = g.ntile_prefix;
+    p.src_rows = g.ids_src1;
+    p.dst_rows = g.ids_dst;
+    p.out = g.dst;
+    p.out_ld = g.n_out;
+    p.hdr = g.hdr;
+    p.bf16 = bf16;
+    moe_status st = run_gemm<0>(p, B, g.x_rows, g.n_in, coltile_bound(g.S, g.E), stream);
+    prof_mark(stream, "gemm");
+    return st;
+}
+
+moe_status launch_gemm_ffn(const GemmFfn& g, cudaStream_t stream) {
+    const void* X = g.x;
+    int bf16 = g.x_type == MOE_BF16;
+    moe_status st;
+    if (g.x_type == MOE_F32) {
+        st = to_f16(g.x, g.x16, g.T * g.n_embd, stream);
+        if (st) return st;
+        prof_mark(stream, "x_to_f16");
+        X = g.x16;
+    }
+    // gate/up -> h (expert-sorted rows), SwiGLU in the epilogue
+    GemmParams p = {};
+    p.A0 = g.Wg;
+    p.A1 = g.Wu;
+    p.L = WLayout(g.n_ff, g.n_embd);
+    p.n_groups = g.E;
+    p.bounds = g.bounds;
+    p.ntile_prefix = g.ntile_prefix;
+    p.src_rows = g.ids_src1;
+    p.h = g.h;
+    p.out_ld = g.n_ff;
+    p.hdr = g.hdr;
+    p.bf16 = bf16;
+    st = run_gemm<1>(p, X, g.T, g.n_embd, coltile_bound(g.S, g.E), stream);
+    if (st) return st;
+    prof_mark(stream, "gemm_gate_up");
+    if (g.n_ff_shared > 0) {
+        GemmParams q = {};
+        q.A0 = g.Sg;
+        q.A1 = g.Su;
+        q.L = WLayout(g.n_ff_shared, g.n_embd);
+        q.n_groups = 0;
+        q.n_rows = (int)g.T;
+        q.h = g.h_sh;
+        q.out_ld = g.n_ff_shared;
+        q.hdr = g.hdr;
+        q.bf16 = bf16;
+        st = run_gemm<1>(q, X, g.T, g.n_embd, (g.T + kGemmBN - 1) / kGemmBN, stream);
+        if (st) return st;
+        prof_mark(stream, "gemm_shared_gate_up");
+    }
+    // down: h rows are already contiguous per expert; scatter to dst by ids_dst
+    GemmParams d = {};
+    d.A0 = g.Wd;
+    d.L = WLayout(g.n_embd, g.n_ff);
+    d.n_groups = g.E;
+    d.bounds = g.bounds;
+    d.ntile_prefix = g.ntile_prefix;
+    d.dst_rows = g.ids_dst;
+    d.out = g.dst;
+    d.out_ld = g.n_embd;
+    d.hdr = g.hdr;
+    d.bf16 = 1;
+    st = run_gemm<0>(d, g.h, g.S, g.n_ff, coltile_bound(g.S, g.E), stream);
+    if (st) return st;
+    prof_mark(stream, "gemm_down");
+    if (g.n_ff_shared > 0) {
+        GemmParams q = {};
+        q.A0 = g.Sd;
+        q.L = WLayout(g.n_embd, g.n_ff_shared);
+        q.n_groups = 0;
+        q.n_rows = (int)g.T;
+        q.out = g.dst_shared;
+        q.out_ld = g.n_embd;
+        q.hdr = g.hdr;
+        q.bf16 = 1;
+        st = run_gemm<0>(q, g.h_sh, g.T, g.n_ff_shared, (g.T + kGemmBN - 1) / kGemmBN, stream);
+        prof_mark(stream, "gemm_shared_down");
+    }
+    return st;
+}
+
+}  // namespace moe

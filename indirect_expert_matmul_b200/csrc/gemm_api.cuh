@@ -1,0 +1,46 @@
+// Host-side argument blocks of the grouped tensor-core GEMM (gemm.cu).
+#pragma once
+#include "common.cuh"
+
+namespace moe {
+
+struct GemmMulMatId {
+    const uint8_t* W;
+    int E, n_out, n_in;
+    const void* x;
+    int x_type;
+    int64_t x_rows;   // rows of x: n_tokens (broadcast) or n_tokens*k (per_slot)
+    void* x16;        // workspace for an fp16 copy of fp32 x (or null)
+    int64_t S;
+    float* dst;
+    const int32_t* bounds;
+    const int32_t* ntile_prefix;
+    const int32_t* ids_src1;
+    const int32_t* ids_dst;
+    int* hdr;
+};
+
+struct GemmFfn {
+    const uint8_t *Wg, *Wu, *Wd;
+    int E, n_embd, n_ff;
+    const uint8_t *Sg, *Su, *Sd;
+    int n_ff_shared;
+    const void* x;
+    int x_type;
+    void* x16;
+    int64_t T, S;
+    float* dst;
+    float* dst_shared;
+    __nv_bfloat16* h;
+    __nv_bfloat16* h_sh;
+    const int32_t* bounds;
+    const int32_t* ntile_prefix;
+    const int32_t* ids_src1;
+    const int32_t* ids_dst;
+    int* hdr;
+};
+
+moe_status launch_gemm_mul_mat_id(const GemmMulMatId& g, cudaStream_t stream);
+moe_status launch_gemm_ffn(const GemmFfn& g, cudaStream_t stream);
+
+}  // namespace moe

@@ -1,0 +1,82 @@
+"""The C-ABI library loads and exports every symbol include/moe.h declares; its
+host-side logic (sizes, argument checks) works without a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import indirect_expert_matmul_b200 as moe
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    src = ""
+    for f in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if f.endswith(".h"):
+            src += open(os.path.join(ROOT, "include", f)).read()
+    return sorted(set(re.findall(r"MOE_API\s+[\w\s\*]*?\b(moe_\w+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    syms = declared_symbols()
+    assert len(syms) >= 14
+    lib = moe.lib()
+    missing = [s for s in syms if not hasattr(lib, s)]
+    assert not missing, missing
+    assert set(syms) == set(moe.ABI_SYMBOLS)
+
+
+def test_status_strings():
+    for code, name in [(0, "MOE_OK"), (-1, "MOE_ERR_INVALID"), (-2, "MOE_ERR_RANGE"), (-3, "MOE_ERR_BAD_ID"),
+                       (-4, "MOE_ERR_CUDA"), (-5, "MOE_ERR_TIMEOUT"), (-6, "MOE_ERR_UNSUPPORTED")]:
+        assert moe.status_string(code) == name
+
+
+def test_prepared_size_is_q8_0_size():
+    for E, n_out, n_in in [(256, 2048, 7168), (256, 7168, 2048), (128, 2880, 2880), (64, 1408, 2048), (8, 512, 256)]:
+        assert moe.weights_prepared_size(E, n_out, n_in) == E * n_out * n_in // 32 * 34
+    # padding: n_out to 16, n_in to 64
+    assert moe.weights_prepared_size(1, 17, 32) == 32 * 1 * 68
+    assert moe.weights_prepared_size(0, 16, 64) == 0
+
+
+def test_workspace_size_covers_tables_and_hidden():
+    T, k, E, n_in, n_ff = 4096, 8, 256, 7168, 2048
+    s = moe.workspace_size(T, k, E, n_in, n_ff, 0)
+    assert s >= 2 * T * k * 4 + T * k * n_ff * 2 + 3 * (E + 1) * 4
+    assert s % 256 == 0
+    assert moe.workspace_size(T, k, E, n_in, 0, 0, __import__("torch").float32) >= T * k * n_in * 2
+
+
+def test_host_argument_checks_without_gpu():
+    lib = moe.lib()
+    nul = None
+    # k > n_experts
+    assert lib.moe_row_ids(nul, 4, 3, 2, 0, nul, nul, nul, nul, nul) == moe.ERR_RANGE
+    # n_tokens >= 2^22
+    assert lib.moe_row_ids(nul, 1 << 22, 1, 2, 0, nul, nul, nul, nul, nul) == moe.ERR_RANGE
+    # k >= 2^10
+    assert lib.moe_mul_mat_id(nul, 2000, 8, 64, nul, 0, nul, 1, 1024, 0, nul, nul, nul) == moe.ERR_RANGE
+    # n_in not a multiple of 32
+    assert lib.moe_mul_mat_id(nul, 4, 8, 48, nul, 0, nul, 1, 1, 0, nul, nul, nul) == moe.ERR_INVALID
+    # bad mode / dtype
+    assert lib.moe_mul_mat_id(nul, 4, 8, 64, nul, 0, nul, 1, 1, 7, nul, nul, nul) == moe.ERR_INVALID
+    assert lib.moe_mul_mat_id(nul, 4, 8, 64, nul, 9, nul, 1, 1, 0, nul, nul, nul) == moe.ERR_INVALID
+    # null workspace
+    assert lib.moe_mul_mat_id(nul, 4, 8, 64, nul, 0, nul, 1, 1, 0, nul, nul, nul) == moe.ERR_INVALID
+    # n_experts above the supported maximum
+    assert lib.moe_row_ids(nul, 1, 1, 20000, 0, nul, nul, nul, nul, nul) == moe.ERR_RANGE
+    # ffn: shared width not a multiple of 32
+    assert lib.moe_ffn(nul, nul, nul, 4, 64, 64, nul, nul, nul, 40, nul, 0, nul, 1, 1, nul, nul, nul,
+                       nul) == moe.ERR_INVALID
+
+
+def test_gemv_threshold_setting():
+    old = moe.get_gemv_threshold()
+    try:
+        moe.set_gemv_threshold(3)
+        assert moe.get_gemv_threshold() == 3
+    finally:
+        moe.set_gemv_threshold(old)

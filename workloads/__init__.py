@@ -83,6 +83,16 @@ def q8_0_weights(n_experts: int, n_out: int, n_in: int, seed: int, tensor: int,
     return out
 
 
+def q8_0_weights_experts(e0: int, n_e: int, n_out: int, n_in: int, seed: int, tensor: int) -> np.ndarray:
+    """Experts e0 .. e0+n_e-1 of a stacked Q8_0 matrix, byte-identical to the
+    same slice of q8_0_weights(...) (the generator is counter-based)."""
+    if n_in % 32:
+        raise ValueError("n_in must be a multiple of 32 for Q8_0")
+    out = np.empty((n_e, n_out, n_in // 32, 34), dtype=np.uint8)
+    _L().wl_fill_q8_0(_ptr(out), e0 * n_out, n_e * n_out, n_in, seed, tensor, D_LO, D_HI)
+    return out
+
+
 def activations(n_rows: int, n_in: int, dtype: str, seed: int, tensor: int, row0: int = 0) -> np.ndarray:
     """N(0,1) activations [n_rows][n_in]; rows numbered globally from row0.
 
