@@ -181,12 +181,18 @@ def run_ours(args):
     hbm_peak, tc_peak, tc_sust, peak_src = load_peaks()
 
     E, k, n_embd, n_ff, T = WL.n_experts, WL.k, WL.n_in, WL.n_out, WL.n_tokens[0]
+    small = args.experts is not None or args.tokens is not None
+    if args.experts is not None:
+        E = args.experts
+    if args.tokens is not None:
+        T = args.tokens
     S = T * k
     t0 = rank * T  # each rank its own batch of tokens
     Wg = upload_prepared(moe, torch, E, n_ff, n_embd, workloads.T_WG)
     Wu = upload_prepared(moe, torch, E, n_ff, n_embd, workloads.T_WU)
     Wd = upload_prepared(moe, torch, E, n_embd, n_ff, workloads.T_WD)
-    ids_np = WL.ids(T, t0=t0)
+    ids_np = workloads.routing(WL.routing, T, E, k, WL.seed, t0=t0, bias_sigma=WL.bias_sigma) if small \
+        else WL.ids(T, t0=t0)
     x_np = WL.x(T, t0=t0)
     x = bf16_dev(torch, x_np)
     ids = torch.from_numpy(ids_np).cuda()
@@ -261,8 +267,9 @@ def run_ours(args):
         "metric": METRIC, "value": round(T * world / (ms * 1e-3), 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": "v3 moe_ffn: 256 experts top-8, n_embd 7168, expert ffn 2048, Q8_0 gate/up/down, "
-                               "bf16 x, 4096 tokens per GPU, biased top-8 routing",
+        "config": {"workload": ("v3 moe_ffn: 256 experts top-8, n_embd 7168, expert ffn 2048, Q8_0 gate/up/down, "
+                                "bf16 x, 4096 tokens per GPU, biased top-8 routing") if not small else
+                               f"profiling case (not a bench line): v3 shape with {E} experts, {T} tokens",
                    "tokens_per_gpu": T, "experts_touched": int(used),
                    "l2": "inputs larger than L2 (12 GB of weights per step)", "parallelism": f"dp{world}"},
         "tflops": round(step_flops * world / (ms * 1e-3) / 1e12, 1),
@@ -422,6 +429,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--decode-layers", type=int, default=16)
+    ap.add_argument("--experts", type=int, default=None, help="profiling only: fewer experts than the V3 layer")
+    ap.add_argument("--tokens", type=int, default=None, help="profiling only: tokens per GPU")
     ap.add_argument("--traffic", type=float, default=None,
                     help="dram bytes per launch of the dominant kernel from an ncu capture (null if stale)")
     args = ap.parse_args()

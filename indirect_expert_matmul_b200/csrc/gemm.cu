@@ -35,27 +35,31 @@
 namespace moe {
 
 constexpr int kGemmThreads = 512;
-constexpr int kWarpProducer = 0;
-constexpr int kWarpMma = 1;
+constexpr int kWarpProdA = 0;   // weight blocks: L2 prefetch + bulk copies
+constexpr int kWarpMma = 1;     // TMEM allocation + tcgen05.mma issue
+constexpr int kWarpProdB = 2;   // activation rows: TMA gather4
 constexpr int kEpiWarp0 = 4;
 constexpr int kDeqWarp0 = 8;
 constexpr int kDeqWarps = 8;
 constexpr uint32_t kATileBytes = kTileM * kTileK * 2;  // 16 KB
 constexpr uint32_t kBTileBytes = kGemmBN * kTileK * 2; // 32 KB
 constexpr uint32_t kRawBytes = kTileM * kRowBytes;     // 8704
-constexpr int kSmemGroups = 1024;                      // schedule tables kept in shared memory up to this
+constexpr int kSmemGroups = 512;                       // schedule tables kept in shared memory up to this
+constexpr int kPrefetchSteps = 8;                      // weight k-steps prefetched into L2 ahead of use
 constexpr long long kWaitLimitCycles = 1ll << 32;      // ~2 s
+constexpr uint32_t kSleepNs = 20000;                   // upper bound of one hardware wait
 
 template <int DUAL>
 struct Cfg {
     static constexpr int NMAT = DUAL + 1;
-    static constexpr int MS = DUAL ? 2 : 3;  // operand stages (A bf16 + B)
-    static constexpr int RS = 4;             // raw weight stages
+    static constexpr int RS = DUAL ? 3 : 4;  // raw weight stages (int8 + scales)
+    static constexpr int MA = DUAL ? 2 : 3;  // dequantised A stages
+    static constexpr int MB = DUAL ? 3 : 4;  // activation (B) stages
     static constexpr uint32_t a_off = 0;
-    static constexpr uint32_t b_off = a_off + MS * NMAT * kATileBytes;
-    static constexpr uint32_t raw_off = b_off + MS * kBTileBytes;
+    static constexpr uint32_t b_off = a_off + MA * NMAT * kATileBytes;
+    static constexpr uint32_t raw_off = b_off + MB * kBTileBytes;
     static constexpr uint32_t bar_off = raw_off + RS * NMAT * kRawBytes;
-    static constexpr int n_bars = 2 * RS + 3 * MS + 4;
+    static constexpr int n_bars = 2 * RS + 2 * MA + 2 * MB + 4;
     static constexpr uint32_t misc_off = bar_off + n_bars * 8;
     static constexpr uint32_t smem_bytes = misc_off + 64 + 1024;  // + alignment slack
 };
@@ -75,7 +79,6 @@ struct GemmParams {
     int out_ld;
     int* hdr;
     int bf16;                   // operand type: 1 bf16, 0 fp16
-    int grid_tiles_hint;
 };
 
 struct Tile {
@@ -108,12 +111,14 @@ __device__ __forceinline__ Tile decode_tile(int t, int mt_count, const GemmParam
     return r;
 }
 
-// Bounded wait by one lane; false when the kernel is aborting.
+// Bounded wait by one lane; false when the kernel is aborting.  The lane
+// sleeps in hardware between polls (suspend-time hint), so waiting roles do
+// not take issue slots from the dequantisation warps.
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {
-        if (ptx::mbar_try_wait(bar, parity)) return true;
+        if (ptx::mbar_try_wait_sleep(bar, parity, kSleepNs)) return true;
         if (*abort_flag) return false;
         if (clock64() - t0 > kWaitLimitCycles) {
             *abort_flag = 1;
@@ -157,12 +162,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmB, const GemmParams p)
     uint64_t* raw_full = bars;
     uint64_t* raw_empty = raw_full + C::RS;
     uint64_t* a_full = raw_empty + C::RS;
-    uint64_t* b_full = a_full + C::MS;
-    uint64_t* mma_empty = b_full + C::MS;
-    uint64_t* tmem_full = mma_empty + C::MS;
+    uint64_t* a_empty = a_full + C::MA;
+    uint64_t* b_full = a_empty + C::MA;
+    uint64_t* b_empty = b_full + C::MB;
+    uint64_t* tmem_full = b_empty + C::MB;
     uint64_t* tmem_empty = tmem_full + 2;
     uint32_t* tmem_base_sh = (uint32_t*)(smem + C::misc_off);
     volatile int* abort_flag = (volatile int*)(smem + C::misc_off + 4);
+    int* status = p.hdr + kHdrStatus;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const WLayout L = p.L;
@@ -173,10 +180,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmB, const GemmParams p)
             ptx::mbar_init(&raw_full[i], 1);
             ptx::mbar_init(&raw_empty[i], kDeqWarps);
         }
-        for (int i = 0; i < C::MS; ++i) {
+        for (int i = 0; i < C::MA; ++i) {
             ptx::mbar_init(&a_full[i], kDeqWarps);
+            ptx::mbar_init(&a_empty[i], 1);
+        }
+        for (int i = 0; i < C::MB; ++i) {
             ptx::mbar_init(&b_full[i], 1);
-            ptx::mbar_init(&mma_empty[i], 1);
+            ptx::mbar_init(&b_empty[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(&tmem_full[i], 1);
@@ -202,11 +212,62 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmB, const GemmParams p)
     ptx::tc_fence_after();
     const uint32_t tmem_base = *tmem_base_sh;
 
-    if (warp == kWarpProducer) {
-        // ------------------------------------------------------------ producer
-        int rs = 0, ms = 0;
-        uint32_t rph = 0, mph = 0;
-        uint32_t raw_used = 0, raw_par = 0, b_used = 0, b_par = 0;  // per-stage issue record, for draining
+    if (warp == kWarpProdA) {
+        // ---------------------------------------------------- weight producer
+        // One lane streams the tiles' weight blocks: an L2 prefetch runs
+        // kPrefetchSteps k-steps ahead of the bulk copies into the raw ring.
+        if (lane == 0) {
+            int rs = 0;
+            uint32_t rph = 0;
+            uint32_t used = 0, par = 0;  // per-stage issue record, for draining
+            int pf_t = blockIdx.x, pf_kt = 0, pf_tile = -1;
+            const uint8_t *pf_a0 = nullptr, *pf_a1 = nullptr;
+            uint32_t pf_bytes = 0;
+            auto prefetch_one = [&]() {
+                if (pf_t >= total) return;
+                if (pf_tile != pf_t) {
+                    const Tile tl = decode_tile(pf_t, MT, p, s_prefix, s_bounds);
+                    pf_bytes = (uint32_t)L.rows(tl.mt) * kRowBytes;
+                    pf_a0 = p.A0 + L.block(tl.e, tl.mt, 0);
+                    pf_a1 = DUAL ? p.A1 + L.block(tl.e, tl.mt, 0) : nullptr;
+                    pf_tile = pf_t;
+                }
+                ptx::bulk_prefetch_l2(pf_a0 + (size_t)pf_kt * pf_bytes, pf_bytes);
+                if (DUAL) ptx::bulk_prefetch_l2(pf_a1 + (size_t)pf_kt * pf_bytes, pf_bytes);
+                if (++pf_kt == KT) { pf_kt = 0; pf_t += gridDim.x; }
+            };
+            for (int i = 0; i < kPrefetchSteps; ++i) prefetch_one();
+            bool ok = true;
+            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+                const Tile tl = decode_tile(t, MT, p, s_prefix, s_bounds);
+                const uint32_t raw_bytes = (uint32_t)L.rows(tl.mt) * kRowBytes;
+                const uint8_t* a0 = p.A0 + L.block(tl.e, tl.mt, 0);
+                const uint8_t* a1 = DUAL ? p.A1 + L.block(tl.e, tl.mt, 0) : nullptr;
+                for (int kt = 0; kt < KT; ++kt) {
+                    prefetch_one();
+                    ok = wait_bar(&raw_empty[rs], rph ^ 1, abort_flag, status);
+                    if (!ok) break;
+                    ptx::mbar_arrive_expect_tx(&raw_full[rs], raw_bytes * C::NMAT);
+                    ptx::bulk_g2s(sRaw + (rs * C::NMAT) * kRawBytes, a0 + (size_t)kt * raw_bytes, raw_bytes,
+                                  &raw_full[rs]);
+                    if (DUAL)
+                        ptx::bulk_g2s(sRaw + (rs * C::NMAT + 1) * kRawBytes, a1 + (size_t)kt * raw_bytes, raw_bytes,
+                                      &raw_full[rs]);
+                    used |= 1u << rs;
+                    par = (par & ~(1u << rs)) | (rph << rs);
+                    if (++rs == C::RS) { rs = 0; rph ^= 1; }
+                }
+            }
+            // let every copy issued land before the CTA can exit (bounded)
+            volatile int never = 0;
+            for (int s = 0; s < C::RS; ++s)
+                if (used >> s & 1) wait_bar(&raw_full[s], (par >> s) & 1, &never, status);
+        }
+    } else if (warp == kWarpProdB) {
+        // ------------------------------------------------ activation producer
+        int bs = 0;
+        uint32_t bph = 0;
+        uint32_t used = 0, par = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
             const Tile tl = decode_tile(t, MT, p, s_prefix, s_bounds);
@@ -221,63 +282,38 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmB, const GemmParams p)
                     rows4[i][r] = p.src_rows ? __ldg(p.src_rows + pos) : pos;
                 }
             }
-            const int rows = L.rows(tl.mt);
-            const uint32_t raw_bytes = (uint32_t)rows * kRowBytes;
-            const uint8_t* a0 = p.A0 + L.block(tl.e, tl.mt, 0);
-            const uint8_t* a1 = DUAL ? p.A1 + L.block(tl.e, tl.mt, 0) : nullptr;
             for (int kt = 0; kt < KT; ++kt) {
-                // weights: raw int8 + scales of both matrices
                 if (lane == 0) {
-                    ok = wait_bar(&raw_empty[rs], rph ^ 1, abort_flag, p.hdr + kHdrStatus);
+                    ok = wait_bar(&b_empty[bs], bph ^ 1, abort_flag, status);
                     if (ok) {
-                        ptx::mbar_arrive_expect_tx(&raw_full[rs], raw_bytes * C::NMAT);
-                        ptx::bulk_g2s(sRaw + (rs * C::NMAT) * kRawBytes, a0 + (size_t)kt * raw_bytes, raw_bytes,
-                                      &raw_full[rs]);
-                        if (DUAL)
-                            ptx::bulk_g2s(sRaw + (rs * C::NMAT + 1) * kRawBytes, a1 + (size_t)kt * raw_bytes,
-                                          raw_bytes, &raw_full[rs]);
-                        raw_used |= 1u << rs;
-                        raw_par = (raw_par & ~(1u << rs)) | (rph << rs);
+                        ptx::mbar_arrive_expect_tx(&b_full[bs], (uint32_t)n16 * 128u);
+                        used |= 1u << bs;
+                        par = (par & ~(1u << bs)) | (bph << bs);
                     }
                 }
                 ok = __shfl_sync(0xffffffffu, (int)ok, 0) != 0;
                 if (!ok) break;
-                if (++rs == C::RS) { rs = 0; rph ^= 1; }
-                // activations: gathered rows of this column tile
-                if (lane == 0) {
-                    ok = wait_bar(&mma_empty[ms], mph ^ 1, abort_flag, p.hdr + kHdrStatus);
-                    if (ok) {
-                        ptx::mbar_arrive_expect_tx(&b_full[ms], (uint32_t)n16 * 128u);
-                        b_used |= 1u << ms;
-                        b_par = (b_par & ~(1u << ms)) | (mph << ms);
-                    }
-                }
-                ok = __shfl_sync(0xffffffffu, (int)ok, 0) != 0;
-                if (!ok) break;
-                uint8_t* bdst = sB + ms * kBTileBytes;
+                uint8_t* bdst = sB + bs * kBTileBytes;
 #pragma unroll
                 for (int i = 0; i < 2; ++i) {
                     const int g = lane + 32 * i;
                     if (4 * g < n16)
                         ptx::tma_gather4(bdst + g * 512, &tmB, kt * kTileK, rows4[i][0], rows4[i][1], rows4[i][2],
-                                         rows4[i][3], &b_full[ms]);
+                                         rows4[i][3], &b_full[bs]);
                 }
-                if (++ms == C::MS) { ms = 0; mph ^= 1; }
+                if (++bs == C::MB) { bs = 0; bph ^= 1; }
             }
         }
-        // before leaving, let every copy this warp issued land (bounded)
         if (lane == 0) {
             volatile int never = 0;
-            for (int s = 0; s < C::RS; ++s)
-                if (raw_used >> s & 1) wait_bar(&raw_full[s], (raw_par >> s) & 1, &never, p.hdr + kHdrStatus);
-            for (int s = 0; s < C::MS; ++s)
-                if (b_used >> s & 1) wait_bar(&b_full[s], (b_par >> s) & 1, &never, p.hdr + kHdrStatus);
+            for (int s = 0; s < C::MB; ++s)
+                if (used >> s & 1) wait_bar(&b_full[s], (par >> s) & 1, &never, status);
         }
     } else if (warp == kWarpMma) {
         // ----------------------------------------------------------------- MMA
         if (lane == 0) {
-            int ms = 0;
-            uint32_t mph = 0;
+            int as = 0, bs = 0;
+            uint32_t aph = 0, bph = 0;
             uint32_t use[2] = {0, 0};
             int it = 0;
             bool ok = true;
@@ -285,20 +321,20 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmB, const GemmParams p)
                 const Tile tl = decode_tile(t, MT, p, s_prefix, s_bounds);
                 const int n16 = (tl.n + 15) & ~15;
                 const int buf = DUAL ? 0 : (it & 1);
-                ok = wait_bar(&tmem_empty[buf], (use[buf] & 1) ^ 1, abort_flag, p.hdr + kHdrStatus);
+                ok = wait_bar(&tmem_empty[buf], (use[buf] & 1) ^ 1, abort_flag, status);
                 if (!ok) break;
                 ptx::tc_fence_after();
                 const uint32_t d0 = tmem_base + (DUAL ? 0u : (uint32_t)buf * 256u);
                 const uint32_t d1 = tmem_base + 256u;
                 const uint32_t idesc = ptx::idesc_f16(p.bf16, n16, 128);
                 for (int kt = 0; kt < KT; ++kt) {
-                    ok = wait_bar(&a_full[ms], mph, abort_flag, p.hdr + kHdrStatus) &&
-                         wait_bar(&b_full[ms], mph, abort_flag, p.hdr + kHdrStatus);
+                    ok = wait_bar(&a_full[as], aph, abort_flag, status) &&
+                         wait_bar(&b_full[bs], bph, abort_flag, status);
                     if (!ok) break;
                     ptx::tc_fence_after();
-                    const uint32_t a0 = ptx::smem_u32(sA + (ms * C::NMAT) * kATileBytes);
+                    const uint32_t a0 = ptx::smem_u32(sA + (as * C::NMAT) * kATileBytes);
                     const uint32_t a1 = a0 + kATileBytes;
-                    const uint32_t b = ptx::smem_u32(sB + ms * kBTileBytes);
+                    const uint32_t b = ptx::smem_u32(sB + bs * kBTileBytes);
 #pragma unroll
                     for (int kk = 0; kk < kTileK / 16; ++kk) {
                         const uint32_t acc = (kt | kk) != 0;
@@ -308,8 +344,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmB, const GemmParams p)
                             ptx::mma_f16_ss(d1, ptx::desc_k_sw128(a1 + kk * 32), ptx::desc_k_sw128(b + kk * 32),
                                             idesc, acc);
                     }
-                    ptx::mma_commit(&mma_empty[ms]);
-                    if (++ms == C::MS) { ms = 0; mph ^= 1; }
+                    ptx::mma_commit(&a_empty[as]);
+                    ptx::mma_commit(&b_empty[bs]);
+                    if (++as == C::MA) { as = 0; aph ^= 1; }
+                    if (++bs == C::MB) { bs = 0; bph ^= 1; }
                 }
                 if (!ok) break;
                 ptx::mma_commit(&tmem_full[buf]);
@@ -325,7 +363,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmB, const GemmParams p)
         for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
             const Tile tl = decode_tile(t, MT, p, s_prefix, s_bounds);
             const int buf = DUAL ? 0 : (it & 1);
-            if (!warp_wait(&tmem_full[buf], use[buf] & 1, abort_flag, p.hdr + kHdrStatus)) break;
+            if (!warp_wait(&tmem_full[buf], use[buf] & 1, abort_flag, status)) break;
             use[buf] += 1;
             ptx::tc_fence_after();
             const int m = tl.mt * kTileM + 32 * ew + lane;
@@ -342,7 +380,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmB, const GemmParams p)
                     for (int i = 0; i < 32; ++i) {
                         if (c0 + i < tl.n && m_ok) {
                             const float g = __uint_as_float(v[i]), up = __uint_as_float(u[i]);
-                            const float hv = g / (1.0f + expf(-g)) * up;
+                            const float hv = g / (1.0f + __expf(-g)) * up;
                             p.h[(int64_t)(tl.p0 + c0 + i) * p.out_ld + m] = __float2bfloat16_rn(hv);
                         }
                     }
@@ -367,20 +405,20 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmB, const GemmParams p)
         const int d = tid - kDeqWarp0 * 32;  // 0..255
         const int r = d >> 1, hlf = d & 1;
         const int first = (d >> 2) & 1;      // alternate read order: conflict-free 16-byte loads
-        int rs = 0, ms = 0;
-        uint32_t rph = 0, mph = 0;
+        int rs = 0, as = 0;
+        uint32_t rph = 0, aph = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
             const Tile tl = decode_tile(t, MT, p, s_prefix, s_bounds);
             const int rows = L.rows(tl.mt);
             for (int kt = 0; kt < KT; ++kt) {
-                ok = warp_wait(&raw_full[rs], rph, abort_flag, p.hdr + kHdrStatus) &&
-                     warp_wait(&mma_empty[ms], mph ^ 1, abort_flag, p.hdr + kHdrStatus);
+                ok = warp_wait(&raw_full[rs], rph, abort_flag, status) &&
+                     warp_wait(&a_empty[as], aph ^ 1, abort_flag, status);
                 if (!ok) break;
 #pragma unroll
                 for (int mat = 0; mat < C::NMAT; ++mat) {
                     const uint8_t* raw = sRaw + (rs * C::NMAT + mat) * kRawBytes;
-                    uint8_t* dstA = sA + (ms * C::NMAT + mat) * kATileBytes + r * 128;
+                    uint8_t* dstA = sA + (as * C::NMAT + mat) * kATileBytes + r * 128;
                     uint32_t pk[16];
                     if (r < rows) {
                         const uint8_t* qrow = raw + r * kTileK + hlf * 32;
@@ -413,10 +451,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmB, const GemmParams p)
                 __syncwarp();
                 if (lane == 0) {
                     ptx::mbar_arrive(&raw_empty[rs]);
-                    ptx::mbar_arrive(&a_full[ms]);
+                    ptx::mbar_arrive(&a_full[as]);
                 }
                 if (++rs == C::RS) { rs = 0; rph ^= 1; }
-                if (++ms == C::MS) { ms = 0; mph ^= 1; }
+                if (++as == C::MA) { as = 0; aph ^= 1; }
             }
         }
     }

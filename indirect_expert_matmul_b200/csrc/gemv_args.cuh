@@ -4,31 +4,36 @@
 
 namespace moe {
 
+constexpr int kGvMaxSlots = 8192;  // the mat-vec path handles n_tokens*k up to this
+
 struct GemvSide {
     const uint8_t* W0;  // prepared weights (single, or gate)
     const uint8_t* W1;  // up (dual) or null
     WLayout L;
     const void* x;      // activations: rows of L.n_in elements
     int x_type;         // MOE_BF16 / MOE_F16 / MOE_F32
-    float* out;         // single: out[row][n], row = ids_dst[p] (routed) or t (shared)
-    __nv_bfloat16* h;   // dual: h[p][n] (routed) or h[t][n] (shared)
-    int row_groups;     // ceil(n_out_pad / 16)
+    int x_per_slot;     // routed x row: 1 -> slot t*k+s, 0 -> token t
+    float* out;         // single: out[slot][n] (routed) or out[t][n] (shared)
+    __nv_bfloat16* h;   // dual: h[slot][n] (routed) or h[t][n] (shared)
+    int rows;           // rows per work item: 16, 32 or 64
+    int items;          // work items per expert: n_out_pad / rows
+    int n_stages;       // weight k-steps resident at once (one activation window)
+    int kw;             // activation window (columns)
 };
 
 struct GemvArgs {
     GemvSide routed, shared;
     int has_shared;
     int dual;
-    int src_from_table;  // routed x row: 1 -> ids_src1[p], 0 -> p
-    int n_tokens;
-    int max_active;
-    const int32_t* bounds;
-    const int32_t* active;
-    const int32_t* ids_src1;
-    const int32_t* ids_dst;
-    const int* hdr;
+    const int32_t* ids;  // [n_tokens][k]
+    int n_tokens, k, n_experts;
+    int max_distinct;    // min(n_tokens*k, n_experts): routed items = max_distinct * routed.items
+    int pdl_secondary;   // launched as a programmatic dependent: wait before reading activations
+    int* hdr;
 };
 
 moe_status launch_gemv(const GemvArgs& a, cudaStream_t stream);
+// Fill rows / items / n_stages / kw of a side for its shape and activation type.
+void gemv_plan_side(GemvSide& s, int dual);
 
 }  // namespace moe

@@ -30,7 +30,8 @@ static moe_status check_sizes(int64_t n_tokens, int k, int n_experts) {
     return MOE_OK;
 }
 
-static bool use_gemv(int64_t n_tokens) {
+static bool use_gemv(int64_t n_tokens, int64_t S) {
+    if (S > kGvMaxSlots) return false;  // beyond the mat-vec kernel's slot scan
     int p = g_path.load();
     if (p == 1) return true;
     if (p == 2) return false;
@@ -124,30 +125,29 @@ moe_status moe_mul_mat_id(const void* W_prepared, int n_experts, int n_out, int 
     int32_t* tiles = (int32_t*)(ws + W.tiles);
     const int64_t S = n_tokens * k;
     prof_begin(s);
-    st = launch_row_ids(ids, S, k, n_experts, mode, src1, dstr, bounds, active, tiles, kGemmBN, hdr, s);
-    if (st) return st;
-    prof_mark(s, "row_ids");
-    if (use_gemv(n_tokens)) {
+    if (use_gemv(n_tokens, S)) {
         GemvArgs a = {};
         a.routed.W0 = (const uint8_t*)W_prepared;
         a.routed.L = WLayout(n_out, n_in);
         a.routed.x = x;
         a.routed.x_type = x_type;
+        a.routed.x_per_slot = mode == MOE_PER_SLOT;
         a.routed.out = dst;
-        a.routed.row_groups = a.routed.L.n_out_pad / 16;
+        gemv_plan_side(a.routed, 0);
         a.dual = 0;
-        a.src_from_table = 1;
+        a.ids = ids;
         a.n_tokens = (int)n_tokens;
-        a.max_active = (int)(S < n_experts ? S : n_experts);
-        a.bounds = bounds;
-        a.active = active;
-        a.ids_src1 = src1;
-        a.ids_dst = dstr;
+        a.k = k;
+        a.n_experts = n_experts;
+        a.max_distinct = (int)(S < n_experts ? S : n_experts);
         a.hdr = hdr;
         st = launch_gemv(a, s);
         prof_mark(s, "gemv");
         return st;
     }
+    st = launch_row_ids(ids, S, k, n_experts, mode, src1, dstr, bounds, active, tiles, kGemmBN, hdr, s);
+    if (st) return st;
+    prof_mark(s, "row_ids");
     GemmMulMatId g = {};
     g.W = (const uint8_t*)W_prepared;
     g.E = n_experts;
@@ -196,29 +196,24 @@ moe_status moe_ffn(const void* Wg, const void* Wu, const void* Wd, int n_experts
     __nv_bfloat16* h_sh = (__nv_bfloat16*)(ws + W.h_sh);
     const int64_t S = n_tokens * k;
     prof_begin(s);
-    st = launch_row_ids(ids, S, k, n_experts, MOE_BROADCAST, src1, dstr, bounds, active, tiles, kGemmBN, hdr, s);
-    if (st) return st;
-    prof_mark(s, "row_ids");
-    if (use_gemv(n_tokens)) {
+    if (use_gemv(n_tokens, S)) {
         GemvArgs a = {};
         a.has_shared = has_shared;
+        a.ids = ids;
         a.n_tokens = (int)n_tokens;
-        a.max_active = (int)(S < n_experts ? S : n_experts);
-        a.bounds = bounds;
-        a.active = active;
-        a.ids_src1 = src1;
-        a.ids_dst = dstr;
+        a.k = k;
+        a.n_experts = n_experts;
+        a.max_distinct = (int)(S < n_experts ? S : n_experts);
         a.hdr = hdr;
-        // gate/up -> h
+        // gate/up -> h[t][s] (SwiGLU), shared -> h_sh[t]
         a.dual = 1;
-        a.src_from_table = 1;
         a.routed.W0 = (const uint8_t*)Wg;
         a.routed.W1 = (const uint8_t*)Wu;
         a.routed.L = WLayout(n_ff, n_embd);
         a.routed.x = x;
         a.routed.x_type = x_type;
         a.routed.h = h;
-        a.routed.row_groups = a.routed.L.n_out_pad / 16;
+        gemv_plan_side(a.routed, 1);
         if (has_shared) {
             a.shared.W0 = (const uint8_t*)Sg;
             a.shared.W1 = (const uint8_t*)Su;
@@ -226,36 +221,44 @@ moe_status moe_ffn(const void* Wg, const void* Wu, const void* Wd, int n_experts
             a.shared.x = x;
             a.shared.x_type = x_type;
             a.shared.h = h_sh;
-            a.shared.row_groups = a.shared.L.n_out_pad / 16;
+            gemv_plan_side(a.shared, 1);
         }
         st = launch_gemv(a, s);
         if (st) return st;
         prof_mark(s, "gemv_gate_up");
-        // down -> dst, dst_shared
-        a.dual = 0;
-        a.src_from_table = 0;
-        a.routed.W0 = (const uint8_t*)Wd;
-        a.routed.W1 = nullptr;
-        a.routed.L = WLayout(n_embd, n_ff);
-        a.routed.x = h;
-        a.routed.x_type = MOE_BF16;
-        a.routed.h = nullptr;
-        a.routed.out = dst;
-        a.routed.row_groups = a.routed.L.n_out_pad / 16;
+        // down -> dst[t][s], dst_shared[t]; a programmatic dependent of gate/up
+        GemvArgs b = {};
+        b.has_shared = has_shared;
+        b.ids = ids;
+        b.n_tokens = (int)n_tokens;
+        b.k = k;
+        b.n_experts = n_experts;
+        b.max_distinct = a.max_distinct;
+        b.hdr = hdr;
+        b.dual = 0;
+        b.pdl_secondary = 1;
+        b.routed.W0 = (const uint8_t*)Wd;
+        b.routed.L = WLayout(n_embd, n_ff);
+        b.routed.x = h;
+        b.routed.x_type = MOE_BF16;
+        b.routed.x_per_slot = 1;
+        b.routed.out = dst;
+        gemv_plan_side(b.routed, 0);
         if (has_shared) {
-            a.shared.W0 = (const uint8_t*)Sd;
-            a.shared.W1 = nullptr;
-            a.shared.L = WLayout(n_embd, n_ff_shared);
-            a.shared.x = h_sh;
-            a.shared.x_type = MOE_BF16;
-            a.shared.h = nullptr;
-            a.shared.out = dst_shared;
-            a.shared.row_groups = a.shared.L.n_out_pad / 16;
+            b.shared.W0 = (const uint8_t*)Sd;
+            b.shared.L = WLayout(n_embd, n_ff_shared);
+            b.shared.x = h_sh;
+            b.shared.x_type = MOE_BF16;
+            b.shared.out = dst_shared;
+            gemv_plan_side(b.shared, 0);
         }
-        st = launch_gemv(a, s);
+        st = launch_gemv(b, s);
         prof_mark(s, "gemv_down");
         return st;
     }
+    st = launch_row_ids(ids, S, k, n_experts, MOE_BROADCAST, src1, dstr, bounds, active, tiles, kGemmBN, hdr, s);
+    if (st) return st;
+    prof_mark(s, "row_ids");
     GemmFfn g = {};
     g.Wg = (const uint8_t*)Wg;
     g.Wu = (const uint8_t*)Wu;
