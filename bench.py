@@ -187,7 +187,8 @@ def run_ours(args):
     if args.tokens is not None:
         T = args.tokens
     S = T * k
-    t0 = rank * T  # each rank its own batch of tokens
+    from indirect_expert_matmul_b200.dist import max_over_ranks, token_shard
+    t0, _ = token_shard(T * world, rank, world)  # each rank its own batch of T tokens
     Wg = upload_prepared(moe, torch, E, n_ff, n_embd, workloads.T_WG)
     Wu = upload_prepared(moe, torch, E, n_ff, n_embd, workloads.T_WU)
     Wd = upload_prepared(moe, torch, E, n_embd, n_ff, workloads.T_WD)
@@ -231,10 +232,7 @@ def run_ours(args):
     st = moe.get_status(ws)
     if st != moe.OK:
         raise RuntimeError(f"device status after timed run: {moe.status_string(st)}")
-    if dist is not None:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, device="cuda")
 
     # algorithmic work of one step
     used, w_bytes = touched_ffn_bytes(ids_np, E, n_embd, n_ff)
@@ -305,10 +303,7 @@ def run_ours(args):
         torch.cuda.synchronize()
         barrier()
         ms_e2e = ev0.elapsed_time(ev1) / n_e2e
-        if dist is not None:
-            t = torch.tensor([ms_e2e], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms_e2e = float(t.item())
+        ms_e2e = max_over_ranks(ms_e2e, device="cuda")
         result["e2e"] = {"value": round(T * world / (ms_e2e * 1e-3), 1), "unit": "tokens/s",
                          "h2d_bytes_per_step": int(x_bytes + ids_np.nbytes), "d2h_bytes_per_step": int(dst_bytes),
                          "ms_per_step": round(ms_e2e, 3)}
