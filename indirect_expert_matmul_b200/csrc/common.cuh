@@ -51,12 +51,25 @@ struct WLayout {
 };
 
 // ------------------------------------------------------------------ workspace
+// Rows of the tile-major activation buffers of the grouped GEMM: every
+// expert's sorted range starts on a multiple of 8 rows (so the 128-byte
+// swizzle of an 8-row atom is position-independent), plus slack for a 16-row
+// rounding of the last column tile.
+inline int64_t tiled_rows(int64_t S, int n_groups) {
+    return S + 8 * (S < n_groups ? S : n_groups) + 32;
+}
 struct WsLayout {
-    int64_t S;
-    size_t hdr, src1, dst, bounds, active, tiles, h, h_sh, x16, total;
+    int64_t S, rows_pad, rows_pad_sh;
+    size_t hdr, src1, dst, bounds, active, tiles, pad, h, h_sh, xt, xt_sh, total;
     static size_t up(size_t v) { return (v + 255) / 256 * 256; }
     WsLayout(int64_t n_tokens, int k, int n_experts, int n_in, int n_hidden, int n_hidden_sh, int x_type) {
+        (void)x_type;
         S = n_tokens * k;
+        rows_pad = tiled_rows(S, n_experts);
+        rows_pad_sh = n_tokens + 32;
+        const int64_t kin = (n_in + 63) / 64, khid = (n_hidden + 63) / 64, khs = (n_hidden_sh + 63) / 64;
+        const size_t h_gemv = (size_t)S * n_hidden * 2, h_gemm = (size_t)rows_pad * khid * 128;
+        const size_t hs_gemv = (size_t)n_tokens * n_hidden_sh * 2, hs_gemm = (size_t)rows_pad_sh * khs * 128;
         size_t o = 0;
         hdr = o; o += 256;
         src1 = o; o += up(S * 4);
@@ -64,9 +77,11 @@ struct WsLayout {
         bounds = o; o += up((size_t)(n_experts + 1) * 4);
         active = o; o += up((size_t)(n_experts + 1) * 4);
         tiles = o; o += up((size_t)(n_experts + 1) * 4);
-        h = o; o += up((size_t)S * n_hidden * 2);
-        h_sh = o; o += up((size_t)n_tokens * n_hidden_sh * 2);
-        x16 = o; o += (x_type == MOE_F32) ? up((size_t)S * n_in * 2) : 0;
+        pad = o; o += up((size_t)(n_experts + 1) * 4);
+        h = o; o += up(h_gemv > h_gemm ? h_gemv : h_gemm);
+        h_sh = o; o += up(hs_gemv > hs_gemm ? hs_gemv : hs_gemm);
+        xt = o; o += up((size_t)rows_pad * kin * 128);
+        xt_sh = o; o += n_hidden_sh > 0 ? up((size_t)rows_pad_sh * kin * 128) : 0;
         total = o;
     }
 };

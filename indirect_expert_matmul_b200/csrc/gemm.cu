@@ -25,9 +25,6 @@
 //               layout the tensor core reads.
 // All waits are bounded; an expired wait sets MOE_ERR_TIMEOUT in the status
 // word and every role leaves its loop.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
 #include "common.cuh"
 #include "gemm_api.cuh"
 #include "ptx.cuh"
@@ -69,35 +66,61 @@ struct GemmParams {
     const uint8_t* A1;
     WLayout L;
     int n_groups;               // > 0: grouped by bounds / ntile_prefix; 0: one group of n_rows
-    const int32_t* bounds;      // [n_groups + 1]
-    const int32_t* ntile_prefix;// [n_groups + 1]
+    const int32_t* bounds;      // [n_groups + 1] sorted-position ranges
+    const int32_t* ntile_prefix;// [n_groups + 1] column-tile prefix
+    const int32_t* pad_start;   // [n_groups + 1] first row of each group in the tile-major buffers
     int n_rows;
-    const int32_t* src_rows;    // B row of sorted position p (null: p)
+    const uint8_t* B;           // activations, tile-major: [kt][b_rows][128 B], 128-byte swizzled
+    int64_t b_rows;             // rows per k-plane of B
     const int32_t* dst_rows;    // output row of sorted position p (null: p)
     float* out;                 // single-matrix output
-    __nv_bfloat16* h;           // dual output (SwiGLU)
+    uint8_t* h;                 // dual output (SwiGLU), tile-major like B: [kt][h_rows][128 B]
+    int64_t h_rows;
     int out_ld;
     int* hdr;
     int bf16;                   // operand type: 1 bf16, 0 fp16
 };
 
 struct Tile {
-    int e, mt, p0, n;
+    int e, mt, p0, n, p0pad;  // p0pad: first row of the tile in the tile-major buffers
 };
 
+// Optional stall accounting (build with -DMOE_GEMM_STATS): per role, the
+// cycles spent waiting on each barrier and the role's total cycles, summed
+// over CTAs into g_gemm_stats[role][slot].
+#ifdef MOE_GEMM_STATS
+__device__ unsigned long long g_gemm_stats[2][6][4];  // [DUAL][role][slot]
+#define STAT_DECL long long st_[4] = {0, 0, 0, 0}; const long long st_t0_ = clock64();
+#define STAT_PTR(i) (&st_[i])
+#define STAT_FLUSH(role)                                                              \
+    do {                                                                              \
+        atomicAdd(&g_gemm_stats[DUAL][role][0], (unsigned long long)st_[0]);                 \
+        atomicAdd(&g_gemm_stats[DUAL][role][1], (unsigned long long)st_[1]);                 \
+        atomicAdd(&g_gemm_stats[DUAL][role][2], (unsigned long long)st_[2]);                 \
+        atomicAdd(&g_gemm_stats[DUAL][role][3], (unsigned long long)(clock64() - st_t0_));   \
+    } while (0)
+#else
+#define STAT_DECL
+#define STAT_PTR(i) nullptr
+#define STAT_FLUSH(role) do {} while (0)
+#endif
+
 __device__ __forceinline__ Tile decode_tile(int t, int mt_count, const GemmParams& p, const int* s_prefix,
-                                            const int* s_bounds) {
+                                            const int* s_bounds, const int* s_pad) {
     Tile r;
     const int q = t / mt_count;
     r.mt = t - q * mt_count;
     if (p.n_groups == 0) {
         r.e = 0;
         r.p0 = q * kGemmBN;
+        r.p0pad = r.p0;
         r.n = min(kGemmBN, p.n_rows - r.p0);
         return r;
     }
-    const int* pre = p.n_groups <= kSmemGroups ? s_prefix : p.ntile_prefix;
-    const int* bnd = p.n_groups <= kSmemGroups ? s_bounds : p.bounds;
+    const bool in_smem = p.n_groups <= kSmemGroups;
+    const int* pre = in_smem ? s_prefix : p.ntile_prefix;
+    const int* bnd = in_smem ? s_bounds : p.bounds;
+    const int* pad = in_smem ? s_pad : p.pad_start;
     // largest e with pre[e] <= q (empty experts share their successor's prefix)
     int lo = 0, hi = p.n_groups;  // invariant: pre[lo] <= q < pre[hi]
     while (hi - lo > 1) {
@@ -107,6 +130,7 @@ __device__ __forceinline__ Tile decode_tile(int t, int mt_count, const GemmParam
     r.e = lo;
     const int j = q - pre[lo];
     r.p0 = bnd[lo] + j * kGemmBN;
+    r.p0pad = pad[lo] + j * kGemmBN;
     r.n = min(kGemmBN, bnd[lo + 1] - r.p0);
     return r;
 }
@@ -114,11 +138,15 @@ __device__ __forceinline__ Tile decode_tile(int t, int mt_count, const GemmParam
 // Bounded wait by one lane; false when the kernel is aborting.  The lane
 // sleeps in hardware between polls (suspend-time hint), so waiting roles do
 // not take issue slots from the dequantisation warps.
-__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status) {
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status,
+                                         long long* stat = nullptr) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {
-        if (ptx::mbar_try_wait_sleep(bar, parity, kSleepNs)) return true;
+        if (ptx::mbar_try_wait_sleep(bar, parity, kSleepNs)) {
+            if (stat) *stat += clock64() - t0;
+            return true;
+        }
         if (*abort_flag) return false;
         if (clock64() - t0 > kWaitLimitCycles) {
             *abort_flag = 1;
@@ -129,9 +157,10 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
 }
 
 // lane 0 waits, the warp learns the outcome
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status) {
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status,
+                                          long long* stat = nullptr) {
     int ok = 1;
-    if ((threadIdx.x & 31) == 0) ok = wait_bar(bar, parity, abort_flag, status);
+    if ((threadIdx.x & 31) == 0) ok = wait_bar(bar, parity, abort_flag, status, stat);
     return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
@@ -146,11 +175,12 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi, int bf16) {
 
 template <int DUAL>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmB, const GemmParams p) {
+grouped_gemm_kernel(const GemmParams p) {
     using C = Cfg<DUAL>;
     extern __shared__ uint8_t smem_dyn[];
     __shared__ int s_prefix[kSmemGroups + 1];
     __shared__ int s_bounds[kSmemGroups + 1];
+    __shared__ int s_pad[kSmemGroups + 1];
 
     if (read_status(p.hdr + kHdrStatus) != 0) return;
 
@@ -203,6 +233,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmB, const GemmParams p)
         for (int i = tid; i <= p.n_groups; i += kGemmThreads) {
             s_prefix[i] = p.ntile_prefix[i];
             s_bounds[i] = p.bounds[i];
+            s_pad[i] = p.pad_start[i];
         }
     }
     const int n_coltiles = p.n_groups > 0 ? p.hdr[kHdrTiles] : (p.n_rows + kGemmBN - 1) / kGemmBN;
@@ -217,6 +248,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmB, const GemmParams p)
         // One lane streams the tiles' weight blocks: an L2 prefetch runs
         // kPrefetchSteps k-steps ahead of the bulk copies into the raw ring.
         if (lane == 0) {
+            STAT_DECL
             int rs = 0;
             uint32_t rph = 0;
             uint32_t used = 0, par = 0;  // per-stage issue record, for draining
@@ -226,7 +258,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmB, const GemmParams p)
             auto prefetch_one = [&]() {
                 if (pf_t >= total) return;
                 if (pf_tile != pf_t) {
-                    const Tile tl = decode_tile(pf_t, MT, p, s_prefix, s_bounds);
+                    const Tile tl = decode_tile(pf_t, MT, p, s_prefix, s_bounds, s_pad);
                     pf_bytes = (uint32_t)L.rows(tl.mt) * kRowBytes;
                     pf_a0 = p.A0 + L.block(tl.e, tl.mt, 0);
                     pf_a1 = DUAL ? p.A1 + L.block(tl.e, tl.mt, 0) : nullptr;
@@ -239,13 +271,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmB, const GemmParams p)
             for (int i = 0; i < kPrefetchSteps; ++i) prefetch_one();
             bool ok = true;
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-                const Tile tl = decode_tile(t, MT, p, s_prefix, s_bounds);
+                const Tile tl = decode_tile(t, MT, p, s_prefix, s_bounds, s_pad);
                 const uint32_t raw_bytes = (uint32_t)L.rows(tl.mt) * kRowBytes;
                 const uint8_t* a0 = p.A0 + L.block(tl.e, tl.mt, 0);
                 const uint8_t* a1 = DUAL ? p.A1 + L.block(tl.e, tl.mt, 0) : nullptr;
                 for (int kt = 0; kt < KT; ++kt) {
                     prefetch_one();
-                    ok = wait_bar(&raw_empty[rs], rph ^ 1, abort_flag, status);
+                    ok = wait_bar(&raw_empty[rs], rph ^ 1, abort_flag, status, STAT_PTR(0));
                     if (!ok) break;
                     ptx::mbar_arrive_expect_tx(&raw_full[rs], raw_bytes * C::NMAT);
                     ptx::bulk_g2s(sRaw + (rs * C::NMAT) * kRawBytes, a0 + (size_t)kt * raw_bytes, raw_bytes,
@@ -262,74 +294,60 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmB, const GemmParams p)
             volatile int never = 0;
             for (int s = 0; s < C::RS; ++s)
                 if (used >> s & 1) wait_bar(&raw_full[s], (par >> s) & 1, &never, status);
+            STAT_FLUSH(0);
         }
     } else if (warp == kWarpProdB) {
         // ------------------------------------------------ activation producer
-        int bs = 0;
-        uint32_t bph = 0;
-        uint32_t used = 0, par = 0;
-        bool ok = true;
-        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-            const Tile tl = decode_tile(t, MT, p, s_prefix, s_bounds);
-            const int n16 = (tl.n + 15) & ~15;
-            int rows4[2][4];
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                const int g = lane + 32 * i;
-#pragma unroll
-                for (int r = 0; r < 4; ++r) {
-                    const int pos = tl.p0 + min(4 * g + r, tl.n - 1);
-                    rows4[i][r] = p.src_rows ? __ldg(p.src_rows + pos) : pos;
-                }
-            }
-            for (int kt = 0; kt < KT; ++kt) {
-                if (lane == 0) {
-                    ok = wait_bar(&b_empty[bs], bph ^ 1, abort_flag, status);
-                    if (ok) {
-                        ptx::mbar_arrive_expect_tx(&b_full[bs], (uint32_t)n16 * 128u);
-                        used |= 1u << bs;
-                        par = (par & ~(1u << bs)) | (bph << bs);
-                    }
-                }
-                ok = __shfl_sync(0xffffffffu, (int)ok, 0) != 0;
-                if (!ok) break;
-                uint8_t* bdst = sB + bs * kBTileBytes;
-#pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    const int g = lane + 32 * i;
-                    if (4 * g < n16)
-                        ptx::tma_gather4(bdst + g * 512, &tmB, kt * kTileK, rows4[i][0], rows4[i][1], rows4[i][2],
-                                         rows4[i][3], &b_full[bs]);
-                }
-                if (++bs == C::MB) { bs = 0; bph ^= 1; }
-            }
-        }
+        // The rows of a column tile are contiguous and already swizzled in the
+        // tile-major activation buffer: one bulk copy per k-step.
         if (lane == 0) {
+            STAT_DECL
+            int bs = 0;
+            uint32_t bph = 0;
+            uint32_t used = 0, par = 0;
+            bool ok = true;
+            const size_t plane = (size_t)p.b_rows * 128u;
+            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+                const Tile tl = decode_tile(t, MT, p, s_prefix, s_bounds, s_pad);
+                const uint32_t bytes = (uint32_t)((tl.n + 15) & ~15) * 128u;
+                const uint8_t* src = p.B + (size_t)tl.p0pad * 128u;
+                for (int kt = 0; kt < KT; ++kt) {
+                    ok = wait_bar(&b_empty[bs], bph ^ 1, abort_flag, status, STAT_PTR(0));
+                    if (!ok) break;
+                    ptx::mbar_arrive_expect_tx(&b_full[bs], bytes);
+                    ptx::bulk_g2s(sB + bs * kBTileBytes, src + kt * plane, bytes, &b_full[bs]);
+                    used |= 1u << bs;
+                    par = (par & ~(1u << bs)) | (bph << bs);
+                    if (++bs == C::MB) { bs = 0; bph ^= 1; }
+                }
+            }
             volatile int never = 0;
             for (int s = 0; s < C::MB; ++s)
                 if (used >> s & 1) wait_bar(&b_full[s], (par >> s) & 1, &never, status);
+            STAT_FLUSH(1);
         }
     } else if (warp == kWarpMma) {
         // ----------------------------------------------------------------- MMA
         if (lane == 0) {
+            STAT_DECL
             int as = 0, bs = 0;
             uint32_t aph = 0, bph = 0;
             uint32_t use[2] = {0, 0};
             int it = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
-                const Tile tl = decode_tile(t, MT, p, s_prefix, s_bounds);
+                const Tile tl = decode_tile(t, MT, p, s_prefix, s_bounds, s_pad);
                 const int n16 = (tl.n + 15) & ~15;
                 const int buf = DUAL ? 0 : (it & 1);
-                ok = wait_bar(&tmem_empty[buf], (use[buf] & 1) ^ 1, abort_flag, status);
+                ok = wait_bar(&tmem_empty[buf], (use[buf] & 1) ^ 1, abort_flag, status, STAT_PTR(2));
                 if (!ok) break;
                 ptx::tc_fence_after();
                 const uint32_t d0 = tmem_base + (DUAL ? 0u : (uint32_t)buf * 256u);
                 const uint32_t d1 = tmem_base + 256u;
                 const uint32_t idesc = ptx::idesc_f16(p.bf16, n16, 128);
                 for (int kt = 0; kt < KT; ++kt) {
-                    ok = wait_bar(&a_full[as], aph, abort_flag, status) &&
-                         wait_bar(&b_full[bs], bph, abort_flag, status);
+                    ok = wait_bar(&a_full[as], aph, abort_flag, status, STAT_PTR(0)) &&
+                         wait_bar(&b_full[bs], bph, abort_flag, status, STAT_PTR(1));
                     if (!ok) break;
                     ptx::tc_fence_after();
                     const uint32_t a0 = ptx::smem_u32(sA + (as * C::NMAT) * kATileBytes);
@@ -353,17 +371,19 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmB, const GemmParams p)
                 ptx::mma_commit(&tmem_full[buf]);
                 use[buf] += 1;
             }
+            STAT_FLUSH(2);
         }
         __syncwarp();
     } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
         // ------------------------------------------------------------ epilogue
         const int ew = warp - kEpiWarp0;
+        STAT_DECL
         uint32_t use[2] = {0, 0};
         int it = 0;
         for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
-            const Tile tl = decode_tile(t, MT, p, s_prefix, s_bounds);
+            const Tile tl = decode_tile(t, MT, p, s_prefix, s_bounds, s_pad);
             const int buf = DUAL ? 0 : (it & 1);
-            if (!warp_wait(&tmem_full[buf], use[buf] & 1, abort_flag, status)) break;
+            if (!warp_wait(&tmem_full[buf], use[buf] & 1, abort_flag, status, STAT_PTR(0))) break;
             use[buf] += 1;
             ptx::tc_fence_after();
             const int m = tl.mt * kTileM + 32 * ew + lane;
@@ -376,12 +396,17 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmB, const GemmParams p)
                     uint32_t u[32];
                     ptx::tmem_ld_32x32b_x32(tbase + 256 + c0, u);
                     ptx::tmem_ld_wait();
+                    // h goes to the tile-major swizzled buffer the down GEMM streams
+                    uint8_t* hplane = p.h + (size_t)(m >> 6) * p.h_rows * 128u + ((m & 7) << 1);
+                    const int mchunk = (m & 63) >> 3;
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
                         if (c0 + i < tl.n && m_ok) {
                             const float g = __uint_as_float(v[i]), up = __uint_as_float(u[i]);
                             const float hv = g / (1.0f + __expf(-g)) * up;
-                            p.h[(int64_t)(tl.p0 + c0 + i) * p.out_ld + m] = __float2bfloat16_rn(hv);
+                            const int prow = tl.p0pad + c0 + i;
+                            *(__nv_bfloat16*)(hplane + (size_t)prow * 128u + ((mchunk ^ (prow & 7)) << 4)) =
+                                __float2bfloat16_rn(hv);
                         }
                     }
                 } else {
@@ -400,20 +425,22 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmB, const GemmParams p)
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&tmem_empty[buf]);
         }
+        if (lane == 0) STAT_FLUSH(3);
     } else if (warp >= kDeqWarp0) {
         // ------------------------------------------------------- dequantisation
         const int d = tid - kDeqWarp0 * 32;  // 0..255
         const int r = d >> 1, hlf = d & 1;
         const int first = (d >> 2) & 1;      // alternate read order: conflict-free 16-byte loads
+        STAT_DECL
         int rs = 0, as = 0;
         uint32_t rph = 0, aph = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-            const Tile tl = decode_tile(t, MT, p, s_prefix, s_bounds);
+            const Tile tl = decode_tile(t, MT, p, s_prefix, s_bounds, s_pad);
             const int rows = L.rows(tl.mt);
             for (int kt = 0; kt < KT; ++kt) {
-                ok = warp_wait(&raw_full[rs], rph, abort_flag, status) &&
-                     warp_wait(&a_empty[as], aph ^ 1, abort_flag, status);
+                ok = warp_wait(&raw_full[rs], rph, abort_flag, status, STAT_PTR(0)) &&
+                     warp_wait(&a_empty[as], aph ^ 1, abort_flag, status, STAT_PTR(1));
                 if (!ok) break;
 #pragma unroll
                 for (int mat = 0; mat < C::NMAT; ++mat) {
@@ -457,6 +484,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmB, const GemmParams p)
                 if (++as == C::MA) { as = 0; aph ^= 1; }
             }
         }
+        if (lane == 0) STAT_FLUSH(4);
     }
 
     ptx::tc_fence_before();
@@ -467,38 +495,60 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmB, const GemmParams p)
     }
 }
 
-// fp32 activations -> fp16 copy (the tensor core reads fp16 operands)
-__global__ void f32_to_f16_kernel(const float* __restrict__ x, __half* __restrict__ y, int64_t n) {
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
-        y[i] = __float2half_rn(x[i]);
+// Gather activation rows into the tile-major, 128-byte-swizzled layout the
+// GEMM streams with one bulk copy per k-step: the row at sorted position p of
+// group e (rank r inside the group) becomes row pad_start[e] + r; k-plane kt
+// holds columns [64*kt, 64*kt + 64) as 128 bytes whose 16-byte chunk c sits at
+// chunk c ^ (row % 8).  fp32 input is rounded to fp16; columns >= n_in are 0.
+__global__ void __launch_bounds__(256)
+gather_tiled_kernel(const void* __restrict__ x, int x_type, int n_in, int KT, const int32_t* __restrict__ src_rows,
+                    const int32_t* __restrict__ bounds, const int32_t* __restrict__ pad_start, int n_groups,
+                    int64_t n_rows, int64_t rows_pad, uint8_t* __restrict__ xt, const int* __restrict__ hdr) {
+    if (read_status(hdr + kHdrStatus) != 0) return;
+    const int lane = threadIdx.x & 31;
+    const int64_t S = n_groups > 0 ? bounds[n_groups] : n_rows;
+    const int64_t nw = (int64_t)gridDim.x * (blockDim.x / 32);
+    for (int64_t p = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); p < S; p += nw) {
+        int64_t prow = p, srow = p;
+        if (n_groups > 0) {
+            int lo = 0, hi = n_groups;  // bounds[lo] <= p < bounds[hi]
+            while (hi - lo > 1) {
+                const int mid = (lo + hi) >> 1;
+                if (__ldg(bounds + mid) <= p) lo = mid; else hi = mid;
+            }
+            prow = __ldg(pad_start + lo) + (p - __ldg(bounds + lo));
+            srow = src_rows ? __ldg(src_rows + p) : p;
+        }
+        for (int seg = lane; seg < KT * 8; seg += 32) {
+            const int kt = seg >> 3, c = seg & 7, col = kt * 64 + c * 8;
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (col < n_in) {
+                if (x_type == MOE_F32) {
+                    const float4* src = (const float4*)((const float*)x + srow * n_in + col);
+                    const float4 a = __ldg(src), b = __ldg(src + 1);
+                    __half2 h0 = __floats2half2_rn(a.x, a.y), h1 = __floats2half2_rn(a.z, a.w);
+                    __half2 h2 = __floats2half2_rn(b.x, b.y), h3 = __floats2half2_rn(b.z, b.w);
+                    v = make_uint4(*(uint32_t*)&h0, *(uint32_t*)&h1, *(uint32_t*)&h2, *(uint32_t*)&h3);
+                } else {
+                    v = __ldg((const uint4*)((const uint16_t*)x + srow * n_in + col));
+                }
+            }
+            *(uint4*)(xt + ((size_t)kt * rows_pad + prow) * 128u + ((c ^ (int)(prow & 7)) << 4)) = v;
+        }
+    }
 }
 
 // ------------------------------------------------------------------- host
-static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        cudaDriverEntryPointQueryResult q;
-        void* f = nullptr;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = (PFN_cuTensorMapEncodeTiled_v12000)f;
+#ifdef MOE_GEMM_STATS
+extern "C" __attribute__((visibility("default"))) int moe_gemm_stats_read(unsigned long long* out48, int reset) {
+    if (cudaMemcpyFromSymbol(out48, g_gemm_stats, sizeof(g_gemm_stats)) != cudaSuccess) return MOE_ERR_CUDA;
+    if (reset) {
+        static const unsigned long long zero[2][6][4] = {};
+        if (cudaMemcpyToSymbol(g_gemm_stats, zero, sizeof(zero)) != cudaSuccess) return MOE_ERR_CUDA;
     }
-    return fn;
+    return MOE_OK;
 }
-
-// 2-D map over rows x n_in 16-bit elements, box = 64 columns x 1 row, 128-byte swizzle
-static bool make_gather_map(CUtensorMap* m, const void* base, int64_t rows, int n_in, int bf16) {
-    auto enc = get_encode();
-    if (!enc) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)n_in, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)n_in * 2};
-    cuuint32_t box[2] = {(cuuint32_t)kTileK, 1};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
-                     const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
+#endif
 
 static int sm_count() {
     static int dev_cached = -1, n = 0;
@@ -512,8 +562,7 @@ static int sm_count() {
 }
 
 template <int DUAL>
-static moe_status run_gemm(const GemmParams& p, const void* B, int64_t b_rows, int b_cols, int64_t max_coltiles,
-                           cudaStream_t stream) {
+static moe_status run_gemm(const GemmParams& p, int64_t max_coltiles, cudaStream_t stream) {
     static int attr_dev = -1;
     int dev = 0;
     cudaGetDevice(&dev);
@@ -523,62 +572,64 @@ static moe_status run_gemm(const GemmParams& p, const void* B, int64_t b_rows, i
             return MOE_ERR_CUDA;
         attr_dev = dev;
     }
-    CUtensorMap map;
-    if (!make_gather_map(&map, B, b_rows, b_cols, p.bf16)) return MOE_ERR_CUDA;
     int64_t tiles = max_coltiles * p.L.mt_count;
     if (tiles <= 0) return MOE_OK;
     int grid = (int)(tiles < sm_count() ? tiles : sm_count());
-    grouped_gemm_kernel<DUAL><<<grid, kGemmThreads, Cfg<DUAL>::smem_bytes, stream>>>(map, p);
+    grouped_gemm_kernel<DUAL><<<grid, kGemmThreads, Cfg<DUAL>::smem_bytes, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 static int64_t coltile_bound(int64_t S, int E) { return (S + kGemmBN - 1) / kGemmBN + (S < E ? S : E); }
 
-static moe_status to_f16(const void* x, void* x16, int64_t n, cudaStream_t s) {
-    int64_t blocks = (n + 255) / 256;
-    if (blocks > 148 * 16) blocks = 148 * 16;
+static moe_status gather(const void* x, int x_type, int n_in, const int32_t* src_rows, const int32_t* bounds,
+                         const int32_t* pad_start, int n_groups, int64_t rows, int64_t rows_pad, void* xt, int* hdr,
+                         cudaStream_t s) {
+    const int KT = (n_in + kTileK - 1) / kTileK;
+    int64_t blocks = (rows + 7) / 8;
+    if (blocks > (int64_t)sm_count() * 8) blocks = (int64_t)sm_count() * 8;
     if (blocks < 1) blocks = 1;
-    f32_to_f16_kernel<<<(unsigned)blocks, 256, 0, s>>>((const float*)x, (__half*)x16, n);
+    gather_tiled_kernel<<<(unsigned)blocks, 256, 0, s>>>(x, x_type, n_in, KT, src_rows, bounds, pad_start, n_groups,
+                                                         rows, rows_pad, (uint8_t*)xt, hdr);
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 moe_status launch_gemm_mul_mat_id(const GemmMulMatId& g, cudaStream_t stream) {
-    const void* B = g.x;
-    int bf16 = g.x_type == MOE_BF16;
-    if (g.x_type == MOE_F32) {
-        moe_status st = to_f16(g.x, g.x16, g.x_rows * g.n_in, stream);
-        if (st) return st;
-        prof_mark(stream, "x_to_f16");
-        B = g.x16;
-    }
+    moe_status st = gather(g.x, g.x_type, g.n_in, g.ids_src1, g.bounds, g.pad_start, g.E, g.S, g.rows_pad, g.xt,
+                           g.hdr, stream);
+    if (st) return st;
+    prof_mark(stream, "gather");
     GemmParams p = {};
     p.A0 = g.W;
     p.L = WLayout(g.n_out, g.n_in);
     p.n_groups = g.E;
     p.bounds = g.bounds;
     p.ntile_prefix = g.ntile_prefix;
-    p.src_rows = g.ids_src1;
+    p.pad_start = g.pad_start;
+    p.B = (const uint8_t*)g.xt;
+    p.b_rows = g.rows_pad;
     p.dst_rows = g.ids_dst;
     p.out = g.dst;
     p.out_ld = g.n_out;
     p.hdr = g.hdr;
-    p.bf16 = bf16;
-    moe_status st = run_gemm<0>(p, B, g.x_rows, g.n_in, coltile_bound(g.S, g.E), stream);
+    p.bf16 = g.x_type == MOE_BF16;
+    st = run_gemm<0>(p, coltile_bound(g.S, g.E), stream);
     prof_mark(stream, "gemm");
     return st;
 }
 
 moe_status launch_gemm_ffn(const GemmFfn& g, cudaStream_t stream) {
-    const void* X = g.x;
-    int bf16 = g.x_type == MOE_BF16;
-    moe_status st;
-    if (g.x_type == MOE_F32) {
-        st = to_f16(g.x, g.x16, g.T * g.n_embd, stream);
-        if (st) return st;
-        prof_mark(stream, "x_to_f16");
-        X = g.x16;
+    const int bf16 = g.x_type == MOE_BF16;
+    const int kt_ff = (g.n_ff + kTileK - 1) / kTileK;
+    moe_status st = gather(g.x, g.x_type, g.n_embd, g.ids_src1, g.bounds, g.pad_start, g.E, g.S, g.rows_pad, g.xt,
+                           g.hdr, stream);
+    if (st) return st;
+    prof_mark(stream, "gather");
+    if (g.n_ff % kTileK) {  // columns past n_ff of the last k-plane of h are read by the down GEMM: keep them 0
+        if (cudaMemsetAsync((uint8_t*)g.h + (size_t)(kt_ff - 1) * g.rows_pad * 128u, 0, (size_t)g.rows_pad * 128u,
+                            stream) != cudaSuccess)
+            return MOE_ERR_CUDA;
     }
-    // gate/up -> h (expert-sorted rows), SwiGLU in the epilogue
+    // gate/up -> h (tile-major, expert-sorted rows), SwiGLU in the epilogue
     GemmParams p = {};
     p.A0 = g.Wg;
     p.A1 = g.Wu;
@@ -586,55 +637,72 @@ moe_status launch_gemm_ffn(const GemmFfn& g, cudaStream_t stream) {
     p.n_groups = g.E;
     p.bounds = g.bounds;
     p.ntile_prefix = g.ntile_prefix;
-    p.src_rows = g.ids_src1;
-    p.h = g.h;
+    p.pad_start = g.pad_start;
+    p.B = (const uint8_t*)g.xt;
+    p.b_rows = g.rows_pad;
+    p.h = (uint8_t*)g.h;
+    p.h_rows = g.rows_pad;
     p.out_ld = g.n_ff;
     p.hdr = g.hdr;
     p.bf16 = bf16;
-    st = run_gemm<1>(p, X, g.T, g.n_embd, coltile_bound(g.S, g.E), stream);
+    st = run_gemm<1>(p, coltile_bound(g.S, g.E), stream);
     if (st) return st;
     prof_mark(stream, "gemm_gate_up");
+    const int kt_sh = (g.n_ff_shared + kTileK - 1) / kTileK;
     if (g.n_ff_shared > 0) {
+        st = gather(g.x, g.x_type, g.n_embd, nullptr, nullptr, nullptr, 0, g.T, g.rows_pad_sh, g.xt_sh, g.hdr, stream);
+        if (st) return st;
+        if (g.n_ff_shared % kTileK) {
+            if (cudaMemsetAsync((uint8_t*)g.h_sh + (size_t)(kt_sh - 1) * g.rows_pad_sh * 128u, 0,
+                                (size_t)g.rows_pad_sh * 128u, stream) != cudaSuccess)
+                return MOE_ERR_CUDA;
+        }
         GemmParams q = {};
         q.A0 = g.Sg;
         q.A1 = g.Su;
         q.L = WLayout(g.n_ff_shared, g.n_embd);
-        q.n_groups = 0;
         q.n_rows = (int)g.T;
-        q.h = g.h_sh;
+        q.B = (const uint8_t*)g.xt_sh;
+        q.b_rows = g.rows_pad_sh;
+        q.h = (uint8_t*)g.h_sh;
+        q.h_rows = g.rows_pad_sh;
         q.out_ld = g.n_ff_shared;
         q.hdr = g.hdr;
         q.bf16 = bf16;
-        st = run_gemm<1>(q, X, g.T, g.n_embd, (g.T + kGemmBN - 1) / kGemmBN, stream);
+        st = run_gemm<1>(q, (g.T + kGemmBN - 1) / kGemmBN, stream);
         if (st) return st;
         prof_mark(stream, "gemm_shared_gate_up");
     }
-    // down: h rows are already contiguous per expert; scatter to dst by ids_dst
+    // down: B = h, contiguous per expert; the epilogue scatters rows to dst by ids_dst
     GemmParams d = {};
     d.A0 = g.Wd;
     d.L = WLayout(g.n_embd, g.n_ff);
     d.n_groups = g.E;
     d.bounds = g.bounds;
     d.ntile_prefix = g.ntile_prefix;
+    d.pad_start = g.pad_start;
+    d.B = (const uint8_t*)g.h;
+    d.b_rows = g.rows_pad;
     d.dst_rows = g.ids_dst;
     d.out = g.dst;
     d.out_ld = g.n_embd;
     d.hdr = g.hdr;
     d.bf16 = 1;
-    st = run_gemm<0>(d, g.h, g.S, g.n_ff, coltile_bound(g.S, g.E), stream);
+    st = run_gemm<0>(d, coltile_bound(g.S, g.E), stream);
     if (st) return st;
     prof_mark(stream, "gemm_down");
     if (g.n_ff_shared > 0) {
         GemmParams q = {};
         q.A0 = g.Sd;
         q.L = WLayout(g.n_embd, g.n_ff_shared);
-        q.n_groups = 0;
         q.n_rows = (int)g.T;
+        q.B = (const uint8_t*)g.h_sh;
+        q.b_rows = g.rows_pad_sh;
         q.out = g.dst_shared;
         q.out_ld = g.n_embd;
         q.hdr = g.hdr;
         q.bf16 = 1;
-        st = run_gemm<0>(q, g.h_sh, g.T, g.n_ff_shared, (g.T + kGemmBN - 1) / kGemmBN, stream);
+        st = run_gemm<0>(q, (g.T + kGemmBN - 1) / kGemmBN, stream);
         prof_mark(stream, "gemm_shared_down");
     }
     return st;

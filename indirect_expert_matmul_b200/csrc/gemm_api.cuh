@@ -10,7 +10,9 @@ struct GemmMulMatId {
     const void* x;
     int x_type;
     int64_t x_rows;   // rows of x: n_tokens (broadcast) or n_tokens*k (per_slot)
-    void* x16;        // workspace for an fp16 copy of fp32 x (or null)
+    void* xt;         // workspace: gathered x, tile-major and swizzled (rows_pad rows)
+    int64_t rows_pad;
+    const int32_t* pad_start;
     int64_t S;
     float* dst;
     const int32_t* bounds;
@@ -27,11 +29,14 @@ struct GemmFfn {
     int n_ff_shared;
     const void* x;
     int x_type;
-    void* x16;
+    void* xt;         // gathered x (routed), tile-major and swizzled
+    void* xt_sh;      // x in token order for the shared expert
+    int64_t rows_pad, rows_pad_sh;
+    const int32_t* pad_start;
     int64_t T, S;
     float* dst;
     float* dst_shared;
-    __nv_bfloat16* h;
+    __nv_bfloat16* h;     // tile-major swizzled hidden activations (GEMM path)
     __nv_bfloat16* h_sh;
     const int32_t* bounds;
     const int32_t* ntile_prefix;

@@ -175,7 +175,9 @@ gemv_kernel(const GemvArgs a) {
         ptx::fence_mbar_init();
     }
     __syncthreads();
-    uint32_t rounds = 0;
+    // stage s completes one phase per arm; windows may arm different numbers of
+    // stages, so each stage keeps its own parity bit
+    uint32_t next_par = 0, wait_par = 0;
     auto issue = [&](int kt0, int kt1) {
         if (tid == 0) {
             for (int kt = kt0; kt < kt1; ++kt) {
@@ -191,7 +193,9 @@ gemv_kernel(const GemvArgs a) {
                 }
             }
         }
-        ++rounds;
+        const uint32_t armed = (kt1 - kt0) >= 32 ? 0xffffffffu : ((1u << (kt1 - kt0)) - 1u);
+        wait_par = next_par;
+        next_par ^= armed;
     };
     if (resident) issue(0, KT);
     if (a.pdl_secondary) asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -257,7 +261,7 @@ gemv_kernel(const GemvArgs a) {
             __syncthreads();
             for (int kt = kt0 + ph; kt < kt1; kt += P) {
                 const int s = kt - kt0;
-                if (!gv_wait(&bars[s], (rounds - 1) & 1, status)) { ok = false; break; }
+                if (!gv_wait(&bars[s], (wait_par >> s) & 1u, status)) { ok = false; break; }
                 const uint8_t* st = sw + (size_t)s * stage_bytes;
                 float w[NMAT][16];
 #pragma unroll

@@ -7,8 +7,8 @@
 
 namespace moe {
 moe_status launch_row_ids(const int32_t* ids, int64_t S, int k, int E, int mode, int32_t* ids_src1,
-                          int32_t* ids_dst, int32_t* bounds, int32_t* active, int32_t* ntile_prefix, int bn, int* hdr,
-                          cudaStream_t stream);
+                          int32_t* ids_dst, int32_t* bounds, int32_t* active, int32_t* ntile_prefix,
+                          int32_t* pad_start, int bn, int* hdr, cudaStream_t stream);
 moe_status launch_prepare(const void* src, int E, int n_out, int n_in, void* dst, cudaStream_t stream);
 }  // namespace moe
 
@@ -98,8 +98,8 @@ moe_status moe_row_ids(const int32_t* ids, int64_t n_tokens, int k, int n_expert
     char* ws = (char*)workspace;
     prof_begin((cudaStream_t)stream);
     st = launch_row_ids(ids, n_tokens * k, k, n_experts, mode, ids_src1, ids_dst, expert_bounds,
-                        (int32_t*)(ws + W.active), (int32_t*)(ws + W.tiles), kGemmBN, (int*)(ws + W.hdr),
-                        (cudaStream_t)stream);
+                        (int32_t*)(ws + W.active), (int32_t*)(ws + W.tiles), (int32_t*)(ws + W.pad), kGemmBN,
+                        (int*)(ws + W.hdr), (cudaStream_t)stream);
     prof_mark((cudaStream_t)stream, "row_ids");
     return st;
 }
@@ -145,7 +145,8 @@ moe_status moe_mul_mat_id(const void* W_prepared, int n_experts, int n_out, int 
         prof_mark(s, "gemv");
         return st;
     }
-    st = launch_row_ids(ids, S, k, n_experts, mode, src1, dstr, bounds, active, tiles, kGemmBN, hdr, s);
+    st = launch_row_ids(ids, S, k, n_experts, mode, src1, dstr, bounds, active, tiles, (int32_t*)(ws + W.pad),
+                        kGemmBN, hdr, s);
     if (st) return st;
     prof_mark(s, "row_ids");
     GemmMulMatId g = {};
@@ -156,7 +157,9 @@ moe_status moe_mul_mat_id(const void* W_prepared, int n_experts, int n_out, int 
     g.x = x;
     g.x_type = x_type;
     g.x_rows = mode == MOE_BROADCAST ? n_tokens : S;
-    g.x16 = (x_type == MOE_F32) ? (void*)(ws + W.x16) : nullptr;
+    g.xt = ws + W.xt;
+    g.rows_pad = W.rows_pad;
+    g.pad_start = (const int32_t*)(ws + W.pad);
     g.S = S;
     g.dst = dst;
     g.bounds = bounds;
@@ -256,7 +259,8 @@ moe_status moe_ffn(const void* Wg, const void* Wu, const void* Wd, int n_experts
         prof_mark(s, "gemv_down");
         return st;
     }
-    st = launch_row_ids(ids, S, k, n_experts, MOE_BROADCAST, src1, dstr, bounds, active, tiles, kGemmBN, hdr, s);
+    st = launch_row_ids(ids, S, k, n_experts, MOE_BROADCAST, src1, dstr, bounds, active, tiles,
+                        (int32_t*)(ws + W.pad), kGemmBN, hdr, s);
     if (st) return st;
     prof_mark(s, "row_ids");
     GemmFfn g = {};
@@ -272,7 +276,11 @@ moe_status moe_ffn(const void* Wg, const void* Wu, const void* Wd, int n_experts
     g.n_ff_shared = n_ff_shared;
     g.x = x;
     g.x_type = x_type;
-    g.x16 = (x_type == MOE_F32) ? (void*)(ws + W.x16) : nullptr;
+    g.xt = ws + W.xt;
+    g.xt_sh = ws + W.xt_sh;
+    g.rows_pad = W.rows_pad;
+    g.rows_pad_sh = W.rows_pad_sh;
+    g.pad_start = (const int32_t*)(ws + W.pad);
     g.T = n_tokens;
     g.S = S;
     g.dst = dst;

@@ -50,12 +50,13 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_sums, int* 
 __global__ void __launch_bounds__(kRowIdThreads, 1)
 row_ids_kernel(const int32_t* __restrict__ ids, int S, int k, int E, int mode, int n_chunks, int bn,
                int32_t* __restrict__ ids_src1, int32_t* __restrict__ ids_dst, int32_t* __restrict__ bounds,
-               int32_t* __restrict__ active, int32_t* __restrict__ ntile_prefix, int* __restrict__ hdr) {
+               int32_t* __restrict__ active, int32_t* __restrict__ ntile_prefix, int32_t* __restrict__ pad_start,
+               int* __restrict__ hdr) {
     extern __shared__ int smem[];
     int* off = smem;                        // [n_chunks][E]
     int* cnt = off + (size_t)n_chunks * E;  // [E]
     __shared__ int warp_sums[32];
-    __shared__ int totals[3];
+    __shared__ int totals[4];
     __shared__ int bad;
 
     if (read_status(hdr + kHdrStatus) != 0) return;  // sticky error: do nothing
@@ -104,24 +105,29 @@ row_ids_kernel(const int32_t* __restrict__ ids, int S, int k, int E, int mode, i
     __syncthreads();
 
     // pass 2b: exclusive prefix over experts (each thread owns a contiguous
-    // segment of experts), the compacted list of non-empty experts, and the
-    // prefix of per-expert column-tile counts ceil(count / bn) for the GEMM
+    // segment of experts), the compacted list of non-empty experts, the
+    // prefix of per-expert column-tile counts ceil(count / bn) for the GEMM,
+    // and each expert's first row in the 8-row-aligned tile-major buffers
     const int seg = (E + blockDim.x - 1) / blockDim.x;
     const int e0 = min(E, tid * seg), e1 = min(E, e0 + seg);
-    int local = 0, local_act = 0, local_tiles = 0;
+    int local = 0, local_act = 0, local_tiles = 0, local_pad = 0;
     for (int e = e0; e < e1; ++e) {
         local += cnt[e];
         local_act += cnt[e] > 0;
         local_tiles += (cnt[e] + bn - 1) / bn;
+        local_pad += (cnt[e] + 7) & ~7;
     }
     int run = block_exclusive_scan(local, warp_sums, &totals[0]);
     int run_act = block_exclusive_scan(local_act, warp_sums, &totals[1]);
     int run_tiles = block_exclusive_scan(local_tiles, warp_sums, &totals[2]);
+    int run_pad = block_exclusive_scan(local_pad, warp_sums, &totals[3]);
     for (int e = e0; e < e1; ++e) {
         int c = cnt[e];
         bounds[e] = run;
         ntile_prefix[e] = run_tiles;
         run_tiles += (c + bn - 1) / bn;
+        pad_start[e] = run_pad;
+        run_pad += (c + 7) & ~7;
         if (c > 0) active[run_act++] = e;
         cnt[e] = run;  // becomes the expert's first position
         run += c;
@@ -129,6 +135,7 @@ row_ids_kernel(const int32_t* __restrict__ ids, int S, int k, int E, int mode, i
     if (tid == 0) {
         bounds[E] = totals[0];
         ntile_prefix[E] = totals[2];
+        pad_start[E] = totals[3];
         hdr[kHdrActive] = totals[1];
         hdr[kHdrTiles] = totals[2];
     }
@@ -160,8 +167,8 @@ row_ids_kernel(const int32_t* __restrict__ ids, int S, int k, int E, int mode, i
 static size_t row_ids_smem(int n_chunks, int E) { return ((size_t)n_chunks + 1) * E * sizeof(int); }
 
 moe_status launch_row_ids(const int32_t* ids, int64_t S, int k, int E, int mode, int32_t* ids_src1,
-                          int32_t* ids_dst, int32_t* bounds, int32_t* active, int32_t* ntile_prefix, int bn, int* hdr,
-                          cudaStream_t stream) {
+                          int32_t* ids_dst, int32_t* bounds, int32_t* active, int32_t* ntile_prefix,
+                          int32_t* pad_start, int bn, int* hdr, cudaStream_t stream) {
     const size_t budget = 200 * 1024;
     int n_chunks = kRowIdWarps;
     while (n_chunks > 1 && row_ids_smem(n_chunks, E) > budget) n_chunks >>= 1;
@@ -181,7 +188,7 @@ moe_status launch_row_ids(const int32_t* ids, int64_t S, int k, int E, int mode,
         attr_dev = dev;
     }
     row_ids_kernel<<<1, kRowIdThreads, smem, stream>>>(ids, (int)S, k, E, mode, n_chunks, bn, ids_src1, ids_dst,
-                                                      bounds, active, ntile_prefix, hdr);
+                                                      bounds, active, ntile_prefix, pad_start, hdr);
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
