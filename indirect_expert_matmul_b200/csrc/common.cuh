@@ -23,8 +23,9 @@ __device__ __forceinline__ int read_status(const int* status) { return *(volatil
 
 // ------------------------------------------------------------ repacked weights
 // Tile-major form: per expert, per 128-row tile mt, per 64-column tile kt, one
-// block of rows(mt) rows: rows*64 bytes of u = q + 128, then rows*4 bytes of
-// scales (two fp16 per row: columns [0,32) and [32,64) of the tile).
+// block of rows(mt) rows: rows*32 bytes of u = q + 128 for columns [0, 32) of
+// each row (32 bytes per row), then rows*32 bytes for columns [32, 64), then
+// rows*4 bytes of scales (two fp16 per row, one per 32-column half).
 // rows(mt) = min(128, n_out_pad - 128*mt), n_out_pad = round_up(n_out, 16).
 constexpr int kTileM = 128;
 constexpr int kTileK = 64;
@@ -89,7 +90,7 @@ struct WsLayout {
 constexpr int kHdrStatus = 0;
 constexpr int kHdrActive = 1;
 constexpr int kHdrTiles = 2;   // total column tiles of the grouped GEMM
-constexpr int kGemmBN = 256;   // column (token) tile of the grouped GEMM
+constexpr int kGemmBN = 192;   // column (token) tile of the grouped GEMM
 
 // ---------------------------------------------------------------- profiling
 void prof_begin(cudaStream_t s);                     // start of an operator call

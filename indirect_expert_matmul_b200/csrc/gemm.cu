@@ -34,29 +34,30 @@ namespace moe {
 constexpr int kGemmThreads = 512;
 constexpr int kWarpProdA = 0;   // weight blocks: L2 prefetch + bulk copies
 constexpr int kWarpMma = 1;     // TMEM allocation + tcgen05.mma issue
-constexpr int kWarpProdB = 2;   // activation rows: TMA gather4
+constexpr int kWarpProdB = 2;   // activation tiles: bulk copies
 constexpr int kEpiWarp0 = 4;
 constexpr int kDeqWarp0 = 8;
 constexpr int kDeqWarps = 8;
-constexpr uint32_t kATileBytes = kTileM * kTileK * 2;  // 16 KB
-constexpr uint32_t kBTileBytes = kGemmBN * kTileK * 2; // 32 KB
+constexpr uint32_t kBTileBytes = kGemmBN * kTileK * 2; // 24 KB
 constexpr uint32_t kRawBytes = kTileM * kRowBytes;     // 8704
 constexpr int kSmemGroups = 512;                       // schedule tables kept in shared memory up to this
 constexpr int kPrefetchSteps = 8;                      // weight k-steps prefetched into L2 ahead of use
 constexpr long long kWaitLimitCycles = 1ll << 32;      // ~2 s
 constexpr uint32_t kSleepNs = 20000;                   // upper bound of one hardware wait
+// Tensor memory (512 columns): two fp32 accumulators of kGemmBN columns, then
+// the dequantised A operand, kMA stages of two 32-column matrices each.
+constexpr uint32_t kAccCols = kGemmBN;
+constexpr uint32_t kACol0 = 2 * kAccCols;
+constexpr int kMA = (512 - (int)kACol0) / 64;
+static_assert(kMA >= 2, "tensor memory holds at least two A stages");
+constexpr int kRS = 4;   // raw weight stages (int8 + scales of both matrices)
+constexpr int kMB = 5;   // activation (B) stages
 
-template <int DUAL>
 struct Cfg {
-    static constexpr int NMAT = DUAL + 1;
-    static constexpr int RS = DUAL ? 3 : 4;  // raw weight stages (int8 + scales)
-    static constexpr int MA = DUAL ? 2 : 3;  // dequantised A stages
-    static constexpr int MB = DUAL ? 3 : 4;  // activation (B) stages
-    static constexpr uint32_t a_off = 0;
-    static constexpr uint32_t b_off = a_off + MA * NMAT * kATileBytes;
-    static constexpr uint32_t raw_off = b_off + MB * kBTileBytes;
-    static constexpr uint32_t bar_off = raw_off + RS * NMAT * kRawBytes;
-    static constexpr int n_bars = 2 * RS + 2 * MA + 2 * MB + 4;
+    static constexpr uint32_t b_off = 0;
+    static constexpr uint32_t raw_off = b_off + kMB * kBTileBytes;
+    static constexpr uint32_t bar_off = raw_off + kRS * 2 * kRawBytes;
+    static constexpr int n_bars = 2 * kRS + 2 * kMA + 2 * kMB + 2;
     static constexpr uint32_t misc_off = bar_off + n_bars * 8;
     static constexpr uint32_t smem_bytes = misc_off + 64 + 1024;  // + alignment slack
 };
@@ -173,10 +174,12 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi, int bf16) {
     return *(uint32_t*)&v;
 }
 
+// Two A operands per tile share each activation tile: DUAL=1 gate and up of
+// one 128-row tile (SwiGLU epilogue into h); DUAL=0 two consecutive 128-row
+// tiles of one matrix (fp32 scatter to dst).
 template <int DUAL>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 grouped_gemm_kernel(const GemmParams p) {
-    using C = Cfg<DUAL>;
     extern __shared__ uint8_t smem_dyn[];
     __shared__ int s_prefix[kSmemGroups + 1];
     __shared__ int s_bounds[kSmemGroups + 1];
@@ -185,43 +188,54 @@ grouped_gemm_kernel(const GemmParams p) {
     if (read_status(p.hdr + kHdrStatus) != 0) return;
 
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_dyn + 1023) & ~(uintptr_t)1023);
-    uint8_t* sA = smem + C::a_off;
-    uint8_t* sB = smem + C::b_off;
-    uint8_t* sRaw = smem + C::raw_off;
-    uint64_t* bars = (uint64_t*)(smem + C::bar_off);
+    uint8_t* sB = smem + Cfg::b_off;
+    uint8_t* sRaw = smem + Cfg::raw_off;
+    uint64_t* bars = (uint64_t*)(smem + Cfg::bar_off);
     uint64_t* raw_full = bars;
-    uint64_t* raw_empty = raw_full + C::RS;
-    uint64_t* a_full = raw_empty + C::RS;
-    uint64_t* a_empty = a_full + C::MA;
-    uint64_t* b_full = a_empty + C::MA;
-    uint64_t* b_empty = b_full + C::MB;
-    uint64_t* tmem_full = b_empty + C::MB;
-    uint64_t* tmem_empty = tmem_full + 2;
-    uint32_t* tmem_base_sh = (uint32_t*)(smem + C::misc_off);
-    volatile int* abort_flag = (volatile int*)(smem + C::misc_off + 4);
+    uint64_t* raw_empty = raw_full + kRS;
+    uint64_t* a_full = raw_empty + kRS;
+    uint64_t* a_empty = a_full + kMA;
+    uint64_t* b_full = a_empty + kMA;
+    uint64_t* b_empty = b_full + kMB;
+    uint64_t* tmem_full = b_empty + kMB;
+    uint64_t* tmem_empty = tmem_full + 1;
+    uint32_t* tmem_base_sh = (uint32_t*)(smem + Cfg::misc_off);
+    volatile int* abort_flag = (volatile int*)(smem + Cfg::misc_off + 4);
     int* status = p.hdr + kHdrStatus;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const WLayout L = p.L;
     const int MT = L.mt_count, KT = L.kt_count;
+    const int MU = DUAL ? MT : (MT + 1) / 2;  // row units per column tile
+
+    // the two A sources of a tile: (block pointer at kt = 0, rows)
+    auto source = [&](const Tile& tl, int i, const uint8_t*& ptr, int& rows, int& mt) {
+        if (DUAL) {
+            mt = tl.mt;
+            rows = L.rows(mt);
+            ptr = (i ? p.A1 : p.A0) + L.block(tl.e, mt, 0);
+        } else {
+            mt = 2 * tl.mt + i;
+            rows = mt < MT ? L.rows(mt) : 0;
+            ptr = p.A0 + (mt < MT ? L.block(tl.e, mt, 0) : 0);
+        }
+    };
 
     if (tid == 0) {
-        for (int i = 0; i < C::RS; ++i) {
+        for (int i = 0; i < kRS; ++i) {
             ptx::mbar_init(&raw_full[i], 1);
             ptx::mbar_init(&raw_empty[i], kDeqWarps);
         }
-        for (int i = 0; i < C::MA; ++i) {
+        for (int i = 0; i < kMA; ++i) {
             ptx::mbar_init(&a_full[i], kDeqWarps);
             ptx::mbar_init(&a_empty[i], 1);
         }
-        for (int i = 0; i < C::MB; ++i) {
+        for (int i = 0; i < kMB; ++i) {
             ptx::mbar_init(&b_full[i], 1);
             ptx::mbar_init(&b_empty[i], 1);
         }
-        for (int i = 0; i < 2; ++i) {
-            ptx::mbar_init(&tmem_full[i], 1);
-            ptx::mbar_init(&tmem_empty[i], 4);
-        }
+        ptx::mbar_init(tmem_full, 1);
+        ptx::mbar_init(tmem_empty, 4);
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
@@ -237,7 +251,7 @@ grouped_gemm_kernel(const GemmParams p) {
         }
     }
     const int n_coltiles = p.n_groups > 0 ? p.hdr[kHdrTiles] : (p.n_rows + kGemmBN - 1) / kGemmBN;
-    const int total = n_coltiles * MT;
+    const int total = n_coltiles * MU;
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
@@ -245,7 +259,7 @@ grouped_gemm_kernel(const GemmParams p) {
 
     if (warp == kWarpProdA) {
         // ---------------------------------------------------- weight producer
-        // One lane streams the tiles' weight blocks: an L2 prefetch runs
+        // One lane streams both sources' weight blocks: an L2 prefetch runs
         // kPrefetchSteps k-steps ahead of the bulk copies into the raw ring.
         if (lane == 0) {
             STAT_DECL
@@ -253,46 +267,51 @@ grouped_gemm_kernel(const GemmParams p) {
             uint32_t rph = 0;
             uint32_t used = 0, par = 0;  // per-stage issue record, for draining
             int pf_t = blockIdx.x, pf_kt = 0, pf_tile = -1;
-            const uint8_t *pf_a0 = nullptr, *pf_a1 = nullptr;
-            uint32_t pf_bytes = 0;
+            const uint8_t* pf_a[2] = {nullptr, nullptr};
+            uint32_t pf_b[2] = {0u, 0u};
             auto prefetch_one = [&]() {
                 if (pf_t >= total) return;
                 if (pf_tile != pf_t) {
-                    const Tile tl = decode_tile(pf_t, MT, p, s_prefix, s_bounds, s_pad);
-                    pf_bytes = (uint32_t)L.rows(tl.mt) * kRowBytes;
-                    pf_a0 = p.A0 + L.block(tl.e, tl.mt, 0);
-                    pf_a1 = DUAL ? p.A1 + L.block(tl.e, tl.mt, 0) : nullptr;
+                    const Tile tl = decode_tile(pf_t, MU, p, s_prefix, s_bounds, s_pad);
+                    for (int i = 0; i < 2; ++i) {
+                        int rows, mt;
+                        source(tl, i, pf_a[i], rows, mt);
+                        pf_b[i] = (uint32_t)rows * kRowBytes;
+                    }
                     pf_tile = pf_t;
                 }
-                ptx::bulk_prefetch_l2(pf_a0 + (size_t)pf_kt * pf_bytes, pf_bytes);
-                if (DUAL) ptx::bulk_prefetch_l2(pf_a1 + (size_t)pf_kt * pf_bytes, pf_bytes);
+                for (int i = 0; i < 2; ++i)
+                    if (pf_b[i]) ptx::bulk_prefetch_l2(pf_a[i] + (size_t)pf_kt * pf_b[i], pf_b[i]);
                 if (++pf_kt == KT) { pf_kt = 0; pf_t += gridDim.x; }
             };
             for (int i = 0; i < kPrefetchSteps; ++i) prefetch_one();
             bool ok = true;
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-                const Tile tl = decode_tile(t, MT, p, s_prefix, s_bounds, s_pad);
-                const uint32_t raw_bytes = (uint32_t)L.rows(tl.mt) * kRowBytes;
-                const uint8_t* a0 = p.A0 + L.block(tl.e, tl.mt, 0);
-                const uint8_t* a1 = DUAL ? p.A1 + L.block(tl.e, tl.mt, 0) : nullptr;
+                const Tile tl = decode_tile(t, MU, p, s_prefix, s_bounds, s_pad);
+                const uint8_t* a[2];
+                uint32_t nb[2];
+                for (int i = 0; i < 2; ++i) {
+                    int rows, mt;
+                    source(tl, i, a[i], rows, mt);
+                    nb[i] = (uint32_t)rows * kRowBytes;
+                }
                 for (int kt = 0; kt < KT; ++kt) {
                     prefetch_one();
                     ok = wait_bar(&raw_empty[rs], rph ^ 1, abort_flag, status, STAT_PTR(0));
                     if (!ok) break;
-                    ptx::mbar_arrive_expect_tx(&raw_full[rs], raw_bytes * C::NMAT);
-                    ptx::bulk_g2s(sRaw + (rs * C::NMAT) * kRawBytes, a0 + (size_t)kt * raw_bytes, raw_bytes,
-                                  &raw_full[rs]);
-                    if (DUAL)
-                        ptx::bulk_g2s(sRaw + (rs * C::NMAT + 1) * kRawBytes, a1 + (size_t)kt * raw_bytes, raw_bytes,
-                                      &raw_full[rs]);
+                    ptx::mbar_arrive_expect_tx(&raw_full[rs], nb[0] + nb[1]);
+                    for (int i = 0; i < 2; ++i)
+                        if (nb[i])
+                            ptx::bulk_g2s(sRaw + (rs * 2 + i) * kRawBytes, a[i] + (size_t)kt * nb[i], nb[i],
+                                          &raw_full[rs]);
                     used |= 1u << rs;
                     par = (par & ~(1u << rs)) | (rph << rs);
-                    if (++rs == C::RS) { rs = 0; rph ^= 1; }
+                    if (++rs == kRS) { rs = 0; rph ^= 1; }
                 }
             }
             // let every copy issued land before the CTA can exit (bounded)
             volatile int never = 0;
-            for (int s = 0; s < C::RS; ++s)
+            for (int s = 0; s < kRS; ++s)
                 if (used >> s & 1) wait_bar(&raw_full[s], (par >> s) & 1, &never, status);
             STAT_FLUSH(0);
         }
@@ -308,7 +327,7 @@ grouped_gemm_kernel(const GemmParams p) {
             bool ok = true;
             const size_t plane = (size_t)p.b_rows * 128u;
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-                const Tile tl = decode_tile(t, MT, p, s_prefix, s_bounds, s_pad);
+                const Tile tl = decode_tile(t, MU, p, s_prefix, s_bounds, s_pad);
                 const uint32_t bytes = (uint32_t)((tl.n + 15) & ~15) * 128u;
                 const uint8_t* src = p.B + (size_t)tl.p0pad * 128u;
                 for (int kt = 0; kt < KT; ++kt) {
@@ -318,58 +337,54 @@ grouped_gemm_kernel(const GemmParams p) {
                     ptx::bulk_g2s(sB + bs * kBTileBytes, src + kt * plane, bytes, &b_full[bs]);
                     used |= 1u << bs;
                     par = (par & ~(1u << bs)) | (bph << bs);
-                    if (++bs == C::MB) { bs = 0; bph ^= 1; }
+                    if (++bs == kMB) { bs = 0; bph ^= 1; }
                 }
             }
             volatile int never = 0;
-            for (int s = 0; s < C::MB; ++s)
+            for (int s = 0; s < kMB; ++s)
                 if (used >> s & 1) wait_bar(&b_full[s], (par >> s) & 1, &never, status);
             STAT_FLUSH(1);
         }
     } else if (warp == kWarpMma) {
         // ----------------------------------------------------------------- MMA
+        // A from tensor memory, B from shared memory; the two accumulators'
+        // instructions interleave so neither chain waits on itself.
         if (lane == 0) {
             STAT_DECL
             int as = 0, bs = 0;
-            uint32_t aph = 0, bph = 0;
-            uint32_t use[2] = {0, 0};
-            int it = 0;
+            uint32_t aph = 0, bph = 0, use = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
-                const Tile tl = decode_tile(t, MT, p, s_prefix, s_bounds, s_pad);
+            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+                const Tile tl = decode_tile(t, MU, p, s_prefix, s_bounds, s_pad);
                 const int n16 = (tl.n + 15) & ~15;
-                const int buf = DUAL ? 0 : (it & 1);
-                ok = wait_bar(&tmem_empty[buf], (use[buf] & 1) ^ 1, abort_flag, status, STAT_PTR(2));
+                const bool has1 = DUAL || (2 * tl.mt + 1 < MT);
+                ok = wait_bar(tmem_empty, (use & 1) ^ 1, abort_flag, status, STAT_PTR(2));
                 if (!ok) break;
                 ptx::tc_fence_after();
-                const uint32_t d0 = tmem_base + (DUAL ? 0u : (uint32_t)buf * 256u);
-                const uint32_t d1 = tmem_base + 256u;
+                const uint32_t d0 = tmem_base, d1 = tmem_base + kAccCols;
                 const uint32_t idesc = ptx::idesc_f16(p.bf16, n16, 128);
                 for (int kt = 0; kt < KT; ++kt) {
                     ok = wait_bar(&a_full[as], aph, abort_flag, status, STAT_PTR(0)) &&
                          wait_bar(&b_full[bs], bph, abort_flag, status, STAT_PTR(1));
                     if (!ok) break;
                     ptx::tc_fence_after();
-                    const uint32_t a0 = ptx::smem_u32(sA + (as * C::NMAT) * kATileBytes);
-                    const uint32_t a1 = a0 + kATileBytes;
+                    const uint32_t a0 = tmem_base + kACol0 + (uint32_t)as * 64u;
                     const uint32_t b = ptx::smem_u32(sB + bs * kBTileBytes);
 #pragma unroll
                     for (int kk = 0; kk < kTileK / 16; ++kk) {
                         const uint32_t acc = (kt | kk) != 0;
-                        ptx::mma_f16_ss(d0, ptx::desc_k_sw128(a0 + kk * 32), ptx::desc_k_sw128(b + kk * 32), idesc,
-                                        acc);
-                        if (DUAL)
-                            ptx::mma_f16_ss(d1, ptx::desc_k_sw128(a1 + kk * 32), ptx::desc_k_sw128(b + kk * 32),
-                                            idesc, acc);
+                        const uint64_t bd = ptx::desc_k_sw128(b + kk * 32);
+                        ptx::mma_f16_ts(d0, a0 + kk * 8, bd, idesc, acc);
+                        if (has1) ptx::mma_f16_ts(d1, a0 + 32 + kk * 8, bd, idesc, acc);
                     }
                     ptx::mma_commit(&a_empty[as]);
                     ptx::mma_commit(&b_empty[bs]);
-                    if (++as == C::MA) { as = 0; aph ^= 1; }
-                    if (++bs == C::MB) { bs = 0; bph ^= 1; }
+                    if (++as == kMA) { as = 0; aph ^= 1; }
+                    if (++bs == kMB) { bs = 0; bph ^= 1; }
                 }
                 if (!ok) break;
-                ptx::mma_commit(&tmem_full[buf]);
-                use[buf] += 1;
+                ptx::mma_commit(tmem_full);
+                use += 1;
             }
             STAT_FLUSH(2);
         }
@@ -378,27 +393,24 @@ grouped_gemm_kernel(const GemmParams p) {
         // ------------------------------------------------------------ epilogue
         const int ew = warp - kEpiWarp0;
         STAT_DECL
-        uint32_t use[2] = {0, 0};
-        int it = 0;
-        for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
-            const Tile tl = decode_tile(t, MT, p, s_prefix, s_bounds, s_pad);
-            const int buf = DUAL ? 0 : (it & 1);
-            if (!warp_wait(&tmem_full[buf], use[buf] & 1, abort_flag, status, STAT_PTR(0))) break;
-            use[buf] += 1;
+        uint32_t use = 0;
+        for (int t = blockIdx.x; t < total; t += gridDim.x) {
+            const Tile tl = decode_tile(t, MU, p, s_prefix, s_bounds, s_pad);
+            if (!warp_wait(tmem_full, use & 1, abort_flag, status, STAT_PTR(0))) break;
+            use += 1;
             ptx::tc_fence_after();
-            const int m = tl.mt * kTileM + 32 * ew + lane;
-            const bool m_ok = m < L.n_out;
-            const uint32_t tbase = tmem_base + ((uint32_t)(32 * ew) << 16) + (DUAL ? 0u : (uint32_t)buf * 256u);
-            for (int c0 = 0; c0 < tl.n; c0 += 32) {
-                uint32_t v[32];
-                ptx::tmem_ld_32x32b_x32(tbase + c0, v);
-                if (DUAL) {
-                    uint32_t u[32];
-                    ptx::tmem_ld_32x32b_x32(tbase + 256 + c0, u);
+            const uint32_t lanes = (uint32_t)(32 * ew) << 16;
+            if (DUAL) {
+                const int m = tl.mt * kTileM + 32 * ew + lane;
+                const bool m_ok = m < L.n_out;
+                // h goes to the tile-major swizzled buffer the down GEMM streams
+                uint8_t* hplane = p.h + (size_t)(m >> 6) * p.h_rows * 128u + ((m & 7) << 1);
+                const int mchunk = (m & 63) >> 3;
+                for (int c0 = 0; c0 < tl.n; c0 += 32) {
+                    uint32_t v[32], u[32];
+                    ptx::tmem_ld_32x32b_x32(tmem_base + lanes + c0, v);
+                    ptx::tmem_ld_32x32b_x32(tmem_base + lanes + kAccCols + c0, u);
                     ptx::tmem_ld_wait();
-                    // h goes to the tile-major swizzled buffer the down GEMM streams
-                    uint8_t* hplane = p.h + (size_t)(m >> 6) * p.h_rows * 128u + ((m & 7) << 1);
-                    const int mchunk = (m & 63) >> 3;
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
                         if (c0 + i < tl.n && m_ok) {
@@ -409,50 +421,71 @@ grouped_gemm_kernel(const GemmParams p) {
                                 __float2bfloat16_rn(hv);
                         }
                     }
-                } else {
-                    ptx::tmem_ld_wait();
-                    const int col = c0 + lane;
-                    int orow = -1;
-                    if (col < tl.n) orow = p.dst_rows ? __ldg(p.dst_rows + tl.p0 + col) : tl.p0 + col;
+                }
+            } else {
+                for (int i = 0; i < 2; ++i) {
+                    const int mt = 2 * tl.mt + i;
+                    if (mt >= MT) break;
+                    const int m = mt * kTileM + 32 * ew + lane;
+                    const bool m_ok = m < L.n_out;
+                    for (int c0 = 0; c0 < tl.n; c0 += 32) {
+                        uint32_t v[32];
+                        ptx::tmem_ld_32x32b_x32(tmem_base + lanes + (uint32_t)i * kAccCols + c0, v);
+                        ptx::tmem_ld_wait();
+                        const int col = c0 + lane;
+                        int orow = -1;
+                        if (col < tl.n) orow = p.dst_rows ? __ldg(p.dst_rows + tl.p0 + col) : tl.p0 + col;
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int r = __shfl_sync(0xffffffffu, orow, i);
-                        if (r >= 0 && m_ok) p.out[(int64_t)r * p.out_ld + m] = __uint_as_float(v[i]);
+                        for (int j = 0; j < 32; ++j) {
+                            const int r = __shfl_sync(0xffffffffu, orow, j);
+                            if (r >= 0 && m_ok) p.out[(int64_t)r * p.out_ld + m] = __uint_as_float(v[j]);
+                        }
                     }
                 }
             }
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&tmem_empty[buf]);
+            if (lane == 0) ptx::mbar_arrive(tmem_empty);
         }
         if (lane == 0) STAT_FLUSH(3);
     } else if (warp >= kDeqWarp0) {
         // ------------------------------------------------------- dequantisation
-        const int d = tid - kDeqWarp0 * 32;  // 0..255
-        const int r = d >> 1, hlf = d & 1;
-        const int first = (d >> 2) & 1;      // alternate read order: conflict-free 16-byte loads
+        // Warp w covers rows 32*(w%4) .. +31 (its tensor-memory lane quarter)
+        // and the 32-column half (w-8)/4 of each k-step: exact fp32 q*d, one
+        // rounding to the operand type, written straight into tensor memory.
+        const int wq = warp & 3, hk = (warp - kDeqWarp0) >> 2;
+        const int r = 32 * wq + lane;
+        const int first = (lane >> 2) & 1;  // alternate read order: conflict-free 16-byte loads
+        const uint32_t lanes = (uint32_t)(32 * wq) << 16;
         STAT_DECL
         int rs = 0, as = 0;
         uint32_t rph = 0, aph = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-            const Tile tl = decode_tile(t, MT, p, s_prefix, s_bounds, s_pad);
-            const int rows = L.rows(tl.mt);
+            const Tile tl = decode_tile(t, MU, p, s_prefix, s_bounds, s_pad);
+            int rows[2];
+            for (int i = 0; i < 2; ++i) {
+                const uint8_t* dummy;
+                int mt;
+                source(tl, i, dummy, rows[i], mt);
+            }
             for (int kt = 0; kt < KT; ++kt) {
                 ok = warp_wait(&raw_full[rs], rph, abort_flag, status, STAT_PTR(0)) &&
                      warp_wait(&a_empty[as], aph ^ 1, abort_flag, status, STAT_PTR(1));
                 if (!ok) break;
+                ptx::tc_fence_after();
 #pragma unroll
-                for (int mat = 0; mat < C::NMAT; ++mat) {
-                    const uint8_t* raw = sRaw + (rs * C::NMAT + mat) * kRawBytes;
-                    uint8_t* dstA = sA + (as * C::NMAT + mat) * kATileBytes + r * 128;
+                for (int mat = 0; mat < 2; ++mat) {
+                    const int nr = rows[mat];
+                    if (nr == 0) continue;
+                    const uint8_t* raw = sRaw + (rs * 2 + mat) * kRawBytes;
                     uint32_t pk[16];
-                    if (r < rows) {
-                        const uint8_t* qrow = raw + r * kTileK + hlf * 32;
+                    if (r < nr) {
+                        const uint8_t* qrow = raw + (size_t)hk * nr * 32 + r * 32;
                         const uint4 qa = *(const uint4*)(qrow + first * 16);
                         const uint4 qb = *(const uint4*)(qrow + (first ^ 1) * 16);
                         const uint4 q0 = first ? qb : qa, q1 = first ? qa : qb;
-                        const float dsc = __half2float(*(const __half*)(raw + rows * kTileK + r * 4 + hlf * 2));
+                        const float dsc = __half2float(*(const __half*)(raw + (size_t)nr * kTileK + r * 4 + hk * 2));
                         const float nd = -32896.0f * dsc;
                         const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
 #pragma unroll
@@ -468,20 +501,17 @@ grouped_gemm_kernel(const GemmParams p) {
 #pragma unroll
                         for (int j = 0; j < 16; ++j) pk[j] = 0u;
                     }
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int phys = (hlf * 4 + i) ^ (r & 7);
-                        *(uint4*)(dstA + phys * 16) = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-                    }
+                    ptx::tmem_st_32x32b_x16(tmem_base + lanes + kACol0 + (uint32_t)as * 64u + mat * 32 + hk * 16, pk);
                 }
-                ptx::fence_proxy_async_smem();
+                ptx::tmem_st_wait();
+                ptx::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) {
                     ptx::mbar_arrive(&raw_empty[rs]);
                     ptx::mbar_arrive(&a_full[as]);
                 }
-                if (++rs == C::RS) { rs = 0; rph ^= 1; }
-                if (++as == C::MA) { as = 0; aph ^= 1; }
+                if (++rs == kRS) { rs = 0; rph ^= 1; }
+                if (++as == kMA) { as = 0; aph ^= 1; }
             }
         }
         if (lane == 0) STAT_FLUSH(4);
@@ -568,14 +598,15 @@ static moe_status run_gemm(const GemmParams& p, int64_t max_coltiles, cudaStream
     cudaGetDevice(&dev);
     if (attr_dev != dev) {
         if (cudaFuncSetAttribute(grouped_gemm_kernel<DUAL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)Cfg<DUAL>::smem_bytes) != cudaSuccess)
+                                 (int)Cfg::smem_bytes) != cudaSuccess)
             return MOE_ERR_CUDA;
         attr_dev = dev;
     }
-    int64_t tiles = max_coltiles * p.L.mt_count;
+    const int64_t units = DUAL ? p.L.mt_count : (p.L.mt_count + 1) / 2;
+    int64_t tiles = max_coltiles * units;
     if (tiles <= 0) return MOE_OK;
     int grid = (int)(tiles < sm_count() ? tiles : sm_count());
-    grouped_gemm_kernel<DUAL><<<grid, kGemmThreads, Cfg<DUAL>::smem_bytes, stream>>>(p);
+    grouped_gemm_kernel<DUAL><<<grid, kGemmThreads, Cfg::smem_bytes, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

@@ -30,6 +30,11 @@ struct GemvArgs {
     int max_distinct;    // min(n_tokens*k, n_experts): routed items = max_distinct * routed.items
     int pdl_secondary;   // launched as a programmatic dependent: wait before reading activations
     int* hdr;
+    // launch plan (filled by launch_gemv)
+    int nt_cap;          // tokens per pass
+    int nbuf;            // 2: double-buffered whole weight slices; 1: windowed
+    uint32_t buf_bytes, x_bytes, red_bytes, bm_words;
+    int max_stages;
 };
 
 moe_status launch_gemv(const GemvArgs& a, cudaStream_t stream);

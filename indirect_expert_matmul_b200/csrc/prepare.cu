@@ -1,7 +1,7 @@
 // One-time repack of Q8_0 expert weights into the tile-major form streamed by
 // the GEMM and mat-vec kernels (layout in common.cuh).  Each thread produces
-// one (expert, row, 64-column tile) piece: 64 bytes u = q + 128 and the two
-// fp16 scales.  Padding rows / columns get u = 128 (q = 0) and d = 0.
+// one (expert, row, 64-column tile) piece: two 32-byte halves of u = q + 128
+// and the two fp16 scales.  Padding rows / columns get u = 128 (q = 0), d = 0.
 #include "common.cuh"
 
 namespace moe {
@@ -18,10 +18,10 @@ __global__ void prepare_kernel(const uint8_t* __restrict__ src, int E, WLayout L
         const int mt = row / kTileM, r = row % kTileM;
         const int rows = L.rows(mt);
         uint8_t* blk = dst + L.block(e, mt, kt);
-        uint8_t* q_out = blk + (size_t)r * kTileK;
         uint16_t* d_out = (uint16_t*)(blk + (size_t)rows * kTileK + (size_t)r * 4);
         for (int h = 0; h < 2; ++h) {
             const int b = kt * 2 + h;  // Q8_0 block index along the row
+            uint8_t* q_out = blk + (size_t)h * rows * 32 + (size_t)r * 32;
             uint16_t d = 0;
             uint32_t words[8];
             if (row < L.n_out && b < nb) {
@@ -35,7 +35,7 @@ __global__ void prepare_kernel(const uint8_t* __restrict__ src, int E, WLayout L
             } else {
                 for (int w = 0; w < 8; ++w) words[w] = 0x80808080u;
             }
-            uint4* o = (uint4*)(q_out + h * 32);
+            uint4* o = (uint4*)q_out;
             o[0] = make_uint4(words[0], words[1], words[2], words[3]);
             o[1] = make_uint4(words[4], words[5], words[6], words[7]);
             d_out[h] = d;
