@@ -159,17 +159,23 @@ def row_ids(ids, n_experts, mode="broadcast", ws=None):
 
 # --------------------------------------------------------------- operators
 def mul_mat_id(W, n_experts, n_out, n_in, x, ids, mode="broadcast", ws=None, out=None):
-    """dst float32 [T][k][n_out] = W[ids[t][s]] . x[t or (t, s)]."""
+    """dst float32 [T][k][n_out] = W[ids[t][s]] . x[t or (t, s)].
+
+    Without `ws` the call makes its own workspace, synchronises and raises
+    MoeError on a device-side error; with `ws` the caller reads get_status."""
     _cuda(W, "W", torch.uint8)
     _cuda(x, "x")
     _cuda(ids, "ids", torch.int32)
     T, k = ids.shape
-    if ws is None:
+    own_ws = ws is None
+    if own_ws:
         ws = workspace(T, k, n_experts, n_in, x_dtype=x.dtype, device=x.device)
     if out is None:
         out = torch.empty((T, k, n_out), dtype=torch.float32, device=x.device)
     _chk(_L().moe_mul_mat_id(_ptr(W), n_experts, n_out, n_in, _ptr(x), _XTYPE[x.dtype], _ptr(ids), T, k,
                              _MODE[mode], _ptr(out), _ptr(ws), _stream(x.device)), "moe_mul_mat_id")
+    if own_ws:
+        _chk(get_status(ws), "moe_mul_mat_id (device status)")
     return out
 
 
@@ -186,7 +192,8 @@ def ffn(Wg, Wu, Wd, n_experts, n_embd, n_ff, x, ids, shared=None, ws=None, out=N
     n_ff_sh = 0
     if shared is not None:
         Sg, Su, Sd, n_ff_sh = shared
-    if ws is None:
+    own_ws = ws is None
+    if own_ws:
         ws = workspace(T, k, n_experts, n_embd, n_ff, n_ff_sh, x.dtype, device=x.device)
     if out is None:
         out = torch.empty((T, k, n_embd), dtype=torch.float32, device=x.device)
@@ -195,6 +202,8 @@ def ffn(Wg, Wu, Wd, n_experts, n_embd, n_ff, x, ids, shared=None, ws=None, out=N
     _chk(_L().moe_ffn(_ptr(Wg), _ptr(Wu), _ptr(Wd), n_experts, n_embd, n_ff, _ptr(Sg), _ptr(Su), _ptr(Sd), n_ff_sh,
                       _ptr(x), _XTYPE[x.dtype], _ptr(ids), T, k, _ptr(out), _ptr(out_shared), _ptr(ws),
                       _stream(x.device)), "moe_ffn")
+    if own_ws:
+        _chk(get_status(ws), "moe_ffn (device status)")
     return out, out_shared
 
 

@@ -151,6 +151,8 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
         if (*abort_flag) return false;
         if (clock64() - t0 > kWaitLimitCycles) {
             *abort_flag = 1;
+            const int site = (1 << 30) | ((int)(threadIdx.x >> 5) << 20) | (int)(ptx::smem_u32(bar) & 0xfffffu);
+            atomicCAS(status + (kHdrWaitSite - kHdrStatus), 0, site);
             set_status(status, MOE_ERR_TIMEOUT);
             return false;
         }
