@@ -170,6 +170,39 @@ MOE_API moe_status moe_ffn(const void *Wg, const void *Wu, const void *Wd, int n
                    const int32_t *ids, int64_t n_tokens, int k, float *dst, float *dst_shared, void *workspace,
                    moe_stream stream);
 
+/*
+ * Decode-size moe_ffn that allocates nothing and takes no workspace.  The
+ * method's description has no counterpart to this entry point: it serves
+ * callers that cannot hand over scratch memory, such as a graph executor that
+ * plans every buffer per tensor before running and gives each operation only
+ * its inputs and outputs, with no allocator at hand while the graph runs.
+ *
+ * Computes what moe_ffn computes, on the mat-vec path, for
+ *   n_tokens * k <= 64, n_ff <= 2048, n_ff_shared <= 2048
+ * (MOE_ERR_RANGE beyond these, checked on the host before any CUDA call).
+ * Scratch is one static device array in the library (256-byte status header +
+ * 256 KB routed hidden activations + 256 KB shared hidden activations, about
+ * 512 KB per device); no call allocates or frees memory.
+ *   - Only the status header must start at zero: each call clears it with an
+ *     asynchronous memset on `stream` before its kernels.  The hidden
+ *     activations need no initial value (the gate/up kernel writes every
+ *     element the down kernel reads).
+ *   - status_out (device int, may be NULL): receives the call's device status
+ *     (MOE_OK, MOE_ERR_BAD_ID, MOE_ERR_TIMEOUT) by an asynchronous
+ *     device-to-device copy at the end of the call; with NULL, device-side
+ *     errors are not observable.
+ *   - All calls on one device share the one scratch array: calls that may
+ *     overlap in time (other streams, other host threads) race on it and give
+ *     undefined results.  Order them on one stream or serialise them.
+ *   - The first call on each device looks up the array's address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     outside any stream capture.
+ */
+MOE_API moe_status moe_ffn_decode_noalloc(const void *Wg, const void *Wu, const void *Wd, int n_experts, int n_embd,
+                                          int n_ff, const void *Sg, const void *Su, const void *Sd, int n_ff_shared,
+                                          const void *x, moe_dtype x_type, const int32_t *ids, int64_t n_tokens, int k,
+                                          float *dst, float *dst_shared, int *status_out, moe_stream stream);
+
 /* ------------------------------------------------------------------ tuning */
 
 /* Token count at or below which the mat-vec path is used (default 8); the

@@ -24,7 +24,7 @@ BF16, F16, F32 = 0, 1, 2
 ABI_SYMBOLS = (
     "moe_status_string", "moe_workspace_size", "moe_workspace_init", "moe_get_status",
     "moe_weights_prepared_size", "moe_weights_prepare", "moe_row_ids", "moe_mul_mat_id", "moe_ffn",
-    "moe_set_gemv_threshold", "moe_get_gemv_threshold", "moe_set_path", "moe_profile_enable", "moe_profile_read",
+    "moe_ffn_decode_noalloc", "moe_set_gemv_threshold", "moe_get_gemv_threshold", "moe_set_path", "moe_profile_enable", "moe_profile_read",
 )
 
 _lib = None
@@ -52,6 +52,8 @@ def _L() -> ctypes.CDLL:
     L.moe_mul_mat_id.argtypes = [_vp, _i32, _i32, _i32, _vp, _i32, _vp, _i64, _i32, _i32, _vp, _vp, _vp]
     L.moe_ffn.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _i32, _vp, _i64, _i32,
                           _vp, _vp, _vp, _vp]
+    L.moe_ffn_decode_noalloc.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _i32, _vp, _i64,
+                                         _i32, _vp, _vp, _vp, _vp]
     L.moe_set_gemv_threshold.argtypes = [_i32]
     L.moe_set_gemv_threshold.restype = None
     L.moe_get_gemv_threshold.argtypes = []
@@ -204,6 +206,32 @@ def ffn(Wg, Wu, Wd, n_experts, n_embd, n_ff, x, ids, shared=None, ws=None, out=N
                       _stream(x.device)), "moe_ffn")
     if own_ws:
         _chk(get_status(ws), "moe_ffn (device status)")
+    return out, out_shared
+
+
+def ffn_decode_noalloc(Wg, Wu, Wd, n_experts, n_embd, n_ff, x, ids, shared=None, out=None, out_shared=None,
+                       status=None):
+    """moe_ffn for decode sizes (n_tokens*k <= 64, n_ff and n_ff_shared <= 2048)
+    through the entry point that takes no workspace.  `status`: optional int32
+    CUDA tensor of one element that receives the device status."""
+    for name, t in (("Wg", Wg), ("Wu", Wu), ("Wd", Wd)):
+        _cuda(t, name, torch.uint8)
+    _cuda(x, "x")
+    _cuda(ids, "ids", torch.int32)
+    if status is not None:
+        _cuda(status, "status", torch.int32)
+    T, k = ids.shape
+    Sg = Su = Sd = None
+    n_ff_sh = 0
+    if shared is not None:
+        Sg, Su, Sd, n_ff_sh = shared
+    if out is None:
+        out = torch.empty((T, k, n_embd), dtype=torch.float32, device=x.device)
+    if shared is not None and out_shared is None:
+        out_shared = torch.empty((T, n_embd), dtype=torch.float32, device=x.device)
+    _chk(_L().moe_ffn_decode_noalloc(_ptr(Wg), _ptr(Wu), _ptr(Wd), n_experts, n_embd, n_ff, _ptr(Sg), _ptr(Su),
+                                     _ptr(Sd), n_ff_sh, _ptr(x), _XTYPE[x.dtype], _ptr(ids), T, k, _ptr(out),
+                                     _ptr(out_shared), _ptr(status), _stream(x.device)), "moe_ffn_decode_noalloc")
     return out, out_shared
 
 
