@@ -206,11 +206,13 @@ MOE_API moe_status moe_ffn_decode_noalloc(const void *Wg, const void *Wu, const 
 /* ------------------------------------------------------------------ tuning */
 
 /* Token count at or below which the mat-vec path is used (default 8); the
- * analogue of ggml's mmq_id threshold ([PR283] section 2.1, ggml-cuda.cu#L2944). */
+ * analogue of ggml's mmq_id threshold ([PR283] section 2.1, ggml-cuda.cu#L2944).
+ * The mat-vec path takes n_tokens*k <= 1024; larger calls use the GEMM. */
 MOE_API void moe_set_gemv_threshold(int n_tokens);
 MOE_API int moe_get_gemv_threshold(void);
 
-/* Force a path for testing: 0 = by threshold, 1 = mat-vec, 2 = grouped GEMM. */
+/* Force a path for testing: 0 = by threshold, 1 = mat-vec (when n_tokens*k <=
+ * 1024, else the GEMM), 2 = grouped GEMM. */
 MOE_API void moe_set_path(int path);
 
 

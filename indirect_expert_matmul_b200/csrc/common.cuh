@@ -59,9 +59,14 @@ struct WLayout {
 inline int64_t tiled_rows(int64_t S, int n_groups) {
     return S + 8 * (S < n_groups ? S : n_groups) + 32;
 }
+// Split-K of the mat-vec kernel (decode FFN gate/up): at most kGvMaxChunks
+// K-chunks per (expert, row tile), only for n_tokens*k <= kGvSplitSlots; the
+// chunks' fp32 partial sums live in the workspace.
+constexpr int kGvSplitSlots = 64;
+constexpr int kGvMaxChunks = 8;
 struct WsLayout {
     int64_t S, rows_pad, rows_pad_sh;
-    size_t hdr, src1, dst, bounds, active, tiles, pad, h, h_sh, xt, xt_sh, total;
+    size_t hdr, src1, dst, bounds, active, tiles, pad, h, h_sh, xt, xt_sh, gv_part, gv_part_sh, total;
     static size_t up(size_t v) { return (v + 255) / 256 * 256; }
     WsLayout(int64_t n_tokens, int k, int n_experts, int n_in, int n_hidden, int n_hidden_sh, int x_type) {
         (void)x_type;
@@ -83,6 +88,9 @@ struct WsLayout {
         h_sh = o; o += up(hs_gemv > hs_gemm ? hs_gemv : hs_gemm);
         xt = o; o += up((size_t)rows_pad * kin * 128);
         xt_sh = o; o += n_hidden_sh > 0 ? up((size_t)rows_pad_sh * kin * 128) : 0;
+        const bool split = S <= kGvSplitSlots;
+        gv_part = o; o += split ? up((size_t)kGvMaxChunks * S * ((n_hidden + 15) / 16 * 16) * 2 * 4) : 0;
+        gv_part_sh = o; o += split ? up((size_t)kGvMaxChunks * n_tokens * ((n_hidden_sh + 15) / 16 * 16) * 2 * 4) : 0;
         total = o;
     }
 };

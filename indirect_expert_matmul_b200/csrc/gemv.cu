@@ -3,48 +3,57 @@
 // llama.cpp PR #29184 ("CUDA: fuse shared experts into MMVQ", release b11370)
 // restated for this library.
 //
-// Work item = (j-th distinct routed expert, slice of 16/32/64 output rows), or
-// (shared expert, slice).  A CTA finds its expert from ids itself (a bitmap of
-// used experts, the j-th set bit), so the decode path needs no row-id launch.
-// It then issues 1-D bulk copies for its whole weight slice (all k-steps of one
-// activation window) into shared memory at once - the largest number of bytes
-// in flight per SM - and stages the activations of its tokens while they
-// land.  Dequantisation is exact (fp32 q*d); dot products accumulate in fp32,
-// partial sums are combined by a fixed shuffle tree and a fixed-order sum, so
-// the result does not depend on timing.
+// Decode is bound by the weight stream, so the kernel is built around moving
+// the repacked weights in large contiguous pieces:
+//  - a work item is (distinct routed expert, 128-row tile, K-chunk) or
+//    (shared expert, 128-row tile, K-chunk); every k-step block of one
+//    (expert, row tile) is contiguous in the repacked layout, so a stage of
+//    up to two k-steps of one matrix is a single bulk copy (17 KB);
+//  - one producer warp streams the stages of the CTA's items through a ring
+//    of shared-memory stages, ahead of the consumers and across items;
+//  - 256 consumer threads dequantise (exact fp32 q*d) and take the dot
+//    products with up to 8 tokens at a time: thread = (row, 32-column half);
+//  - when there are fewer (expert, row tile) groups than SMs (a single decode
+//    token), K is split into chunks; each chunk writes fp32 partial sums and
+//    the CTA that finishes a group last adds the chunks in chunk order and
+//    applies the epilogue.  Every sum has a fixed order, so results do not
+//    depend on timing.
+// A CTA finds the distinct experts and their slots from ids itself (bitmap +
+// a per-CTA slot table), so the decode path needs no row-id launch.
 //
 // Modes: single matrix (mul_mat_id rows, or the down projection writing
 // dst[t][s]), or dual gate/up with a SwiGLU epilogue writing bf16 h[t][s].
-// The down launch is a programmatic dependent of the gate/up launch: its CTAs
-// start while gate/up runs, issue their weight copies, and only then wait for
-// gate/up to finish before reading h.
+// The down launch is a programmatic dependent of the gate/up launch: its
+// producer streams weights while gate/up finishes; its consumers wait for
+// gate/up before reading h.
 #include "common.cuh"
 #include "gemv_args.cuh"
 #include "ptx.cuh"
 
 namespace moe {
 
-constexpr int kGvThreads = 256;
-constexpr int kGvNT = 8;                   // tokens per pass, at most
-constexpr int kGvWeightBudget = 72 * 1024; // weight bytes of one work item (one buffer)
+constexpr int kGvConsumers = 256;
+constexpr int kGvThreads = 32 + kGvConsumers;  // warp 0: producer
+constexpr uint32_t kGvBlock = kTileM * kRowBytes;  // 8704: one k-step of a full row tile
+constexpr uint32_t kGvSmemBudget = 200 * 1024;
 constexpr long long kGvWaitLimit = 1ll << 32;
 
 struct GvLay {
-    uint32_t buf0, buf1, x, red, bm, wp, bars, misc, total;
+    uint32_t ring, x, red, bm, wp, tab, bars, misc, total;
 };
 
 __host__ __device__ inline GvLay gv_lay(const GemvArgs& a) {
     GvLay m;
     uint32_t o = 0;
-    m.buf0 = o; o += a.buf_bytes;
-    m.buf1 = o; o += a.nbuf == 2 ? a.buf_bytes : 0u;
+    m.ring = o; o += (uint32_t)a.ns * a.stage_bytes;
     m.x = o; o += a.x_bytes;
     m.red = o; o += a.red_bytes;
     m.bm = o; o += a.bm_words * 4u;
     m.wp = o; o += (a.bm_words + 1u) * 4u;
+    m.tab = o; o += a.tab_words * 4u;
     o = (o + 15u) & ~15u;
-    m.bars = o; o += 2u * a.max_stages * 8u;
-    m.misc = o; o += 64u * 4u;
+    m.bars = o; o += 2u * (uint32_t)a.ns * 8u;
+    m.misc = o; o += 16u * 4u;
     m.total = o;
     return m;
 }
@@ -53,11 +62,15 @@ __device__ __forceinline__ float ld_x16(uint32_t bits16, int x_type) {
     return x_type == MOE_BF16 ? __uint_as_float(bits16 << 16) : __half2float(__ushort_as_half((unsigned short)bits16));
 }
 
-__device__ __forceinline__ bool gv_wait(uint64_t* bar, uint32_t parity, int* status) {
+// Bounded wait by one thread: false on expiry (status set, abort raised) or
+// when another thread has raised abort.
+__device__ __forceinline__ bool gv_wait(uint64_t* bar, uint32_t parity, int* status, volatile int* abort_flag) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (!ptx::mbar_try_wait_sleep(bar, parity, 20000)) {
+        if (*abort_flag) return false;
         if (clock64() - t0 > kGvWaitLimit) {
+            *abort_flag = 1;
             set_status(status, MOE_ERR_TIMEOUT);
             return false;
         }
@@ -65,14 +78,38 @@ __device__ __forceinline__ bool gv_wait(uint64_t* bar, uint32_t parity, int* sta
     return true;
 }
 
-// One work item: a slice of `R` output rows of one expert's matrix (or two).
+// Named barrier 1 over the consumer warps; consumers_and also returns the AND
+// of every consumer's flag, so exits decided from it are uniform.
+__device__ __forceinline__ void consumers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kGvConsumers) : "memory"); }
+__device__ __forceinline__ bool consumers_and(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.and.pred p, 1, %2, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v), "n"(kGvConsumers)
+        : "memory");
+    return r != 0;
+}
+
+// One work item.
 struct GvItem {
     const GemvSide* sd;
-    int shared, e, mt, r0, rows_mt;
+    int shared;   // 1: shared expert
+    int e;        // expert of the weights
+    int mt;       // 128-row tile
+    int c;        // K-chunk
+    int kt0, nk;  // first k-step and k-steps of the chunk
+    int rows;     // rows of the tile
+    int nsl;      // slots (routed) or tokens (shared)
+    int sbase;    // first entry of the expert's slots in the slot list
+    int group;    // split-K counter index
 };
 
 template <int DUAL, int XB>
-__global__ void __launch_bounds__(kGvThreads)
+__global__ void __launch_bounds__(kGvThreads, 1)
 gemv_kernel(const GemvArgs a) {
     extern __shared__ __align__(128) uint8_t sm[];
     constexpr int NMAT = DUAL + 1;
@@ -82,22 +119,30 @@ gemv_kernel(const GemvArgs a) {
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const GvLay lay = gv_lay(a);
-    uint8_t* sbuf[2] = {sm + lay.buf0, sm + lay.buf1};
+    uint8_t* ring = sm + lay.ring;
     uint8_t* sx = sm + lay.x;
     float* red = (float*)(sm + lay.red);
     uint32_t* bm = (uint32_t*)(sm + lay.bm);
     int* wp = (int*)(sm + lay.wp);
-    uint64_t* bars = (uint64_t*)(sm + lay.bars);
-    int* misc = (int*)(sm + lay.misc);  // [0..7] reduce scratch, [16..23] rows of the token group
-    int* rows_sh = misc + 16;
+    int* tab = (int*)(sm + lay.tab);
+    uint64_t* full = (uint64_t*)(sm + lay.bars);
+    uint64_t* empty = full + a.ns;
+    int* misc = (int*)(sm + lay.misc);
+    volatile int* abort_flag = misc;   // misc[0]
+    int* last_flag = misc + 1;
     const int S = a.n_tokens * a.k;
     const int nwords = (int)a.bm_words;
 
-    // ---- the distinct routed experts, once per CTA: bitmap + per-word prefix
+    // ---- the distinct routed experts: bitmap + per-word prefix of popcounts
     for (int w = tid; w < nwords; w += kGvThreads) bm[w] = 0u;
-    if (tid == 0)
-        for (int s = 0; s < 2 * a.max_stages; ++s) ptx::mbar_init(&bars[s], 1);
-    ptx::fence_mbar_init();
+    if (tid == 0) {
+        for (int s = 0; s < a.ns; ++s) {
+            ptx::mbar_init(&full[s], 1);
+            ptx::mbar_init(&empty[s], kGvConsumers / 32);
+        }
+        *abort_flag = 0;
+        ptx::fence_mbar_init();
+    }
     __syncthreads();
     for (int i = tid; i < S; i += kGvThreads) {
         const int v = __ldg(a.ids + i);
@@ -105,7 +150,7 @@ gemv_kernel(const GemvArgs a) {
         else set_status(status, MOE_ERR_BAD_ID);
     }
     __syncthreads();
-    if (warp == 0) {  // exclusive prefix of popcounts, 32 words per step
+    if (warp == 0) {  // exclusive prefix, 32 words per step
         int run = 0;
         for (int w0 = 0; w0 < nwords; w0 += 32) {
             const int w = w0 + lane;
@@ -123,15 +168,60 @@ gemv_kernel(const GemvArgs a) {
     }
     __syncthreads();
     const int n_distinct = wp[nwords];
-    const int routed_items = n_distinct * a.routed.items;
-    const int n_items = routed_items + (a.has_shared ? a.shared.items : 0);
+    // ---- slot table: the slots of distinct expert j are list[off[j] .. off[j+1])
+    int* cnt = tab;                      // [n_distinct + 1]
+    int* off = tab + (a.max_distinct + 1);
+    int* list = off + (a.max_distinct + 1);
+    auto rank_of = [&](int v) { return wp[v >> 5] + __popc(bm[v >> 5] & ((1u << (v & 31)) - 1u)); };
+    for (int j = tid; j <= n_distinct; j += kGvThreads) cnt[j] = 0;
+    __syncthreads();
+    for (int i = tid; i < S; i += kGvThreads) {
+        const int v = __ldg(a.ids + i);
+        if (v >= 0 && v < a.n_experts) atomicAdd(&cnt[rank_of(v)], 1);
+    }
+    __syncthreads();
+    if (warp == 0) {
+        int run = 0;
+        for (int j0 = 0; j0 < n_distinct; j0 += 32) {
+            const int j = j0 + lane;
+            const int c = j < n_distinct ? cnt[j] : 0;
+            int incl = c;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int n = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += n;
+            }
+            if (j < n_distinct) off[j] = run + incl - c;
+            run += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) off[n_distinct] = run;
+    }
+    __syncthreads();
+    for (int j = tid; j < n_distinct; j += kGvThreads) cnt[j] = 0;
+    __syncthreads();
+    for (int i = tid; i < S; i += kGvThreads) {  // order inside an expert is free: slots are independent
+        const int v = __ldg(a.ids + i);
+        if (v >= 0 && v < a.n_experts) {
+            const int j = rank_of(v);
+            list[off[j] + atomicAdd(&cnt[j], 1)] = i;
+        }
+    }
+    __syncthreads();
+
+    const GemvSide& R = a.routed;
+    const GemvSide& Sh = a.shared;
+    const int per_e = R.L.mt_count * R.chunks;
+    const int n_items_r = n_distinct * per_e;
+    const int n_items = n_items_r + (a.has_shared ? Sh.L.mt_count * Sh.chunks : 0);
 
     auto item_of = [&](int it) {
         GvItem f;
-        int slice;
-        if (it < routed_items) {
-            const int j = it / a.routed.items;
-            slice = it - j * a.routed.items;
+        if (it < n_items_r) {
+            const int j = it / per_e, rem = it - j * per_e;
+            f.sd = &R;
+            f.shared = 0;
+            f.mt = rem / R.chunks;
+            f.c = rem - f.mt * R.chunks;
             int lo = 0, hi = nwords;  // wp[lo] <= j < wp[hi]
             while (hi - lo > 1) {
                 const int mid = (lo + hi) >> 1;
@@ -140,244 +230,237 @@ gemv_kernel(const GemvArgs a) {
             uint32_t bits = bm[lo];
             for (int q = j - wp[lo]; q > 0; --q) bits &= bits - 1;
             f.e = lo * 32 + __ffs(bits) - 1;
-            f.shared = 0;
-            f.sd = &a.routed;
+            f.sbase = off[j];
+            f.nsl = off[j + 1] - off[j];
+            f.group = R.group0 + j * R.L.mt_count + f.mt;
         } else {
-            slice = it - routed_items;
-            f.e = 0;
+            const int i2 = it - n_items_r;
+            f.sd = &Sh;
             f.shared = 1;
-            f.sd = &a.shared;
+            f.mt = i2 / Sh.chunks;
+            f.c = i2 - f.mt * Sh.chunks;
+            f.e = 0;
+            f.sbase = 0;
+            f.nsl = a.n_tokens;
+            f.group = Sh.group0 + f.mt;
         }
-        const int r = slice * f.sd->rows;
-        f.mt = r / kTileM;
-        f.r0 = r % kTileM;
-        f.rows_mt = f.sd->L.rows(f.mt);
+        f.kt0 = f.c * f.sd->kc;
+        f.nk = min(f.sd->kc, f.sd->L.kt_count - f.kt0);
+        f.rows = f.sd->L.rows(f.mt);
         return f;
     };
+    const int sk = a.sk, ns = a.ns;
 
-    // stage s of buffer b completes one phase per arm; each keeps its own parity bit
-    uint32_t next_par[2] = {0u, 0u}, wait_par[2] = {0u, 0u};
-    auto issue = [&](const GvItem& f, int b, int kt0, int kt1) {
-        const GemvSide& sd = *f.sd;
-        const uint32_t pq = (uint32_t)sd.rows * kTileK, pd = (uint32_t)sd.rows * 4u;
-        const uint32_t stage_bytes = (uint32_t)NMAT * (pq + pd);
-        if (warp == 0) {
-            for (int s = lane; s < kt1 - kt0; s += 32) {
-                uint8_t* dst = sbuf[b] + (size_t)s * stage_bytes;
-                uint64_t* bar = &bars[b * a.max_stages + s];
-                ptx::mbar_arrive_expect_tx(bar, stage_bytes);
+    if (warp == 0) {
+        // ------------------------------------------------------- producer
+        if (lane == 0) {
+            uint32_t sc = 0;
+            bool ok = true;
+            for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+                const GvItem f = item_of(it);
+                const GemvSide& sd = *f.sd;
+                const int G = (f.nsl + kGvNT - 1) / kGvNT;
+                for (int g = 0; g < G && ok; ++g)
+                    for (int ks = 0; ks < f.nk; ks += sk, ++sc) {
+                        const int nks = min(sk, f.nk - ks);
+                        const int s = (int)(sc % (uint32_t)ns);
+                        if (!gv_wait(&empty[s], ((sc / ns) & 1u) ^ 1u, status, abort_flag)) { ok = false; break; }
+                        const uint32_t bytes = (uint32_t)nks * f.rows * kRowBytes;
+                        ptx::mbar_arrive_expect_tx(&full[s], NMAT * bytes);
 #pragma unroll
-                for (int m = 0; m < NMAT; ++m) {
-                    // the slice's rows of both 32-column halves, then their scales
-                    const uint8_t* blk = (m ? sd.W1 : sd.W0) + sd.L.block(f.e, f.mt, kt0 + s);
-                    uint8_t* o = dst + m * (pq + pd);
-                    ptx::bulk_g2s(o, blk + (size_t)f.r0 * 32, pq / 2, bar);
-                    ptx::bulk_g2s(o + pq / 2, blk + (size_t)f.rows_mt * 32 + (size_t)f.r0 * 32, pq / 2, bar);
-                    ptx::bulk_g2s(o + pq, blk + (size_t)f.rows_mt * kTileK + f.r0 * 4, pd, bar);
-                }
+                        for (int m = 0; m < NMAT; ++m)
+                            ptx::bulk_g2s(ring + (size_t)s * a.stage_bytes + (size_t)m * sk * kGvBlock,
+                                          (m ? sd.W1 : sd.W0) + sd.L.block(f.e, f.mt, f.kt0 + ks), bytes, &full[s]);
+                    }
             }
+            // every copy issued lands before the CTA can exit (bounded)
+            volatile int never = 0;
+            const uint32_t first = sc > (uint32_t)ns ? sc - ns : 0u;
+            for (uint32_t q = first; q < sc; ++q) gv_wait(&full[q % ns], (q / ns) & 1u, status, &never);
         }
-        const int ns = kt1 - kt0;
-        const uint32_t armed = ns >= 32 ? 0xffffffffu : ((1u << ns) - 1u);
-        wait_par[b] = next_par[b];
-        next_par[b] ^= armed;
-    };
-
-    const bool resident = a.nbuf == 2;
-    const int step = gridDim.x;
-    int it = blockIdx.x;
-    if (resident) {
-        if (it < n_items) { const GvItem f = item_of(it); issue(f, 0, 0, f.sd->L.kt_count); }
-        if (it + step < n_items) { const GvItem f = item_of(it + step); issue(f, 1, 0, f.sd->L.kt_count); }
+        return;
     }
-    if (a.pdl_secondary) asm volatile("griddepcontrol.wait;" ::: "memory");
 
-    bool ok = true;
-    for (int i = 0; it < n_items && ok; ++i, it += step) {
-        const int b = resident ? (i & 1) : 0;
+    // ----------------------------------------------------------- consumers
+    const int ct = tid - 32;
+    const int r = ct & (kTileM - 1), hh = ct >> 7;
+    const int first = (lane >> 2) & 1;  // alternate 16-byte order: conflict-free shared loads
+    const uint32_t xrow = (uint32_t)a.xw * kTileK;  // activation window row, elements
+    uint32_t sc = 0;
+    bool waited_primary = !a.pdl_secondary;
+
+    for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
         const GvItem f = item_of(it);
         const GemvSide& sd = *f.sd;
         const WLayout L = sd.L;
-        const int R = sd.rows, KT = L.kt_count, NW = sd.kw / kTileK;
-        const uint32_t pq = (uint32_t)R * kTileK, pd = (uint32_t)R * 4u;
-        const uint32_t stage_bytes = (uint32_t)NMAT * (pq + pd);
-        const int c = tid & 3, r = (tid >> 2) % R, ph = tid / (R * 4);
-        const int P = kGvThreads / (R * 4);
-        const int ntc = a.nt_cap;
-
-        // slots of this expert (routed) or tokens (shared)
-        int n_sl = a.n_tokens;
-        if (!f.shared) {
-            int cnt = 0;
-            for (int q = tid; q < S; q += kGvThreads) cnt += (__ldg(a.ids + q) == f.e);
-            cnt = __reduce_add_sync(0xffffffffu, cnt);
-            if (lane == 0) misc[warp] = cnt;
-            __syncthreads();
-            n_sl = 0;
-            for (int w = 0; w < kGvThreads / 32; ++w) n_sl += misc[w];
-            __syncthreads();
-        }
-        for (int g0 = 0; g0 < n_sl && ok; g0 += ntc) {
-            const int nt = min(ntc, n_sl - g0);
-            if (f.shared) {
-                if (tid < nt) rows_sh[tid] = g0 + tid;
-            } else {
-                int base = 0;
-                for (int q0 = 0; q0 < S; q0 += kGvThreads) {
-                    const int q = q0 + tid;
-                    const bool hit = q < S && __ldg(a.ids + q) == f.e;
-                    const unsigned bal = __ballot_sync(0xffffffffu, hit);
-                    if (lane == 0) misc[warp] = __popc(bal);
-                    __syncthreads();
-                    int before = base;
-                    for (int w = 0; w < warp; ++w) before += misc[w];
-                    const int rank = before + __popc(bal & ((1u << lane) - 1u));
-                    if (hit && rank >= g0 && rank < g0 + nt) rows_sh[rank - g0] = q;
-                    int tot = 0;
-                    for (int w = 0; w < kGvThreads / 32; ++w) tot += misc[w];
-                    base += tot;
-                    __syncthreads();
-                }
-            }
+        const int G = (f.nsl + kGvNT - 1) / kGvNT;
+        const int S_side = f.shared ? a.n_tokens : S;
+        auto slot_of = [&](int q) { return f.shared ? q : list[f.sbase + q]; };
+        for (int g = 0; g < G; ++g) {
+            const int nt = min(kGvNT, f.nsl - g * kGvNT);
             float acc[NMAT][kGvNT];
 #pragma unroll
             for (int m = 0; m < NMAT; ++m)
 #pragma unroll
                 for (int q = 0; q < kGvNT; ++q) acc[m][q] = 0.f;
-
-            for (int kt0 = 0; kt0 < KT && ok; kt0 += NW) {
-                const int kt1 = min(KT, kt0 + NW);
-                __syncthreads();  // previous window's stages and activations are free
-                if (!resident) issue(f, b, kt0, kt1);
-                const int cols = (kt1 - kt0) * kTileK;
-                if (XB == 2) {
-                    const uint16_t* xg = (const uint16_t*)sd.x;
-                    for (int idx = tid; idx < nt * cols / 8; idx += kGvThreads) {
-                        const int q = idx / (cols / 8), c8 = (idx % (cols / 8)) * 8, col = kt0 * kTileK + c8;
-                        const int row = f.shared ? rows_sh[q] : (sd.x_per_slot ? rows_sh[q] : rows_sh[q] / a.k);
-                        uint4 v = make_uint4(0, 0, 0, 0);
-                        if (col < L.n_in) v = __ldg((const uint4*)(xg + (size_t)row * L.n_in + col));
-                        *(uint4*)(sx + ((size_t)q * sd.kw + c8) * 2) = v;
-                    }
-                } else {
-                    const float* xg = (const float*)sd.x;
-                    for (int idx = tid; idx < nt * cols / 4; idx += kGvThreads) {
-                        const int q = idx / (cols / 4), c4 = (idx % (cols / 4)) * 4, col = kt0 * kTileK + c4;
-                        const int row = f.shared ? rows_sh[q] : (sd.x_per_slot ? rows_sh[q] : rows_sh[q] / a.k);
-                        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-                        if (col < L.n_in) v = __ldg((const float4*)(xg + (size_t)row * L.n_in + col));
-                        *(float4*)(sx + ((size_t)q * sd.kw + c4) * 4) = v;
+            bool ok = true;
+            for (int w0 = 0; w0 < f.nk; w0 += a.xw) {
+                const int nw = min(a.xw, f.nk - w0);
+                // the previous window's activations are no longer read; stop together on abort
+                ok = consumers_and(ok && !*abort_flag);
+                if (!ok) break;
+                if (!waited_primary) {
+                    asm volatile("griddepcontrol.wait;" ::: "memory");
+                    waited_primary = true;
+                }
+                // stage the activations of the nt tokens for this window, as fp32
+                const int cols = nw * kTileK, col0 = (f.kt0 + w0) * kTileK;
+                constexpr int VE = 16 / XB;  // elements per 16-byte vector
+                for (int idx = ct; idx < nt * cols / VE; idx += kGvConsumers) {
+                    const int q = idx / (cols / VE), cc = (idx - q * (cols / VE)) * VE, col = col0 + cc;
+                    const int sl = slot_of(g * kGvNT + q);
+                    const int row = f.shared ? sl : (sd.x_per_slot ? sl : sl / a.k);
+                    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                    if (col < L.n_in) v = __ldg((const uint4*)((const uint8_t*)sd.x + ((size_t)row * L.n_in + col) * XB));
+                    float* dst = (float*)sx + (size_t)q * xrow + cc;
+                    if (XB == 4) {
+                        *(uint4*)dst = v;
+                    } else {
+                        const uint32_t uw[4] = {v.x, v.y, v.z, v.w};
+                        float e[8];
+#pragma unroll
+                        for (int b = 0; b < 4; ++b) {
+                            e[2 * b] = ld_x16(uw[b] & 0xffffu, sd.x_type);
+                            e[2 * b + 1] = ld_x16(uw[b] >> 16, sd.x_type);
+                        }
+                        *(float4*)dst = make_float4(e[0], e[1], e[2], e[3]);
+                        *(float4*)(dst + 4) = make_float4(e[4], e[5], e[6], e[7]);
                     }
                 }
-                __syncthreads();
-                for (int kt = kt0 + ph; kt < kt1; kt += P) {
-                    const int s = kt - kt0;
-                    if (!gv_wait(&bars[b * a.max_stages + s], (wait_par[b] >> s) & 1u, status)) { ok = false; break; }
-                    const uint8_t* st = sbuf[b] + (size_t)s * stage_bytes;
-                    float w[NMAT][16];
-#pragma unroll
-                    for (int m = 0; m < NMAT; ++m) {
-                        const uint8_t* pm = st + m * (pq + pd);
-                        const uint4 qv = *(const uint4*)(pm + (c >> 1) * (pq / 2) + r * 32 + (c & 1) * 16);
-                        const float d = __half2float(*(const __half*)(pm + pq + r * 4 + (c >> 1) * 2));
-                        const float nd = -32896.0f * d;
-                        const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
-#pragma unroll
-                        for (int bb = 0; bb < 16; ++bb) w[m][bb] = fmaf(magic_byte(qw[bb >> 2], bb & 3), d, nd);
-                    }
-                    const int xc = s * kTileK + c * 16;
-#pragma unroll
-                    for (int q = 0; q < kGvNT; ++q) {
-                        if (q < nt) {
-                            float xv[16];
-                            if (XB == 2) {
-                                const uint4 u0 = *(const uint4*)(sx + ((size_t)q * sd.kw + xc) * 2);
-                                const uint4 u1 = *(const uint4*)(sx + ((size_t)q * sd.kw + xc + 8) * 2);
-                                const uint32_t uw[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-#pragma unroll
-                                for (int bb = 0; bb < 8; ++bb) {
-                                    xv[2 * bb] = ld_x16(uw[bb] & 0xffffu, sd.x_type);
-                                    xv[2 * bb + 1] = ld_x16(uw[bb] >> 16, sd.x_type);
-                                }
-                            } else {
-#pragma unroll
-                                for (int bb = 0; bb < 16; bb += 4) {
-                                    const float4 vv = *(const float4*)(sx + ((size_t)q * sd.kw + xc + bb) * 4);
-                                    xv[bb] = vv.x; xv[bb + 1] = vv.y; xv[bb + 2] = vv.z; xv[bb + 3] = vv.w;
-                                }
-                            }
+                consumers_sync();
+                for (int ks = w0; ks < w0 + nw; ks += sk, ++sc) {
+                    const int nks = min(sk, f.nk - ks);
+                    const int s = (int)(sc % (uint32_t)ns);
+                    int okw = 1;
+                    if (lane == 0) okw = gv_wait(&full[s], (sc / ns) & 1u, status, abort_flag);
+                    if (!__shfl_sync(0xffffffffu, okw, 0)) { ok = false; break; }
+                    if (r < f.rows) {
+                        for (int kk = 0; kk < nks; ++kk) {
+                            float w[NMAT][32];
 #pragma unroll
                             for (int m = 0; m < NMAT; ++m) {
-                                float t = 0.f;
+                                const uint8_t* blk = ring + (size_t)s * a.stage_bytes + (size_t)m * sk * kGvBlock +
+                                                     (size_t)kk * f.rows * kRowBytes;
+                                const uint8_t* qrow = blk + (size_t)hh * f.rows * 32 + r * 32;
+                                const uint4 qa = *(const uint4*)(qrow + first * 16);
+                                const uint4 qb = *(const uint4*)(qrow + (first ^ 1) * 16);
+                                const uint4 q0 = first ? qb : qa, q1 = first ? qa : qb;
+                                const float d =
+                                    __half2float(*(const __half*)(blk + (size_t)f.rows * kTileK + r * 4 + hh * 2));
+                                const float nd = -32896.0f * d;
+                                const uint32_t qw[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
 #pragma unroll
-                                for (int bb = 0; bb < 16; ++bb) t = fmaf(w[m][bb], xv[bb], t);
-                                acc[m][q] += t;
+                                for (int i = 0; i < 32; ++i) w[m][i] = fmaf(magic_byte(qw[i >> 2], i & 3), d, nd);
+                            }
+                            const float* xk = (const float*)sx + (size_t)(ks - w0 + kk) * kTileK + hh * 32;
+#pragma unroll
+                            for (int q = 0; q < kGvNT; ++q) {
+                                if (q >= nt) break;
+                                const float4* xv = (const float4*)(xk + (size_t)q * xrow);
+                                float t[NMAT];
+#pragma unroll
+                                for (int m = 0; m < NMAT; ++m) t[m] = 0.f;
+#pragma unroll
+                                for (int v4 = 0; v4 < 8; ++v4) {
+                                    const float4 u = xv[v4];
+#pragma unroll
+                                    for (int m = 0; m < NMAT; ++m) {
+                                        t[m] = fmaf(w[m][v4 * 4], u.x, t[m]);
+                                        t[m] = fmaf(w[m][v4 * 4 + 1], u.y, t[m]);
+                                        t[m] = fmaf(w[m][v4 * 4 + 2], u.z, t[m]);
+                                        t[m] = fmaf(w[m][v4 * 4 + 3], u.w, t[m]);
+                                    }
+                                }
+#pragma unroll
+                                for (int m = 0; m < NMAT; ++m) acc[m][q] += t[m];
                             }
                         }
                     }
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(&empty[s]);
                 }
-                // every thread leaves a timed-out wait the same way (no divergent barriers)
-                ok = __syncthreads_and(ok) != 0;
             }
-            // reduce: the 4 chunk lanes by a fixed butterfly, then the k phases in order
+            // the two column halves of each row, in a fixed order
 #pragma unroll
             for (int m = 0; m < NMAT; ++m)
 #pragma unroll
-                for (int q = 0; q < kGvNT; ++q) {
-                    float v = acc[m][q];
-                    v += __shfl_xor_sync(0xffffffffu, v, 1);
-                    v += __shfl_xor_sync(0xffffffffu, v, 2);
-                    acc[m][q] = v;
-                }
-            if (c == 0)
+                for (int q = 0; q < kGvNT; ++q)
+                    if (q < nt) red[((hh * kTileM + r) * kGvNT + q) * NMAT + m] = acc[m][q];
+            if (!consumers_and(ok && !*abort_flag)) return;  // uniform
+            if (hh == 0 && r < f.rows) {
+                const int n = f.mt * kTileM + r;
+                if (n < L.n_out)
+                    for (int q = 0; q < nt; ++q) {
+                        const int sl = slot_of(g * kGvNT + q);
+                        float v[NMAT];
 #pragma unroll
-                for (int m = 0; m < NMAT; ++m)
+                        for (int m = 0; m < NMAT; ++m)
+                            v[m] = red[((0 * kTileM + r) * kGvNT + q) * NMAT + m] +
+                                   red[((1 * kTileM + r) * kGvNT + q) * NMAT + m];
+                        if (sd.chunks > 1) {
+                            float* pp = sd.part + (((size_t)f.c * S_side + sl) * L.n_out_pad + n) * NMAT;
 #pragma unroll
-                    for (int q = 0; q < kGvNT; ++q)
-                        if (q < ntc) red[((ph * R + r) * ntc + q) * NMAT + m] = acc[m][q];
-            __syncthreads();
-            for (int idx = tid; idx < R * ntc; idx += kGvThreads) {
-                const int row = idx / ntc, q = idx % ntc;
-                const int n = f.mt * kTileM + f.r0 + row;
-                if (q < nt && n < L.n_out) {
+                            for (int m = 0; m < NMAT; ++m) pp[m] = v[m];
+                        } else if (DUAL) {
+                            const float gt = v[0], up = v[NMAT - 1];
+                            sd.h[(int64_t)sl * L.n_out + n] = __float2bfloat16_rn(gt / (1.0f + expf(-gt)) * up);
+                        } else {
+                            sd.out[(int64_t)sl * L.n_out + n] = v[0];
+                        }
+                    }
+            }
+            consumers_sync();  // red is free again
+        }
+        if (sd.chunks > 1) {
+            // the last chunk of this (expert, row tile) to finish adds all chunks in order
+            __threadfence();
+            consumers_sync();
+            if (ct == 0) *last_flag = atomicAdd(a.hdr + kHdrCnt0 + f.group, 1) == sd.chunks - 1;
+            consumers_sync();
+            if (*last_flag) {
+                __threadfence();
+                for (int idx = ct; idx < f.nsl * f.rows; idx += kGvConsumers) {
+                    const int q = idx / f.rows, rr = idx - q * f.rows;
+                    const int n = f.mt * kTileM + rr;
+                    if (n >= L.n_out) continue;
+                    const int sl = slot_of(q);
                     float v[NMAT];
 #pragma unroll
-                    for (int m = 0; m < NMAT; ++m) {
-                        v[m] = 0.f;
-                        for (int p2 = 0; p2 < P; ++p2) v[m] += red[((p2 * R + row) * ntc + q) * NMAT + m];
+                    for (int m = 0; m < NMAT; ++m) v[m] = 0.f;
+                    for (int c = 0; c < sd.chunks; ++c) {
+                        const volatile float* pp = sd.part + (((size_t)c * S_side + sl) * L.n_out_pad + n) * NMAT;
+#pragma unroll
+                        for (int m = 0; m < NMAT; ++m) v[m] += pp[m];
                     }
-                    const int64_t orow = rows_sh[q];
                     if (DUAL) {
-                        const float g = v[0], u = v[NMAT - 1];
-                        sd.h[orow * L.n_out + n] = __float2bfloat16_rn(g / (1.0f + expf(-g)) * u);
+                        const float gt = v[0], up = v[NMAT - 1];
+                        sd.h[(int64_t)sl * L.n_out + n] = __float2bfloat16_rn(gt / (1.0f + expf(-gt)) * up);
                     } else {
-                        sd.out[orow * L.n_out + n] = v[0];
+                        sd.out[(int64_t)sl * L.n_out + n] = v[0];
                     }
                 }
+                if (ct == 0) atomicExch(a.hdr + kHdrCnt0 + f.group, 0);
             }
-            __syncthreads();
-        }
-        __syncthreads();  // this item's buffer is free
-        if (resident && it + 2 * step < n_items) {
-            const GvItem nf = item_of(it + 2 * step);
-            issue(nf, b, 0, nf.sd->L.kt_count);
+            consumers_sync();  // last_flag is free again
         }
     }
 }
 
 void gemv_plan_side(GemvSide& s, int dual) {
-    const int nmat = dual + 1;
-    const int xb = s.x_type == MOE_F32 ? 4 : 2;
-    s.kw = xb == 2 ? 2048 : 1024;
-    s.n_stages = s.L.kt_count < s.kw / kTileK ? s.L.kt_count : s.kw / kTileK;
-    s.rows = 16;
-    for (int R : {64, 32}) {
-        if (s.L.n_out_pad % R == 0 && s.n_stages * nmat * R * kRowBytes <= kGvWeightBudget) {
-            s.rows = R;
-            break;
-        }
-    }
-    s.items = s.L.n_out_pad / s.rows;
+    (void)dual;
+    s.kc = s.L.kt_count;
+    s.chunks = 1;
+    s.group0 = 0;
 }
 
 template <int DUAL, int XB>
@@ -386,8 +469,8 @@ static moe_status launch_t(const GemvArgs& a, size_t smem, unsigned grid, cudaSt
     int dev = 0;
     cudaGetDevice(&dev);
     if (attr_dev != dev) {
-        if (cudaFuncSetAttribute(gemv_kernel<DUAL, XB>, cudaFuncAttributeMaxDynamicSharedMemorySize, 220 * 1024) !=
-            cudaSuccess)
+        if (cudaFuncSetAttribute(gemv_kernel<DUAL, XB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kGvSmemBudget + 16 * 1024) != cudaSuccess)
             return MOE_ERR_CUDA;
         attr_dev = dev;
     }
@@ -417,41 +500,59 @@ static int gv_sm_count() {
 
 moe_status launch_gemv(const GemvArgs& in, cudaStream_t stream) {
     GemvArgs a = in;
-    const int64_t items_max = (int64_t)a.max_distinct * a.routed.items + (a.has_shared ? a.shared.items : 0);
-    if (items_max == 0) return MOE_OK;
+    const int S = a.n_tokens * a.k;
+    if (S > kGvMaxSlots) return MOE_ERR_UNSUPPORTED;
+    const int64_t groups_r = (int64_t)a.max_distinct * a.routed.L.mt_count;
+    const int64_t groups_s = a.has_shared ? a.shared.L.mt_count : 0;
+    if (groups_r + groups_s == 0) return MOE_OK;
     const bool f32 = a.routed.x_type == MOE_F32 || (a.has_shared && a.shared.x_type == MOE_F32);
     if (f32 && a.has_shared && a.routed.x_type != a.shared.x_type) return MOE_ERR_UNSUPPORTED;
     const int nmat = a.dual + 1;
-    const int xb = f32 ? 4 : 2;
-    a.nt_cap = a.n_tokens < kGvNT ? (a.n_tokens > 0 ? a.n_tokens : 1) : kGvNT;
-    const GemvSide* sides[2] = {&a.routed, a.has_shared ? &a.shared : nullptr};
-    uint32_t buf = 0, red = 0;
-    int kw = 0, max_stages = 0;
-    bool resident = true;
-    for (const GemvSide* s : sides) {
-        if (!s) continue;
-        const uint32_t b = (uint32_t)s->n_stages * nmat * s->rows * kRowBytes;
-        const int P = kGvThreads / (s->rows * 4);
-        const uint32_t rb = (uint32_t)P * s->rows * a.nt_cap * nmat * 4;
-        if (b > buf) buf = b;
-        if (rb > red) red = rb;
-        if (s->kw > kw) kw = s->kw;
-        if (s->n_stages > max_stages) max_stages = s->n_stages;
-        if (s->L.kt_count > s->kw / kTileK) resident = false;
+    const int sms = gv_sm_count();
+
+    // Split K when the (expert, row tile) groups alone cannot cover the SMs.
+    // Shared-expert items carry every token, so that side is split further.
+    // Split groups count arrivals in the header (kGvMaxGroups counters).
+    GemvSide* sides[2] = {&a.routed, a.has_shared ? &a.shared : nullptr};
+    for (GemvSide* s : sides)
+        if (s) s->kc = s->L.kt_count, s->chunks = 1;
+    const bool small = S <= kGvSplitSlots;
+    int chunks_r = 1, chunks_s = 1;
+    if (small) {
+        chunks_r = (int)((sms + groups_r + groups_s - 1) / (groups_r + groups_s));
+        chunks_s = chunks_r > 2 * a.n_tokens ? chunks_r : 2 * a.n_tokens;
     }
-    a.buf_bytes = buf;
-    a.red_bytes = red;
-    a.x_bytes = (uint32_t)a.nt_cap * kw * xb;
+    int counters = 0;
+    auto split = [&](GemvSide* s, int64_t groups, int want) {
+        if (!s || !s->part || want <= 1 || counters + groups > kGvMaxGroups) return;
+        const int KT = s->L.kt_count;
+        if (want > kGvMaxChunks) want = kGvMaxChunks;
+        if (want > KT) want = KT;
+        s->kc = (KT + want - 1) / want;
+        s->chunks = (KT + s->kc - 1) / s->kc;
+        s->group0 = counters;
+        counters += (int)groups;
+    };
+    split(&a.routed, groups_r, chunks_r);
+    if (a.has_shared) split(&a.shared, groups_s, chunks_s);
+
+    a.sk = 2;
+    a.xw = 16;
+    a.stage_bytes = (uint32_t)nmat * a.sk * kGvBlock;
+    a.x_bytes = (uint32_t)kGvNT * a.xw * kTileK * 4;  // fp32 after staging
+    a.red_bytes = (uint32_t)2 * kTileM * kGvNT * nmat * 4;
     a.bm_words = (uint32_t)((a.n_experts + 31) / 32);
-    a.max_stages = max_stages;
-    a.nbuf = resident ? 2 : 1;
-    size_t smem = gv_lay(a).total;
-    if (smem > 200 * 1024) {
-        a.nbuf = 1;
-        smem = gv_lay(a).total;
-    }
-    const int per_sm = (int)((228 * 1024) / (smem + 1024)) > 0 ? (int)((228 * 1024) / (smem + 1024)) : 1;
-    int64_t grid = (int64_t)gv_sm_count() * per_sm;
+    a.tab_words = (uint32_t)(2 * (a.max_distinct + 1) + S);
+    a.ns = 1;
+    const uint32_t fixed = gv_lay(a).total - a.stage_bytes;
+    int ns = (int)((kGvSmemBudget - fixed) / a.stage_bytes);
+    if (ns > 8) ns = 8;
+    if (ns < 2) return MOE_ERR_UNSUPPORTED;
+    a.ns = ns;
+    const size_t smem = gv_lay(a).total;
+
+    const int64_t items_max = groups_r * a.routed.chunks + groups_s * (a.has_shared ? a.shared.chunks : 0);
+    int64_t grid = sms;
     if (grid > items_max) grid = items_max;
     if (a.dual)
         return f32 ? launch_t<1, 4>(a, smem, (unsigned)grid, stream) : launch_t<1, 2>(a, smem, (unsigned)grid, stream);

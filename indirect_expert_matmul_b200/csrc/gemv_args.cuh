@@ -4,7 +4,10 @@
 
 namespace moe {
 
-constexpr int kGvMaxSlots = 8192;  // the mat-vec path handles n_tokens*k up to this
+constexpr int kGvMaxSlots = 1024;   // the mat-vec path handles n_tokens*k up to this
+constexpr int kGvNT = 8;            // tokens per pass over a weight chunk
+constexpr int kHdrCnt0 = 16;        // header words [16, 64): split-K arrival counters
+constexpr int kGvMaxGroups = 48;    // (expert, row tile) groups that may be split
 
 struct GemvSide {
     const uint8_t* W0;  // prepared weights (single, or gate)
@@ -15,10 +18,10 @@ struct GemvSide {
     int x_per_slot;     // routed x row: 1 -> slot t*k+s, 0 -> token t
     float* out;         // single: out[slot][n] (routed) or out[t][n] (shared)
     __nv_bfloat16* h;   // dual: h[slot][n] (routed) or h[t][n] (shared)
-    int rows;           // rows per work item: 16, 32 or 64
-    int items;          // work items per expert: n_out_pad / rows
-    int n_stages;       // weight k-steps resident at once (one activation window)
-    int kw;             // activation window (columns)
+    float* part;        // split-K partial sums [chunk][slot][n_out_pad][1 + dual], or null (no split)
+    int kc;             // k-steps per chunk (filled by launch_gemv)
+    int chunks;         // ceil(kt_count / kc)
+    int group0;         // first counter index of this side's (expert, row tile) groups
 };
 
 struct GemvArgs {
@@ -27,18 +30,18 @@ struct GemvArgs {
     int dual;
     const int32_t* ids;  // [n_tokens][k]
     int n_tokens, k, n_experts;
-    int max_distinct;    // min(n_tokens*k, n_experts): routed items = max_distinct * routed.items
+    int max_distinct;    // min(n_tokens*k, n_experts)
     int pdl_secondary;   // launched as a programmatic dependent: wait before reading activations
     int* hdr;
     // launch plan (filled by launch_gemv)
-    int nt_cap;          // tokens per pass
-    int nbuf;            // 2: double-buffered whole weight slices; 1: windowed
-    uint32_t buf_bytes, x_bytes, red_bytes, bm_words;
-    int max_stages;
+    int sk;              // k-steps per ring stage
+    int ns;              // ring stages
+    int xw;              // activation window, in k-steps (a multiple of sk)
+    uint32_t stage_bytes, x_bytes, red_bytes, tab_words, bm_words;
 };
 
 moe_status launch_gemv(const GemvArgs& a, cudaStream_t stream);
-// Fill rows / items / n_stages / kw of a side for its shape and activation type.
+// Reset the split fields of a side (no split); launch_gemv chooses the split.
 void gemv_plan_side(GemvSide& s, int dual);
 
 }  // namespace moe

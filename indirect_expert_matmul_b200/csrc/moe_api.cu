@@ -217,6 +217,7 @@ moe_status moe_ffn(const void* Wg, const void* Wu, const void* Wd, int n_experts
         a.routed.x_type = x_type;
         a.routed.h = h;
         gemv_plan_side(a.routed, 1);
+        a.routed.part = S <= kGvSplitSlots ? (float*)(ws + W.gv_part) : nullptr;  // split-K partial sums
         if (has_shared) {
             a.shared.W0 = (const uint8_t*)Sg;
             a.shared.W1 = (const uint8_t*)Su;
@@ -225,6 +226,7 @@ moe_status moe_ffn(const void* Wg, const void* Wu, const void* Wd, int n_experts
             a.shared.x_type = x_type;
             a.shared.h = h_sh;
             gemv_plan_side(a.shared, 1);
+            a.shared.part = S <= kGvSplitSlots ? (float*)(ws + W.gv_part_sh) : nullptr;
         }
         st = launch_gemv(a, s);
         if (st) return st;
