@@ -8,11 +8,12 @@
 //  - a work item is (distinct routed expert, 128-row tile, K-chunk) or
 //    (shared expert, 128-row tile, K-chunk); every k-step block of one
 //    (expert, row tile) is contiguous in the repacked layout, so a stage of
-//    up to two k-steps of one matrix is a single bulk copy (17 KB);
+//    up to two (dual) or four (single) k-steps of one matrix is a single bulk
+//    copy of up to 34 KB;
 //  - one producer warp streams the stages of the CTA's items through a ring
 //    of shared-memory stages, ahead of the consumers and across items;
-//  - 256 consumer threads dequantise (exact fp32 q*d) and take the dot
-//    products with up to 8 tokens at a time: thread = (row, 32-column half);
+//  - 512 consumer threads dequantise (exact fp32 q*d) and take the dot
+//    products with up to 8 tokens at a time: thread = (row, 16 columns);
 //  - when there are fewer (expert, row tile) groups than SMs (a single decode
 //    token), K is split into chunks; each chunk writes fp32 partial sums and
 //    the CTA that finishes a group last adds the chunks in chunk order and
@@ -32,7 +33,7 @@
 
 namespace moe {
 
-constexpr int kGvConsumers = 256;
+constexpr int kGvConsumers = 512;
 constexpr int kGvThreads = 32 + kGvConsumers;  // warp 0: producer
 constexpr uint32_t kGvBlock = kTileM * kRowBytes;  // 8704: one k-step of a full row tile
 constexpr uint32_t kGvSmemBudget = 200 * 1024;
@@ -56,6 +57,24 @@ __host__ __device__ inline GvLay gv_lay(const GemvArgs& a) {
     m.misc = o; o += 16u * 4u;
     m.total = o;
     return m;
+}
+
+// Packed fp32 pairs (two lanes of one 64-bit register): fma.rn.f32x2 does two
+// independent round-to-nearest fp32 fmas, the same as two fmaf calls.
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ float f2sum(uint64_t v) {
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+    return lo + hi;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
 }
 
 __device__ __forceinline__ float ld_x16(uint32_t bits16, int x_type) {
@@ -144,8 +163,10 @@ gemv_kernel(const GemvArgs a) {
         ptx::fence_mbar_init();
     }
     __syncthreads();
+    int* ids_sh = tab + 2 * (a.max_distinct + 1) + S;  // ids, read from global memory once
     for (int i = tid; i < S; i += kGvThreads) {
         const int v = __ldg(a.ids + i);
+        ids_sh[i] = v;
         if (v >= 0 && v < a.n_experts) atomicOr(&bm[v >> 5], 1u << (v & 31));
         else set_status(status, MOE_ERR_BAD_ID);
     }
@@ -176,7 +197,7 @@ gemv_kernel(const GemvArgs a) {
     for (int j = tid; j <= n_distinct; j += kGvThreads) cnt[j] = 0;
     __syncthreads();
     for (int i = tid; i < S; i += kGvThreads) {
-        const int v = __ldg(a.ids + i);
+        const int v = ids_sh[i];
         if (v >= 0 && v < a.n_experts) atomicAdd(&cnt[rank_of(v)], 1);
     }
     __syncthreads();
@@ -200,7 +221,7 @@ gemv_kernel(const GemvArgs a) {
     for (int j = tid; j < n_distinct; j += kGvThreads) cnt[j] = 0;
     __syncthreads();
     for (int i = tid; i < S; i += kGvThreads) {  // order inside an expert is free: slots are independent
-        const int v = __ldg(a.ids + i);
+        const int v = ids_sh[i];
         if (v >= 0 && v < a.n_experts) {
             const int j = rank_of(v);
             list[off[j] + atomicAdd(&cnt[j], 1)] = i;
@@ -282,9 +303,10 @@ gemv_kernel(const GemvArgs a) {
     }
 
     // ----------------------------------------------------------- consumers
+    // thread = (32-column half hh, row r, 16-column chunk c16): eight lanes read
+    // four rows' 128 contiguous bytes, so the 16-byte shared loads do not conflict
     const int ct = tid - 32;
-    const int r = ct & (kTileM - 1), hh = ct >> 7;
-    const int first = (lane >> 2) & 1;  // alternate 16-byte order: conflict-free shared loads
+    const int c16 = ct & 1, r = (ct >> 1) & (kTileM - 1), hh = ct >> 8;
     const uint32_t xrow = (uint32_t)a.xw * kTileK;  // activation window row, elements
     uint32_t sc = 0;
     bool waited_primary = !a.pdl_secondary;
@@ -346,43 +368,44 @@ gemv_kernel(const GemvArgs a) {
                     if (!__shfl_sync(0xffffffffu, okw, 0)) { ok = false; break; }
                     if (r < f.rows) {
                         for (int kk = 0; kk < nks; ++kk) {
-                            float w[NMAT][32];
+                            // w = q*d for this thread's 16 columns of each matrix, as 8 packed pairs
+                            uint64_t w2[NMAT][8];
 #pragma unroll
                             for (int m = 0; m < NMAT; ++m) {
                                 const uint8_t* blk = ring + (size_t)s * a.stage_bytes + (size_t)m * sk * kGvBlock +
                                                      (size_t)kk * f.rows * kRowBytes;
-                                const uint8_t* qrow = blk + (size_t)hh * f.rows * 32 + r * 32;
-                                const uint4 qa = *(const uint4*)(qrow + first * 16);
-                                const uint4 qb = *(const uint4*)(qrow + (first ^ 1) * 16);
-                                const uint4 q0 = first ? qb : qa, q1 = first ? qa : qb;
+                                const uint4 qv = *(const uint4*)(blk + (size_t)hh * f.rows * 32 + r * 32 + c16 * 16);
                                 const float d =
                                     __half2float(*(const __half*)(blk + (size_t)f.rows * kTileK + r * 4 + hh * 2));
-                                const float nd = -32896.0f * d;
-                                const uint32_t qw[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+                                const uint64_t dd = f2pack(d, d), nd = f2pack(-32896.0f * d, -32896.0f * d);
+                                const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
 #pragma unroll
-                                for (int i = 0; i < 32; ++i) w[m][i] = fmaf(magic_byte(qw[i >> 2], i & 3), d, nd);
+                                for (int i = 0; i < 8; ++i) {
+                                    const uint32_t wd = qw[i >> 1];
+                                    const int b0 = (2 * i) & 3;
+                                    w2[m][i] = fma2(f2pack(magic_byte(wd, b0), magic_byte(wd, b0 + 1)), dd, nd);
+                                }
                             }
-                            const float* xk = (const float*)sx + (size_t)(ks - w0 + kk) * kTileK + hh * 32;
+                            const float* xk = (const float*)sx + (size_t)(ks - w0 + kk) * kTileK + hh * 32 + c16 * 16;
 #pragma unroll
                             for (int q = 0; q < kGvNT; ++q) {
                                 if (q >= nt) break;
-                                const float4* xv = (const float4*)(xk + (size_t)q * xrow);
-                                float t[NMAT];
+                                const ulonglong2* xv = (const ulonglong2*)(xk + (size_t)q * xrow);
+                                // two independent packed chains per matrix, added in a fixed order
+                                uint64_t t0[NMAT], t1[NMAT];
 #pragma unroll
-                                for (int m = 0; m < NMAT; ++m) t[m] = 0.f;
+                                for (int m = 0; m < NMAT; ++m) t0[m] = t1[m] = 0ull;
 #pragma unroll
-                                for (int v4 = 0; v4 < 8; ++v4) {
-                                    const float4 u = xv[v4];
+                                for (int v4 = 0; v4 < 4; ++v4) {
+                                    const ulonglong2 u = xv[v4];
 #pragma unroll
                                     for (int m = 0; m < NMAT; ++m) {
-                                        t[m] = fmaf(w[m][v4 * 4], u.x, t[m]);
-                                        t[m] = fmaf(w[m][v4 * 4 + 1], u.y, t[m]);
-                                        t[m] = fmaf(w[m][v4 * 4 + 2], u.z, t[m]);
-                                        t[m] = fmaf(w[m][v4 * 4 + 3], u.w, t[m]);
+                                        t0[m] = fma2(w2[m][2 * v4], u.x, t0[m]);
+                                        t1[m] = fma2(w2[m][2 * v4 + 1], u.y, t1[m]);
                                     }
                                 }
 #pragma unroll
-                                for (int m = 0; m < NMAT; ++m) acc[m][q] += t[m];
+                                for (int m = 0; m < NMAT; ++m) acc[m][q] += f2sum(t0[m]) + f2sum(t1[m]);
                             }
                         }
                     }
@@ -390,14 +413,17 @@ gemv_kernel(const GemvArgs a) {
                     if (lane == 0) ptx::mbar_arrive(&empty[s]);
                 }
             }
-            // the two column halves of each row, in a fixed order
+            // the two 16-column chunks (adjacent lanes; a + b == b + a), then the
+            // two 32-column halves of each row, in a fixed order
 #pragma unroll
             for (int m = 0; m < NMAT; ++m)
 #pragma unroll
-                for (int q = 0; q < kGvNT; ++q)
-                    if (q < nt) red[((hh * kTileM + r) * kGvNT + q) * NMAT + m] = acc[m][q];
+                for (int q = 0; q < kGvNT; ++q) {
+                    const float v = acc[m][q] + __shfl_xor_sync(0xffffffffu, acc[m][q], 1);
+                    if (c16 == 0 && q < nt) red[((hh * kTileM + r) * kGvNT + q) * NMAT + m] = v;
+                }
             if (!consumers_and(ok && !*abort_flag)) return;  // uniform
-            if (hh == 0 && r < f.rows) {
+            if (hh == 0 && c16 == 0 && r < f.rows) {
                 const int n = f.mt * kTileM + r;
                 if (n < L.n_out)
                     for (int q = 0; q < nt; ++q) {
@@ -536,13 +562,15 @@ moe_status launch_gemv(const GemvArgs& in, cudaStream_t stream) {
     split(&a.routed, groups_r, chunks_r);
     if (a.has_shared) split(&a.shared, groups_s, chunks_s);
 
-    a.sk = 2;
+    // A stage carries ~34 KB whatever the mode (per-stage costs are fixed): two
+    // k-steps of both matrices, or four of one.
+    a.sk = a.dual ? 2 : 4;
     a.xw = 16;
     a.stage_bytes = (uint32_t)nmat * a.sk * kGvBlock;
     a.x_bytes = (uint32_t)kGvNT * a.xw * kTileK * 4;  // fp32 after staging
     a.red_bytes = (uint32_t)2 * kTileM * kGvNT * nmat * 4;
     a.bm_words = (uint32_t)((a.n_experts + 31) / 32);
-    a.tab_words = (uint32_t)(2 * (a.max_distinct + 1) + S);
+    a.tab_words = (uint32_t)(2 * (a.max_distinct + 1) + 2 * S);  // cnt, off, slot list, ids
     a.ns = 1;
     const uint32_t fixed = gv_lay(a).total - a.stage_bytes;
     int ns = (int)((kGvSmemBudget - fixed) / a.stage_bytes);
