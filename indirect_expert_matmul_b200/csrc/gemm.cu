@@ -167,8 +167,11 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
     return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
-__device__ __forceinline__ uint32_t pack2(float lo, float hi, int bf16) {
-    if (bf16) {
+// Operand type is a template parameter: a runtime choice inside the unrolled
+// dequantisation loop costs a compare and branch per packed pair.
+template <int BF16>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+    if (BF16) {
         __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
         return *(uint32_t*)&v;
     }
@@ -178,8 +181,9 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi, int bf16) {
 
 // Two A operands per tile share each activation tile: DUAL=1 gate and up of
 // one 128-row tile (SwiGLU epilogue into h); DUAL=0 two consecutive 128-row
-// tiles of one matrix (fp32 scatter to dst).
-template <int DUAL>
+// tiles of one matrix (fp32 scatter to dst).  BF16: operand type bf16 (1) or
+// fp16 (0), which must equal p.bf16.
+template <int DUAL, int BF16>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 grouped_gemm_kernel(const GemmParams p) {
     extern __shared__ uint8_t smem_dyn[];
@@ -364,7 +368,7 @@ grouped_gemm_kernel(const GemmParams p) {
                 if (!ok) break;
                 ptx::tc_fence_after();
                 const uint32_t d0 = tmem_base, d1 = tmem_base + kAccCols;
-                const uint32_t idesc = ptx::idesc_f16(p.bf16, n16, 128);
+                const uint32_t idesc = ptx::idesc_f16(BF16, n16, 128);
                 for (int kt = 0; kt < KT; ++kt) {
                     ok = wait_bar(&a_full[as], aph, abort_flag, status, STAT_PTR(0)) &&
                          wait_bar(&b_full[bs], bph, abort_flag, status, STAT_PTR(1));
@@ -496,8 +500,8 @@ grouped_gemm_kernel(const GemmParams p) {
                             const float v1 = fmaf(magic_byte(w[j], 1), dsc, nd);
                             const float v2 = fmaf(magic_byte(w[j], 2), dsc, nd);
                             const float v3 = fmaf(magic_byte(w[j], 3), dsc, nd);
-                            pk[2 * j] = pack2(v0, v1, p.bf16);
-                            pk[2 * j + 1] = pack2(v2, v3, p.bf16);
+                            pk[2 * j] = pack2<BF16>(v0, v1);
+                            pk[2 * j + 1] = pack2<BF16>(v2, v3);
                         }
                     } else {
 #pragma unroll
@@ -599,7 +603,9 @@ static moe_status run_gemm(const GemmParams& p, int64_t max_coltiles, cudaStream
     int dev = 0;
     cudaGetDevice(&dev);
     if (attr_dev != dev) {
-        if (cudaFuncSetAttribute(grouped_gemm_kernel<DUAL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(grouped_gemm_kernel<DUAL, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)Cfg::smem_bytes) != cudaSuccess ||
+            cudaFuncSetAttribute(grouped_gemm_kernel<DUAL, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)Cfg::smem_bytes) != cudaSuccess)
             return MOE_ERR_CUDA;
         attr_dev = dev;
@@ -608,7 +614,10 @@ static moe_status run_gemm(const GemmParams& p, int64_t max_coltiles, cudaStream
     int64_t tiles = max_coltiles * units;
     if (tiles <= 0) return MOE_OK;
     int grid = (int)(tiles < sm_count() ? tiles : sm_count());
-    grouped_gemm_kernel<DUAL><<<grid, kGemmThreads, Cfg::smem_bytes, stream>>>(p);
+    if (p.bf16)
+        grouped_gemm_kernel<DUAL, 1><<<grid, kGemmThreads, Cfg::smem_bytes, stream>>>(p);
+    else
+        grouped_gemm_kernel<DUAL, 0><<<grid, kGemmThreads, Cfg::smem_bytes, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
