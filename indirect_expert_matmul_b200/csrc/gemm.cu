@@ -179,6 +179,14 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
     return *(uint32_t*)&v;
 }
 
+// pack2 of a packed fp32 pair (low lane first)
+template <int BF16>
+__device__ __forceinline__ uint32_t pack2x(uint64_t v) {
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+    return pack2<BF16>(lo, hi);
+}
+
 // Two A operands per tile share each activation tile: DUAL=1 gate and up of
 // one 128-row tile (SwiGLU epilogue into h); DUAL=0 two consecutive 128-row
 // tiles of one matrix (fp32 scatter to dst).  BF16: operand type bf16 (1) or
@@ -196,6 +204,7 @@ grouped_gemm_kernel(const GemmParams p) {
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_dyn + 1023) & ~(uintptr_t)1023);
     uint8_t* sB = smem + Cfg::b_off;
     uint8_t* sRaw = smem + Cfg::raw_off;
+    const uint32_t raw_sa = ptx::smem_u32(sRaw);
     uint64_t* bars = (uint64_t*)(smem + Cfg::bar_off);
     uint64_t* raw_full = bars;
     uint64_t* raw_empty = raw_full + kRS;
@@ -480,32 +489,38 @@ grouped_gemm_kernel(const GemmParams p) {
                      warp_wait(&a_empty[as], aph ^ 1, abort_flag, status, STAT_PTR(1));
                 if (!ok) break;
                 ptx::tc_fence_after();
+                // both sources' bytes and scales first (shared-window loads), then the arithmetic
+                uint4 qv[2][2];
+                float dsc[2];
 #pragma unroll
                 for (int mat = 0; mat < 2; ++mat) {
                     const int nr = rows[mat];
-                    if (nr == 0) continue;
-                    const uint8_t* raw = sRaw + (rs * 2 + mat) * kRawBytes;
-                    uint32_t pk[16];
+                    qv[mat][0] = qv[mat][1] = make_uint4(0x80808080u, 0x80808080u, 0x80808080u, 0x80808080u);
+                    dsc[mat] = 0.f;
                     if (r < nr) {
-                        const uint8_t* qrow = raw + (size_t)hk * nr * 32 + r * 32;
-                        const uint4 qa = *(const uint4*)(qrow + first * 16);
-                        const uint4 qb = *(const uint4*)(qrow + (first ^ 1) * 16);
-                        const uint4 q0 = first ? qb : qa, q1 = first ? qa : qb;
-                        const float dsc = __half2float(*(const __half*)(raw + (size_t)nr * kTileK + r * 4 + hk * 2));
-                        const float nd = -32896.0f * dsc;
-                        const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+                        const uint32_t raw = raw_sa + (uint32_t)(rs * 2 + mat) * kRawBytes;
+                        const uint32_t qrow = raw + (uint32_t)(hk * nr * 32 + r * 32);
+                        const uint4 x0 = ptx::lds128(qrow + first * 16);
+                        const uint4 x1 = ptx::lds128(qrow + (first ^ 1) * 16);
+                        qv[mat][0] = first ? x1 : x0;
+                        qv[mat][1] = first ? x0 : x1;
+                        dsc[mat] = __half2float(__ushort_as_half(ptx::lds16(raw + (uint32_t)(nr * kTileK + r * 4 + hk * 2))));
+                    }
+                }
 #pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            const float v0 = fmaf(magic_byte(w[j], 0), dsc, nd);
-                            const float v1 = fmaf(magic_byte(w[j], 1), dsc, nd);
-                            const float v2 = fmaf(magic_byte(w[j], 2), dsc, nd);
-                            const float v3 = fmaf(magic_byte(w[j], 3), dsc, nd);
-                            pk[2 * j] = pack2<BF16>(v0, v1);
-                            pk[2 * j + 1] = pack2<BF16>(v2, v3);
-                        }
-                    } else {
+                for (int mat = 0; mat < 2; ++mat) {
+                    if (rows[mat] == 0) continue;
+                    const uint64_t dd = ptx::f2pack(dsc[mat], dsc[mat]);
+                    const uint64_t nd = ptx::f2pack(-32896.0f * dsc[mat], -32896.0f * dsc[mat]);
+                    const uint32_t w[8] = {qv[mat][0].x, qv[mat][0].y, qv[mat][0].z, qv[mat][0].w,
+                                           qv[mat][1].x, qv[mat][1].y, qv[mat][1].z, qv[mat][1].w};
+                    uint32_t pk[16];
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) pk[j] = 0u;
+                    for (int j = 0; j < 8; ++j) {
+                        const uint64_t v01 = ptx::fma2(ptx::f2pack(magic_byte(w[j], 0), magic_byte(w[j], 1)), dd, nd);
+                        const uint64_t v23 = ptx::fma2(ptx::f2pack(magic_byte(w[j], 2), magic_byte(w[j], 3)), dd, nd);
+                        pk[2 * j] = pack2x<BF16>(v01);
+                        pk[2 * j + 1] = pack2x<BF16>(v23);
                     }
                     ptx::tmem_st_32x32b_x16(tmem_base + lanes + kACol0 + (uint32_t)as * 64u + mat * 32 + hk * 16, pk);
                 }
