@@ -31,11 +31,14 @@
 
 namespace moe {
 
-constexpr int kGemmThreads = 512;
+constexpr int kGemmThreads = 640;
 constexpr int kWarpProdA = 0;   // weight blocks: L2 prefetch + bulk copies
 constexpr int kWarpMma = 1;     // TMEM allocation + tcgen05.mma issue
 constexpr int kWarpProdB = 2;   // activation tiles: bulk copies
-constexpr int kEpiWarp0 = 4;
+constexpr int kEpiWarp0 = 4;   // warps 4-7 and 16-19: epilogue, two per lane quarter
+constexpr int kEpiWarp1 = 16;
+constexpr int kEpiWarps = 8;
+static_assert(kGemmBN <= 6 * 32, "the epilogue holds six 32-column chunk pairs of output rows");
 constexpr int kDeqWarp0 = 8;
 constexpr int kDeqWarps = 8;
 constexpr uint32_t kBTileBytes = kGemmBN * kTileK * 2; // 24 KB
@@ -250,7 +253,7 @@ grouped_gemm_kernel(const GemmParams p) {
             ptx::mbar_init(&b_empty[i], 1);
         }
         ptx::mbar_init(tmem_full, 1);
-        ptx::mbar_init(tmem_empty, 4);
+        ptx::mbar_init(tmem_empty, kEpiWarps);
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
@@ -404,33 +407,45 @@ grouped_gemm_kernel(const GemmParams p) {
             STAT_FLUSH(2);
         }
         __syncwarp();
-    } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
+    } else if ((warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) || (warp >= kEpiWarp1 && warp < kEpiWarp1 + 4)) {
         // ------------------------------------------------------------ epilogue
-        const int ew = warp - kEpiWarp0;
+        // Two warps per tensor-memory lane quarter (warp % 4), taking alternate
+        // 16-column chunks of the tile.
+        const int eq = warp & 3, ehalf = warp >= kEpiWarp1;
         STAT_DECL
         uint32_t use = 0;
         for (int t = blockIdx.x; t < total; t += gridDim.x) {
             const Tile tl = decode_tile(t, MU, p, s_prefix, s_bounds, s_pad);
+            // output rows of this warp's chunks, fetched before the accumulators are ready
+            int orow[6];
+            if (!DUAL) {
+#pragma unroll
+                for (int q = 0; q < 6; ++q) {
+                    const int col = (2 * q + ehalf) * 16 + (lane & 15);
+                    orow[q] = -1;
+                    if (col < tl.n) orow[q] = p.dst_rows ? __ldg(p.dst_rows + tl.p0 + col) : tl.p0 + col;
+                }
+            }
             if (!warp_wait(tmem_full, use & 1, abort_flag, status, STAT_PTR(0))) break;
             use += 1;
             ptx::tc_fence_after();
-            const uint32_t lanes = (uint32_t)(32 * ew) << 16;
+            const uint32_t lanes = (uint32_t)(32 * eq) << 16;
             if (DUAL) {
-                const int m = tl.mt * kTileM + 32 * ew + lane;
+                const int m = tl.mt * kTileM + 32 * eq + lane;
                 const bool m_ok = m < L.n_out;
                 // h goes to the tile-major swizzled buffer the down GEMM streams
                 uint8_t* hplane = p.h + (size_t)(m >> 6) * p.h_rows * 128u + ((m & 7) << 1);
                 const int mchunk = (m & 63) >> 3;
-                for (int c0 = 0; c0 < tl.n; c0 += 32) {
-                    uint32_t v[32], u[32];
-                    ptx::tmem_ld_32x32b_x32(tmem_base + lanes + c0, v);
-                    ptx::tmem_ld_32x32b_x32(tmem_base + lanes + kAccCols + c0, u);
+                for (int c0 = ehalf * 16; c0 < tl.n; c0 += 32) {
+                    uint32_t v[16], u[16];
+                    ptx::tmem_ld_32x32b_x16(tmem_base + lanes + c0, v);
+                    ptx::tmem_ld_32x32b_x16(tmem_base + lanes + kAccCols + c0, u);
                     ptx::tmem_ld_wait();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
+                    for (int i = 0; i < 16; ++i) {
                         if (c0 + i < tl.n && m_ok) {
                             const float g = __uint_as_float(v[i]), up = __uint_as_float(u[i]);
-                            const float hv = g / (1.0f + __expf(-g)) * up;
+                            const float hv = __fdividef(g, 1.0f + __expf(-g)) * up;
                             const int prow = tl.p0pad + c0 + i;
                             *(__nv_bfloat16*)(hplane + (size_t)prow * 128u + ((mchunk ^ (prow & 7)) << 4)) =
                                 __float2bfloat16_rn(hv);
@@ -441,18 +456,18 @@ grouped_gemm_kernel(const GemmParams p) {
                 for (int i = 0; i < 2; ++i) {
                     const int mt = 2 * tl.mt + i;
                     if (mt >= MT) break;
-                    const int m = mt * kTileM + 32 * ew + lane;
+                    const int m = mt * kTileM + 32 * eq + lane;
                     const bool m_ok = m < L.n_out;
-                    for (int c0 = 0; c0 < tl.n; c0 += 32) {
-                        uint32_t v[32];
-                        ptx::tmem_ld_32x32b_x32(tmem_base + lanes + (uint32_t)i * kAccCols + c0, v);
-                        ptx::tmem_ld_wait();
-                        const int col = c0 + lane;
-                        int orow = -1;
-                        if (col < tl.n) orow = p.dst_rows ? __ldg(p.dst_rows + tl.p0 + col) : tl.p0 + col;
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const int r = __shfl_sync(0xffffffffu, orow, j);
+                    for (int q = 0; q < 6; ++q) {
+                        const int c0 = (2 * q + ehalf) * 16;
+                        if (c0 >= tl.n) break;
+                        uint32_t v[16];
+                        ptx::tmem_ld_32x32b_x16(tmem_base + lanes + (uint32_t)i * kAccCols + c0, v);
+                        ptx::tmem_ld_wait();
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int r = __shfl_sync(0xffffffffu, orow[q], j);
                             if (r >= 0 && m_ok) p.out[(int64_t)r * p.out_ld + m] = __uint_as_float(v[j]);
                         }
                     }
@@ -463,7 +478,7 @@ grouped_gemm_kernel(const GemmParams p) {
             if (lane == 0) ptx::mbar_arrive(tmem_empty);
         }
         if (lane == 0) STAT_FLUSH(3);
-    } else if (warp >= kDeqWarp0) {
+    } else if (warp >= kDeqWarp0 && warp < kDeqWarp0 + kDeqWarps) {
         // ------------------------------------------------------- dequantisation
         // Warp w covers rows 32*(w%4) .. +31 (its tensor-memory lane quarter)
         // and the 32-column half (w-8)/4 of each k-step: exact fp32 q*d, one
