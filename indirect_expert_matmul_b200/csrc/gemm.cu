@@ -35,12 +35,9 @@ constexpr int kGemmThreads = 640;
 constexpr int kWarpProdA = 0;   // weight blocks: L2 prefetch + bulk copies
 constexpr int kWarpMma = 1;     // TMEM allocation + tcgen05.mma issue
 constexpr int kWarpProdB = 2;   // activation tiles: bulk copies
-constexpr int kEpiWarp0 = 4;   // warps 4-7 and 16-19: epilogue, two per lane quarter
-constexpr int kEpiWarp1 = 16;
-constexpr int kEpiWarps = 8;
-static_assert(kGemmBN <= 6 * 32, "the epilogue holds six 32-column chunk pairs of output rows");
-constexpr int kDeqWarp0 = 8;
-constexpr int kDeqWarps = 8;
+constexpr int kWorkWarp0 = 4;   // warps 4-19: dequantisation and epilogue, four per lane quarter
+constexpr int kWorkWarps = 16;
+static_assert(kGemmBN <= 3 * 64, "a worker holds the output rows of three 16-column chunks");
 constexpr uint32_t kBTileBytes = kGemmBN * kTileK * 2; // 24 KB
 constexpr uint32_t kRawBytes = kTileM * kRowBytes;     // 8704
 constexpr int kSmemGroups = 512;                       // schedule tables kept in shared memory up to this
@@ -242,10 +239,10 @@ grouped_gemm_kernel(const GemmParams p) {
     if (tid == 0) {
         for (int i = 0; i < kRS; ++i) {
             ptx::mbar_init(&raw_full[i], 1);
-            ptx::mbar_init(&raw_empty[i], kDeqWarps);
+            ptx::mbar_init(&raw_empty[i], kWorkWarps);
         }
         for (int i = 0; i < kMA; ++i) {
-            ptx::mbar_init(&a_full[i], kDeqWarps);
+            ptx::mbar_init(&a_full[i], kWorkWarps);
             ptx::mbar_init(&a_empty[i], 1);
         }
         for (int i = 0; i < kMB; ++i) {
@@ -253,7 +250,7 @@ grouped_gemm_kernel(const GemmParams p) {
             ptx::mbar_init(&b_empty[i], 1);
         }
         ptx::mbar_init(tmem_full, 1);
-        ptx::mbar_init(tmem_empty, kEpiWarps);
+        ptx::mbar_init(tmem_empty, kWorkWarps);
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
@@ -407,36 +404,94 @@ grouped_gemm_kernel(const GemmParams p) {
             STAT_FLUSH(2);
         }
         __syncwarp();
-    } else if ((warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) || (warp >= kEpiWarp1 && warp < kEpiWarp1 + 4)) {
-        // ------------------------------------------------------------ epilogue
-        // Two warps per tensor-memory lane quarter (warp % 4), taking alternate
-        // 16-column chunks of the tile.
-        const int eq = warp & 3, ehalf = warp >= kEpiWarp1;
+    } else if (warp >= kWorkWarp0 && warp < kWorkWarp0 + kWorkWarps) {
+        // ---------------------------------------------- dequantisation + epilogue
+        // 16 worker warps, four per tensor-memory lane quarter (warp % 4).  In
+        // every k-step each dequantises one piece - rows 32*wq .. +31 of one
+        // source, one 32-column half - exactly (fp32 q*d, one rounding to the
+        // operand type) straight into tensor memory.  At the end of a tile the
+        // same warps run the epilogue, each on a quarter of the 16-column chunks.
+        // (Dequantisation is latency-bound per warp: more warps, not more
+        // arithmetic per warp, is what raises its rate.)
+        const int wq = warp & 3, wj = (warp - kWorkWarp0) >> 2;  // wj: piece (source, half), epilogue chunk phase
+        const int mat = wj >> 1, hk = wj & 1;
+        const int r = 32 * wq + lane;
+        const int first = (lane >> 2) & 1;  // alternate read order: conflict-free 16-byte loads
+        const uint32_t lanes = (uint32_t)(32 * wq) << 16;
         STAT_DECL
-        uint32_t use = 0;
-        for (int t = blockIdx.x; t < total; t += gridDim.x) {
+        int rs = 0, as = 0;
+        uint32_t rph = 0, aph = 0, use = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
             const Tile tl = decode_tile(t, MU, p, s_prefix, s_bounds, s_pad);
-            // output rows of this warp's chunks, fetched before the accumulators are ready
-            int orow[6];
+            int nr;
+            {
+                const uint8_t* dummy;
+                int mt;
+                source(tl, mat, dummy, nr, mt);
+            }
+            // output rows of this warp's epilogue chunks, fetched ahead of time
+            int orow[3];
             if (!DUAL) {
 #pragma unroll
-                for (int q = 0; q < 6; ++q) {
-                    const int col = (2 * q + ehalf) * 16 + (lane & 15);
+                for (int q = 0; q < 3; ++q) {
+                    const int col = (4 * q + wj) * 16 + (lane & 15);
                     orow[q] = -1;
                     if (col < tl.n) orow[q] = p.dst_rows ? __ldg(p.dst_rows + tl.p0 + col) : tl.p0 + col;
                 }
             }
-            if (!warp_wait(tmem_full, use & 1, abort_flag, status, STAT_PTR(0))) break;
+            for (int kt = 0; kt < KT; ++kt) {
+                ok = warp_wait(&raw_full[rs], rph, abort_flag, status, STAT_PTR(0)) &&
+                     warp_wait(&a_empty[as], aph ^ 1, abort_flag, status, STAT_PTR(1));
+                if (!ok) break;
+                if (nr > 0) {
+                    ptx::tc_fence_after();
+                    uint4 q0 = make_uint4(0x80808080u, 0x80808080u, 0x80808080u, 0x80808080u), q1 = q0;
+                    float dsc = 0.f;
+                    if (r < nr) {
+                        const uint32_t raw = raw_sa + (uint32_t)(rs * 2 + mat) * kRawBytes;
+                        const uint32_t qrow = raw + (uint32_t)(hk * nr * 32 + r * 32);
+                        const uint4 x0 = ptx::lds128(qrow + first * 16);
+                        const uint4 x1 = ptx::lds128(qrow + (first ^ 1) * 16);
+                        q0 = first ? x1 : x0;
+                        q1 = first ? x0 : x1;
+                        dsc = __half2float(__ushort_as_half(ptx::lds16(raw + (uint32_t)(nr * kTileK + r * 4 + hk * 2))));
+                    }
+                    const uint64_t dd = ptx::f2pack(dsc, dsc);
+                    const uint64_t nd = ptx::f2pack(-32896.0f * dsc, -32896.0f * dsc);
+                    const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const uint64_t v01 = ptx::fma2(ptx::f2pack(magic_byte(w[j], 0), magic_byte(w[j], 1)), dd, nd);
+                        const uint64_t v23 = ptx::fma2(ptx::f2pack(magic_byte(w[j], 2), magic_byte(w[j], 3)), dd, nd);
+                        pk[2 * j] = pack2x<BF16>(v01);
+                        pk[2 * j + 1] = pack2x<BF16>(v23);
+                    }
+                    ptx::tmem_st_32x32b_x16(tmem_base + lanes + kACol0 + (uint32_t)as * 64u + mat * 32 + hk * 16, pk);
+                    ptx::tmem_st_wait();
+                    ptx::tc_fence_before();
+                }
+                __syncwarp();
+                if (lane == 0) {
+                    ptx::mbar_arrive(&raw_empty[rs]);
+                    ptx::mbar_arrive(&a_full[as]);
+                }
+                if (++rs == kRS) { rs = 0; rph ^= 1; }
+                if (++as == kMA) { as = 0; aph ^= 1; }
+            }
+            if (!ok) break;
+            // ---- epilogue of this tile
+            if (!warp_wait(tmem_full, use & 1, abort_flag, status, STAT_PTR(2))) break;
             use += 1;
             ptx::tc_fence_after();
-            const uint32_t lanes = (uint32_t)(32 * eq) << 16;
             if (DUAL) {
-                const int m = tl.mt * kTileM + 32 * eq + lane;
+                const int m = tl.mt * kTileM + 32 * wq + lane;
                 const bool m_ok = m < L.n_out;
                 // h goes to the tile-major swizzled buffer the down GEMM streams
                 uint8_t* hplane = p.h + (size_t)(m >> 6) * p.h_rows * 128u + ((m & 7) << 1);
                 const int mchunk = (m & 63) >> 3;
-                for (int c0 = ehalf * 16; c0 < tl.n; c0 += 32) {
+                for (int c0 = wj * 16; c0 < tl.n; c0 += 64) {
                     uint32_t v[16], u[16];
                     ptx::tmem_ld_32x32b_x16(tmem_base + lanes + c0, v);
                     ptx::tmem_ld_32x32b_x16(tmem_base + lanes + kAccCols + c0, u);
@@ -454,21 +509,21 @@ grouped_gemm_kernel(const GemmParams p) {
                 }
             } else {
                 for (int i = 0; i < 2; ++i) {
-                    const int mt = 2 * tl.mt + i;
-                    if (mt >= MT) break;
-                    const int m = mt * kTileM + 32 * eq + lane;
+                    const int mt2 = 2 * tl.mt + i;
+                    if (mt2 >= MT) break;
+                    const int m = mt2 * kTileM + 32 * wq + lane;
                     const bool m_ok = m < L.n_out;
 #pragma unroll
-                    for (int q = 0; q < 6; ++q) {
-                        const int c0 = (2 * q + ehalf) * 16;
+                    for (int q = 0; q < 3; ++q) {
+                        const int c0 = (4 * q + wj) * 16;
                         if (c0 >= tl.n) break;
                         uint32_t v[16];
                         ptx::tmem_ld_32x32b_x16(tmem_base + lanes + (uint32_t)i * kAccCols + c0, v);
                         ptx::tmem_ld_wait();
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
-                            const int r = __shfl_sync(0xffffffffu, orow[q], j);
-                            if (r >= 0 && m_ok) p.out[(int64_t)r * p.out_ld + m] = __uint_as_float(v[j]);
+                            const int rr = __shfl_sync(0xffffffffu, orow[q], j);
+                            if (rr >= 0 && m_ok) p.out[(int64_t)rr * p.out_ld + m] = __uint_as_float(v[j]);
                         }
                     }
                 }
@@ -476,79 +531,6 @@ grouped_gemm_kernel(const GemmParams p) {
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(tmem_empty);
-        }
-        if (lane == 0) STAT_FLUSH(3);
-    } else if (warp >= kDeqWarp0 && warp < kDeqWarp0 + kDeqWarps) {
-        // ------------------------------------------------------- dequantisation
-        // Warp w covers rows 32*(w%4) .. +31 (its tensor-memory lane quarter)
-        // and the 32-column half (w-8)/4 of each k-step: exact fp32 q*d, one
-        // rounding to the operand type, written straight into tensor memory.
-        const int wq = warp & 3, hk = (warp - kDeqWarp0) >> 2;
-        const int r = 32 * wq + lane;
-        const int first = (lane >> 2) & 1;  // alternate read order: conflict-free 16-byte loads
-        const uint32_t lanes = (uint32_t)(32 * wq) << 16;
-        STAT_DECL
-        int rs = 0, as = 0;
-        uint32_t rph = 0, aph = 0;
-        bool ok = true;
-        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-            const Tile tl = decode_tile(t, MU, p, s_prefix, s_bounds, s_pad);
-            int rows[2];
-            for (int i = 0; i < 2; ++i) {
-                const uint8_t* dummy;
-                int mt;
-                source(tl, i, dummy, rows[i], mt);
-            }
-            for (int kt = 0; kt < KT; ++kt) {
-                ok = warp_wait(&raw_full[rs], rph, abort_flag, status, STAT_PTR(0)) &&
-                     warp_wait(&a_empty[as], aph ^ 1, abort_flag, status, STAT_PTR(1));
-                if (!ok) break;
-                ptx::tc_fence_after();
-                // both sources' bytes and scales first (shared-window loads), then the arithmetic
-                uint4 qv[2][2];
-                float dsc[2];
-#pragma unroll
-                for (int mat = 0; mat < 2; ++mat) {
-                    const int nr = rows[mat];
-                    qv[mat][0] = qv[mat][1] = make_uint4(0x80808080u, 0x80808080u, 0x80808080u, 0x80808080u);
-                    dsc[mat] = 0.f;
-                    if (r < nr) {
-                        const uint32_t raw = raw_sa + (uint32_t)(rs * 2 + mat) * kRawBytes;
-                        const uint32_t qrow = raw + (uint32_t)(hk * nr * 32 + r * 32);
-                        const uint4 x0 = ptx::lds128(qrow + first * 16);
-                        const uint4 x1 = ptx::lds128(qrow + (first ^ 1) * 16);
-                        qv[mat][0] = first ? x1 : x0;
-                        qv[mat][1] = first ? x0 : x1;
-                        dsc[mat] = __half2float(__ushort_as_half(ptx::lds16(raw + (uint32_t)(nr * kTileK + r * 4 + hk * 2))));
-                    }
-                }
-#pragma unroll
-                for (int mat = 0; mat < 2; ++mat) {
-                    if (rows[mat] == 0) continue;
-                    const uint64_t dd = ptx::f2pack(dsc[mat], dsc[mat]);
-                    const uint64_t nd = ptx::f2pack(-32896.0f * dsc[mat], -32896.0f * dsc[mat]);
-                    const uint32_t w[8] = {qv[mat][0].x, qv[mat][0].y, qv[mat][0].z, qv[mat][0].w,
-                                           qv[mat][1].x, qv[mat][1].y, qv[mat][1].z, qv[mat][1].w};
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const uint64_t v01 = ptx::fma2(ptx::f2pack(magic_byte(w[j], 0), magic_byte(w[j], 1)), dd, nd);
-                        const uint64_t v23 = ptx::fma2(ptx::f2pack(magic_byte(w[j], 2), magic_byte(w[j], 3)), dd, nd);
-                        pk[2 * j] = pack2x<BF16>(v01);
-                        pk[2 * j + 1] = pack2x<BF16>(v23);
-                    }
-                    ptx::tmem_st_32x32b_x16(tmem_base + lanes + kACol0 + (uint32_t)as * 64u + mat * 32 + hk * 16, pk);
-                }
-                ptx::tmem_st_wait();
-                ptx::tc_fence_before();
-                __syncwarp();
-                if (lane == 0) {
-                    ptx::mbar_arrive(&raw_empty[rs]);
-                    ptx::mbar_arrive(&a_full[as]);
-                }
-                if (++rs == kRS) { rs = 0; rph ^= 1; }
-                if (++as == kMA) { as = 0; aph ^= 1; }
-            }
         }
         if (lane == 0) STAT_FLUSH(4);
     }
