@@ -545,7 +545,10 @@ moe_status launch_gemv(const GemvArgs& in, cudaStream_t stream) {
     const bool small = S <= kGvSplitSlots;
     int chunks_r = 1, chunks_s = 1;
     if (small) {
-        chunks_r = (int)((sms + groups_r + groups_s - 1) / (groups_r + groups_s));
+        // as many chunks as fit in one wave of CTAs (a second, partial wave would
+        // double the time of the CTAs that run it)
+        chunks_r = (int)(sms / (groups_r + groups_s));
+        if (chunks_r < 1) chunks_r = 1;
         chunks_s = chunks_r > 2 * a.n_tokens ? chunks_r : 2 * a.n_tokens;
     }
     int counters = 0;
