@@ -35,12 +35,12 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 # profiles/grouped_gemm_gate_up_v3_shape_32experts.md.  It describes only the kernel
 # sources it was measured on; when any of them changes the bench reports null.
 GATE_UP_TRAFFIC = {
-    "bytes_per_launch": 8 * (1168412928 + 16517376),
+    "bytes_per_launch": 8 * (1100119808 + 16582912),
     "sources_sha256": {
-        "gemm.cu": "f6b6bbc53ad38039d5858a81fe1400005e8cf50af628b8fbc3c326444ee0a8bb",
+        "gemm.cu": "3ca9e7abf2d82acd03c96e77d4aed79a404aa447963a1f22345a222ba6dbd179",
         "gemm_api.cuh": "eee6bb8b5679e86a69cddeb281c294fcd3a03522b1b133650d1cd4bfe798c573",
         "common.cuh": "96ddf2fe1497db4e5f7ab02d2d1817a44a47549c5cbae59c2b1a3397242cc87f",
-        "ptx.cuh": "6e2b814ce63361130ffa9f366941b4db03da296fa6d5573406ff101a7368606d",
+        "ptx.cuh": "13ef7fadc6faf28e59029f6a76aadc57d333f8845fa948e909e3debccbd6bb9f",
     },
 }
 
@@ -368,7 +368,7 @@ def run_decode(moe, torch, args, hbm_peak):
     per_expert = 3 * n_embd * n_ff * Q8_BYTES_PER_W
     per_shared = 3 * n_embd * n_sh * Q8_BYTES_PER_W
     out = {}
-    for T in DEC.n_tokens:
+    for T in (DEC.n_tokens if args.decode_tokens is None else (args.decode_tokens,)):
         x = bf16_dev(torch, DEC.x(T))
         ids = [torch.from_numpy(DEC.ids(T, layer=l)).cuda() for l in range(L)]
         touched = sum(np.unique(i.cpu().numpy()).size for i in ids)
@@ -453,6 +453,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--decode-layers", type=int, default=16)
+    ap.add_argument("--decode-only", action="store_true", help="profiling only: the decode measurement alone")
+    ap.add_argument("--decode-tokens", type=int, default=None, help="profiling only: one decode token count")
     ap.add_argument("--experts", type=int, default=None, help="profiling only: fewer experts than the V3 layer")
     ap.add_argument("--tokens", type=int, default=None, help="profiling only: tokens per GPU")
     ap.add_argument("--traffic", type=float, default=None,
@@ -460,6 +462,12 @@ def main():
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)
+    elif args.decode_only:
+        import torch
+
+        import indirect_expert_matmul_b200 as moe
+        hbm_peak = load_peaks()[0]
+        print(json.dumps({"decode": run_decode(moe, torch, args, hbm_peak)}), flush=True)
     else:
         run_ours(args)
 
