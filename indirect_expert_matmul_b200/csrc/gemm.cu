@@ -162,9 +162,25 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
 // lane 0 waits, the warp learns the outcome
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status,
                                           long long* stat = nullptr) {
-    int ok = 1;
-    if ((threadIdx.x & 31) == 0) ok = wait_bar(bar, parity, abort_flag, status, stat);
-    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+    // every lane polls (no lane-0 branch); lanes that see different phases simply poll again
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (true) {
+        if (ptx::mbar_try_wait_sleep(bar, parity, kSleepNs)) {
+            if (stat) *stat += clock64() - t0;
+            return true;
+        }
+        if (*abort_flag) return false;
+        if (clock64() - t0 > kWaitLimitCycles) {
+            if ((threadIdx.x & 31) == 0) {
+                *abort_flag = 1;
+                const int site = (1 << 30) | ((int)(threadIdx.x >> 5) << 20) | (int)(ptx::smem_u32(bar) & 0xfffffu);
+                atomicCAS(status + (kHdrWaitSite - kHdrStatus), 0, site);
+                set_status(status, MOE_ERR_TIMEOUT);
+            }
+            return false;
+        }
+    }
 }
 
 // Operand type is a template parameter: a runtime choice inside the unrolled
