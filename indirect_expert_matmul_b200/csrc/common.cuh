@@ -66,7 +66,7 @@ constexpr int kGvSplitSlots = 64;
 constexpr int kGvMaxChunks = 8;
 struct WsLayout {
     int64_t S, rows_pad, rows_pad_sh;
-    size_t hdr, src1, dst, bounds, active, tiles, pad, h, h_sh, xt, xt_sh, gv_part, gv_part_sh, total;
+    size_t hdr, src1, dst, bounds, active, tiles, pad, h, h_sh, xt, xt_sh, xs, xs_sh, gv_part, gv_part_sh, total;
     static size_t up(size_t v) { return (v + 255) / 256 * 256; }
     WsLayout(int64_t n_tokens, int k, int n_experts, int n_in, int n_hidden, int n_hidden_sh, int x_type) {
         (void)x_type;
@@ -88,6 +88,8 @@ struct WsLayout {
         h_sh = o; o += up(hs_gemv > hs_gemm ? hs_gemv : hs_gemm);
         xt = o; o += up((size_t)rows_pad * kin * 128);
         xt_sh = o; o += n_hidden_sh > 0 ? up((size_t)rows_pad_sh * kin * 128) : 0;
+        xs = o; o += up((size_t)rows_pad * 4);  // power-of-two scale of each tiled activation row
+        xs_sh = o; o += n_hidden_sh > 0 ? up((size_t)rows_pad_sh * 4) : 0;
         const bool split = S <= kGvSplitSlots;
         gv_part = o; o += split ? up((size_t)kGvMaxChunks * S * ((n_hidden + 15) / 16 * 16) * 2 * 4) : 0;
         gv_part_sh = o; o += split ? up((size_t)kGvMaxChunks * n_tokens * ((n_hidden_sh + 15) / 16 * 16) * 2 * 4) : 0;

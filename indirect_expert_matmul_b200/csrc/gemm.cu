@@ -80,6 +80,7 @@ struct GemmParams {
     int out_ld;
     int* hdr;
     int bf16;                   // operand type: 1 bf16, 0 fp16
+    const float* col_scale;     // per tiled row of B (a tile column): factor the accumulator takes (null: 1)
 };
 
 struct Tile {
@@ -448,12 +449,17 @@ grouped_gemm_kernel(const GemmParams p) {
             }
             // output rows of this warp's epilogue chunks, fetched ahead of time
             int orow[3];
+            float oscale[3];
             if (!DUAL) {
 #pragma unroll
                 for (int q = 0; q < 3; ++q) {
                     const int col = (4 * q + wj) * 16 + (lane & 15);
                     orow[q] = -1;
-                    if (col < tl.n) orow[q] = p.dst_rows ? __ldg(p.dst_rows + tl.p0 + col) : tl.p0 + col;
+                    oscale[q] = 1.0f;
+                    if (col < tl.n) {
+                        orow[q] = p.dst_rows ? __ldg(p.dst_rows + tl.p0 + col) : tl.p0 + col;
+                        if (p.col_scale) oscale[q] = __ldg(p.col_scale + tl.p0pad + col);
+                    }
                 }
             }
             for (int kt = 0; kt < KT; ++kt) {
@@ -473,16 +479,35 @@ grouped_gemm_kernel(const GemmParams p) {
                         q1 = first ? x0 : x1;
                         dsc = __half2float(__ushort_as_half(ptx::lds16(raw + (uint32_t)(nr * kTileK + r * 4 + hk * 2))));
                     }
-                    const uint64_t dd = ptx::f2pack(dsc, dsc);
-                    const uint64_t nd = ptx::f2pack(-32896.0f * dsc, -32896.0f * dsc);
                     const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
                     uint32_t pk[16];
+                    if (BF16) {
+                        const uint64_t dd = ptx::f2pack(dsc, dsc);
+                        const uint64_t nd = ptx::f2pack(-32896.0f * dsc, -32896.0f * dsc);
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const uint64_t v01 = ptx::fma2(ptx::f2pack(magic_byte(w[j], 0), magic_byte(w[j], 1)), dd, nd);
-                        const uint64_t v23 = ptx::fma2(ptx::f2pack(magic_byte(w[j], 2), magic_byte(w[j], 3)), dd, nd);
-                        pk[2 * j] = pack2x<BF16>(v01);
-                        pk[2 * j + 1] = pack2x<BF16>(v23);
+                        for (int j = 0; j < 8; ++j) {
+                            const uint64_t v01 =
+                                ptx::fma2(ptx::f2pack(magic_byte(w[j], 0), magic_byte(w[j], 1)), dd, nd);
+                            const uint64_t v23 =
+                                ptx::fma2(ptx::f2pack(magic_byte(w[j], 2), magic_byte(w[j], 3)), dd, nd);
+                            pk[2 * j] = pack2x<BF16>(v01);
+                            pk[2 * j + 1] = pack2x<BF16>(v23);
+                        }
+                    } else {
+                        // fp16 pairs: {0x64, u} is 1024 + u, minus 1152 is q (exact), times d
+                        // rounds q*d once - the same value as the fp32 route rounded to fp16
+                        const __half2 d2 = __half2half2(__float2half_rn(dsc));
+                        const __half2 off = __float2half2_rn(1152.0f);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            uint32_t lo, hi;
+                            asm("prmt.b32 %0, %1, %2, 0x7170;" : "=r"(lo) : "r"(w[j]), "r"(0x64646464u));
+                            asm("prmt.b32 %0, %1, %2, 0x7372;" : "=r"(hi) : "r"(w[j]), "r"(0x64646464u));
+                            const __half2 vlo = __hmul2(__hsub2(*(const __half2*)&lo, off), d2);
+                            const __half2 vhi = __hmul2(__hsub2(*(const __half2*)&hi, off), d2);
+                            pk[2 * j] = *(const uint32_t*)&vlo;
+                            pk[2 * j + 1] = *(const uint32_t*)&vhi;
+                        }
                     }
                     ptx::tmem_st_32x32b_x16(tmem_base + lanes + kACol0 + (uint32_t)as * 64u + mat * 32 + hk * 16, pk);
                     ptx::tmem_st_wait();
@@ -511,11 +536,13 @@ grouped_gemm_kernel(const GemmParams p) {
                     uint32_t v[16], u[16];
                     ptx::tmem_ld_32x32b_x16(tmem_base + lanes + c0, v);
                     ptx::tmem_ld_32x32b_x16(tmem_base + lanes + kAccCols + c0, u);
+                    const float csc = p.col_scale && c0 + (lane & 15) < tl.n ? __ldg(p.col_scale + tl.p0pad + c0 + (lane & 15)) : 1.0f;
                     ptx::tmem_ld_wait();
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
+                        const float sc = __shfl_sync(0xffffffffu, csc, i);
                         if (c0 + i < tl.n && m_ok) {
-                            const float g = __uint_as_float(v[i]), up = __uint_as_float(u[i]);
+                            const float g = __uint_as_float(v[i]) * sc, up = __uint_as_float(u[i]) * sc;
                             const float hv = __fdividef(g, 1.0f + __expf(-g)) * up;
                             const int prow = tl.p0pad + c0 + i;
                             *(__nv_bfloat16*)(hplane + (size_t)prow * 128u + ((mchunk ^ (prow & 7)) << 4)) =
@@ -539,7 +566,8 @@ grouped_gemm_kernel(const GemmParams p) {
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
                             const int rr = __shfl_sync(0xffffffffu, orow[q], j);
-                            if (rr >= 0 && m_ok) p.out[(int64_t)rr * p.out_ld + m] = __uint_as_float(v[j]);
+                            const float sc = __shfl_sync(0xffffffffu, oscale[q], j);
+                            if (rr >= 0 && m_ok) p.out[(int64_t)rr * p.out_ld + m] = __uint_as_float(v[j]) * sc;
                         }
                     }
                 }
@@ -564,10 +592,48 @@ grouped_gemm_kernel(const GemmParams p) {
 // group e (rank r inside the group) becomes row pad_start[e] + r; k-plane kt
 // holds columns [64*kt, 64*kt + 64) as 128 bytes whose 16-byte chunk c sits at
 // chunk c ^ (row % 8).  fp32 input is rounded to fp16; columns >= n_in are 0.
+// Eight activations of row `row`, columns col .. col+7, as fp32 (zeros past n_in).
+__device__ __forceinline__ void load8(const void* x, int x_type, int64_t row, int n_in, int col, float (&e)[8]) {
+    if (col >= n_in) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) e[i] = 0.f;
+        return;
+    }
+    if (x_type == MOE_F32) {
+        const float4* src = (const float4*)((const float*)x + row * n_in + col);
+        const float4 a = __ldg(src), b = __ldg(src + 1);
+        e[0] = a.x; e[1] = a.y; e[2] = a.z; e[3] = a.w;
+        e[4] = b.x; e[5] = b.y; e[6] = b.z; e[7] = b.w;
+        return;
+    }
+    const uint4 v = __ldg((const uint4*)((const uint16_t*)x + row * n_in + col));
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t lo = w[i] & 0xffffu, hi = w[i] >> 16;
+        if (x_type == MOE_BF16) {
+            e[2 * i] = __uint_as_float(lo << 16);
+            e[2 * i + 1] = __uint_as_float(hi << 16);
+        } else {
+            e[2 * i] = __half2float(__ushort_as_half((unsigned short)lo));
+            e[2 * i + 1] = __half2float(__ushort_as_half((unsigned short)hi));
+        }
+    }
+}
+
+// Gather activation rows into the tile-major, 128-byte-swizzled fp16 layout the
+// GEMM streams with one bulk copy per k-step: the row at sorted position p of
+// group e (rank r inside the group) becomes row pad_start[e] + r; k-plane kt
+// holds columns [64*kt, 64*kt + 64) as 128 bytes whose 16-byte chunk c sits at
+// chunk c ^ (row % 8); columns >= n_in are 0.  Each row is multiplied by the
+// power of two 2^-e that puts its largest magnitude in [2^14, 2^15) - exact,
+// and inside the fp16 range whatever the input type - and xs[row] = 2^e is what
+// the GEMM epilogue multiplies that token's results by.
 __global__ void __launch_bounds__(256)
 gather_tiled_kernel(const void* __restrict__ x, int x_type, int n_in, int KT, const int32_t* __restrict__ src_rows,
                     const int32_t* __restrict__ bounds, const int32_t* __restrict__ pad_start, int n_groups,
-                    int64_t n_rows, int64_t rows_pad, uint8_t* __restrict__ xt, const int* __restrict__ hdr) {
+                    int64_t n_rows, int64_t rows_pad, uint8_t* __restrict__ xt, float* __restrict__ xs,
+                    const int* __restrict__ hdr) {
     if (read_status(hdr + kHdrStatus) != 0) return;
     const int lane = threadIdx.x & 31;
     const int64_t S = n_groups > 0 ? bounds[n_groups] : n_rows;
@@ -583,21 +649,34 @@ gather_tiled_kernel(const void* __restrict__ x, int x_type, int n_in, int KT, co
             prow = __ldg(pad_start + lo) + (p - __ldg(bounds + lo));
             srow = src_rows ? __ldg(src_rows + p) : p;
         }
+        float mx = 0.f;
         for (int seg = lane; seg < KT * 8; seg += 32) {
-            const int kt = seg >> 3, c = seg & 7, col = kt * 64 + c * 8;
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (col < n_in) {
-                if (x_type == MOE_F32) {
-                    const float4* src = (const float4*)((const float*)x + srow * n_in + col);
-                    const float4 a = __ldg(src), b = __ldg(src + 1);
-                    __half2 h0 = __floats2half2_rn(a.x, a.y), h1 = __floats2half2_rn(a.z, a.w);
-                    __half2 h2 = __floats2half2_rn(b.x, b.y), h3 = __floats2half2_rn(b.z, b.w);
-                    v = make_uint4(*(uint32_t*)&h0, *(uint32_t*)&h1, *(uint32_t*)&h2, *(uint32_t*)&h3);
-                } else {
-                    v = __ldg((const uint4*)((const uint16_t*)x + srow * n_in + col));
-                }
+            float e[8];
+            load8(x, x_type, srow, n_in, (seg >> 3) * 64 + (seg & 7) * 8, e);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(e[i]));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        int ex = 0;
+        if (mx > 0.f && mx <= 3.402823466e38f) {
+            ex = ilogbf(mx) - 14;
+            ex = ex < -100 ? -100 : ex;
+        }
+        const float sc = ldexpf(1.0f, -ex);
+        if (lane == 0) xs[prow] = ldexpf(1.0f, ex);
+        for (int seg = lane; seg < KT * 8; seg += 32) {
+            const int kt = seg >> 3, c = seg & 7;
+            float e[8];
+            load8(x, x_type, srow, n_in, kt * 64 + c * 8, e);
+            uint32_t h[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const __half2 v2 = __floats2half2_rn(e[2 * i] * sc, e[2 * i + 1] * sc);
+                h[i] = *(const uint32_t*)&v2;
             }
-            *(uint4*)(xt + ((size_t)kt * rows_pad + prow) * 128u + ((c ^ (int)(prow & 7)) << 4)) = v;
+            *(uint4*)(xt + ((size_t)kt * rows_pad + prow) * 128u + ((c ^ (int)(prow & 7)) << 4)) =
+                make_uint4(h[0], h[1], h[2], h[3]);
         }
     }
 }
@@ -652,20 +731,20 @@ static moe_status run_gemm(const GemmParams& p, int64_t max_coltiles, cudaStream
 static int64_t coltile_bound(int64_t S, int E) { return (S + kGemmBN - 1) / kGemmBN + (S < E ? S : E); }
 
 static moe_status gather(const void* x, int x_type, int n_in, const int32_t* src_rows, const int32_t* bounds,
-                         const int32_t* pad_start, int n_groups, int64_t rows, int64_t rows_pad, void* xt, int* hdr,
-                         cudaStream_t s) {
+                         const int32_t* pad_start, int n_groups, int64_t rows, int64_t rows_pad, void* xt, float* xs,
+                         int* hdr, cudaStream_t s) {
     const int KT = (n_in + kTileK - 1) / kTileK;
     int64_t blocks = (rows + 7) / 8;
     if (blocks > (int64_t)sm_count() * 8) blocks = (int64_t)sm_count() * 8;
     if (blocks < 1) blocks = 1;
     gather_tiled_kernel<<<(unsigned)blocks, 256, 0, s>>>(x, x_type, n_in, KT, src_rows, bounds, pad_start, n_groups,
-                                                         rows, rows_pad, (uint8_t*)xt, hdr);
+                                                         rows, rows_pad, (uint8_t*)xt, xs, hdr);
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 moe_status launch_gemm_mul_mat_id(const GemmMulMatId& g, cudaStream_t stream) {
     moe_status st = gather(g.x, g.x_type, g.n_in, g.ids_src1, g.bounds, g.pad_start, g.E, g.S, g.rows_pad, g.xt,
-                           g.hdr, stream);
+                           g.xs, g.hdr, stream);
     if (st) return st;
     prof_mark(stream, "gather");
     GemmParams p = {};
@@ -681,17 +760,17 @@ moe_status launch_gemm_mul_mat_id(const GemmMulMatId& g, cudaStream_t stream) {
     p.out = g.dst;
     p.out_ld = g.n_out;
     p.hdr = g.hdr;
-    p.bf16 = g.x_type == MOE_BF16;
+    p.bf16 = 0;  // fp16 activation tiles (scaled rows)
+    p.col_scale = g.xs;
     st = run_gemm<0>(p, coltile_bound(g.S, g.E), stream);
     prof_mark(stream, "gemm");
     return st;
 }
 
 moe_status launch_gemm_ffn(const GemmFfn& g, cudaStream_t stream) {
-    const int bf16 = g.x_type == MOE_BF16;
     const int kt_ff = (g.n_ff + kTileK - 1) / kTileK;
     moe_status st = gather(g.x, g.x_type, g.n_embd, g.ids_src1, g.bounds, g.pad_start, g.E, g.S, g.rows_pad, g.xt,
-                           g.hdr, stream);
+                           g.xs, g.hdr, stream);
     if (st) return st;
     prof_mark(stream, "gather");
     if (g.n_ff % kTileK) {  // columns past n_ff of the last k-plane of h are read by the down GEMM: keep them 0
@@ -714,13 +793,15 @@ moe_status launch_gemm_ffn(const GemmFfn& g, cudaStream_t stream) {
     p.h_rows = g.rows_pad;
     p.out_ld = g.n_ff;
     p.hdr = g.hdr;
-    p.bf16 = bf16;
+    p.bf16 = 0;  // fp16 activation tiles (scaled rows)
+    p.col_scale = g.xs;
     st = run_gemm<1>(p, coltile_bound(g.S, g.E), stream);
     if (st) return st;
     prof_mark(stream, "gemm_gate_up");
     const int kt_sh = (g.n_ff_shared + kTileK - 1) / kTileK;
     if (g.n_ff_shared > 0) {
-        st = gather(g.x, g.x_type, g.n_embd, nullptr, nullptr, nullptr, 0, g.T, g.rows_pad_sh, g.xt_sh, g.hdr, stream);
+        st = gather(g.x, g.x_type, g.n_embd, nullptr, nullptr, nullptr, 0, g.T, g.rows_pad_sh, g.xt_sh, g.xs_sh,
+                    g.hdr, stream);
         if (st) return st;
         if (g.n_ff_shared % kTileK) {
             if (cudaMemsetAsync((uint8_t*)g.h_sh + (size_t)(kt_sh - 1) * g.rows_pad_sh * 128u, 0,
@@ -738,7 +819,8 @@ moe_status launch_gemm_ffn(const GemmFfn& g, cudaStream_t stream) {
         q.h_rows = g.rows_pad_sh;
         q.out_ld = g.n_ff_shared;
         q.hdr = g.hdr;
-        q.bf16 = bf16;
+        q.bf16 = 0;
+        q.col_scale = g.xs_sh;
         st = run_gemm<1>(q, (g.T + kGemmBN - 1) / kGemmBN, stream);
         if (st) return st;
         prof_mark(stream, "gemm_shared_gate_up");

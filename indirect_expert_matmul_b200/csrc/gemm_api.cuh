@@ -10,7 +10,8 @@ struct GemmMulMatId {
     const void* x;
     int x_type;
     int64_t x_rows;   // rows of x: n_tokens (broadcast) or n_tokens*k (per_slot)
-    void* xt;         // workspace: gathered x, tile-major and swizzled (rows_pad rows)
+    void* xt;         // workspace: gathered x, tile-major and swizzled (rows_pad rows), fp16
+    float* xs;        // workspace: per tiled row, the power of two that undoes its scaling
     int64_t rows_pad;
     const int32_t* pad_start;
     int64_t S;
@@ -29,8 +30,10 @@ struct GemmFfn {
     int n_ff_shared;
     const void* x;
     int x_type;
-    void* xt;         // gathered x (routed), tile-major and swizzled
-    void* xt_sh;      // x in token order for the shared expert
+    void* xt;         // gathered x (routed), tile-major and swizzled, fp16
+    void* xt_sh;      // x in token order for the shared expert, fp16
+    float* xs;        // per tiled row of xt / xt_sh: the power of two that undoes its scaling
+    float* xs_sh;
     int64_t rows_pad, rows_pad_sh;
     const int32_t* pad_start;
     int64_t T, S;

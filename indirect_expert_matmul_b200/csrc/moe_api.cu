@@ -158,6 +158,7 @@ moe_status moe_mul_mat_id(const void* W_prepared, int n_experts, int n_out, int 
     g.x_type = x_type;
     g.x_rows = mode == MOE_BROADCAST ? n_tokens : S;
     g.xt = ws + W.xt;
+    g.xs = (float*)(ws + W.xs);
     g.rows_pad = W.rows_pad;
     g.pad_start = (const int32_t*)(ws + W.pad);
     g.S = S;
@@ -280,6 +281,8 @@ moe_status moe_ffn(const void* Wg, const void* Wu, const void* Wd, int n_experts
     g.x_type = x_type;
     g.xt = ws + W.xt;
     g.xt_sh = ws + W.xt_sh;
+    g.xs = (float*)(ws + W.xs);
+    g.xs_sh = (float*)(ws + W.xs_sh);
     g.rows_pad = W.rows_pad;
     g.rows_pad_sh = W.rows_pad_sh;
     g.pad_start = (const int32_t*)(ws + W.pad);

@@ -135,6 +135,26 @@ def test_f32_activations_ffn(path):
     check_close(dst.reshape(T * k, n_embd), ref, tol, f"f32 ffn path {path}")
 
 
+@pytest.mark.parametrize("x_type", ["bf16", "f32"])
+def test_gemm_rows_far_from_unit_scale(x_type):
+    """The GEMM path stores activations as fp16 after scaling each row by a power
+    of two; rows near 2^20 (beyond the fp16 range unscaled), rows near 2^-20 and
+    an all-zero row still agree with the oracle element by element."""
+    E, k, T, n_in, n_out = 6, 2, 40, 256, 192
+    W = workloads.q8_0_weights(E, n_out, n_in, 11, 1)
+    x = workloads.activations(T, n_in, x_type, 11, 2)
+    f = x.astype(np.uint32).__lshift__(16).view(np.float32) if x_type == "bf16" else x.copy()
+    for t in range(T):
+        f[t] *= {1: 2.0 ** 20, 2: 2.0 ** -20}.get(t % 4, 1.0) if t != 3 else 0.0
+    x = (f.view(np.uint32) >> 16).astype(np.uint16) if x_type == "bf16" else f.astype(np.float32)
+    ids = workloads.routing("uniform", T, E, k, 11)
+    ref, tol = oracle.mul_mat_id(W, x, x_type, ids)
+    with paths(2):
+        dst = moe.mul_mat_id(prep(W), E, n_out, n_in, to_dev_x(x, x_type), torch.from_numpy(ids).cuda())
+    check_close(dst, ref, tol, f"scaled rows {x_type}")
+    assert np.all(ref[3] == 0) and float(dst[3].abs().max()) == 0.0
+
+
 def test_gemm_is_repeatable():
     wl = workloads.WORKLOADS["tiny"]
     W = workloads.q8_0_weights(wl.n_experts, wl.n_out, wl.n_in, wl.seed, workloads.T_W)
