@@ -35,11 +35,11 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 # profiles/grouped_gemm_gate_up_v3_shape_32experts.md.  It describes only the kernel
 # sources it was measured on; when any of them changes the bench reports null.
 GATE_UP_TRAFFIC = {
-    "bytes_per_launch": 8 * (1100119808 + 16582912),
+    "bytes_per_launch": 8 * (1103577344 + 16493568),
     "sources_sha256": {
-        "gemm.cu": "3ca9e7abf2d82acd03c96e77d4aed79a404aa447963a1f22345a222ba6dbd179",
-        "gemm_api.cuh": "eee6bb8b5679e86a69cddeb281c294fcd3a03522b1b133650d1cd4bfe798c573",
-        "common.cuh": "96ddf2fe1497db4e5f7ab02d2d1817a44a47549c5cbae59c2b1a3397242cc87f",
+        "gemm.cu": "a19ec5a686425844b2490fe62449589a8a671716d54f5134fa78ff8c3b458bee",
+        "gemm_api.cuh": "640350de47f592462e8f6833a3d97ecc1aca101afc65d89f35685ade1cb3cc78",
+        "common.cuh": "480438163b25ce334fe7c403f5a3d6869cc5661f046be943194a695426eba16d",
         "ptx.cuh": "13ef7fadc6faf28e59029f6a76aadc57d333f8845fa948e909e3debccbd6bb9f",
     },
 }
@@ -293,10 +293,12 @@ def run_ours(args):
     result = {
         "metric": METRIC, "value": round(T * world / (ms * 1e-3), 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16+bf16", "data": "synthetic",
         "config": {"workload": ("v3 moe_ffn: 256 experts top-8, n_embd 7168, expert ffn 2048, Q8_0 gate/up/down, "
                                 "bf16 x, 4096 tokens per GPU, biased top-8 routing") if not small else
                                f"profiling case (not a bench line): v3 shape with {E} experts, {T} tokens",
+                   "arithmetic": "gate/up: fp16 operands (activation rows scaled by exact powers of two), "
+                                 "down: bf16 operands; Q8_0 dequantised exactly then rounded once; fp32 accumulation",
                    "tokens_per_gpu": T, "experts_touched": int(used),
                    "l2": "inputs larger than L2 (12 GB of weights per step)", "parallelism": f"dp{world}"},
         "tflops": round(step_flops * world / (ms * 1e-3) / 1e12, 1),

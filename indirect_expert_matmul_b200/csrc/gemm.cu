@@ -447,19 +447,17 @@ grouped_gemm_kernel(const GemmParams p) {
                 int mt;
                 source(tl, mat, dummy, nr, mt);
             }
-            // output rows of this warp's epilogue chunks, fetched ahead of time
+            // output rows and column scales of this warp's epilogue chunks, fetched ahead of time
             int orow[3];
             float oscale[3];
-            if (!DUAL) {
 #pragma unroll
-                for (int q = 0; q < 3; ++q) {
-                    const int col = (4 * q + wj) * 16 + (lane & 15);
-                    orow[q] = -1;
-                    oscale[q] = 1.0f;
-                    if (col < tl.n) {
-                        orow[q] = p.dst_rows ? __ldg(p.dst_rows + tl.p0 + col) : tl.p0 + col;
-                        if (p.col_scale) oscale[q] = __ldg(p.col_scale + tl.p0pad + col);
-                    }
+            for (int q = 0; q < 3; ++q) {
+                const int col = (4 * q + wj) * 16 + (lane & 15);
+                orow[q] = -1;
+                oscale[q] = 1.0f;
+                if (col < tl.n) {
+                    if (!DUAL) orow[q] = p.dst_rows ? __ldg(p.dst_rows + tl.p0 + col) : tl.p0 + col;
+                    if (p.col_scale) oscale[q] = __ldg(p.col_scale + tl.p0pad + col);
                 }
             }
             for (int kt = 0; kt < KT; ++kt) {
@@ -532,15 +530,17 @@ grouped_gemm_kernel(const GemmParams p) {
                 // h goes to the tile-major swizzled buffer the down GEMM streams
                 uint8_t* hplane = p.h + (size_t)(m >> 6) * p.h_rows * 128u + ((m & 7) << 1);
                 const int mchunk = (m & 63) >> 3;
-                for (int c0 = wj * 16; c0 < tl.n; c0 += 64) {
+#pragma unroll
+                for (int q = 0; q < 3; ++q) {
+                    const int c0 = (4 * q + wj) * 16;
+                    if (c0 >= tl.n) break;
                     uint32_t v[16], u[16];
                     ptx::tmem_ld_32x32b_x16(tmem_base + lanes + c0, v);
                     ptx::tmem_ld_32x32b_x16(tmem_base + lanes + kAccCols + c0, u);
-                    const float csc = p.col_scale && c0 + (lane & 15) < tl.n ? __ldg(p.col_scale + tl.p0pad + c0 + (lane & 15)) : 1.0f;
                     ptx::tmem_ld_wait();
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        const float sc = __shfl_sync(0xffffffffu, csc, i);
+                        const float sc = __shfl_sync(0xffffffffu, oscale[q], i);
                         if (c0 + i < tl.n && m_ok) {
                             const float g = __uint_as_float(v[i]) * sc, up = __uint_as_float(u[i]) * sc;
                             const float hv = __fdividef(g, 1.0f + __expf(-g)) * up;
