@@ -4,25 +4,28 @@
 // sections 2.1 and 6: gather src1 rows by ids_src1, multiply per expert, write
 // dst rows by ids_dst), restated for Blackwell.
 //
-// Tile = (expert e, column tile j of up to 256 of the expert's sorted slots,
-// row tile mt of 128 output rows).  One persistent CTA per SM walks tiles in
-// (e, j, mt) order, so CTAs running together share the gathered activations
-// (and an expert's later column tiles find its weights in L2).  Every output
-// element is produced by exactly one CTA with one fixed reduction order: the
-// result is bit-identical from run to run.
+// Tile = (expert e, column tile j of up to 192 of the expert's sorted slots,
+// row unit mt).  One persistent CTA per SM walks tiles in (e, j, mt) order, so
+// CTAs running together share the gathered activations (and an expert's later
+// column tiles find its weights in L2).  Every output element is produced by
+// exactly one CTA with one fixed reduction order: the result is bit-identical
+// from run to run.
 //
-// Warp roles (512 threads):
-//   warp 0      producer: 1-D bulk copies of the repacked int8+scale weight
-//               blocks, and TMA tile::gather4 loads of the activation rows
-//               named by the row table (4 rows per instruction, 32 lanes
-//               issuing in parallel).
+// Both operands come from shared memory (128-byte-swizzled, K-major); the two
+// fp32 accumulators live in tensor memory.  Warp roles (768 threads):
+//   warp 0      weight producer: L2 prefetch and 1-D bulk copies of the
+//               repacked int8+scale blocks of both A sources.
 //   warp 1      TMEM allocation and the single thread issuing tcgen05.mma
-//               (M=128, N=16..256, K=16 per instruction, fp32 accumulators).
-//   warps 4-7   epilogue: tcgen05.ld of the accumulators; scatter fp32 rows to
-//               dst by ids_dst, or SwiGLU of the gate/up pair to bf16 h.
-//   warps 8-15  dequantisation: int8 q + fp16 d in shared memory -> exact fp32
-//               q*d -> bf16 or fp16, written in the 128-byte-swizzled K-major
-//               layout the tensor core reads.
+//               (M=128, N=16..192, K=16 per instruction).  Its sub-partition
+//               runs no arithmetic: work there stretches every k-step.
+//   warp 2      activation producer: one bulk copy per k-step of the
+//               pre-swizzled, tile-major activation rows.
+//   warps 3-23 but 5, 9, 13, 17, 21 (16 warps on sub-partitions 0, 2, 3):
+//               dequantisation, int8 q + fp16 d -> q*d rounded once to the
+//               operand type, stored in the layout the tensor core reads.
+//   warps 4-19  epilogue, four per tensor-memory lane quarter (warp % 4):
+//               tcgen05.ld of the accumulators; SwiGLU of the gate/up pair to
+//               bf16 h, or fp32 rows scattered to dst by ids_dst.
 // All waits are bounded; an expired wait sets MOE_ERR_TIMEOUT in the status
 // word and every role leaves its loop.
 #include "common.cuh"
@@ -31,31 +34,40 @@
 
 namespace moe {
 
-constexpr int kGemmThreads = 640;
+constexpr int kGemmThreads = 768;
 constexpr int kWarpProdA = 0;   // weight blocks: L2 prefetch + bulk copies
 constexpr int kWarpMma = 1;     // TMEM allocation + tcgen05.mma issue
 constexpr int kWarpProdB = 2;   // activation tiles: bulk copies
-constexpr int kWorkWarp0 = 4;   // warps 4-19: dequantisation and epilogue, four per lane quarter
+constexpr int kWorkWarp0 = 4;   // warps 4-19: epilogue, four per lane quarter
 constexpr int kWorkWarps = 16;
+constexpr int kDeqWarps = 16;   // warps 3-23 off the MMA warp's sub-partition: dequantisation
+// Dequantisation warp index 0..15 of warp w, or -1 (the MMA warp's sub-partition, w % 4 == 1,
+// is left to tcgen05.mma issue: arithmetic there stretches every k-step).
+__host__ __device__ constexpr int deq_index(int w) {
+    return (w < 3 || w > 23 || (w & 3) == 1) ? -1 : (w - 3) - ((w - 3 + 2) >> 2);
+}
 static_assert(kGemmBN <= 3 * 64, "a worker holds the output rows of three 16-column chunks");
 constexpr uint32_t kBTileBytes = kGemmBN * kTileK * 2; // 24 KB
 constexpr uint32_t kRawBytes = kTileM * kRowBytes;     // 8704
-constexpr int kSmemGroups = 512;                       // schedule tables kept in shared memory up to this
+constexpr int kSmemGroups = 256;                       // schedule tables kept in shared memory up to this
 constexpr int kPrefetchSteps = 8;                      // weight k-steps prefetched into L2 ahead of use
 constexpr long long kWaitLimitCycles = 1ll << 32;      // ~2 s
 constexpr uint32_t kSleepNs = 20000;                   // upper bound of one hardware wait
-// Tensor memory (512 columns): two fp32 accumulators of kGemmBN columns, then
-// the dequantised A operand, kMA stages of two 32-column matrices each.
+// Tensor memory (512 columns): two fp32 accumulators of kGemmBN columns.
 constexpr uint32_t kAccCols = kGemmBN;
-constexpr uint32_t kACol0 = 2 * kAccCols;
-constexpr int kMA = (512 - (int)kACol0) / 64;
-static_assert(kMA >= 2, "tensor memory holds at least two A stages");
+constexpr int kMA = 2;   // dequantised A stages in shared memory: two 128 x 64 matrices, SW128 K-major
+constexpr uint32_t kATileBytes = kTileM * kTileK * 2;  // 16 KB per matrix
 constexpr int kRS = 4;   // raw weight stages (int8 + scales of both matrices)
-constexpr int kMB = 5;   // activation (B) stages
+constexpr int kMB = 3;   // activation (B) stages
+// Dequantisation warps take alternate k-steps by parity: with an even number
+// of raw and A stages every stage is always filled and drained by the same
+// group, so no group can mistake another phase of a stage for its own.
+static_assert(kRS % 2 == 0 && kMA % 2 == 0, "ring stages are owned by one k-step parity");
 
 struct Cfg {
     static constexpr uint32_t b_off = 0;
-    static constexpr uint32_t raw_off = b_off + kMB * kBTileBytes;
+    static constexpr uint32_t a_off = b_off + kMB * kBTileBytes;
+    static constexpr uint32_t raw_off = a_off + kMA * 2 * kATileBytes;
     static constexpr uint32_t bar_off = raw_off + kRS * 2 * kRawBytes;
     static constexpr int n_bars = 2 * kRS + 2 * kMA + 2 * kMB + 2;
     static constexpr uint32_t misc_off = bar_off + n_bars * 8;
@@ -208,6 +220,40 @@ __device__ __forceinline__ uint32_t pack2x(uint64_t v) {
 // one 128-row tile (SwiGLU epilogue into h); DUAL=0 two consecutive 128-row
 // tiles of one matrix (fp32 scatter to dst).  BF16: operand type bf16 (1) or
 // fp16 (0), which must equal p.bf16.
+// 16 quantised bytes (16 consecutive K values of one row) -> two 16-byte
+// chunks of operand values, exact: q*d rounded once to the operand type.
+// d2: the row's fp16 scale in both halves (fp16 route); dsc: the same as fp32.
+template <int BF16>
+__device__ __forceinline__ void dequant16_sts(uint4 x, uint32_t d2, float dsc, uint32_t dst0, uint32_t dst1) {
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+    uint32_t pk[8];
+    if (BF16) {
+        const uint64_t dd = ptx::f2pack(dsc, dsc);
+        const uint64_t nd = ptx::f2pack(-32896.0f * dsc, -32896.0f * dsc);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            pk[2 * j] = pack2x<BF16>(ptx::fma2(ptx::f2pack(magic_byte(w[j], 0), magic_byte(w[j], 1)), dd, nd));
+            pk[2 * j + 1] = pack2x<BF16>(ptx::fma2(ptx::f2pack(magic_byte(w[j], 2), magic_byte(w[j], 3)), dd, nd));
+        }
+    } else {
+        // {0x64, u} is the fp16 value 1024 + u; minus 1152 is q (exact); times d rounds once
+        const __half2 off = __float2half2_rn(1152.0f);
+        const __half2 d = *(const __half2*)&d2;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            uint32_t lo, hi;
+            asm("prmt.b32 %0, %1, %2, 0x7170;" : "=r"(lo) : "r"(w[j]), "r"(0x64646464u));
+            asm("prmt.b32 %0, %1, %2, 0x7372;" : "=r"(hi) : "r"(w[j]), "r"(0x64646464u));
+            const __half2 vlo = __hmul2(__hsub2(*(const __half2*)&lo, off), d);
+            const __half2 vhi = __hmul2(__hsub2(*(const __half2*)&hi, off), d);
+            pk[2 * j] = *(const uint32_t*)&vlo;
+            pk[2 * j + 1] = *(const uint32_t*)&vhi;
+        }
+    }
+    ptx::sts128(dst0, make_uint4(pk[0], pk[1], pk[2], pk[3]));
+    ptx::sts128(dst1, make_uint4(pk[4], pk[5], pk[6], pk[7]));
+}
+
 template <int DUAL, int BF16>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 grouped_gemm_kernel(const GemmParams p) {
@@ -221,6 +267,7 @@ grouped_gemm_kernel(const GemmParams p) {
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_dyn + 1023) & ~(uintptr_t)1023);
     uint8_t* sB = smem + Cfg::b_off;
     uint8_t* sRaw = smem + Cfg::raw_off;
+    const uint32_t a_sa = ptx::smem_u32(smem + Cfg::a_off);
     const uint32_t raw_sa = ptx::smem_u32(sRaw);
     uint64_t* bars = (uint64_t*)(smem + Cfg::bar_off);
     uint64_t* raw_full = bars;
@@ -256,10 +303,10 @@ grouped_gemm_kernel(const GemmParams p) {
     if (tid == 0) {
         for (int i = 0; i < kRS; ++i) {
             ptx::mbar_init(&raw_full[i], 1);
-            ptx::mbar_init(&raw_empty[i], kWorkWarps);
+            ptx::mbar_init(&raw_empty[i], kDeqWarps / 2);
         }
         for (int i = 0; i < kMA; ++i) {
-            ptx::mbar_init(&a_full[i], kWorkWarps);
+            ptx::mbar_init(&a_full[i], kDeqWarps / 2);
             ptx::mbar_init(&a_empty[i], 1);
         }
         for (int i = 0; i < kMB; ++i) {
@@ -379,8 +426,8 @@ grouped_gemm_kernel(const GemmParams p) {
         }
     } else if (warp == kWarpMma) {
         // ----------------------------------------------------------------- MMA
-        // A from tensor memory, B from shared memory; the two accumulators'
-        // instructions interleave so neither chain waits on itself.
+        // A and B from shared memory; the two accumulators' instructions
+        // interleave so neither chain waits on itself.
         if (lane == 0) {
             STAT_DECL
             int as = 0, bs = 0;
@@ -400,14 +447,14 @@ grouped_gemm_kernel(const GemmParams p) {
                          wait_bar(&b_full[bs], bph, abort_flag, status, STAT_PTR(1));
                     if (!ok) break;
                     ptx::tc_fence_after();
-                    const uint32_t a0 = tmem_base + kACol0 + (uint32_t)as * 64u;
+                    const uint32_t a0 = a_sa + (uint32_t)as * 2u * kATileBytes;
                     const uint32_t b = ptx::smem_u32(sB + bs * kBTileBytes);
 #pragma unroll
                     for (int kk = 0; kk < kTileK / 16; ++kk) {
                         const uint32_t acc = (kt | kk) != 0;
                         const uint64_t bd = ptx::desc_k_sw128(b + kk * 32);
-                        ptx::mma_f16_ts(d0, a0 + kk * 8, bd, idesc, acc);
-                        if (has1) ptx::mma_f16_ts(d1, a0 + 32 + kk * 8, bd, idesc, acc);
+                        ptx::mma_f16_ss(d0, ptx::desc_k_sw128(a0 + kk * 32), bd, idesc, acc);
+                        if (has1) ptx::mma_f16_ss(d1, ptx::desc_k_sw128(a0 + kATileBytes + kk * 32), bd, idesc, acc);
                     }
                     ptx::mma_commit(&a_empty[as]);
                     ptx::mma_commit(&b_empty[bs]);
@@ -421,32 +468,30 @@ grouped_gemm_kernel(const GemmParams p) {
             STAT_FLUSH(2);
         }
         __syncwarp();
-    } else if (warp >= kWorkWarp0 && warp < kWorkWarp0 + kWorkWarps) {
-        // ---------------------------------------------- dequantisation + epilogue
-        // 16 worker warps, four per tensor-memory lane quarter (warp % 4).  In
-        // every k-step each dequantises one piece - rows 32*wq .. +31 of one
-        // source, one 32-column half - exactly (fp32 q*d, one rounding to the
-        // operand type) straight into tensor memory.  At the end of a tile the
-        // same warps run the epilogue, each on a quarter of the 16-column chunks.
-        // (Dequantisation is latency-bound per warp: more warps, not more
-        // arithmetic per warp, is what raises its rate.)
-        const int wq = warp & 3, wj = (warp - kWorkWarp0) >> 2;  // wj: piece (source, half), epilogue chunk phase
-        const int mat = wj >> 1, hk = wj & 1;
-        const int r = 32 * wq + lane;
+    } else if (deq_index(warp) >= 0 || (warp >= kWorkWarp0 && warp < kWorkWarp0 + kWorkWarps)) {
+        // ------------------------------------- dequantisation and epilogue warps
+        // Dequantisation (16 warps on sub-partitions 0, 2, 3, two groups of eight
+        // taking alternate k-steps): each warp converts 32 rows of one source,
+        // all 64 columns, exactly (q*d rounded once to the operand type) into the
+        // SW128 K-major A stage in shared memory.  Epilogue (warps 4-19, four per
+        // tensor-memory lane quarter warp % 4): at the end of a tile each drains a
+        // quarter of the 16-column chunks of its lanes; warps 5, 9, 13, 17 do only
+        // this.
+        const int di = deq_index(warp);
+        const bool epi = warp >= kWorkWarp0 && warp < kWorkWarp0 + kWorkWarps;
+        const int wq = warp & 3, wj = (warp - kWorkWarp0) >> 2;  // epilogue lane quarter, chunk phase
+        const int kpar = di >> 3, mat = (di >> 2) & 1;
+        const int r = 32 * (di & 3) + lane;
         const int first = (lane >> 2) & 1;  // alternate read order: conflict-free 16-byte loads
         const uint32_t lanes = (uint32_t)(32 * wq) << 16;
+        const uint32_t a_row = (uint32_t)mat * kATileBytes + (uint32_t)(r >> 3) * 1024u + (uint32_t)(r & 7) * 128u;
+        const uint32_t rx = (uint32_t)(r & 7);
         STAT_DECL
         int rs = 0, as = 0;
         uint32_t rph = 0, aph = 0, use = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
             const Tile tl = decode_tile(t, MU, p, s_prefix, s_bounds, s_pad);
-            int nr;
-            {
-                const uint8_t* dummy;
-                int mt;
-                source(tl, mat, dummy, nr, mt);
-            }
             // output rows and column scales of this warp's epilogue chunks, fetched ahead of time
             int orow[3];
             float oscale[3];
@@ -455,71 +500,66 @@ grouped_gemm_kernel(const GemmParams p) {
                 const int col = (4 * q + wj) * 16 + (lane & 15);
                 orow[q] = -1;
                 oscale[q] = 1.0f;
-                if (col < tl.n) {
+                if (epi && col < tl.n) {
                     if (!DUAL) orow[q] = p.dst_rows ? __ldg(p.dst_rows + tl.p0 + col) : tl.p0 + col;
                     if (p.col_scale) oscale[q] = __ldg(p.col_scale + tl.p0pad + col);
                 }
             }
-            for (int kt = 0; kt < KT; ++kt) {
-                ok = warp_wait(&raw_full[rs], rph, abort_flag, status, STAT_PTR(0)) &&
-                     warp_wait(&a_empty[as], aph ^ 1, abort_flag, status, STAT_PTR(1));
-                if (!ok) break;
-                if (nr > 0) {
-                    ptx::tc_fence_after();
-                    uint4 q0 = make_uint4(0x80808080u, 0x80808080u, 0x80808080u, 0x80808080u), q1 = q0;
-                    float dsc = 0.f;
-                    if (r < nr) {
-                        const uint32_t raw = raw_sa + (uint32_t)(rs * 2 + mat) * kRawBytes;
-                        const uint32_t qrow = raw + (uint32_t)(hk * nr * 32 + r * 32);
-                        const uint4 x0 = ptx::lds128(qrow + first * 16);
-                        const uint4 x1 = ptx::lds128(qrow + (first ^ 1) * 16);
-                        q0 = first ? x1 : x0;
-                        q1 = first ? x0 : x1;
-                        dsc = __half2float(__ushort_as_half(ptx::lds16(raw + (uint32_t)(nr * kTileK + r * 4 + hk * 2))));
-                    }
-                    const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-                    uint32_t pk[16];
-                    if (BF16) {
-                        const uint64_t dd = ptx::f2pack(dsc, dsc);
-                        const uint64_t nd = ptx::f2pack(-32896.0f * dsc, -32896.0f * dsc);
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            const uint64_t v01 =
-                                ptx::fma2(ptx::f2pack(magic_byte(w[j], 0), magic_byte(w[j], 1)), dd, nd);
-                            const uint64_t v23 =
-                                ptx::fma2(ptx::f2pack(magic_byte(w[j], 2), magic_byte(w[j], 3)), dd, nd);
-                            pk[2 * j] = pack2x<BF16>(v01);
-                            pk[2 * j + 1] = pack2x<BF16>(v23);
-                        }
-                    } else {
-                        // fp16 pairs: {0x64, u} is 1024 + u, minus 1152 is q (exact), times d
-                        // rounds q*d once - the same value as the fp32 route rounded to fp16
-                        const __half2 d2 = __half2half2(__float2half_rn(dsc));
-                        const __half2 off = __float2half2_rn(1152.0f);
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            uint32_t lo, hi;
-                            asm("prmt.b32 %0, %1, %2, 0x7170;" : "=r"(lo) : "r"(w[j]), "r"(0x64646464u));
-                            asm("prmt.b32 %0, %1, %2, 0x7372;" : "=r"(hi) : "r"(w[j]), "r"(0x64646464u));
-                            const __half2 vlo = __hmul2(__hsub2(*(const __half2*)&lo, off), d2);
-                            const __half2 vhi = __hmul2(__hsub2(*(const __half2*)&hi, off), d2);
-                            pk[2 * j] = *(const uint32_t*)&vlo;
-                            pk[2 * j + 1] = *(const uint32_t*)&vhi;
-                        }
-                    }
-                    ptx::tmem_st_32x32b_x16(tmem_base + lanes + kACol0 + (uint32_t)as * 64u + mat * 32 + hk * 16, pk);
-                    ptx::tmem_st_wait();
-                    ptx::tc_fence_before();
+            if (di >= 0) {
+                int nr;
+                {
+                    const uint8_t* dummy;
+                    int mt;
+                    source(tl, mat, dummy, nr, mt);
                 }
-                __syncwarp();
-                if (lane == 0) {
-                    ptx::mbar_arrive(&raw_empty[rs]);
-                    ptx::mbar_arrive(&a_full[as]);
+                for (int kt = 0; kt < KT; ++kt) {
+                    if ((as & 1) == kpar) {  // the k-step count's parity, continued across tiles
+                        ok = warp_wait(&raw_full[rs], rph, abort_flag, status, STAT_PTR(0)) &&
+                             warp_wait(&a_empty[as], aph ^ 1, abort_flag, status, STAT_PTR(1));
+                        if (!ok) break;
+                        if (nr > 0) {
+                            const uint32_t raw = raw_sa + (uint32_t)(rs * 2 + mat) * kRawBytes;
+                            const uint32_t dst = a_sa + (uint32_t)as * 2u * kATileBytes + a_row;
+                            uint4 x[4];
+                            uint32_t sc = 0u;
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) x[i] = make_uint4(0x80808080u, 0x80808080u, 0x80808080u, 0x80808080u);
+                            if (r < nr) {
+                                // half h, 16-byte chunk c at raw + h*nr*32 + r*32 + c*16; lanes alternate
+                                // the chunk order so that the 16-byte loads are conflict-free
+                                const uint32_t q = raw + (uint32_t)r * 32u;
+                                const uint32_t h1 = (uint32_t)nr * 32u;
+                                x[0] = ptx::lds128(q + first * 16);
+                                x[1] = ptx::lds128(q + (first ^ 1) * 16);
+                                x[2] = ptx::lds128(q + h1 + first * 16);
+                                x[3] = ptx::lds128(q + h1 + (first ^ 1) * 16);
+                                sc = ptx::lds32(raw + (uint32_t)nr * kTileK + (uint32_t)r * 4u);
+                            }
+                            uint32_t d0, d1;
+                            asm("prmt.b32 %0, %1, %1, 0x1010;" : "=r"(d0) : "r"(sc));
+                            asm("prmt.b32 %0, %1, %1, 0x3232;" : "=r"(d1) : "r"(sc));
+                            const float f0 = BF16 ? __half2float(__ushort_as_half((unsigned short)(sc & 0xffffu))) : 0.f;
+                            const float f1 = BF16 ? __half2float(__ushort_as_half((unsigned short)(sc >> 16))) : 0.f;
+                            // raw chunk c of half h holds operand chunks 4h + 2c and 4h + 2c + 1 of the row
+                            const uint32_t c0 = (uint32_t)first * 2u, c1 = (uint32_t)(first ^ 1) * 2u;
+                            dequant16_sts<BF16>(x[0], d0, f0, dst + (((c0 + 0u) ^ rx) << 4), dst + (((c0 + 1u) ^ rx) << 4));
+                            dequant16_sts<BF16>(x[1], d0, f0, dst + (((c1 + 0u) ^ rx) << 4), dst + (((c1 + 1u) ^ rx) << 4));
+                            dequant16_sts<BF16>(x[2], d1, f1, dst + (((4u + c0) ^ rx) << 4), dst + (((5u + c0) ^ rx) << 4));
+                            dequant16_sts<BF16>(x[3], d1, f1, dst + (((4u + c1) ^ rx) << 4), dst + (((5u + c1) ^ rx) << 4));
+                            ptx::fence_proxy_async_smem();  // generic writes -> tensor-core reads
+                        }
+                        __syncwarp();
+                        if (lane == 0) {
+                            ptx::mbar_arrive(&raw_empty[rs]);
+                            ptx::mbar_arrive(&a_full[as]);
+                        }
+                    }
+                    if (++rs == kRS) { rs = 0; rph ^= 1; }
+                    if (++as == kMA) { as = 0; aph ^= 1; }
                 }
-                if (++rs == kRS) { rs = 0; rph ^= 1; }
-                if (++as == kMA) { as = 0; aph ^= 1; }
             }
             if (!ok) break;
+            if (!epi) continue;
             // ---- epilogue of this tile
             if (!warp_wait(tmem_full, use & 1, abort_flag, status, STAT_PTR(2))) break;
             use += 1;
