@@ -66,7 +66,7 @@ constexpr int kGvSplitSlots = 64;
 constexpr int kGvMaxChunks = 8;
 struct WsLayout {
     int64_t S, rows_pad, rows_pad_sh;
-    size_t hdr, src1, dst, bounds, active, tiles, pad, h, h_sh, xt, xt_sh, xs, xs_sh, gv_part, gv_part_sh, total;
+    size_t hdr, src1, dst, sprow, bounds, active, tiles, pad, h, h_sh, xt, xt_sh, xs, xs_sh, gv_part, gv_part_sh, total;
     static size_t up(size_t v) { return (v + 255) / 256 * 256; }
     WsLayout(int64_t n_tokens, int k, int n_experts, int n_in, int n_hidden, int n_hidden_sh, int x_type) {
         (void)x_type;
@@ -80,6 +80,7 @@ struct WsLayout {
         hdr = o; o += 256;
         src1 = o; o += up(S * 4);
         dst = o; o += up(S * 4);
+        sprow = o; o += up(S * 4);  // tiled row of each slot t*k+s
         bounds = o; o += up((size_t)(n_experts + 1) * 4);
         active = o; o += up((size_t)(n_experts + 1) * 4);
         tiles = o; o += up((size_t)(n_experts + 1) * 4);

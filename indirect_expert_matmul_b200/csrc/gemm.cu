@@ -721,6 +721,55 @@ gather_tiled_kernel(const void* __restrict__ x, int x_type, int n_in, int KT, co
     }
 }
 
+// Broadcast gather, one warp per token: the token's row is read (and its scale
+// found) once and written to the tiled rows of all k of its slots.
+__global__ void __launch_bounds__(256)
+gather_tokens_kernel(const void* __restrict__ x, int x_type, int n_in, int KT, const int32_t* __restrict__ slot_prow,
+                     int k, int64_t n_tokens, int64_t rows_pad, uint8_t* __restrict__ xt, float* __restrict__ xs,
+                     const int* __restrict__ hdr) {
+    if (read_status(hdr + kHdrStatus) != 0) return;
+    const int lane = threadIdx.x & 31;
+    const int64_t nw = (int64_t)gridDim.x * (blockDim.x / 32);
+    for (int64_t t = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); t < n_tokens; t += nw) {
+        const int32_t* pr = slot_prow + t * k;
+        float mx = 0.f;
+#pragma unroll 4
+        for (int seg = lane; seg < KT * 8; seg += 32) {
+            float e[8];
+            load8(x, x_type, t, n_in, (seg >> 3) * 64 + (seg & 7) * 8, e);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(e[i]));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        int ex = 0;
+        if (mx > 0.f && mx <= 3.402823466e38f) {
+            ex = ilogbf(mx) - 14;
+            ex = ex < -100 ? -100 : ex;
+        }
+        const float sc = ldexpf(1.0f, -ex);
+        for (int j = lane; j < k; j += 32) xs[__ldg(pr + j)] = ldexpf(1.0f, ex);
+#pragma unroll 2
+        for (int seg = lane; seg < KT * 8; seg += 32) {
+            const int kt = seg >> 3, c = seg & 7;
+            float e[8];
+            load8(x, x_type, t, n_in, kt * 64 + c * 8, e);
+            uint32_t h[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const __half2 v2 = __floats2half2_rn(e[2 * i] * sc, e[2 * i + 1] * sc);
+                h[i] = *(const uint32_t*)&v2;
+            }
+            const uint4 v = make_uint4(h[0], h[1], h[2], h[3]);
+            uint8_t* plane = xt + (size_t)kt * rows_pad * 128u;
+            for (int j = 0; j < k; ++j) {
+                const int prow = __ldg(pr + j);
+                *(uint4*)(plane + (size_t)prow * 128u + ((c ^ (prow & 7)) << 4)) = v;
+            }
+        }
+    }
+}
+
 // ------------------------------------------------------------------- host
 #ifdef MOE_GEMM_STATS
 extern "C" __attribute__((visibility("default"))) int moe_gemm_stats_read(unsigned long long* out48, int reset) {
@@ -770,6 +819,18 @@ static moe_status run_gemm(const GemmParams& p, int64_t max_coltiles, cudaStream
 
 static int64_t coltile_bound(int64_t S, int E) { return (S + kGemmBN - 1) / kGemmBN + (S < E ? S : E); }
 
+// Broadcast mode (every slot of a token reads the token's row): per token.
+static moe_status gather_tokens(const void* x, int x_type, int n_in, const int32_t* slot_prow, int k, int64_t n_tokens,
+                                int64_t rows_pad, void* xt, float* xs, int* hdr, cudaStream_t s) {
+    const int KT = (n_in + kTileK - 1) / kTileK;
+    int64_t blocks = (n_tokens + 7) / 8;
+    if (blocks > (int64_t)sm_count() * 8) blocks = (int64_t)sm_count() * 8;
+    if (blocks < 1) blocks = 1;
+    gather_tokens_kernel<<<(unsigned)blocks, 256, 0, s>>>(x, x_type, n_in, KT, slot_prow, k, n_tokens, rows_pad,
+                                                          (uint8_t*)xt, xs, hdr);
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
 static moe_status gather(const void* x, int x_type, int n_in, const int32_t* src_rows, const int32_t* bounds,
                          const int32_t* pad_start, int n_groups, int64_t rows, int64_t rows_pad, void* xt, float* xs,
                          int* hdr, cudaStream_t s) {
@@ -783,8 +844,11 @@ static moe_status gather(const void* x, int x_type, int n_in, const int32_t* src
 }
 
 moe_status launch_gemm_mul_mat_id(const GemmMulMatId& g, cudaStream_t stream) {
-    moe_status st = gather(g.x, g.x_type, g.n_in, g.ids_src1, g.bounds, g.pad_start, g.E, g.S, g.rows_pad, g.xt,
-                           g.xs, g.hdr, stream);
+    moe_status st = g.x_rows * g.k == g.S
+                        ? gather_tokens(g.x, g.x_type, g.n_in, g.slot_prow, g.k, g.x_rows, g.rows_pad, g.xt, g.xs,
+                                        g.hdr, stream)
+                        : gather(g.x, g.x_type, g.n_in, g.ids_src1, g.bounds, g.pad_start, g.E, g.S, g.rows_pad, g.xt,
+                                 g.xs, g.hdr, stream);
     if (st) return st;
     prof_mark(stream, "gather");
     GemmParams p = {};
@@ -809,8 +873,8 @@ moe_status launch_gemm_mul_mat_id(const GemmMulMatId& g, cudaStream_t stream) {
 
 moe_status launch_gemm_ffn(const GemmFfn& g, cudaStream_t stream) {
     const int kt_ff = (g.n_ff + kTileK - 1) / kTileK;
-    moe_status st = gather(g.x, g.x_type, g.n_embd, g.ids_src1, g.bounds, g.pad_start, g.E, g.S, g.rows_pad, g.xt,
-                           g.xs, g.hdr, stream);
+    moe_status st =
+        gather_tokens(g.x, g.x_type, g.n_embd, g.slot_prow, g.k, g.T, g.rows_pad, g.xt, g.xs, g.hdr, stream);
     if (st) return st;
     prof_mark(stream, "gather");
     if (g.n_ff % kTileK) {  // columns past n_ff of the last k-plane of h are read by the down GEMM: keep them 0

@@ -20,6 +20,8 @@ struct GemmMulMatId {
     const int32_t* ntile_prefix;
     const int32_t* ids_src1;
     const int32_t* ids_dst;
+    const int32_t* slot_prow;  // tiled row of each slot t*k+s
+    int k;
     int* hdr;
 };
 
@@ -45,6 +47,8 @@ struct GemmFfn {
     const int32_t* ntile_prefix;
     const int32_t* ids_src1;
     const int32_t* ids_dst;
+    const int32_t* slot_prow;  // tiled row of each slot t*k+s
+    int k;
     int* hdr;
 };
 

@@ -8,7 +8,7 @@
 namespace moe {
 moe_status launch_row_ids(const int32_t* ids, int64_t S, int k, int E, int mode, int32_t* ids_src1,
                           int32_t* ids_dst, int32_t* bounds, int32_t* active, int32_t* ntile_prefix,
-                          int32_t* pad_start, int bn, int* hdr, cudaStream_t stream);
+                          int32_t* pad_start, int32_t* slot_prow, int bn, int* hdr, cudaStream_t stream);
 moe_status launch_prepare(const void* src, int E, int n_out, int n_in, void* dst, cudaStream_t stream);
 }  // namespace moe
 
@@ -98,8 +98,8 @@ moe_status moe_row_ids(const int32_t* ids, int64_t n_tokens, int k, int n_expert
     char* ws = (char*)workspace;
     prof_begin((cudaStream_t)stream);
     st = launch_row_ids(ids, n_tokens * k, k, n_experts, mode, ids_src1, ids_dst, expert_bounds,
-                        (int32_t*)(ws + W.active), (int32_t*)(ws + W.tiles), (int32_t*)(ws + W.pad), kGemmBN,
-                        (int*)(ws + W.hdr), (cudaStream_t)stream);
+                        (int32_t*)(ws + W.active), (int32_t*)(ws + W.tiles), (int32_t*)(ws + W.pad),
+                        (int32_t*)(ws + W.sprow), kGemmBN, (int*)(ws + W.hdr), (cudaStream_t)stream);
     prof_mark((cudaStream_t)stream, "row_ids");
     return st;
 }
@@ -146,7 +146,7 @@ moe_status moe_mul_mat_id(const void* W_prepared, int n_experts, int n_out, int 
         return st;
     }
     st = launch_row_ids(ids, S, k, n_experts, mode, src1, dstr, bounds, active, tiles, (int32_t*)(ws + W.pad),
-                        kGemmBN, hdr, s);
+                        (int32_t*)(ws + W.sprow), kGemmBN, hdr, s);
     if (st) return st;
     prof_mark(s, "row_ids");
     GemmMulMatId g = {};
@@ -167,6 +167,8 @@ moe_status moe_mul_mat_id(const void* W_prepared, int n_experts, int n_out, int 
     g.ntile_prefix = tiles;
     g.ids_src1 = src1;
     g.ids_dst = dstr;
+    g.slot_prow = (const int32_t*)(ws + W.sprow);
+    g.k = k;
     g.hdr = hdr;
     return launch_gemm_mul_mat_id(g, s);
 }
@@ -263,7 +265,7 @@ moe_status moe_ffn(const void* Wg, const void* Wu, const void* Wd, int n_experts
         return st;
     }
     st = launch_row_ids(ids, S, k, n_experts, MOE_BROADCAST, src1, dstr, bounds, active, tiles,
-                        (int32_t*)(ws + W.pad), kGemmBN, hdr, s);
+                        (int32_t*)(ws + W.pad), (int32_t*)(ws + W.sprow), kGemmBN, hdr, s);
     if (st) return st;
     prof_mark(s, "row_ids");
     GemmFfn g = {};
@@ -296,6 +298,8 @@ moe_status moe_ffn(const void* Wg, const void* Wu, const void* Wd, int n_experts
     g.ntile_prefix = tiles;
     g.ids_src1 = src1;
     g.ids_dst = dstr;
+    g.slot_prow = (const int32_t*)(ws + W.sprow);
+    g.k = k;
     g.hdr = hdr;
     return launch_gemm_ffn(g, s);
 }

@@ -51,10 +51,11 @@ __global__ void __launch_bounds__(kRowIdThreads, 1)
 row_ids_kernel(const int32_t* __restrict__ ids, int S, int k, int E, int mode, int n_chunks, int bn,
                int32_t* __restrict__ ids_src1, int32_t* __restrict__ ids_dst, int32_t* __restrict__ bounds,
                int32_t* __restrict__ active, int32_t* __restrict__ ntile_prefix, int32_t* __restrict__ pad_start,
-               int* __restrict__ hdr) {
+               int32_t* __restrict__ slot_prow, int* __restrict__ hdr) {
     extern __shared__ int smem[];
     int* off = smem;                        // [n_chunks][E]
     int* cnt = off + (size_t)n_chunks * E;  // [E]
+    int* pad_delta = cnt + E;               // [E]: pad_start[e] - bounds[e]
     __shared__ int warp_sums[32];
     __shared__ int totals[4];
     __shared__ int bad;
@@ -127,6 +128,7 @@ row_ids_kernel(const int32_t* __restrict__ ids, int S, int k, int E, int mode, i
         ntile_prefix[e] = run_tiles;
         run_tiles += (c + bn - 1) / bn;
         pad_start[e] = run_pad;
+        pad_delta[e] = run_pad - run;
         run_pad += (c + 7) & ~7;
         if (c > 0) active[run_act++] = e;
         cnt[e] = run;  // becomes the expert's first position
@@ -156,6 +158,7 @@ row_ids_kernel(const int32_t* __restrict__ ids, int S, int k, int E, int mode, i
             if (e >= 0) {
                 ids_dst[p] = i;
                 ids_src1[p] = (mode == MOE_BROADCAST) ? i / k : i;
+                if (slot_prow) slot_prow[i] = p + pad_delta[e];
                 if ((m & lt_mask) == 0) row[e] += __popc(m);
             }
             __syncwarp();
@@ -164,11 +167,11 @@ row_ids_kernel(const int32_t* __restrict__ ids, int S, int k, int E, int mode, i
 }
 
 // Shared memory needed for a given chunk count.
-static size_t row_ids_smem(int n_chunks, int E) { return ((size_t)n_chunks + 1) * E * sizeof(int); }
+static size_t row_ids_smem(int n_chunks, int E) { return ((size_t)n_chunks + 2) * E * sizeof(int); }
 
 moe_status launch_row_ids(const int32_t* ids, int64_t S, int k, int E, int mode, int32_t* ids_src1,
                           int32_t* ids_dst, int32_t* bounds, int32_t* active, int32_t* ntile_prefix,
-                          int32_t* pad_start, int bn, int* hdr, cudaStream_t stream) {
+                          int32_t* pad_start, int32_t* slot_prow, int bn, int* hdr, cudaStream_t stream) {
     const size_t budget = 200 * 1024;
     int n_chunks = kRowIdWarps;
     while (n_chunks > 1 && row_ids_smem(n_chunks, E) > budget) n_chunks >>= 1;
@@ -188,7 +191,7 @@ moe_status launch_row_ids(const int32_t* ids, int64_t S, int k, int E, int mode,
         attr_dev = dev;
     }
     row_ids_kernel<<<1, kRowIdThreads, smem, stream>>>(ids, (int)S, k, E, mode, n_chunks, bn, ids_src1, ids_dst,
-                                                      bounds, active, ntile_prefix, pad_start, hdr);
+                                                      bounds, active, ntile_prefix, pad_start, slot_prow, hdr);
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
