@@ -50,6 +50,8 @@ def _L():
         _lib.oracle_ffn_hidden.argtypes = [vp, vp, i32, i32, i32, vp, i32, vp, i64, i32, vp, i64, vp, vp, vp]
         _lib.oracle_dequant.argtypes = [vp, i32, i32, i32, vp]
         _lib.oracle_dequant.restype = None
+        _lib.oracle_combine.argtypes = [vp, vp, vp, i64, i32, i64, vp, vp]
+        _lib.oracle_combine.restype = None
     return _lib
 
 
@@ -169,3 +171,29 @@ def ffn_hidden(Wg, Wu, x, x_type, ids, slots):
     _chk(_L().oracle_ffn_hidden(_p(Wg), _p(Wu), E, nb * 32, n_ff, _p(x), DTYPES[x_type], _p(ids), T, k,
                                 _p(slots), len(slots), _p(h), _p(g), _p(u)))
     return h, g, u
+
+
+def combine(dst, r, dst_shared=None):
+    """Weighted combine y[t] = sum_s r[t][s]*dst[t][s] (+ dst_shared[t]), fp64,
+    ascending s (moe_oracle.c: oracle_combine).  dst float32 [T][k][n] (or
+    [T*k][n]), r float32 [T][k], dst_shared float32 [T][n] or None.  Returns
+    (y, mag): y float64 [T][n] and mag = sum of the terms' magnitudes."""
+    r = np.ascontiguousarray(r, dtype=np.float32)
+    T, k = r.shape
+    dst = np.ascontiguousarray(dst, dtype=np.float32)
+    n = dst.shape[-1]
+    dst = dst.reshape(T, k, n)
+    sh = None if dst_shared is None else np.ascontiguousarray(dst_shared, dtype=np.float32).reshape(T, n)
+    y = np.empty((T, n), dtype=np.float64)
+    mag = np.empty((T, n), dtype=np.float64)
+    _L().oracle_combine(_p(dst), _p(r), _p(sh), T, k, n, _p(y), _p(mag))
+    return y, mag
+
+
+def combine_tolerance(mag, k, shared):
+    """Bound on |float32 evaluation - exact| for the combine as the library
+    evaluates it: k fused multiply-adds in ascending s, then one add of the
+    shared term, each rounding once (relative 2^-24 of the running magnitude,
+    at most mag): (k + 1 + shared) * 2^-24 * mag, plus the smallest normal float
+    for sums that vanish."""
+    return (k + 1 + (1 if shared else 0)) * 2.0 ** -24 * mag + 1.2e-38

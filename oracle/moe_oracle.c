@@ -17,6 +17,9 @@
  *           "CUDA: better MoE implementation"), sections 1.2, 2, 2.1, 5, 6.
  *   [b11370] "llama.cpp 發布 b11370，CUDA 後端將共享專家融合進 MMVQ"
  *           (release note of PR #29184 "CUDA: fuse shared experts into MMVQ").
+ *   [cmoe]  "Optimalizace MoE modelů na slabém GPU: spuštění GPT-OSS-120B s 6 GB
+ *           VRAM až 30 t/s", section "Architektura Mixture of Experts" (a router
+ *           picks a few experts per token in every layer).
  *
  * Readings where the pages are silent (each also listed in the design notes):
  *   - Q8_0 block = fp16 scale d, then 32 int8 q; weight = d*q.
@@ -29,6 +32,8 @@
  *   - SwiGLU: h = silu(gate) * up, silu(z) = z / (1 + exp(-z)).
  *   - The shared expert is an always-on FFN on x[t] with its own weights,
  *     written to its own output.
+ *   - Combine (the step after the path): y[t] = sum_s r[t][s] * dst[t][s] +
+ *     dst_shared[t], the slots taken in ascending s.
  *
  * Tolerances returned beside every output element follow the bound
  * |gpu - oracle| <= 2e-3 * sum|w*x| + 1e-5; for the two-stage FFN the bound is
@@ -343,4 +348,35 @@ int oracle_ffn_hidden(const uint8_t *Wg, const uint8_t *Wu, int n_experts, int n
 void oracle_dequant(const uint8_t *W, int n_out, int n_in, int e, double *out) {
     for (int64_t n = 0; n < n_out; ++n)
         for (int64_t j = 0; j < n_in; ++j) out[n * n_in + j] = w_value(W, n_out, n_in, e, n, j);
+}
+
+/*
+ * Weighted combine of a token's expert outputs ([cmoe], "Architektura Mixture
+ * of Experts": the router picks k experts per token; the layer's output is
+ * their outputs weighted by the router, plus the always-on shared expert of
+ * [b11370]).  dst is [T][k][n] float, r is [T][k] float, dst_shared is [T][n]
+ * float or NULL.  For every (t, j), in fp64 and ascending s:
+ *   y[t][j]   = sum_s r[t][s] * dst[t][s][j]  (+ dst_shared[t][j])
+ *   mag[t][j] = sum_s |r[t][s] * dst[t][s][j]| (+ |dst_shared[t][j]|)
+ * mag is what a tolerance for a float evaluation of the same sum scales with.
+ */
+void oracle_combine(const float *dst, const float *r, const float *dst_shared, int64_t n_tokens, int k, int64_t n,
+                    double *y, double *mag) {
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < n_tokens; ++t) {
+        for (int64_t j = 0; j < n; ++j) {
+            double acc = 0.0, m = 0.0;
+            for (int s = 0; s < k; ++s) {
+                const double term = (double)r[t * k + s] * (double)dst[(t * k + s) * n + j];
+                acc += term;
+                m += fabs(term);
+            }
+            if (dst_shared) {
+                acc += (double)dst_shared[t * n + j];
+                m += fabs((double)dst_shared[t * n + j]);
+            }
+            y[t * n + j] = acc;
+            mag[t * n + j] = m;
+        }
+    }
 }

@@ -300,3 +300,76 @@ def test_workload_inputs_are_deterministic_and_shardable():
     sk = workloads.WORKLOADS["skew"]
     c = np.bincount(sk.ids(2048).reshape(-1), minlength=sk.n_experts)
     assert (c == 0).sum() >= sk.n_zero
+
+
+# ----------------------------------------------------------- weighted combine
+def _combine_inputs(T, k, n, seed):
+    rng = np.random.default_rng(seed)
+    dst = rng.normal(size=(T, k, n)).astype(np.float32)
+    r = rng.uniform(0.05, 1.0, size=(T, k)).astype(np.float32)
+    sh = rng.normal(size=(T, n)).astype(np.float32)
+    return dst, r, sh
+
+
+def test_combine_one_hot_weights_select_a_slot():
+    # r = e_s picks slot s exactly; plus the shared term exactly (one fp64 add of two floats)
+    dst, _, sh = _combine_inputs(5, 4, 33, 1)
+    for s in range(4):
+        r = np.zeros((5, 4), np.float32)
+        r[:, s] = 1.0
+        y, _ = oracle.combine(dst, r)
+        assert np.array_equal(y, dst[:, s, :].astype(np.float64))
+        y, _ = oracle.combine(dst, r, sh)
+        assert np.array_equal(y, dst[:, s, :].astype(np.float64) + sh.astype(np.float64))
+
+
+def test_combine_matches_numpy_einsum_and_is_linear():
+    dst, r, sh = _combine_inputs(7, 6, 40, 2)
+    y, mag = oracle.combine(dst, r, sh)
+    ref = np.einsum("tk,tkn->tn", r.astype(np.float64), dst.astype(np.float64)) + sh.astype(np.float64)
+    assert np.allclose(y, ref, rtol=0, atol=1e-12)
+    ref_mag = np.einsum("tk,tkn->tn", np.abs(r.astype(np.float64)), np.abs(dst.astype(np.float64))) + np.abs(sh)
+    assert np.allclose(mag, ref_mag, rtol=1e-14, atol=0)
+    y2, _ = oracle.combine(dst, 2 * r, 2 * sh)  # scaling by 2 is exact in float
+    assert np.array_equal(y2, 2 * y)
+
+
+def test_combine_slot_order_and_tokens_are_not_mixed():
+    # permuting the slots of one token together with their weights leaves y unchanged
+    # up to fp64 reordering; token rows stay separate
+    dst, r, _ = _combine_inputs(4, 5, 16, 3)
+    perm = np.array([3, 0, 4, 1, 2])
+    y, _ = oracle.combine(dst, r)
+    yp, _ = oracle.combine(dst[:, perm, :], r[:, perm])
+    assert np.allclose(y, yp, rtol=0, atol=1e-12)
+    dst2 = dst.copy()
+    dst2[1] += 1.0  # touching token 1 changes only row 1, by about sum_s r[1][s]
+    y2, _ = oracle.combine(dst2, r)
+    assert np.array_equal(np.delete(y2, 1, axis=0), np.delete(y, 1, axis=0))
+    assert np.allclose(y2[1] - y[1], r[1].astype(np.float64).sum(), rtol=0, atol=1e-6)
+
+
+def test_combine_edge_cases_and_tolerance():
+    dst, r, sh = _combine_inputs(3, 1, 8, 4)
+    y, mag = oracle.combine(dst, r)  # k = 1: one product, exact in fp64
+    assert np.array_equal(y, r.astype(np.float64) * dst[:, 0, :].astype(np.float64))
+    y0, _ = oracle.combine(np.zeros((0, 2, 8), np.float32), np.zeros((0, 2), np.float32))
+    assert y0.shape == (0, 8)
+    # the tolerance covers a float32 evaluation in the library's order
+    dst, r, sh = _combine_inputs(6, 8, 64, 5)
+    y, mag = oracle.combine(dst, r, sh)
+    acc = np.zeros((6, 64), np.float32)
+    for s in range(8):  # float32 multiply-add per slot (product exact in float64, one rounding)
+        acc = (acc.astype(np.float64) + r[:, s:s + 1].astype(np.float64) * dst[:, s, :]).astype(np.float32)
+    acc = (acc + sh).astype(np.float32)
+    tol = oracle.combine_tolerance(mag, 8, True)
+    assert np.all(np.abs(acc - y) <= tol)
+
+
+def test_router_weights_are_seeded_and_normalised():
+    a = workloads.router_weights(9, 8, 0)
+    b = workloads.router_weights(9, 8, 0)
+    assert np.array_equal(a, b) and a.dtype == np.float32
+    assert np.allclose(a.sum(axis=1), 1.0, atol=1e-6) and np.all(a > 0)
+    # rows are independent of how many tokens are generated (counter-based)
+    assert np.array_equal(workloads.router_weights(4, 8, 0, t0=5), a[5:9])

@@ -31,6 +31,7 @@ T_SG, T_SU, T_SD = 5, 6, 7          # shared expert gate / up / down
 T_X = 100          # activations, one row per token
 T_X_SLOT = 102     # activations, one row per (token, slot)
 T_ROUTE = 200      # routing keys (uses T_ROUTE and T_ROUTE + 1)
+T_RW = 300         # router weights of the routed slots
 LAYER_STRIDE = 1000  # decode layers l use tensor ids + l * LAYER_STRIDE
 
 D_LO, D_HI = 0.001, 0.01   # Q8_0 scale range
@@ -56,6 +57,7 @@ def _L():
         _lib.wl_fill_q8_0.argtypes = [vp, i64, i64, i64, u64, u64, dbl, dbl]
         for f in (_lib.wl_fill_normal_f32, _lib.wl_fill_normal_bf16, _lib.wl_fill_normal_f16):
             f.argtypes = [vp, i64, i64, u64, u64]
+        _lib.wl_fill_uniform_f32.argtypes = [vp, i64, i64, dbl, dbl, u64, u64]
         _lib.wl_route_topk_normal.argtypes = [vp, i64, i64, i32, i32, dbl, u64, u64]
         _lib.wl_route_uniform.argtypes = [vp, i64, i64, i32, i32, u64, u64]
         _lib.wl_route_zipf.argtypes = [vp, i64, i64, i32, i32, dbl, i32, u64, u64]
@@ -110,6 +112,24 @@ def activations(n_rows: int, n_in: int, dtype: str, seed: int, tensor: int, row0
     else:
         raise ValueError(dtype)
     return out
+
+
+def uniform_f32(n: int, lo: float, hi: float, seed: int, tensor: int, i0: int = 0) -> np.ndarray:
+    """U[lo, hi) float32 samples i0 .. i0+n-1 of a tensor."""
+    out = np.empty(n, dtype=np.float32)
+    if n:
+        _L().wl_fill_uniform_f32(_ptr(out), i0, n, lo, hi, seed, tensor)
+    return out
+
+
+def router_weights(n_tokens: int, k: int, seed: int, tensor: int = T_RW, t0: int = 0) -> np.ndarray:
+    """Router weights float32 [n_tokens][k]: U[0.05, 1) per slot, scaled in fp64 so
+    that each token's weights sum to one (the shape a softmax over the chosen
+    experts gives), then rounded to float32."""
+    u = uniform_f32(n_tokens * k, 0.05, 1.0, seed, tensor, i0=t0 * k).astype(np.float64).reshape(n_tokens, k)
+    if n_tokens == 0:
+        return u.astype(np.float32)
+    return (u / u.sum(axis=1, keepdims=True)).astype(np.float32)
 
 
 def routing(kind: str, n_tokens: int, n_experts: int, k: int, seed: int, tensor: int = T_ROUTE,

@@ -121,6 +121,13 @@ void wl_fill_normal_bf16(uint16_t *out, int64_t i0, int64_t n, uint64_t seed, ui
     for (int64_t i = 0; i < n; ++i) out[i] = f32_to_bf16((float)normal(key, (uint64_t)(i0 + i)));
 }
 
+/* U[lo, hi) samples i0 .. i0+n-1 of a tensor, stored as float. */
+void wl_fill_uniform_f32(float *out, int64_t i0, int64_t n, double lo, double hi, uint64_t seed, uint64_t tensor) {
+    const uint64_t key = stream_key(seed, tensor);
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) out[i] = (float)(lo + (hi - lo) * unif01(draw(key, (uint64_t)(i0 + i))));
+}
+
 /* N(0,1) samples stored as fp16 (for fp16-activation cases). */
 void wl_fill_normal_f16(uint16_t *out, int64_t i0, int64_t n, uint64_t seed, uint64_t tensor) {
     const uint64_t key = stream_key(seed, tensor);
