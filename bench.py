@@ -78,18 +78,59 @@ def load_peaks():
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons while running."""
+    """SM clock and clock-event (throttle) reasons of one GPU while running:
+    read-only NVML queries every few milliseconds from a background thread
+    (the timed region can be only tens of milliseconds), else nvidia-smi.
+    The samples are also written to gpurun_out/clocks_gpu<i>.csv."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASON_BITS = (("sw_power_cap", 0x4), ("hw_slowdown", 0x8), ("sw_thermal_slowdown", 0x20),
+                   ("hw_thermal_slowdown", 0x40))
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
+        self.nv = None
+        self.samples = []  # (sm MHz, reason bits)
+        self.smax = None
         self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
 
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(self.gpu).uuid)
+            return pynvml, pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+
+    def _poll(self):
+        nv, h = self.nv, self.h
+        while not self.stop.is_set():
+            try:
+                self.samples.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM),
+                                     nv.nvmlDeviceGetCurrentClocksEventReasons(h)))
+            except Exception:
+                break
+            self.stop.wait(0.004)
+
     def __enter__(self):
+        import threading
+        try:
+            self.nv, self.h = self._nvml_handle()
+            self.smax = self.nv.nvmlDeviceGetMaxClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+            self.stop = threading.Event()
+            self.thread = threading.Thread(target=self._poll, daemon=True)
+            self.thread.start()
+            t0 = time.time()
+            while not self.samples and time.time() - t0 < 2.0:
+                time.sleep(0.002)
+            return self
+        except Exception:
+            self.nv = None
         try:
             os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.f = open(self.path, "w")
@@ -102,6 +143,18 @@ class ClockSampler:
         return self
 
     def __exit__(self, *a):
+        if self.nv is not None:
+            self.stop.set()
+            self.thread.join(timeout=2)
+            try:
+                os.makedirs(os.path.dirname(self.path), exist_ok=True)
+                with open(self.path, "w") as f:
+                    f.write("# sm_mhz, sm_max_mhz, clock event reason bits (NVML), one line per sample\n")
+                    for sm, bits in self.samples:
+                        f.write(f"{sm}, {self.smax}, {bits:#x}\n")
+            except OSError:
+                pass
+            return
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -111,6 +164,13 @@ class ClockSampler:
             self.f.close()
 
     def summary(self):
+        if self.nv is not None:
+            sm = [float(x) for x, _ in self.samples]
+            reasons = sorted({nm for _, bits in self.samples for nm, b in self.REASON_BITS if bits & b})
+            smax = float(self.smax) if self.smax else None
+            load = [x for x in sm if smax and x > 0.3 * smax] or sm
+            return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": smax,
+                    "reasons": reasons, "samples": len(sm), "source": "nvml"}
         if self.proc is None or not os.path.exists(self.path):
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         sm, smax, reasons = [], None, set()
@@ -129,7 +189,7 @@ class ClockSampler:
                     reasons.add(nm)
         load = [s for s in sm if smax and s > 0.3 * smax] or sm
         return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "source": "nvidia-smi"}
 
 
 # ------------------------------------------------------------ CPU baseline
@@ -340,6 +400,29 @@ def run_ours(args):
                          "ms_per_step": round(ms_e2e, 3)}
         del x_pin, dst_pin
 
+    # ---- the weighted combine that follows the path (its own kernel, timed alone):
+    # y[t] = sum_s r[t][s] * dst[t][s] over this step's output, HBM-bound
+    if not args.no_combine:
+        r_dev = torch.from_numpy(workloads.router_weights(T, k, WL.seed)).cuda()
+        y = torch.empty((T, n_embd), dtype=torch.float32, device="cuda")
+        for _ in range(3):
+            moe.combine(dst, r_dev, out=y)
+        torch.cuda.synchronize()
+        n_c = 10
+        ev0.record()
+        for _ in range(n_c):
+            moe.combine(dst, r_dev, out=y)
+        ev1.record()
+        torch.cuda.synchronize()
+        ms_c = max_over_ranks(ev0.elapsed_time(ev1) / n_c, device="cuda")
+        c_bytes = dst_bytes + S * 4 + T * n_embd * 4
+        c_gbs = c_bytes / (ms_c * 1e-3) / 1e9
+        result["combine"] = {"ms": round(ms_c, 4), "GB/s": round(c_gbs, 1), "frac_of_hbm": round(c_gbs / hbm_peak, 4),
+                             "algorithmic_bytes": int(c_bytes), "kernel": "combine_kernel",
+                             "config": f"dst [{T}][{k}][{n_embd}] fp32 of this step, router weights, no shared "
+                                       "expert; inputs larger than L2"}
+        del y, r_dev
+
     del Wg, Wu, Wd
     torch.cuda.empty_cache()
     if not args.no_decode:
@@ -452,6 +535,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-combine", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--decode-layers", type=int, default=16)

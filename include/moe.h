@@ -203,6 +203,30 @@ MOE_API moe_status moe_ffn_decode_noalloc(const void *Wg, const void *Wu, const 
                                           const void *x, moe_dtype x_type, const int32_t *ids, int64_t n_tokens, int k,
                                           float *dst, float *dst_shared, int *status_out, moe_stream stream);
 
+/* ----------------------------------------------------------------- combine */
+
+/*
+ * Weighted combine of each token's expert outputs - the step after the
+ * indirect matmul in a MoE layer ("Optimalizace MoE modelů na slabém GPU:
+ * spuštění GPT-OSS-120B s 6 GB VRAM až 30 t/s", section "Architektura Mixture
+ * of Experts": a router picks k experts per token; the layer output weights
+ * their outputs), plus the always-on shared expert ([b11370]):
+ *   y[t][j] = sum_s weights[t][s] * dst[t][s][j]  (+ dst_shared[t][j])
+ * dst: float [n_tokens][k][n] (moe_mul_mat_id / moe_ffn output); weights:
+ * float [n_tokens][k] (the router's weights, any values); dst_shared: float
+ * [n_tokens][n] or NULL; y: float [n_tokens][n], caller-owned, must not
+ * overlap dst or weights (it may be dst_shared itself).  All pointers 4-byte
+ * aligned; 16-byte alignment and n % 4 == 0 take the vector path.
+ * Evaluation: per output one fused multiply-add per slot in ascending s, then
+ * one add of the shared term - bit-identical from run to run; within
+ * (k + 1 + shared) * 2^-24 * sum of the terms' magnitudes of the exact sum.
+ * Errors (host, before any launch): MOE_ERR_INVALID for null pointers,
+ * misalignment, k < 1 or n < 1; MOE_ERR_RANGE for n_tokens >= 2^22,
+ * k >= 1024 or n >= 2^31.  n_tokens == 0 does nothing.
+ */
+MOE_API moe_status moe_combine(const float *dst, const float *weights, const float *dst_shared, int64_t n_tokens,
+                               int k, int64_t n, float *y, moe_stream stream);
+
 /* ------------------------------------------------------------------ tuning */
 
 /* Token count at or below which the mat-vec path is used (default 8); the

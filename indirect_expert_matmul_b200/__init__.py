@@ -24,7 +24,7 @@ BF16, F16, F32 = 0, 1, 2
 ABI_SYMBOLS = (
     "moe_status_string", "moe_workspace_size", "moe_workspace_init", "moe_get_status",
     "moe_weights_prepared_size", "moe_weights_prepare", "moe_row_ids", "moe_mul_mat_id", "moe_ffn",
-    "moe_ffn_decode_noalloc", "moe_set_gemv_threshold", "moe_get_gemv_threshold", "moe_set_path", "moe_profile_enable", "moe_profile_read",
+    "moe_ffn_decode_noalloc", "moe_combine", "moe_set_gemv_threshold", "moe_get_gemv_threshold", "moe_set_path", "moe_profile_enable", "moe_profile_read",
 )
 
 _lib = None
@@ -54,6 +54,7 @@ def _L() -> ctypes.CDLL:
                           _vp, _vp, _vp, _vp]
     L.moe_ffn_decode_noalloc.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _i32, _vp, _i64,
                                          _i32, _vp, _vp, _vp, _vp]
+    L.moe_combine.argtypes = [_vp, _vp, _vp, _i64, _i32, _i64, _vp, _vp]
     L.moe_set_gemv_threshold.argtypes = [_i32]
     L.moe_set_gemv_threshold.restype = None
     L.moe_get_gemv_threshold.argtypes = []
@@ -233,6 +234,25 @@ def ffn_decode_noalloc(Wg, Wu, Wd, n_experts, n_embd, n_ff, x, ids, shared=None,
                                      _ptr(Sd), n_ff_sh, _ptr(x), _XTYPE[x.dtype], _ptr(ids), T, k, _ptr(out),
                                      _ptr(out_shared), _ptr(status), _stream(x.device)), "moe_ffn_decode_noalloc")
     return out, out_shared
+
+
+def combine(dst, weights, shared=None, out=None):
+    """y[t] = sum_s weights[t][s] * dst[t][s] (+ shared[t]) through moe_combine.
+    dst: float32 CUDA [T][k][n] (or [T*k][n] with weights [T][k]); weights:
+    float32 [T][k]; shared: float32 [T][n] or None; out: float32 [T][n] or None."""
+    _cuda(dst, "dst", torch.float32)
+    _cuda(weights, "weights", torch.float32)
+    T, k = weights.shape
+    n = dst.shape[-1]
+    if dst.numel() != T * k * n:
+        raise ValueError("dst must hold n_tokens*k rows of n")
+    if shared is not None:
+        _cuda(shared, "shared", torch.float32)
+    if out is None:
+        out = torch.empty((T, n), dtype=torch.float32, device=dst.device)
+    _chk(_L().moe_combine(_ptr(dst), _ptr(weights), _ptr(shared), T, k, n, _ptr(out), _stream(dst.device)),
+         "moe_combine")
+    return out
 
 
 # ------------------------------------------------------------------ tuning

@@ -67,6 +67,18 @@ def test_v3_sampled_rows_within_tolerance(v3_run):
     check_close(got, ref, tol, "v3 moe_ffn")
 
 
+def test_v3_combine_sampled_tokens(v3_run):
+    wl, _, _, _, dst = v3_run
+    T = wl.n_tokens[0]
+    r = workloads.router_weights(T, wl.k, wl.seed)
+    y = moe.combine(dst, torch.from_numpy(r).cuda())
+    rng = np.random.default_rng(0)
+    toks = np.unique(np.concatenate([[0, T - 1], rng.choice(T, 62, replace=False)]))
+    sel = torch.from_numpy(toks).cuda()
+    y_ref, mag = oracle.combine(dst[sel].cpu().numpy(), r[toks])
+    check_close(y[sel], y_ref, oracle.combine_tolerance(mag, wl.k, False), "combine V3")
+
+
 def test_v3_ten_runs_bit_identical(v3_run):
     wl, _, _, (Wg, Wu, Wd, x, ids, ws), dst = v3_run
     ref = dst.clone()
