@@ -52,6 +52,7 @@ def _L():
         _lib.oracle_dequant.restype = None
         _lib.oracle_combine.argtypes = [vp, vp, vp, i64, i32, i64, vp, vp]
         _lib.oracle_combine.restype = None
+        _lib.oracle_route.argtypes = [vp, vp, i64, i32, i32, i32, vp, vp]
     return _lib
 
 
@@ -197,3 +198,31 @@ def combine_tolerance(mag, k, shared):
     at most mag): (k + 1 + shared) * 2^-24 * mag, plus the smallest normal float
     for sums that vanish."""
     return (k + 1 + (1 if shared else 0)) * 2.0 ** -24 * mag + 1.2e-38
+
+
+def route(logits, k, bias=None, normalize=True):
+    """Router (moe_oracle.c: oracle_route).  logits float32 [T][E], bias float32
+    [E] or None.  Returns (ids int32 [T][k], w float64 [T][k], tol float64
+    [T][k]): the k largest float32 keys logit + bias in descending order (ties to
+    the lower index), their softmax probabilities (renormalised over the k when
+    `normalize`), and the bound a float32 evaluation of the weights meets."""
+    logits = np.ascontiguousarray(logits, dtype=np.float32)
+    T, E = logits.shape
+    b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32).reshape(E)
+    ids = np.empty((T, k), dtype=np.int32)
+    w = np.empty((T, k), dtype=np.float64)
+    st = _L().oracle_route(_p(logits), _p(b), T, E, k, 1 if normalize else 0, _p(ids), _p(w))
+    if st != 0:
+        raise ValueError("need 1 <= k <= n_experts")
+    return ids, w, route_tolerance(w, logits, E, k, normalize)
+
+
+def route_tolerance(w, logits, E, k, normalize):
+    """Relative bound for float32 softmax weights: the exponent's argument
+    l - max rounds once (2^-24 of |l - max|, at most the row's logit span), the
+    exponential is within a few units in the last place, the sum of E terms
+    and of the k chosen ones round once per addition, and the divisions once
+    each: (span + 4 + E + k + 4) * 2^-24, applied to |w|."""
+    span = (logits.max(axis=1) - logits.min(axis=1)).astype(np.float64)[:, None]
+    rel = (span + 8.0 + E + (k if normalize else 0)) * 2.0 ** -24
+    return rel * np.abs(w) + 1e-30

@@ -34,6 +34,9 @@
  *     written to its own output.
  *   - Combine (the step after the path): y[t] = sum_s r[t][s] * dst[t][s] +
  *     dst_shared[t], the slots taken in ascending s.
+ *   - Router (the step before it): softmax over all experts' logits; the k
+ *     largest of logit + bias chosen (descending, ties to the lower index);
+ *     weights = the chosen experts' probabilities, optionally renormalised.
  *
  * Tolerances returned beside every output element follow the bound
  * |gpu - oracle| <= 2e-3 * sum|w*x| + 1e-5; for the two-stage FFN the bound is
@@ -379,4 +382,52 @@ void oracle_combine(const float *dst, const float *r, const float *dst_shared, i
             mag[t * n + j] = m;
         }
     }
+}
+
+/*
+ * Router ([cmoe], "Architektura Mixture of Experts": a gating network picks k
+ * of the experts for every token).  logits float [T][E]; bias float [E] or
+ * NULL (a per-expert selection bias).  For every token t:
+ *   key[e]  = logits[t][e] + bias[e], evaluated as one float addition - the
+ *             selection is a decision on these float values, made from the
+ *             same bits on both sides;
+ *   ids[t]  = the k experts with the largest keys, in descending key order,
+ *             equal keys taken in ascending expert index;
+ *   p[e]    = exp(logits[t][e] - m) / sum_j exp(logits[t][j] - m), m = max_j
+ *             logits[t][j] (softmax over all experts, fp64);
+ *   w[t][i] = p[ids[t][i]], divided by sum_i p[ids[t][i]] when normalize != 0.
+ * Returns 0, or -1 for k outside [1, E].
+ */
+int oracle_route(const float *logits, const float *bias, int64_t n_tokens, int n_experts, int k, int normalize,
+                 int32_t *ids, double *w) {
+    if (k < 1 || k > n_experts) return -1;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < n_tokens; ++t) {
+        const float *l = logits + t * n_experts;
+        unsigned char *taken = (unsigned char *)calloc((size_t)n_experts, 1);
+        for (int i = 0; i < k; ++i) {
+            int best = -1;
+            float bk = 0.0f;
+            for (int e = 0; e < n_experts; ++e) {
+                if (taken[e]) continue;
+                const float key = bias ? l[e] + bias[e] : l[e];
+                if (best < 0 || key > bk) { best = e; bk = key; }  /* ascending e keeps the lower index on ties */
+            }
+            taken[best] = 1;
+            ids[t * k + i] = best;
+        }
+        free(taken);
+        double m = l[0];
+        for (int e = 1; e < n_experts; ++e) if (l[e] > m) m = l[e];
+        double z = 0.0;
+        for (int e = 0; e < n_experts; ++e) z += exp((double)l[e] - m);
+        double sel = 0.0;
+        for (int i = 0; i < k; ++i) {
+            w[t * k + i] = exp((double)l[ids[t * k + i]] - m) / z;
+            sel += w[t * k + i];
+        }
+        if (normalize)
+            for (int i = 0; i < k; ++i) w[t * k + i] /= sel;
+    }
+    return 0;
 }

@@ -373,3 +373,70 @@ def test_router_weights_are_seeded_and_normalised():
     assert np.allclose(a.sum(axis=1), 1.0, atol=1e-6) and np.all(a > 0)
     # rows are independent of how many tokens are generated (counter-based)
     assert np.array_equal(workloads.router_weights(4, 8, 0, t0=5), a[5:9])
+
+
+# ------------------------------------------------------------------- router
+def _np_route(logits, k, bias=None, normalize=True):
+    # independent restatement with numpy: float32 keys, a stable sort, float64 softmax
+    key = logits if bias is None else (logits + bias[None, :]).astype(np.float32)
+    T, E = logits.shape
+    order = np.array([np.lexsort((np.arange(E), -key[t].astype(np.float64)))[:k] for t in range(T)], np.int32)
+    l64 = logits.astype(np.float64)
+    p = np.exp(l64 - l64.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    w = np.take_along_axis(p, order, axis=1)
+    if normalize:
+        w = w / w.sum(axis=1, keepdims=True)
+    return order, w
+
+
+@pytest.mark.parametrize("normalize", [True, False])
+@pytest.mark.parametrize("with_bias", [False, True])
+def test_route_matches_numpy(normalize, with_bias):
+    rng = np.random.default_rng(11)
+    logits = rng.normal(size=(50, 40)).astype(np.float32)
+    bias = rng.normal(scale=0.5, size=40).astype(np.float32) if with_bias else None
+    ids, w, tol = oracle.route(logits, 6, bias, normalize)
+    ref_ids, ref_w = _np_route(logits, 6, bias, normalize)
+    assert np.array_equal(ids, ref_ids)
+    assert np.allclose(w, ref_w, rtol=1e-13, atol=0)
+
+
+def test_route_ties_bias_and_full_k():
+    logits = np.zeros((3, 10), np.float32)
+    ids, w, _ = oracle.route(logits, 4, normalize=False)
+    assert np.array_equal(ids, np.tile(np.arange(4, dtype=np.int32), (3, 1)))  # equal keys: lower index first
+    assert np.allclose(w, 0.1, rtol=1e-15)
+    _, wn, _ = oracle.route(logits, 4)
+    assert np.allclose(wn, 0.25, rtol=1e-15)
+    # the bias moves the choice, not the probabilities
+    bias = np.zeros(10, np.float32)
+    bias[7] = 1.0
+    ids_b, w_b, _ = oracle.route(logits, 2, bias, normalize=False)
+    assert list(ids_b[0]) == [7, 0] and np.allclose(w_b, 0.1, rtol=1e-15)
+    # k = E: every expert, probabilities summing to one
+    rng = np.random.default_rng(3)
+    l = rng.normal(size=(5, 12)).astype(np.float32)
+    ids_f, w_f, _ = oracle.route(l, 12, normalize=False)
+    assert all(sorted(r) == list(range(12)) for r in ids_f)
+    assert np.allclose(w_f.sum(axis=1), 1.0, atol=1e-14)
+    with pytest.raises(ValueError):
+        oracle.route(l, 13)
+
+
+def test_route_tolerance_covers_a_float32_softmax():
+    rng = np.random.default_rng(5)
+    logits = (rng.normal(size=(40, 64)) * 3).astype(np.float32)
+    ids, w, tol = oracle.route(logits, 8)
+    m = logits.max(axis=1, keepdims=True)
+    e = np.exp((logits - m).astype(np.float32)).astype(np.float32)
+    z = np.zeros((40, 1), np.float32)
+    for j in range(64):  # float32 sum, one rounding per addition
+        z = (z + e[:, j:j + 1]).astype(np.float32)
+    p = (e / z).astype(np.float32)
+    sel = np.take_along_axis(p, ids, axis=1)
+    s = np.zeros((40, 1), np.float32)
+    for i in range(8):
+        s = (s + sel[:, i:i + 1]).astype(np.float32)
+    w32 = (sel / s).astype(np.float32)
+    assert np.all(np.abs(w32 - w) <= tol)
