@@ -423,6 +423,39 @@ def run_ours(args):
                                        "expert; inputs larger than L2"}
         del y, r_dev
 
+    # ---- the router that precedes the path (its own kernel, timed alone): top-k of
+    # logit + bias over the experts and softmax weights, at the V3 routing shape
+    if not args.no_combine:
+        logits = torch.from_numpy(workloads.activations(T, E, "f32", WL.seed, 51)).cuda()
+        bias_e = torch.from_numpy((workloads.activations(1, E, "f32", WL.seed, 52)[0] * 0.5).astype(np.float32)).cuda()
+        r_ids = torch.empty((T, k), dtype=torch.int32, device="cuda")
+        r_w = torch.empty((T, k), dtype=torch.float32, device="cuda")
+        for _ in range(3):
+            moe.route(logits, k, bias_e, True, ids=r_ids, weights=r_w)
+        torch.cuda.synchronize()
+        # one launch is a few microseconds: replay them from a CUDA graph so that host
+        # launch overhead is not what is timed
+        n_r = 20
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for _ in range(n_r):
+                moe.route(logits, k, bias_e, True, ids=r_ids, weights=r_w)
+        graph.replay()
+        torch.cuda.synchronize()
+        ev0.record()
+        graph.replay()
+        ev1.record()
+        torch.cuda.synchronize()
+        us_r = max_over_ranks(ev0.elapsed_time(ev1) / n_r, device="cuda") * 1e3
+        del graph
+        r_bytes = T * E * 4 + E * 4 + T * k * 8
+        result["route"] = {"us": round(us_r, 2), "GB/s": round(r_bytes / (us_r * 1e-6) / 1e9, 1),
+                           "frac_of_hbm": round(r_bytes / (us_r * 1e-6) / 1e9 / hbm_peak, 4),
+                           "algorithmic_bytes": int(r_bytes), "kernel": "route_kernel",
+                           "config": f"logits [{T}][{E}] fp32 + bias, top-{k}, softmax weights renormalised; "
+                                     f"{n_r} launches replayed from one CUDA graph"}
+        del logits, bias_e, r_ids, r_w
+
     del Wg, Wu, Wd
     torch.cuda.empty_cache()
     if not args.no_decode:

@@ -203,6 +203,30 @@ MOE_API moe_status moe_ffn_decode_noalloc(const void *Wg, const void *Wu, const 
                                           const void *x, moe_dtype x_type, const int32_t *ids, int64_t n_tokens, int k,
                                           float *dst, float *dst_shared, int *status_out, moe_stream stream);
 
+/* ------------------------------------------------------------------ router */
+
+/*
+ * Router - the step before the indirect matmul ("Optimalizace MoE modelů na
+ * slabém GPU: spuštění GPT-OSS-120B s 6 GB VRAM až 30 t/s", section
+ * "Architektura Mixture of Experts": a gating network picks k experts per
+ * token).  For every token t:
+ *   key[e]     = logits[t][e] + bias[e]      (one float addition; bias may be NULL)
+ *   ids[t][:]  = the k largest keys in descending order, equal keys in
+ *                ascending expert index      (int32 [n_tokens][k])
+ *   weights[t][i] = softmax(logits[t])[ids[t][i]], divided by their sum over
+ *                the k when normalize != 0   (float [n_tokens][k])
+ * logits: float [n_tokens][n_experts]; bias: float [n_experts] or NULL.  The
+ * choice is a pure function of the float keys (bit-identical to any exact
+ * evaluation of the rule above); the weights are within
+ * (span + 8 + n_experts + k) * 2^-24 relative of the exact softmax, span being
+ * the row's largest minus smallest logit.  NaN logits give unspecified ids.
+ * Errors (host): MOE_ERR_INVALID for null pointers, 4-byte misalignment,
+ * n_experts < 1 or k outside [1, n_experts]; MOE_ERR_RANGE for n_tokens >= 2^22,
+ * n_experts > 1024 or k >= 1024.  n_tokens == 0 does nothing.
+ */
+MOE_API moe_status moe_route(const float *logits, const float *bias, int64_t n_tokens, int n_experts, int k,
+                             int normalize, int32_t *ids, float *weights, moe_stream stream);
+
 /* ----------------------------------------------------------------- combine */
 
 /*

@@ -24,7 +24,7 @@ BF16, F16, F32 = 0, 1, 2
 ABI_SYMBOLS = (
     "moe_status_string", "moe_workspace_size", "moe_workspace_init", "moe_get_status",
     "moe_weights_prepared_size", "moe_weights_prepare", "moe_row_ids", "moe_mul_mat_id", "moe_ffn",
-    "moe_ffn_decode_noalloc", "moe_combine", "moe_set_gemv_threshold", "moe_get_gemv_threshold", "moe_set_path", "moe_profile_enable", "moe_profile_read",
+    "moe_ffn_decode_noalloc", "moe_route", "moe_combine", "moe_set_gemv_threshold", "moe_get_gemv_threshold", "moe_set_path", "moe_profile_enable", "moe_profile_read",
 )
 
 _lib = None
@@ -54,6 +54,7 @@ def _L() -> ctypes.CDLL:
                           _vp, _vp, _vp, _vp]
     L.moe_ffn_decode_noalloc.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _i32, _vp, _i64,
                                          _i32, _vp, _vp, _vp, _vp]
+    L.moe_route.argtypes = [_vp, _vp, _i64, _i32, _i32, _i32, _vp, _vp, _vp]
     L.moe_combine.argtypes = [_vp, _vp, _vp, _i64, _i32, _i64, _vp, _vp]
     L.moe_set_gemv_threshold.argtypes = [_i32]
     L.moe_set_gemv_threshold.restype = None
@@ -234,6 +235,23 @@ def ffn_decode_noalloc(Wg, Wu, Wd, n_experts, n_embd, n_ff, x, ids, shared=None,
                                      _ptr(Sd), n_ff_sh, _ptr(x), _XTYPE[x.dtype], _ptr(ids), T, k, _ptr(out),
                                      _ptr(out_shared), _ptr(status), _stream(x.device)), "moe_ffn_decode_noalloc")
     return out, out_shared
+
+
+def route(logits, k, bias=None, normalize=True, ids=None, weights=None):
+    """Router through moe_route: the k largest logit + bias per token (ties to
+    the lower expert) and their softmax weights.  logits: float32 CUDA [T][E];
+    bias: float32 [E] or None.  Returns (ids int32 [T][k], weights float32 [T][k])."""
+    _cuda(logits, "logits", torch.float32)
+    T, E = logits.shape
+    if bias is not None:
+        _cuda(bias, "bias", torch.float32)
+    if ids is None:
+        ids = torch.empty((T, k), dtype=torch.int32, device=logits.device)
+    if weights is None:
+        weights = torch.empty((T, k), dtype=torch.float32, device=logits.device)
+    _chk(_L().moe_route(_ptr(logits), _ptr(bias), T, E, k, 1 if normalize else 0, _ptr(ids), _ptr(weights),
+                        _stream(logits.device)), "moe_route")
+    return ids, weights
 
 
 def combine(dst, weights, shared=None, out=None):
