@@ -8,6 +8,9 @@
  *            "CUDA: better MoE implementation" (sections 1.2, 2, 2.1, 5, 6).
  *   [b11370] "llama.cpp 發布 b11370，CUDA 後端將共享專家融合進 MMVQ" - release
  *            note of llama.cpp PR #29184 "CUDA: fuse shared experts into MMVQ".
+ *   [cmoe]   "Optimalizace MoE modelů na slabém GPU: spuštění GPT-OSS-120B s
+ *            6 GB VRAM až 30 t/s", section "Architektura Mixture of Experts"
+ *            (the router before the path and the weighted combine after it).
  *
  * Conventions shared by every entry point
  * ---------------------------------------
