@@ -81,7 +81,7 @@ class ClockSampler:
     """SM clock and clock-event (throttle) reasons of one GPU while running:
     read-only NVML queries every few milliseconds from a background thread
     (the timed region can be only tens of milliseconds), else nvidia-smi.
-    The samples are also written to gpurun_out/clocks_gpu<i>.csv."""
+    The samples are also written out as clocks_gpu<i>.csv."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
