@@ -63,6 +63,24 @@ def test_ragged_shapes(path, mode, x_type):
 
 
 @pytest.mark.parametrize("path", PATHS)
+@pytest.mark.parametrize("E,k,T", [(300, 4, 40), (16384, 6, 24), (1024, 1023, 2)])
+def test_expert_and_slot_count_limits(path, E, k, T):
+    """Beyond 256 experts the GEMM reads its schedule tables from global memory
+    (300 experts); the largest expert count (16384) runs the row-id pass with
+    one counting chunk; the largest k (1023: 2046 slots, past the mat-vec
+    kernel's slot limit, so both settings run the GEMM).  Small matrices keep
+    the oracle fast."""
+    n_in, n_out = 64, 48
+    W = workloads.q8_0_weights(E, n_out, n_in, 17, 13)
+    ids = workloads.routing("uniform", T, E, k, 17)
+    x = workloads.activations(T, n_in, "bf16", 17, 14)
+    ref, tol = oracle.mul_mat_id(W, x, "bf16", ids)
+    with paths(path):
+        dst = moe.mul_mat_id(prep(W), E, n_out, n_in, to_dev_x(x, "bf16"), torch.from_numpy(ids).cuda())
+    check_close(dst, ref, tol, f"limits path {path} E={E} k={k} T={T}")
+
+
+@pytest.mark.parametrize("path", PATHS)
 @pytest.mark.parametrize("mode", ["broadcast", "per_slot"])
 def test_skew_shape_small_batch(path, mode):
     """The skewed-load expert shape (2880 x 2880, 128 experts, top-4 Zipf) on
