@@ -73,6 +73,26 @@ def test_host_argument_checks_without_gpu():
                        nul) == moe.ERR_INVALID
 
 
+def test_router_and_combine_argument_checks_without_gpu():
+    lib = moe.lib()
+    nul = None
+    # router: k outside [1, n_experts], no logits, more than 1024 experts, too many tokens
+    assert lib.moe_route(nul, nul, 4, 8, 0, 1, nul, nul, nul) == moe.ERR_INVALID
+    assert lib.moe_route(nul, nul, 4, 8, 9, 1, nul, nul, nul) == moe.ERR_INVALID
+    assert lib.moe_route(nul, nul, 4, 8, 2, 1, nul, nul, nul) == moe.ERR_INVALID
+    assert lib.moe_route(nul, nul, 4, 1025, 2, 1, nul, nul, nul) == moe.ERR_RANGE
+    assert lib.moe_route(nul, nul, 1 << 22, 8, 2, 1, nul, nul, nul) == moe.ERR_RANGE
+    assert lib.moe_route(nul, nul, 0, 8, 2, 1, nul, nul, nul) == moe.OK  # nothing to do
+    # combine: k < 1, n < 1, null pointers, misaligned, k >= 2^10, too many tokens
+    assert lib.moe_combine(nul, nul, nul, 4, 0, 8, nul, nul) == moe.ERR_INVALID
+    assert lib.moe_combine(nul, nul, nul, 4, 2, 0, nul, nul) == moe.ERR_INVALID
+    assert lib.moe_combine(nul, nul, nul, 4, 2, 8, nul, nul) == moe.ERR_INVALID
+    assert lib.moe_combine(4098, 4096, nul, 4, 2, 8, 4096, nul) == moe.ERR_INVALID
+    assert lib.moe_combine(nul, nul, nul, 4, 1024, 8, nul, nul) == moe.ERR_RANGE
+    assert lib.moe_combine(nul, nul, nul, 1 << 22, 2, 8, nul, nul) == moe.ERR_RANGE
+    assert lib.moe_combine(nul, nul, nul, 0, 2, 8, nul, nul) == moe.OK
+
+
 def test_gemv_threshold_setting():
     old = moe.get_gemv_threshold()
     try:
