@@ -440,3 +440,21 @@ def test_route_tolerance_covers_a_float32_softmax():
         s = (s + sel[:, i:i + 1]).astype(np.float32)
     w32 = (sel / s).astype(np.float32)
     assert np.all(np.abs(w32 - w) <= tol)
+
+
+def test_float32_bounds_are_tight_enough_to_mean_something():
+    # the combine and router bounds stay within a few hundred float32 units, so a
+    # dropped term or a wrong weight (errors of order the values) cannot hide in them
+    rng = np.random.default_rng(8)
+    dst = rng.normal(size=(4, 8, 32)).astype(np.float32)
+    r = rng.uniform(0.05, 1.0, size=(4, 8)).astype(np.float32)
+    y, mag = oracle.combine(dst, r)
+    tol = oracle.combine_tolerance(mag, 8, False)
+    assert np.all(tol <= 1e-5 * mag + 1e-30)
+    y_drop, _ = oracle.combine(dst[:, :7, :], r[:, :7])  # one slot missing
+    assert np.any(np.abs(y_drop - y) > tol)
+    logits = rng.normal(size=(6, 256)).astype(np.float32)
+    ids, w, tol_w = oracle.route(logits, 8)
+    assert np.all(tol_w <= 1e-4 * w)
+    _, w_un, _ = oracle.route(logits, 8, normalize=False)  # forgetting the renormalisation
+    assert np.all(np.abs(w_un - w) > tol_w)
