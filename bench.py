@@ -209,7 +209,13 @@ def cpu_baseline(budget_s: float = 12.0, t0: int = 0):
     while elapsed < budget_s and i < len(order):
         batch = order[i:i + cores]
         i += len(batch)
-        es = sorted(set(int(flat[s]) for s in batch))
+        es = set(int(flat[s]) for s in batch)
+        # the oracle checks k <= n_experts: a small batch may touch fewer than k
+        # experts, so pad the set with unused ones (their rows are never computed)
+        pad = (e for e in range(WL.n_experts) if e not in es)
+        while len(es) < WL.k:
+            es.add(next(pad))
+        es = sorted(es)
         remap = {e: j for j, e in enumerate(es)}
         Wg = np.concatenate([workloads.q8_0_weights_experts(e, 1, WL.n_out, WL.n_in, WL.seed, workloads.T_WG)
                              for e in es])

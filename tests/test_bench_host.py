@@ -84,3 +84,10 @@ def test_traffic_is_null_once_a_gemm_source_changes(monkeypatch, tmp_path):
     assert bench.gate_up_traffic() == bench.GATE_UP_TRAFFIC["bytes_per_launch"]
     (csrc / "gemm.cu").write_bytes(b"changed")
     assert bench.gate_up_traffic() is None
+
+
+def test_cpu_baseline_survives_batches_with_fewer_experts_than_k(monkeypatch):
+    # with 2 host cores a batch holds 2 slots, so fewer than k = 8 distinct experts
+    monkeypatch.setattr(bench.os, "sched_getaffinity", lambda pid: {0, 1})
+    r = bench.cpu_baseline(budget_s=0.01)
+    assert r["value"] > 0 and r["cores"] == 2 and r["kind"] == "oracle"
