@@ -204,7 +204,9 @@ def cpu_baseline(budget_s: float = 12.0, t0: int = 0):
     flat = ids.reshape(-1)
     rng = np.random.default_rng(1)
     order = rng.permutation(len(flat))
-    cores = len(os.sched_getaffinity(0))
+    # all host cores, whatever a launcher set OMP_NUM_THREADS to; report the threads used
+    oracle.set_num_threads(len(os.sched_getaffinity(0)))
+    cores = oracle.num_threads()
     done, elapsed, i = 0, 0.0, 0
     while elapsed < budget_s and i < len(order):
         batch = order[i:i + cores]

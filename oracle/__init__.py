@@ -53,6 +53,9 @@ def _L():
         _lib.oracle_combine.argtypes = [vp, vp, vp, i64, i32, i64, vp, vp]
         _lib.oracle_combine.restype = None
         _lib.oracle_route.argtypes = [vp, vp, i64, i32, i32, i32, vp, vp]
+        _lib.oracle_num_threads.argtypes = []
+        _lib.oracle_set_num_threads.argtypes = [i32]
+        _lib.oracle_set_num_threads.restype = None
     return _lib
 
 
@@ -226,3 +229,14 @@ def route_tolerance(w, logits, E, k, normalize):
     span = (logits.max(axis=1) - logits.min(axis=1)).astype(np.float64)[:, None]
     rel = (span + 8.0 + E + (k if normalize else 0)) * 2.0 ** -24
     return rel * np.abs(w) + 1e-30
+
+
+def num_threads() -> int:
+    """OpenMP threads the oracle's parallel loops use."""
+    return int(_L().oracle_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """Set the oracle's OpenMP thread count (e.g. to all host cores when a
+    launcher capped OMP_NUM_THREADS)."""
+    _L().oracle_set_num_threads(int(n))

@@ -43,6 +43,7 @@
  * propagated through SwiGLU (see oracle_ffn_rows).
  */
 #include <math.h>
+#include <omp.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -431,3 +432,8 @@ int oracle_route(const float *logits, const float *bias, int64_t n_tokens, int n
     }
     return 0;
 }
+
+/* Threads the parallel loops above use (timing runs report it), and a way to
+ * set it to the host's cores when a launcher has capped it. */
+int oracle_num_threads(void) { return omp_get_max_threads(); }
+void oracle_set_num_threads(int n) { if (n > 0) omp_set_num_threads(n); }
