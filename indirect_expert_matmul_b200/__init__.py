@@ -110,6 +110,15 @@ def _cuda(t, name, dtype=None):
     return t
 
 
+def _need(t, name, dtype, numel):
+    """A caller-supplied output or workspace: CUDA, contiguous, of `dtype`, and
+    at least `numel` elements (the library writes that many)."""
+    _cuda(t, name, dtype)
+    if t.numel() < numel:
+        raise ValueError(f"{name} holds {t.numel()} elements; the call writes {numel}")
+    return t
+
+
 # ----------------------------------------------------------------- memory
 def workspace_size(n_tokens, k, n_experts, n_in, n_hidden=0, n_hidden_shared=0, x_dtype=torch.bfloat16) -> int:
     return _L().moe_workspace_size(n_tokens, k, n_experts, n_in, n_hidden, n_hidden_shared, _XTYPE[x_dtype])
@@ -139,6 +148,7 @@ def weights_prepare(q8_0, n_experts, n_out, n_in, out=None):
     n = weights_prepared_size(n_experts, n_out, n_in)
     if out is None:
         out = torch.empty(n, dtype=torch.uint8, device=q8_0.device)
+    _need(out, "out", torch.uint8, n)
     _chk(_L().moe_weights_prepare(_ptr(q8_0), n_experts, n_out, n_in, _ptr(out), _stream(q8_0.device)),
          "moe_weights_prepare")
     return out
@@ -156,6 +166,7 @@ def row_ids(ids, n_experts, mode="broadcast", ws=None):
     bounds = torch.empty(n_experts + 1, dtype=torch.int32, device=dev)
     if ws is None:
         ws = workspace(T, k, n_experts, 0, device=dev)
+    _need(ws, "ws", torch.uint8, workspace_size(T, k, n_experts, 0))
     _chk(_L().moe_row_ids(_ptr(ids), T, k, n_experts, _MODE[mode], _ptr(src1), _ptr(dst), _ptr(bounds), _ptr(ws),
                           _stream(dev)), "moe_row_ids")
     return src1[:S], dst[:S], bounds
@@ -167,15 +178,18 @@ def mul_mat_id(W, n_experts, n_out, n_in, x, ids, mode="broadcast", ws=None, out
 
     Without `ws` the call makes its own workspace, synchronises and raises
     MoeError on a device-side error; with `ws` the caller reads get_status."""
-    _cuda(W, "W", torch.uint8)
     _cuda(x, "x")
     _cuda(ids, "ids", torch.int32)
     T, k = ids.shape
+    _need(W, "W", torch.uint8, weights_prepared_size(n_experts, n_out, n_in))
+    _need(x, "x", x.dtype, (T if _MODE[mode] == BROADCAST else T * k) * n_in)
     own_ws = ws is None
     if own_ws:
         ws = workspace(T, k, n_experts, n_in, x_dtype=x.dtype, device=x.device)
+    _need(ws, "ws", torch.uint8, workspace_size(T, k, n_experts, n_in, x_dtype=x.dtype))
     if out is None:
         out = torch.empty((T, k, n_out), dtype=torch.float32, device=x.device)
+    _need(out, "out", torch.float32, T * k * n_out)
     _chk(_L().moe_mul_mat_id(_ptr(W), n_experts, n_out, n_in, _ptr(x), _XTYPE[x.dtype], _ptr(ids), T, k,
                              _MODE[mode], _ptr(out), _ptr(ws), _stream(x.device)), "moe_mul_mat_id")
     if own_ws:
@@ -183,12 +197,21 @@ def mul_mat_id(W, n_experts, n_out, n_in, x, ids, mode="broadcast", ws=None, out
     return out
 
 
+def _check_ffn_inputs(Wg, Wu, Wd, Sg, Su, Sd, n_experts, n_embd, n_ff, n_ff_sh, x, T):
+    _need(Wg, "Wg", torch.uint8, weights_prepared_size(n_experts, n_ff, n_embd))
+    _need(Wu, "Wu", torch.uint8, weights_prepared_size(n_experts, n_ff, n_embd))
+    _need(Wd, "Wd", torch.uint8, weights_prepared_size(n_experts, n_embd, n_ff))
+    if n_ff_sh:
+        _need(Sg, "Sg", torch.uint8, weights_prepared_size(1, n_ff_sh, n_embd))
+        _need(Su, "Su", torch.uint8, weights_prepared_size(1, n_ff_sh, n_embd))
+        _need(Sd, "Sd", torch.uint8, weights_prepared_size(1, n_embd, n_ff_sh))
+    _need(x, "x", x.dtype, T * n_embd)
+
+
 def ffn(Wg, Wu, Wd, n_experts, n_embd, n_ff, x, ids, shared=None, ws=None, out=None, out_shared=None):
     """Routed SwiGLU expert FFN (+ optional shared expert (Sg, Su, Sd, n_ff_shared)).
 
     Returns (dst [T][k][n_embd], dst_shared [T][n_embd] or None), float32."""
-    for name, t in (("Wg", Wg), ("Wu", Wu), ("Wd", Wd)):
-        _cuda(t, name, torch.uint8)
     _cuda(x, "x")
     _cuda(ids, "ids", torch.int32)
     T, k = ids.shape
@@ -196,13 +219,18 @@ def ffn(Wg, Wu, Wd, n_experts, n_embd, n_ff, x, ids, shared=None, ws=None, out=N
     n_ff_sh = 0
     if shared is not None:
         Sg, Su, Sd, n_ff_sh = shared
+    _check_ffn_inputs(Wg, Wu, Wd, Sg, Su, Sd, n_experts, n_embd, n_ff, n_ff_sh, x, T)
     own_ws = ws is None
     if own_ws:
         ws = workspace(T, k, n_experts, n_embd, n_ff, n_ff_sh, x.dtype, device=x.device)
+    _need(ws, "ws", torch.uint8, workspace_size(T, k, n_experts, n_embd, n_ff, n_ff_sh, x.dtype))
     if out is None:
         out = torch.empty((T, k, n_embd), dtype=torch.float32, device=x.device)
+    _need(out, "out", torch.float32, T * k * n_embd)
     if shared is not None and out_shared is None:
         out_shared = torch.empty((T, n_embd), dtype=torch.float32, device=x.device)
+    if shared is not None:
+        _need(out_shared, "out_shared", torch.float32, T * n_embd)
     _chk(_L().moe_ffn(_ptr(Wg), _ptr(Wu), _ptr(Wd), n_experts, n_embd, n_ff, _ptr(Sg), _ptr(Su), _ptr(Sd), n_ff_sh,
                       _ptr(x), _XTYPE[x.dtype], _ptr(ids), T, k, _ptr(out), _ptr(out_shared), _ptr(ws),
                       _stream(x.device)), "moe_ffn")
@@ -216,21 +244,23 @@ def ffn_decode_noalloc(Wg, Wu, Wd, n_experts, n_embd, n_ff, x, ids, shared=None,
     """moe_ffn for decode sizes (n_tokens*k <= 64, n_ff and n_ff_shared <= 2048)
     through the entry point that takes no workspace.  `status`: optional int32
     CUDA tensor of one element that receives the device status."""
-    for name, t in (("Wg", Wg), ("Wu", Wu), ("Wd", Wd)):
-        _cuda(t, name, torch.uint8)
     _cuda(x, "x")
     _cuda(ids, "ids", torch.int32)
-    if status is not None:
-        _cuda(status, "status", torch.int32)
     T, k = ids.shape
     Sg = Su = Sd = None
     n_ff_sh = 0
     if shared is not None:
         Sg, Su, Sd, n_ff_sh = shared
+    _check_ffn_inputs(Wg, Wu, Wd, Sg, Su, Sd, n_experts, n_embd, n_ff, n_ff_sh, x, T)
     if out is None:
         out = torch.empty((T, k, n_embd), dtype=torch.float32, device=x.device)
+    _need(out, "out", torch.float32, T * k * n_embd)
     if shared is not None and out_shared is None:
         out_shared = torch.empty((T, n_embd), dtype=torch.float32, device=x.device)
+    if shared is not None:
+        _need(out_shared, "out_shared", torch.float32, T * n_embd)
+    if status is not None:
+        _need(status, "status", torch.int32, 1)
     _chk(_L().moe_ffn_decode_noalloc(_ptr(Wg), _ptr(Wu), _ptr(Wd), n_experts, n_embd, n_ff, _ptr(Sg), _ptr(Su),
                                      _ptr(Sd), n_ff_sh, _ptr(x), _XTYPE[x.dtype], _ptr(ids), T, k, _ptr(out),
                                      _ptr(out_shared), _ptr(status), _stream(x.device)), "moe_ffn_decode_noalloc")
@@ -245,10 +275,14 @@ def route(logits, k, bias=None, normalize=True, ids=None, weights=None):
     T, E = logits.shape
     if bias is not None:
         _cuda(bias, "bias", torch.float32)
+    if bias is not None:
+        _need(bias, "bias", torch.float32, E)
     if ids is None:
         ids = torch.empty((T, k), dtype=torch.int32, device=logits.device)
     if weights is None:
         weights = torch.empty((T, k), dtype=torch.float32, device=logits.device)
+    _need(ids, "ids", torch.int32, T * k)
+    _need(weights, "weights", torch.float32, T * k)
     _chk(_L().moe_route(_ptr(logits), _ptr(bias), T, E, k, 1 if normalize else 0, _ptr(ids), _ptr(weights),
                         _stream(logits.device)), "moe_route")
     return ids, weights
@@ -265,9 +299,10 @@ def combine(dst, weights, shared=None, out=None):
     if dst.numel() != T * k * n:
         raise ValueError("dst must hold n_tokens*k rows of n")
     if shared is not None:
-        _cuda(shared, "shared", torch.float32)
+        _need(shared, "shared", torch.float32, T * n)
     if out is None:
         out = torch.empty((T, n), dtype=torch.float32, device=dst.device)
+    _need(out, "out", torch.float32, T * n)
     _chk(_L().moe_combine(_ptr(dst), _ptr(weights), _ptr(shared), T, k, n, _ptr(out), _stream(dst.device)),
          "moe_combine")
     return out

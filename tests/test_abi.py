@@ -100,3 +100,12 @@ def test_gemv_threshold_setting():
         assert moe.get_gemv_threshold() == 3
     finally:
         moe.set_gemv_threshold(old)
+
+
+def test_caller_buffers_are_checked_before_any_launch(monkeypatch):
+    # outputs and workspaces handed in by the caller must hold what the call writes
+    import torch
+    monkeypatch.setattr(moe, "_cuda", lambda t, name, dtype=None: t)  # no GPU here: skip the device check
+    moe._need(torch.empty(10), "out", torch.float32, 10)
+    with pytest.raises(ValueError, match="holds 9 elements"):
+        moe._need(torch.empty(9), "out", torch.float32, 10)

@@ -74,6 +74,13 @@ def test_noalloc_refuses_sizes_past_its_scratch():
     with pytest.raises(moe.MoeError) as e:
         moe.ffn_decode_noalloc(dWg, dWu, dWd, wl.n_experts, wl.n_in, wl.n_out, big_x, big_ids)
     assert e.value.code == moe.ERR_RANGE
-    with pytest.raises(moe.MoeError) as e:  # n_ff past 2048 (checked before the weights are touched)
-        moe.ffn_decode_noalloc(dWg, dWu, dWd, wl.n_experts, wl.n_in, 2080, xd, torch.from_numpy(ids).cuda())
-    assert e.value.code == moe.ERR_RANGE
+    # n_ff past 2048: the entry point refuses it on the host, before any weight is read
+    ids_d = torch.from_numpy(ids).cuda()
+    out = torch.empty((1, wl.k, wl.n_in), dtype=torch.float32, device="cuda")
+    st = moe.lib().moe_ffn_decode_noalloc(dWg.data_ptr(), dWu.data_ptr(), dWd.data_ptr(), wl.n_experts, wl.n_in, 2080,
+                                          None, None, None, 0, xd.data_ptr(), moe.BF16, ids_d.data_ptr(), 1, wl.k,
+                                          out.data_ptr(), None, None, None)
+    assert st == moe.ERR_RANGE
+    # through the binding, weights too small for the stated n_ff are refused before the call
+    with pytest.raises(ValueError):
+        moe.ffn_decode_noalloc(dWg, dWu, dWd, wl.n_experts, wl.n_in, 2080, xd, ids_d)
