@@ -274,8 +274,6 @@ def route(logits, k, bias=None, normalize=True, ids=None, weights=None):
     _cuda(logits, "logits", torch.float32)
     T, E = logits.shape
     if bias is not None:
-        _cuda(bias, "bias", torch.float32)
-    if bias is not None:
         _need(bias, "bias", torch.float32, E)
     if ids is None:
         ids = torch.empty((T, k), dtype=torch.int32, device=logits.device)
