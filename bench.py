@@ -30,10 +30,10 @@ import numpy as np
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 
-# dram__bytes_read.sum + dram__bytes_write.sum of one V3 gate/up launch: the 32-expert,
-# 512-token capture (same per-expert load) times 8, as summarised in
-# profiles/grouped_gemm_gate_up_v3_shape_32experts.md.  It describes only the kernel
-# sources it was measured on; when any of them changes the bench reports null.
+# dram__bytes_read.sum + dram__bytes_write.sum of one V3 gate/up launch: an ncu
+# capture of the 32-expert, 512-token case (same per-expert load) times 8.  It
+# describes only the kernel sources it was measured on; when any of them changes
+# the bench reports null.
 GATE_UP_TRAFFIC = {
     "bytes_per_launch": 8 * (1112740864 + 16419584),
     "sources_sha256": {
@@ -80,8 +80,8 @@ def load_peaks():
 class ClockSampler:
     """SM clock and clock-event (throttle) reasons of one GPU while running:
     read-only NVML queries every few milliseconds from a background thread
-    (the timed region can be only tens of milliseconds), else nvidia-smi.
-    The samples are also written out as clocks_gpu<i>.csv."""
+    (the timed region can be only tens of milliseconds), else nvidia-smi
+    writing into a temporary file that is removed afterwards."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -95,7 +95,7 @@ class ClockSampler:
         self.nv = None
         self.samples = []  # (sm MHz, reason bits)
         self.smax = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+        self.path = None
 
     def _nvml_handle(self):
         import pynvml
@@ -132,8 +132,9 @@ class ClockSampler:
         except Exception:
             self.nv = None
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.f = open(self.path, "w")
+            import tempfile
+            fd, self.path = tempfile.mkstemp(prefix=f"clocks_gpu{self.gpu}_", suffix=".csv")
+            self.f = os.fdopen(fd, "w")
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
                                           "--format=csv,noheader,nounits", "-lms", "100"],
                                          stdout=self.f, stderr=subprocess.DEVNULL)
@@ -146,14 +147,6 @@ class ClockSampler:
         if self.nv is not None:
             self.stop.set()
             self.thread.join(timeout=2)
-            try:
-                os.makedirs(os.path.dirname(self.path), exist_ok=True)
-                with open(self.path, "w") as f:
-                    f.write("# sm_mhz, sm_max_mhz, clock event reason bits (NVML), one line per sample\n")
-                    for sm, bits in self.samples:
-                        f.write(f"{sm}, {self.smax}, {bits:#x}\n")
-            except OSError:
-                pass
             return
         if self.proc is not None:
             self.proc.terminate()
@@ -171,11 +164,17 @@ class ClockSampler:
             load = [x for x in sm if smax and x > 0.3 * smax] or sm
             return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": smax,
                     "reasons": reasons, "samples": len(sm), "source": "nvml"}
-        if self.proc is None or not os.path.exists(self.path):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         sm, smax, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in open(self.path):
+        with open(self.path) as f:
+            lines = f.readlines()
+        try:
+            os.unlink(self.path)
+        except OSError:
+            pass
+        for line in lines:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
                 continue
@@ -350,7 +349,7 @@ def run_ours(args):
     else:
         roof = {"bound": "tensor", "achieved": round(gu_tflops, 1), "peak": tc_peak, "unit": "TFLOP/s",
                 "frac": round(gu_tflops / tc_peak, 4)}
-    traffic = args.traffic if args.traffic is not None else (None if small else gate_up_traffic())
+    traffic = None if small else gate_up_traffic()
     roof.update({"traffic": traffic, "kernel": "grouped_gemm_kernel<1> (gate/up + SwiGLU)",
                  "peak_source": peak_src, "ms_per_launch": round(t_gu * 1e3, 4),
                  "tensor_tflops": round(gu_tflops, 1), "tensor_frac": round(gu_tflops / tc_peak, 4),
@@ -584,8 +583,6 @@ def main():
     ap.add_argument("--decode-tokens", type=int, default=None, help="profiling only: one decode token count")
     ap.add_argument("--experts", type=int, default=None, help="profiling only: fewer experts than the V3 layer")
     ap.add_argument("--tokens", type=int, default=None, help="profiling only: tokens per GPU")
-    ap.add_argument("--traffic", type=float, default=None,
-                    help="dram bytes per launch of the dominant kernel from an ncu capture (null if stale)")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)

@@ -217,7 +217,11 @@ MOE_API moe_status moe_ffn_decode_noalloc(const void *Wg, const void *Wu, const 
  *   ids[t][:]  = the k largest keys in descending order, equal keys in
  *                ascending expert index      (int32 [n_tokens][k])
  *   weights[t][i] = softmax(logits[t])[ids[t][i]], divided by their sum over
- *                the k when normalize != 0   (float [n_tokens][k])
+ *                the k when normalize != 0   (float [n_tokens][k]).  The
+ *                renormalised form is evaluated as the softmax over the k
+ *                chosen logits (the same quantity), so it stays finite and
+ *                sums to one even where the chosen experts' probabilities
+ *                underflow in float (chosen logits far below the row's top).
  * logits: float [n_tokens][n_experts]; bias: float [n_experts] or NULL.  The
  * choice is a pure function of the float keys (bit-identical to any exact
  * evaluation of the rule above); the weights are within

@@ -100,20 +100,30 @@ _XTYPE = {torch.bfloat16: BF16, torch.float16: F16, torch.float32: F32}
 _MODE = {"broadcast": BROADCAST, "per_slot": PER_SLOT, BROADCAST: BROADCAST, PER_SLOT: PER_SLOT}
 
 
-def _cuda(t, name, dtype=None):
+def _gpu(t, name):
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
+
+
+def _cuda(t, name, dtype=None, device=None):
+    """A CUDA tensor, contiguous, of `dtype` (if given) and on `device` (if
+    given: the device whose stream the call launches on - a tensor elsewhere
+    would reach the kernels as another GPU's or an unmapped address)."""
+    _gpu(t, name)
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     if dtype is not None and t.dtype != dtype:
         raise ValueError(f"{name} must be {dtype}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}; the call runs on {device}")
     return t
 
 
-def _need(t, name, dtype, numel):
-    """A caller-supplied output or workspace: CUDA, contiguous, of `dtype`, and
-    at least `numel` elements (the library writes that many)."""
-    _cuda(t, name, dtype)
+def _need(t, name, dtype, numel, device=None):
+    """A caller-supplied input, output or workspace: CUDA, contiguous, of
+    `dtype`, on `device`, and at least `numel` elements (the library reads or
+    writes that many)."""
+    _cuda(t, name, dtype, device)
     if t.numel() < numel:
         raise ValueError(f"{name} holds {t.numel()} elements; the call writes {numel}")
     return t
@@ -148,7 +158,7 @@ def weights_prepare(q8_0, n_experts, n_out, n_in, out=None):
     n = weights_prepared_size(n_experts, n_out, n_in)
     if out is None:
         out = torch.empty(n, dtype=torch.uint8, device=q8_0.device)
-    _need(out, "out", torch.uint8, n)
+    _need(out, "out", torch.uint8, n, q8_0.device)
     _chk(_L().moe_weights_prepare(_ptr(q8_0), n_experts, n_out, n_in, _ptr(out), _stream(q8_0.device)),
          "moe_weights_prepare")
     return out
@@ -166,7 +176,7 @@ def row_ids(ids, n_experts, mode="broadcast", ws=None):
     bounds = torch.empty(n_experts + 1, dtype=torch.int32, device=dev)
     if ws is None:
         ws = workspace(T, k, n_experts, 0, device=dev)
-    _need(ws, "ws", torch.uint8, workspace_size(T, k, n_experts, 0))
+    _need(ws, "ws", torch.uint8, workspace_size(T, k, n_experts, 0), dev)
     _chk(_L().moe_row_ids(_ptr(ids), T, k, n_experts, _MODE[mode], _ptr(src1), _ptr(dst), _ptr(bounds), _ptr(ws),
                           _stream(dev)), "moe_row_ids")
     return src1[:S], dst[:S], bounds
@@ -179,17 +189,18 @@ def mul_mat_id(W, n_experts, n_out, n_in, x, ids, mode="broadcast", ws=None, out
     Without `ws` the call makes its own workspace, synchronises and raises
     MoeError on a device-side error; with `ws` the caller reads get_status."""
     _cuda(x, "x")
-    _cuda(ids, "ids", torch.int32)
+    dev = x.device
+    _cuda(ids, "ids", torch.int32, dev)
     T, k = ids.shape
-    _need(W, "W", torch.uint8, weights_prepared_size(n_experts, n_out, n_in))
+    _need(W, "W", torch.uint8, weights_prepared_size(n_experts, n_out, n_in), dev)
     _need(x, "x", x.dtype, (T if _MODE[mode] == BROADCAST else T * k) * n_in)
     own_ws = ws is None
     if own_ws:
-        ws = workspace(T, k, n_experts, n_in, x_dtype=x.dtype, device=x.device)
-    _need(ws, "ws", torch.uint8, workspace_size(T, k, n_experts, n_in, x_dtype=x.dtype))
+        ws = workspace(T, k, n_experts, n_in, x_dtype=x.dtype, device=dev)
+    _need(ws, "ws", torch.uint8, workspace_size(T, k, n_experts, n_in, x_dtype=x.dtype), dev)
     if out is None:
-        out = torch.empty((T, k, n_out), dtype=torch.float32, device=x.device)
-    _need(out, "out", torch.float32, T * k * n_out)
+        out = torch.empty((T, k, n_out), dtype=torch.float32, device=dev)
+    _need(out, "out", torch.float32, T * k * n_out, dev)
     _chk(_L().moe_mul_mat_id(_ptr(W), n_experts, n_out, n_in, _ptr(x), _XTYPE[x.dtype], _ptr(ids), T, k,
                              _MODE[mode], _ptr(out), _ptr(ws), _stream(x.device)), "moe_mul_mat_id")
     if own_ws:
@@ -198,13 +209,14 @@ def mul_mat_id(W, n_experts, n_out, n_in, x, ids, mode="broadcast", ws=None, out
 
 
 def _check_ffn_inputs(Wg, Wu, Wd, Sg, Su, Sd, n_experts, n_embd, n_ff, n_ff_sh, x, T):
-    _need(Wg, "Wg", torch.uint8, weights_prepared_size(n_experts, n_ff, n_embd))
-    _need(Wu, "Wu", torch.uint8, weights_prepared_size(n_experts, n_ff, n_embd))
-    _need(Wd, "Wd", torch.uint8, weights_prepared_size(n_experts, n_embd, n_ff))
+    dev = x.device
+    _need(Wg, "Wg", torch.uint8, weights_prepared_size(n_experts, n_ff, n_embd), dev)
+    _need(Wu, "Wu", torch.uint8, weights_prepared_size(n_experts, n_ff, n_embd), dev)
+    _need(Wd, "Wd", torch.uint8, weights_prepared_size(n_experts, n_embd, n_ff), dev)
     if n_ff_sh:
-        _need(Sg, "Sg", torch.uint8, weights_prepared_size(1, n_ff_sh, n_embd))
-        _need(Su, "Su", torch.uint8, weights_prepared_size(1, n_ff_sh, n_embd))
-        _need(Sd, "Sd", torch.uint8, weights_prepared_size(1, n_embd, n_ff_sh))
+        _need(Sg, "Sg", torch.uint8, weights_prepared_size(1, n_ff_sh, n_embd), dev)
+        _need(Su, "Su", torch.uint8, weights_prepared_size(1, n_ff_sh, n_embd), dev)
+        _need(Sd, "Sd", torch.uint8, weights_prepared_size(1, n_embd, n_ff_sh), dev)
     _need(x, "x", x.dtype, T * n_embd)
 
 
@@ -213,7 +225,8 @@ def ffn(Wg, Wu, Wd, n_experts, n_embd, n_ff, x, ids, shared=None, ws=None, out=N
 
     Returns (dst [T][k][n_embd], dst_shared [T][n_embd] or None), float32."""
     _cuda(x, "x")
-    _cuda(ids, "ids", torch.int32)
+    dev = x.device
+    _cuda(ids, "ids", torch.int32, dev)
     T, k = ids.shape
     Sg = Su = Sd = None
     n_ff_sh = 0
@@ -222,15 +235,15 @@ def ffn(Wg, Wu, Wd, n_experts, n_embd, n_ff, x, ids, shared=None, ws=None, out=N
     _check_ffn_inputs(Wg, Wu, Wd, Sg, Su, Sd, n_experts, n_embd, n_ff, n_ff_sh, x, T)
     own_ws = ws is None
     if own_ws:
-        ws = workspace(T, k, n_experts, n_embd, n_ff, n_ff_sh, x.dtype, device=x.device)
-    _need(ws, "ws", torch.uint8, workspace_size(T, k, n_experts, n_embd, n_ff, n_ff_sh, x.dtype))
+        ws = workspace(T, k, n_experts, n_embd, n_ff, n_ff_sh, x.dtype, device=dev)
+    _need(ws, "ws", torch.uint8, workspace_size(T, k, n_experts, n_embd, n_ff, n_ff_sh, x.dtype), dev)
     if out is None:
-        out = torch.empty((T, k, n_embd), dtype=torch.float32, device=x.device)
-    _need(out, "out", torch.float32, T * k * n_embd)
+        out = torch.empty((T, k, n_embd), dtype=torch.float32, device=dev)
+    _need(out, "out", torch.float32, T * k * n_embd, dev)
     if shared is not None and out_shared is None:
-        out_shared = torch.empty((T, n_embd), dtype=torch.float32, device=x.device)
+        out_shared = torch.empty((T, n_embd), dtype=torch.float32, device=dev)
     if shared is not None:
-        _need(out_shared, "out_shared", torch.float32, T * n_embd)
+        _need(out_shared, "out_shared", torch.float32, T * n_embd, dev)
     _chk(_L().moe_ffn(_ptr(Wg), _ptr(Wu), _ptr(Wd), n_experts, n_embd, n_ff, _ptr(Sg), _ptr(Su), _ptr(Sd), n_ff_sh,
                       _ptr(x), _XTYPE[x.dtype], _ptr(ids), T, k, _ptr(out), _ptr(out_shared), _ptr(ws),
                       _stream(x.device)), "moe_ffn")
@@ -245,7 +258,8 @@ def ffn_decode_noalloc(Wg, Wu, Wd, n_experts, n_embd, n_ff, x, ids, shared=None,
     through the entry point that takes no workspace.  `status`: optional int32
     CUDA tensor of one element that receives the device status."""
     _cuda(x, "x")
-    _cuda(ids, "ids", torch.int32)
+    dev = x.device
+    _cuda(ids, "ids", torch.int32, dev)
     T, k = ids.shape
     Sg = Su = Sd = None
     n_ff_sh = 0
@@ -253,14 +267,14 @@ def ffn_decode_noalloc(Wg, Wu, Wd, n_experts, n_embd, n_ff, x, ids, shared=None,
         Sg, Su, Sd, n_ff_sh = shared
     _check_ffn_inputs(Wg, Wu, Wd, Sg, Su, Sd, n_experts, n_embd, n_ff, n_ff_sh, x, T)
     if out is None:
-        out = torch.empty((T, k, n_embd), dtype=torch.float32, device=x.device)
-    _need(out, "out", torch.float32, T * k * n_embd)
+        out = torch.empty((T, k, n_embd), dtype=torch.float32, device=dev)
+    _need(out, "out", torch.float32, T * k * n_embd, dev)
     if shared is not None and out_shared is None:
-        out_shared = torch.empty((T, n_embd), dtype=torch.float32, device=x.device)
+        out_shared = torch.empty((T, n_embd), dtype=torch.float32, device=dev)
     if shared is not None:
-        _need(out_shared, "out_shared", torch.float32, T * n_embd)
+        _need(out_shared, "out_shared", torch.float32, T * n_embd, dev)
     if status is not None:
-        _need(status, "status", torch.int32, 1)
+        _need(status, "status", torch.int32, 1, dev)
     _chk(_L().moe_ffn_decode_noalloc(_ptr(Wg), _ptr(Wu), _ptr(Wd), n_experts, n_embd, n_ff, _ptr(Sg), _ptr(Su),
                                      _ptr(Sd), n_ff_sh, _ptr(x), _XTYPE[x.dtype], _ptr(ids), T, k, _ptr(out),
                                      _ptr(out_shared), _ptr(status), _stream(x.device)), "moe_ffn_decode_noalloc")
@@ -272,15 +286,16 @@ def route(logits, k, bias=None, normalize=True, ids=None, weights=None):
     the lower expert) and their softmax weights.  logits: float32 CUDA [T][E];
     bias: float32 [E] or None.  Returns (ids int32 [T][k], weights float32 [T][k])."""
     _cuda(logits, "logits", torch.float32)
+    dev = logits.device
     T, E = logits.shape
     if bias is not None:
-        _need(bias, "bias", torch.float32, E)
+        _need(bias, "bias", torch.float32, E, dev)
     if ids is None:
-        ids = torch.empty((T, k), dtype=torch.int32, device=logits.device)
+        ids = torch.empty((T, k), dtype=torch.int32, device=dev)
     if weights is None:
-        weights = torch.empty((T, k), dtype=torch.float32, device=logits.device)
-    _need(ids, "ids", torch.int32, T * k)
-    _need(weights, "weights", torch.float32, T * k)
+        weights = torch.empty((T, k), dtype=torch.float32, device=dev)
+    _need(ids, "ids", torch.int32, T * k, dev)
+    _need(weights, "weights", torch.float32, T * k, dev)
     _chk(_L().moe_route(_ptr(logits), _ptr(bias), T, E, k, 1 if normalize else 0, _ptr(ids), _ptr(weights),
                         _stream(logits.device)), "moe_route")
     return ids, weights
@@ -291,16 +306,17 @@ def combine(dst, weights, shared=None, out=None):
     dst: float32 CUDA [T][k][n] (or [T*k][n] with weights [T][k]); weights:
     float32 [T][k]; shared: float32 [T][n] or None; out: float32 [T][n] or None."""
     _cuda(dst, "dst", torch.float32)
-    _cuda(weights, "weights", torch.float32)
+    dev = dst.device
+    _cuda(weights, "weights", torch.float32, dev)
     T, k = weights.shape
     n = dst.shape[-1]
     if dst.numel() != T * k * n:
         raise ValueError("dst must hold n_tokens*k rows of n")
     if shared is not None:
-        _need(shared, "shared", torch.float32, T * n)
+        _need(shared, "shared", torch.float32, T * n, dev)
     if out is None:
-        out = torch.empty((T, n), dtype=torch.float32, device=dst.device)
-    _need(out, "out", torch.float32, T * n)
+        out = torch.empty((T, n), dtype=torch.float32, device=dev)
+    _need(out, "out", torch.float32, T * n, dev)
     _chk(_L().moe_combine(_ptr(dst), _ptr(weights), _ptr(shared), T, k, n, _ptr(out), _stream(dst.device)),
          "moe_combine")
     return out

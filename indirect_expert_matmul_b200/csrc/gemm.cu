@@ -99,26 +99,6 @@ struct Tile {
     int e, mt, p0, n, p0pad;  // p0pad: first row of the tile in the tile-major buffers
 };
 
-// Optional stall accounting (build with -DMOE_GEMM_STATS): per role, the
-// cycles spent waiting on each barrier and the role's total cycles, summed
-// over CTAs into g_gemm_stats[role][slot].
-#ifdef MOE_GEMM_STATS
-__device__ unsigned long long g_gemm_stats[2][6][4];  // [DUAL][role][slot]
-#define STAT_DECL long long st_[4] = {0, 0, 0, 0}; const long long st_t0_ = clock64();
-#define STAT_PTR(i) (&st_[i])
-#define STAT_FLUSH(role)                                                              \
-    do {                                                                              \
-        atomicAdd(&g_gemm_stats[DUAL][role][0], (unsigned long long)st_[0]);                 \
-        atomicAdd(&g_gemm_stats[DUAL][role][1], (unsigned long long)st_[1]);                 \
-        atomicAdd(&g_gemm_stats[DUAL][role][2], (unsigned long long)st_[2]);                 \
-        atomicAdd(&g_gemm_stats[DUAL][role][3], (unsigned long long)(clock64() - st_t0_));   \
-    } while (0)
-#else
-#define STAT_DECL
-#define STAT_PTR(i) nullptr
-#define STAT_FLUSH(role) do {} while (0)
-#endif
-
 __device__ __forceinline__ Tile decode_tile(int t, int mt_count, const GemmParams& p, const int* s_prefix,
                                             const int* s_bounds, const int* s_pad) {
     Tile r;
@@ -152,15 +132,11 @@ __device__ __forceinline__ Tile decode_tile(int t, int mt_count, const GemmParam
 // Bounded wait by one lane; false when the kernel is aborting.  The lane
 // sleeps in hardware between polls (suspend-time hint), so waiting roles do
 // not take issue slots from the dequantisation warps.
-__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status,
-                                         long long* stat = nullptr) {
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {
-        if (ptx::mbar_try_wait_sleep(bar, parity, kSleepNs)) {
-            if (stat) *stat += clock64() - t0;
-            return true;
-        }
+        if (ptx::mbar_try_wait_sleep(bar, parity, kSleepNs)) return true;
         if (*abort_flag) return false;
         if (clock64() - t0 > kWaitLimitCycles) {
             *abort_flag = 1;
@@ -173,16 +149,12 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
 }
 
 // lane 0 waits, the warp learns the outcome
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status,
-                                          long long* stat = nullptr) {
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status) {
     // every lane polls (no lane-0 branch); lanes that see different phases simply poll again
     if (ptx::mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {
-        if (ptx::mbar_try_wait_sleep(bar, parity, kSleepNs)) {
-            if (stat) *stat += clock64() - t0;
-            return true;
-        }
+        if (ptx::mbar_try_wait_sleep(bar, parity, kSleepNs)) return true;
         if (*abort_flag) return false;
         if (clock64() - t0 > kWaitLimitCycles) {
             if ((threadIdx.x & 31) == 0) {
@@ -341,7 +313,6 @@ grouped_gemm_kernel(const GemmParams p) {
         // One lane streams both sources' weight blocks: an L2 prefetch runs
         // kPrefetchSteps k-steps ahead of the bulk copies into the raw ring.
         if (lane == 0) {
-            STAT_DECL
             int rs = 0;
             uint32_t rph = 0;
             uint32_t used = 0, par = 0;  // per-stage issue record, for draining
@@ -376,7 +347,7 @@ grouped_gemm_kernel(const GemmParams p) {
                 }
                 for (int kt = 0; kt < KT; ++kt) {
                     prefetch_one();
-                    ok = wait_bar(&raw_empty[rs], rph ^ 1, abort_flag, status, STAT_PTR(0));
+                    ok = wait_bar(&raw_empty[rs], rph ^ 1, abort_flag, status);
                     if (!ok) break;
                     ptx::mbar_arrive_expect_tx(&raw_full[rs], nb[0] + nb[1]);
                     for (int i = 0; i < 2; ++i)
@@ -392,14 +363,12 @@ grouped_gemm_kernel(const GemmParams p) {
             volatile int never = 0;
             for (int s = 0; s < kRS; ++s)
                 if (used >> s & 1) wait_bar(&raw_full[s], (par >> s) & 1, &never, status);
-            STAT_FLUSH(0);
         }
     } else if (warp == kWarpProdB) {
         // ------------------------------------------------ activation producer
         // The rows of a column tile are contiguous and already swizzled in the
         // tile-major activation buffer: one bulk copy per k-step.
         if (lane == 0) {
-            STAT_DECL
             int bs = 0;
             uint32_t bph = 0;
             uint32_t used = 0, par = 0;
@@ -410,7 +379,7 @@ grouped_gemm_kernel(const GemmParams p) {
                 const uint32_t bytes = (uint32_t)((tl.n + 15) & ~15) * 128u;
                 const uint8_t* src = p.B + (size_t)tl.p0pad * 128u;
                 for (int kt = 0; kt < KT; ++kt) {
-                    ok = wait_bar(&b_empty[bs], bph ^ 1, abort_flag, status, STAT_PTR(0));
+                    ok = wait_bar(&b_empty[bs], bph ^ 1, abort_flag, status);
                     if (!ok) break;
                     ptx::mbar_arrive_expect_tx(&b_full[bs], bytes);
                     ptx::bulk_g2s(sB + bs * kBTileBytes, src + kt * plane, bytes, &b_full[bs]);
@@ -422,14 +391,12 @@ grouped_gemm_kernel(const GemmParams p) {
             volatile int never = 0;
             for (int s = 0; s < kMB; ++s)
                 if (used >> s & 1) wait_bar(&b_full[s], (par >> s) & 1, &never, status);
-            STAT_FLUSH(1);
         }
     } else if (warp == kWarpMma) {
         // ----------------------------------------------------------------- MMA
         // A and B from shared memory; the two accumulators' instructions
         // interleave so neither chain waits on itself.
         if (lane == 0) {
-            STAT_DECL
             int as = 0, bs = 0;
             uint32_t aph = 0, bph = 0, use = 0;
             bool ok = true;
@@ -437,14 +404,14 @@ grouped_gemm_kernel(const GemmParams p) {
                 const Tile tl = decode_tile(t, MU, p, s_prefix, s_bounds, s_pad);
                 const int n16 = (tl.n + 15) & ~15;
                 const bool has1 = DUAL || (2 * tl.mt + 1 < MT);
-                ok = wait_bar(tmem_empty, (use & 1) ^ 1, abort_flag, status, STAT_PTR(2));
+                ok = wait_bar(tmem_empty, (use & 1) ^ 1, abort_flag, status);
                 if (!ok) break;
                 ptx::tc_fence_after();
                 const uint32_t d0 = tmem_base, d1 = tmem_base + kAccCols;
                 const uint32_t idesc = ptx::idesc_f16(BF16, n16, 128);
                 for (int kt = 0; kt < KT; ++kt) {
-                    ok = wait_bar(&a_full[as], aph, abort_flag, status, STAT_PTR(0)) &&
-                         wait_bar(&b_full[bs], bph, abort_flag, status, STAT_PTR(1));
+                    ok = wait_bar(&a_full[as], aph, abort_flag, status) &&
+                         wait_bar(&b_full[bs], bph, abort_flag, status);
                     if (!ok) break;
                     ptx::tc_fence_after();
                     const uint32_t a0 = a_sa + (uint32_t)as * 2u * kATileBytes;
@@ -465,7 +432,6 @@ grouped_gemm_kernel(const GemmParams p) {
                 ptx::mma_commit(tmem_full);
                 use += 1;
             }
-            STAT_FLUSH(2);
         }
         __syncwarp();
     } else if (deq_index(warp) >= 0 || (warp >= kWorkWarp0 && warp < kWorkWarp0 + kWorkWarps)) {
@@ -486,7 +452,6 @@ grouped_gemm_kernel(const GemmParams p) {
         const uint32_t lanes = (uint32_t)(32 * wq) << 16;
         const uint32_t a_row = (uint32_t)mat * kATileBytes + (uint32_t)(r >> 3) * 1024u + (uint32_t)(r & 7) * 128u;
         const uint32_t rx = (uint32_t)(r & 7);
-        STAT_DECL
         int rs = 0, as = 0;
         uint32_t rph = 0, aph = 0, use = 0;
         bool ok = true;
@@ -514,8 +479,8 @@ grouped_gemm_kernel(const GemmParams p) {
                 }
                 for (int kt = 0; kt < KT; ++kt) {
                     if ((as & 1) == kpar) {  // the k-step count's parity, continued across tiles
-                        ok = warp_wait(&raw_full[rs], rph, abort_flag, status, STAT_PTR(0)) &&
-                             warp_wait(&a_empty[as], aph ^ 1, abort_flag, status, STAT_PTR(1));
+                        ok = warp_wait(&raw_full[rs], rph, abort_flag, status) &&
+                             warp_wait(&a_empty[as], aph ^ 1, abort_flag, status);
                         if (!ok) break;
                         if (nr > 0) {
                             const uint32_t raw = raw_sa + (uint32_t)(rs * 2 + mat) * kRawBytes;
@@ -561,7 +526,7 @@ grouped_gemm_kernel(const GemmParams p) {
             if (!ok) break;
             if (!epi) continue;
             // ---- epilogue of this tile
-            if (!warp_wait(tmem_full, use & 1, abort_flag, status, STAT_PTR(2))) break;
+            if (!warp_wait(tmem_full, use & 1, abort_flag, status)) break;
             use += 1;
             ptx::tc_fence_after();
             if (DUAL) {
@@ -616,7 +581,6 @@ grouped_gemm_kernel(const GemmParams p) {
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(tmem_empty);
         }
-        if (lane == 0) STAT_FLUSH(4);
     }
 
     ptx::tc_fence_before();
@@ -771,17 +735,6 @@ gather_tokens_kernel(const void* __restrict__ x, int x_type, int n_in, int KT, c
 }
 
 // ------------------------------------------------------------------- host
-#ifdef MOE_GEMM_STATS
-extern "C" __attribute__((visibility("default"))) int moe_gemm_stats_read(unsigned long long* out48, int reset) {
-    if (cudaMemcpyFromSymbol(out48, g_gemm_stats, sizeof(g_gemm_stats)) != cudaSuccess) return MOE_ERR_CUDA;
-    if (reset) {
-        static const unsigned long long zero[2][6][4] = {};
-        if (cudaMemcpyToSymbol(g_gemm_stats, zero, sizeof(zero)) != cudaSuccess) return MOE_ERR_CUDA;
-    }
-    return MOE_OK;
-}
-#endif
-
 static int sm_count() {
     static int dev_cached = -1, n = 0;
     int dev = 0;

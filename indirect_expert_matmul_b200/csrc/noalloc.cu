@@ -57,6 +57,8 @@ extern "C" moe_status moe_ffn_decode_noalloc(const void* Wg, const void* Wu, con
                                               moe_stream stream) {
     // host checks, before any CUDA call
     if (n_tokens < 0 || k < 1 || n_experts < 1) return MOE_ERR_INVALID;
+    // the library-wide limits first, so that n_tokens * k below cannot overflow
+    if (n_tokens >= kMaxTokens || k >= kMaxK) return MOE_ERR_RANGE;
     if (k > n_experts || n_experts > kMaxExperts) return MOE_ERR_RANGE;
     if (n_tokens * (int64_t)k > kNaMaxSlots || n_ff > kNaMaxFF || n_ff_shared > kNaMaxFF) return MOE_ERR_RANGE;
     if (x_type != MOE_BF16 && x_type != MOE_F16 && x_type != MOE_F32) return MOE_ERR_INVALID;

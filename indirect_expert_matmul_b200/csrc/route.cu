@@ -6,7 +6,8 @@
 //   key[e]  = logits[t][e] + bias[e]     (one float addition)
 //   ids[t]  = the k largest keys, descending, equal keys in ascending e
 //   p[e]    = softmax over all experts of logits[t]
-//   w[t][i] = p[ids[t][i]]  (divided by the sum over the k when normalising)
+//   w[t][i] = p[ids[t][i]]  (divided by the sum over the k when normalising,
+//             evaluated as the softmax over the k chosen logits)
 //
 // One warp per token.  The keys and logits of a token live in registers
 // (ceil(n_experts / 32) per lane, rounded up to a power of two; n_experts <= 1024); each of the k rounds is a per-lane pairwise
@@ -51,15 +52,17 @@ route_kernel(const float* __restrict__ logits, const float* __restrict__ bias, i
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    float z = 0.f;
+    float z = 0.f;  // softmax denominator over all experts (unnormalised weights only)
+    if (!normalize) {
 #pragma unroll
-    for (int j = 0; j < NPL; ++j)
-        if (j * 32 + lane < n_experts) z = __fadd_rn(z, expf(__fsub_rn(l[j], mx)));
+        for (int j = 0; j < NPL; ++j)
+            if (j * 32 + lane < n_experts) z = __fadd_rn(z, expf(__fsub_rn(l[j], mx)));
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) z = __fadd_rn(z, __shfl_xor_sync(0xffffffffu, z, o));
+        for (int o = 16; o > 0; o >>= 1) z = __fadd_rn(z, __shfl_xor_sync(0xffffffffu, z, o));
+    }
 
     uint32_t taken = 0u;  // bit j: expert j*32 + lane chosen
-    float sel = 0.f;      // lane 0: sum of the chosen probabilities, in choice order
+    float mc = -INFINITY; // lane 0: largest chosen logit (renormalised weights)
     int32_t* it = ids + t * k;
     float* wt = weights + t * k;
     for (int i = 0; i < k; ++i) {
@@ -99,16 +102,27 @@ route_kernel(const float* __restrict__ logits, const float* __restrict__ bias, i
         }
         if ((be & 31) == lane) taken |= 1u << (be >> 5);
         if (lane == 0) {
-            const float p = __fdiv_rn(expf(__fsub_rn(bl, mx)), z);
             it[i] = be;
-            wt[i] = p;
-            sel = __fadd_rn(sel, p);
+            if (normalize) {
+                wt[i] = bl;  // the chosen logit, turned into its weight below
+                mc = fmaxf(mc, bl);
+            } else {
+                wt[i] = __fdiv_rn(expf(__fsub_rn(bl, mx)), z);
+            }
         }
     }
-    if (normalize) {
-        sel = __shfl_sync(0xffffffffu, sel, 0);
-        __syncwarp();  // lane 0's weights are visible to the warp
-        for (int i = lane; i < k; i += 32) wt[i] = __fdiv_rn(wt[i], sel);
+    // Renormalised weights p_i / sum_chosen p_j are the softmax over the chosen
+    // logits alone; taken relative to the largest chosen logit, the sum is at
+    // least 1, so it cannot underflow to zero however far the chosen logits sit
+    // below the row's maximum.  Lane 0, in choice order.
+    if (normalize && lane == 0) {
+        float sel = 0.f;
+        for (int i = 0; i < k; ++i) {
+            const float e = expf(__fsub_rn(wt[i], mc));
+            wt[i] = e;
+            sel = __fadd_rn(sel, e);
+        }
+        for (int i = 0; i < k; ++i) wt[i] = __fdiv_rn(wt[i], sel);
     }
 }
 

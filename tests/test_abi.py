@@ -71,6 +71,13 @@ def test_host_argument_checks_without_gpu():
     # ffn: shared width not a multiple of 32
     assert lib.moe_ffn(nul, nul, nul, 4, 64, 64, nul, nul, nul, 40, nul, 0, nul, 1, 1, nul, nul, nul,
                        nul) == moe.ERR_INVALID
+    # the no-workspace entry point: n_tokens far past 2^22 is refused before n_tokens*k is formed
+    # (2^61 + 1 times 8 would wrap to 8, under its 64-slot limit)
+    for T in ((1 << 61) + 1, 1 << 22):
+        assert lib.moe_ffn_decode_noalloc(nul, nul, nul, 256, 2048, 512, nul, nul, nul, 0, nul, 0, nul, T, 8, nul,
+                                          nul, nul, nul) == moe.ERR_RANGE
+    assert lib.moe_ffn_decode_noalloc(nul, nul, nul, 2048, 2048, 512, nul, nul, nul, 0, nul, 0, nul, 1, 1024, nul,
+                                      nul, nul, nul) == moe.ERR_RANGE
 
 
 def test_router_and_combine_argument_checks_without_gpu():
@@ -105,7 +112,47 @@ def test_gemv_threshold_setting():
 def test_caller_buffers_are_checked_before_any_launch(monkeypatch):
     # outputs and workspaces handed in by the caller must hold what the call writes
     import torch
-    monkeypatch.setattr(moe, "_cuda", lambda t, name, dtype=None: t)  # no GPU here: skip the device check
+    monkeypatch.setattr(moe, "_gpu", lambda t, name: None)  # no GPU here: accept host tensors as device ones
     moe._need(torch.empty(10), "out", torch.float32, 10)
     with pytest.raises(ValueError, match="holds 9 elements"):
         moe._need(torch.empty(9), "out", torch.float32, 10)
+
+
+def test_tensors_on_another_device_are_refused(monkeypatch):
+    # every tensor of a call must sit on the device whose stream the call uses;
+    # "meta" stands in for a second GPU (no GPU here)
+    import torch
+    monkeypatch.setattr(moe, "_gpu", lambda t, name: None)
+    here, other = torch.device("cpu"), torch.device("meta")
+    moe._need(torch.empty(4), "out", torch.float32, 4, here)
+    with pytest.raises(ValueError, match="is on meta"):
+        moe._need(torch.empty(4, device=other), "out", torch.float32, 4, here)
+    # through the operators, before the library is called
+    called = []
+    real = moe.lib()
+
+    class SizesOnly:  # the library's size queries run; any other entry point is recorded
+        def __getattr__(self, name):
+            if name.endswith("_size") or name == "moe_status_string":
+                return getattr(real, name)
+            return lambda *a: called.append(name) or 0
+
+    monkeypatch.setattr(moe, "_L", lambda: SizesOnly())
+    x = torch.zeros((2, 64), dtype=torch.bfloat16)
+    ids = torch.zeros((2, 1), dtype=torch.int32)
+    W = torch.empty(moe_prepared_bytes(4, 32, 64), dtype=torch.uint8, device=other)
+    with pytest.raises(ValueError, match="W is on meta"):
+        moe.mul_mat_id(W, 4, 32, 64, x, ids, ws=torch.empty(1, dtype=torch.uint8))
+    with pytest.raises(ValueError, match="ids is on meta"):
+        moe.mul_mat_id(W, 4, 32, 64, x, ids.to(other), ws=torch.empty(1, dtype=torch.uint8))
+    with pytest.raises(ValueError, match="Wg is on meta"):
+        moe.ffn(W, W, W, 4, 64, 32, x, ids, ws=torch.empty(1, dtype=torch.uint8))
+    with pytest.raises(ValueError, match="weights is on meta"):
+        moe.combine(torch.zeros((2, 1, 8)), torch.zeros((2, 1), device=other))
+    with pytest.raises(ValueError, match="bias is on meta"):
+        moe.route(torch.zeros((2, 8)), 2, bias=torch.zeros(8, device=other))
+    assert not called
+
+
+def moe_prepared_bytes(E, n_out, n_in):
+    return E * ((n_out + 15) // 16 * 16) * ((n_in + 63) // 64) * 68

@@ -48,7 +48,6 @@ def test_nvml_summary_maps_reason_bits_and_takes_the_loaded_median(monkeypatch, 
     monkeypatch.setattr(bench.ClockSampler, "_nvml_handle", lambda self: (fake, "h"))
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     c = bench.ClockSampler(0)
-    c.path = str(tmp_path / "clocks.csv")
     with c:
         while fake.i < 5:
             pass
@@ -56,7 +55,7 @@ def test_nvml_summary_maps_reason_bits_and_takes_the_loaded_median(monkeypatch, 
     assert s["source"] == "nvml" and s["sm_max_mhz"] == 1965.0 and s["samples"] >= 5
     assert s["sm_mhz"] == 1965.0  # the idle 210 MHz sample is not under load
     assert s["reasons"] == ["hw_slowdown", "sw_power_cap"]  # 0x8 and 0x4; 0x1 (idle) is not a reason
-    assert open(c.path).read().startswith("# sm_mhz")
+    assert list(tmp_path.iterdir()) == []  # the samples stay in memory: nothing is written
 
 
 def test_nvidia_smi_csv_summary(monkeypatch, tmp_path):
@@ -70,6 +69,7 @@ def test_nvidia_smi_csv_summary(monkeypatch, tmp_path):
     s = c.summary()
     assert s["samples"] == 3 and s["sm_mhz"] == 1965.0 and s["sm_max_mhz"] == 1965.0
     assert s["reasons"] == ["sw_power_cap", "sw_thermal_slowdown"]
+    assert not os.path.exists(c.path)  # the temporary sample file is removed once read
 
 
 def test_traffic_is_null_once_a_gemm_source_changes(monkeypatch, tmp_path):

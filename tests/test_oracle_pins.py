@@ -424,6 +424,33 @@ def test_route_ties_bias_and_full_k():
         oracle.route(l, 13)
 
 
+def _wide_span_logits():
+    # a row spanning ~200: the top expert far above the rest, and a bias that
+    # makes the chosen experts ones whose probabilities are about e^-190 - far
+    # below float32's smallest value, but not float64's
+    logits = np.zeros((4, 16), np.float32)
+    logits[:, 0] = 100.0
+    logits[:, 1:] = np.linspace(-100.0, -90.0, 15, dtype=np.float32)[None, :] + np.arange(4, dtype=np.float32)[:, None]
+    bias = np.zeros(16, np.float32)
+    bias[0] = -1000.0  # expert 0 never chosen
+    return logits, bias
+
+
+def test_route_renormalised_weights_are_the_softmax_over_the_chosen_logits():
+    # renormalising the chosen probabilities is the softmax over the chosen
+    # logits alone (the common factor exp(-max) / sum cancels): checked against
+    # that closed form, on a row whose chosen probabilities underflow in float32
+    logits, bias = _wide_span_logits()
+    ids, w, tol = oracle.route(logits, 4, bias)
+    chosen = np.take_along_axis(logits.astype(np.float64), ids, axis=1)
+    e = np.exp(chosen - chosen.max(axis=1, keepdims=True))
+    assert np.all(ids != 0)
+    assert np.allclose(w, e / e.sum(axis=1, keepdims=True), rtol=1e-13, atol=0)
+    assert np.allclose(w.sum(axis=1), 1.0, atol=1e-15) and np.all(np.isfinite(tol))
+    p32 = np.exp((chosen - 100.0).astype(np.float32))  # what a float32 softmax over all experts gives
+    assert np.all(p32 == 0.0)
+
+
 def test_route_tolerance_covers_a_float32_softmax():
     rng = np.random.default_rng(5)
     logits = (rng.normal(size=(40, 64)) * 3).astype(np.float32)

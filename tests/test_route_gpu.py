@@ -38,6 +38,20 @@ def test_route_matches_oracle(T, E, k, normalize):
     assert torch.equal(ids2, ids) and torch.equal(w2.view(torch.int32), w.view(torch.int32))
 
 
+def test_route_renormalised_weights_stay_finite_when_probabilities_underflow():
+    # chosen logits ~190 below the row's top: their float32 probabilities are 0,
+    # yet the renormalised weights (the softmax over the chosen logits) are finite,
+    # sum to one and match the oracle within the float32 bound
+    from tests.test_oracle_pins import _wide_span_logits
+    logits, bias = _wide_span_logits()
+    ref_ids, ref_w, tol = oracle.route(logits, 4, bias)
+    ids, w = moe.route(torch.from_numpy(logits).cuda(), 4, torch.from_numpy(bias).cuda())
+    assert np.array_equal(ids.cpu().numpy(), ref_ids)
+    assert torch.isfinite(w).all()
+    check_close(w, ref_w, tol, "router weights, span 200")
+    assert np.allclose(w.cpu().numpy().sum(axis=1), 1.0, atol=1e-6)
+
+
 def test_route_exact_ties_take_the_lower_expert():
     logits = np.zeros((6, 96), np.float32)
     logits[:, 50] = 1.0

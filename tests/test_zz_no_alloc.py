@@ -1,11 +1,12 @@
 """moe_ffn_decode_noalloc - the decode FFN with its scratch in a static
-device array - against moe_ffn with a caller workspace, on the decode
-workload with a shared expert.  Two calls in a row each agree with the
-workspace entry point within the oracle's per-element tolerance (the two can
-differ by at most the sum of their distances to the exact result), report a
-zero device status, and sizes past the static array's capacity are refused
-on the host.  This file is named to be collected last so that it also runs
-after every other GPU test in the same process.
+device array - on the decode workload with a shared expert.  Two calls in a
+row: each is within the oracle's per-element tolerance of the exact result,
+each agrees with moe_ffn (the workspace entry point) within the sum of their
+two distances to it, the second is bit-identical to the first (a stale
+scratch array would show here), and each reports a zero device status.
+Sizes past the static array's capacity are refused on the host.  This file
+is named to be collected last so that it also runs after every other GPU
+test in the same process.
 """
 import numpy as np
 import pytest
@@ -33,8 +34,8 @@ def _inputs(wl, T):
 def test_noalloc_matches_workspace_entry_point(T):
     wl = workloads.WORKLOADS["decode"]
     Wg, Wu, Wd, sh, x, ids = _inputs(wl, T)
-    _, tol = oracle.ffn(Wg, Wu, Wd, x, "bf16", ids)
-    _, tol_sh = oracle.shared_ffn(*sh, x, "bf16")
+    exact, tol = oracle.ffn(Wg, Wu, Wd, x, "bf16", ids)
+    exact_sh, tol_sh = oracle.shared_ffn(*sh, x, "bf16")
     dWg, dWu, dWd = prep(Wg), prep(Wu), prep(Wd)
     shared = (prep(sh[0]), prep(sh[1]), prep(sh[2]), wl.n_ff_shared)
     xd, idd = to_dev_x(x, "bf16"), torch.from_numpy(ids).cuda()
@@ -42,6 +43,7 @@ def test_noalloc_matches_workspace_entry_point(T):
     ref = ref.cpu().numpy().reshape(T * wl.k, wl.n_in).astype(np.float64)
     ref_sh = ref_sh.cpu().numpy().astype(np.float64)
     status = torch.full((1,), 12345, dtype=torch.int32, device="cuda")
+    first = None
     for call in range(2):  # two calls in a row share the one static scratch
         dst, dsh = moe.ffn_decode_noalloc(dWg, dWu, dWd, wl.n_experts, wl.n_in, wl.n_out, xd, idd, shared=shared,
                                           status=status)
@@ -49,8 +51,14 @@ def test_noalloc_matches_workspace_entry_point(T):
         assert int(status.item()) == moe.OK, f"call {call}: {moe.status_string(int(status.item()))}"
         got = dst.cpu().numpy().reshape(T * wl.k, wl.n_in).astype(np.float64)
         got_sh = dsh.cpu().numpy().astype(np.float64)
-        assert np.all(np.abs(got - ref) <= 2 * tol), f"call {call}: routed rows differ beyond tolerance"
-        assert np.all(np.abs(got_sh - ref_sh) <= 2 * tol_sh), f"call {call}: shared rows differ beyond tolerance"
+        assert np.all(np.abs(got - exact) <= tol), f"call {call}: routed rows outside the oracle's tolerance"
+        assert np.all(np.abs(got_sh - exact_sh) <= tol_sh), f"call {call}: shared rows outside the oracle's tolerance"
+        assert np.all(np.abs(got - ref) <= 2 * tol), f"call {call}: routed rows differ from moe_ffn beyond tolerance"
+        assert np.all(np.abs(got_sh - ref_sh) <= 2 * tol_sh), f"call {call}: shared rows differ from moe_ffn"
+        if first is None:
+            first = (got.copy(), got_sh.copy())
+        else:
+            assert np.array_equal(got, first[0]) and np.array_equal(got_sh, first[1]), "calls differ bit for bit"
 
 
 def test_noalloc_reports_bad_id():
