@@ -76,3 +76,98 @@ def test_two_gloo_ranks_match_unsharded(tmp_path):
     assert np.array_equal(got["ids"], ids)
     assert np.array_equal(got["dst"], dst)       # bit-identical: tokens are independent
     assert float(got["slow"]) == 1.5              # max over ranks
+
+
+# ------------------------------------------------------- expert parallelism
+def _ep_rank_main(rank, world, port, out_dir, what):
+    import torch
+    import torch.distributed as dist
+
+    import oracle
+    import workloads
+    from indirect_expert_matmul_b200.dist import token_shard
+    from indirect_expert_matmul_b200.expert_parallel import ep_forward, expert_range
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    e0, e1 = expert_range(EP_E, rank, world)
+    t0, T = token_shard(EP_T, rank, world)
+    ids_all = workloads.routing("uniform", EP_T, EP_E, EP_K, 21)
+    if what == "mul_mat_id":
+        W = workloads.q8_0_weights(EP_E, EP_NOUT, EP_NIN, 21, workloads.T_W)[e0:e1]  # this rank's experts only
+        x = workloads.activations(EP_T, EP_NIN, "f32", 21, workloads.T_X)[t0:t0 + T]
+        n_out = EP_NOUT
+
+        def compute(xr, ir):
+            out, _ = oracle.mul_mat_id(W, xr.numpy(), "f32", ir.numpy())
+            return torch.from_numpy(out.astype(np.float32))
+        x_t = torch.from_numpy(np.ascontiguousarray(x))
+    else:  # the routed SwiGLU FFN, bf16 activations (bit patterns carried as int32)
+        Wg = workloads.q8_0_weights(EP_E, EP_NFF, EP_NIN, 21, workloads.T_WG)[e0:e1]
+        Wu = workloads.q8_0_weights(EP_E, EP_NFF, EP_NIN, 21, workloads.T_WU)[e0:e1]
+        Wd = workloads.q8_0_weights(EP_E, EP_NIN, EP_NFF, 21, workloads.T_WD)[e0:e1]
+        x = workloads.activations(EP_T, EP_NIN, "bf16", 21, workloads.T_X)[t0:t0 + T]
+        n_out = EP_NIN
+
+        def compute(xr, ir):
+            out, _ = oracle.ffn(Wg, Wu, Wd, xr.numpy().astype(np.uint16), "bf16", ir.numpy())
+            return torch.from_numpy(out.astype(np.float32))
+        x_t = torch.from_numpy(np.ascontiguousarray(x).astype(np.int32))
+    dst = ep_forward(x_t, torch.from_numpy(ids_all[t0:t0 + T].copy()), EP_T, EP_E, n_out, compute)
+    np.save(os.path.join(out_dir, f"ep_{rank}.npy"), dst.numpy())
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+EP_E, EP_K, EP_T, EP_NIN, EP_NOUT, EP_NFF = 10, 3, 23, 96, 40, 64
+
+
+@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("what", ["mul_mat_id", "ffn"])
+def test_expert_parallel_matches_unsharded(tmp_path, world, what):
+    """Experts split into contiguous ranges across gloo ranks, tokens sharded:
+    after the all-to-all every rank holds exactly the unsharded oracle's rows
+    for its tokens, bit for bit (each slot is computed once, from the same
+    weights and activation row, and the exchange does no arithmetic)."""
+    import oracle
+    import workloads
+
+    mp.start_processes(_ep_rank_main, args=(world, _free_port(), str(tmp_path), what), nprocs=world,
+                       start_method="spawn")
+    got = np.concatenate([np.load(tmp_path / f"ep_{r}.npy") for r in range(world)])
+    ids = workloads.routing("uniform", EP_T, EP_E, EP_K, 21)
+    if what == "mul_mat_id":
+        W = workloads.q8_0_weights(EP_E, EP_NOUT, EP_NIN, 21, workloads.T_W)
+        ref, _ = oracle.mul_mat_id(W, workloads.activations(EP_T, EP_NIN, "f32", 21, workloads.T_X), "f32", ids)
+        ref = ref.reshape(EP_T, EP_K, EP_NOUT)
+    else:
+        Wg = workloads.q8_0_weights(EP_E, EP_NFF, EP_NIN, 21, workloads.T_WG)
+        Wu = workloads.q8_0_weights(EP_E, EP_NFF, EP_NIN, 21, workloads.T_WU)
+        Wd = workloads.q8_0_weights(EP_E, EP_NIN, EP_NFF, 21, workloads.T_WD)
+        ref, _ = oracle.ffn(Wg, Wu, Wd, workloads.activations(EP_T, EP_NIN, "bf16", 21, workloads.T_X), "bf16", ids)
+        ref = ref.reshape(EP_T, EP_K, EP_NIN)
+    assert got.shape == ref.shape
+    assert np.array_equal(got, ref.astype(np.float32))
+
+
+def test_expert_ranges_partition_the_experts():
+    from indirect_expert_matmul_b200.expert_parallel import expert_range, owned_slot_range
+    import oracle
+    import workloads
+    for E in (1, 8, 10, 256):
+        for W in (1, 2, 3, 8):
+            if W > E:
+                continue
+            rs = [expert_range(E, r, W) for r in range(W)]
+            assert rs[0][0] == 0 and rs[-1][1] == E
+            assert all(a[1] == b[0] for a, b in zip(rs, rs[1:]))
+    # a contiguous expert range owns a contiguous range of sorted positions
+    ids = workloads.routing("uniform", 40, 10, 3, 5)
+    _, ids_dst, bounds = oracle.row_ids(ids, 10)
+    for W in (2, 3):
+        for r in range(W):
+            e0, e1 = expert_range(10, r, W)
+            p0, p1 = owned_slot_range(bounds, e0, e1)
+            flat = ids.reshape(-1)
+            assert sorted(ids_dst[p0:p1].tolist()) == [i for i in range(flat.size) if e0 <= flat[i] < e1]
