@@ -43,12 +43,12 @@ def _L():
         _lib.oracle_check_args.argtypes = [i64, i32, i32]
         _lib.oracle_row_ids.argtypes = [vp, i64, i32, i32, i32, vp, vp, vp]
         for f in (_lib.oracle_mul_mat_id_brute, _lib.oracle_mul_mat_id_grouped):
-            f.argtypes = [vp, i32, i32, i32, vp, i32, vp, i64, i32, i32, vp, vp]
-        _lib.oracle_mul_mat_id_rows.argtypes = [vp, i32, i32, i32, vp, i32, vp, i64, i32, i32, vp, i64, vp, vp]
-        _lib.oracle_ffn_rows.argtypes = [vp, vp, vp, i32, i32, i32, vp, i32, vp, i64, i32, vp, i64, vp, vp]
-        _lib.oracle_shared_rows.argtypes = [vp, vp, vp, i32, i32, vp, i32, vp, i64, vp, vp]
-        _lib.oracle_ffn_hidden.argtypes = [vp, vp, i32, i32, i32, vp, i32, vp, i64, i32, vp, i64, vp, vp, vp]
-        _lib.oracle_dequant.argtypes = [vp, i32, i32, i32, vp]
+            f.argtypes = [vp, i32, i32, i32, vp, i32, vp, i64, i32, i32, vp, vp, i32]
+        _lib.oracle_mul_mat_id_rows.argtypes = [vp, i32, i32, i32, vp, i32, vp, i64, i32, i32, vp, i64, vp, vp, i32]
+        _lib.oracle_ffn_rows.argtypes = [vp, vp, vp, i32, i32, i32, vp, i32, vp, i64, i32, vp, i64, vp, vp, i32]
+        _lib.oracle_shared_rows.argtypes = [vp, vp, vp, i32, i32, vp, i32, vp, i64, vp, vp, i32]
+        _lib.oracle_ffn_hidden.argtypes = [vp, vp, i32, i32, i32, vp, i32, vp, i64, i32, vp, i64, vp, vp, vp, i32]
+        _lib.oracle_dequant.argtypes = [vp, i32, i32, i32, vp, i32]
         _lib.oracle_dequant.restype = None
         _lib.oracle_combine.argtypes = [vp, vp, vp, i64, i32, i64, vp, vp]
         _lib.oracle_combine.restype = None
@@ -68,6 +68,20 @@ def _p(a):
 
 def _mode(mode):
     return {"broadcast": BROADCAST, "per_slot": PER_SLOT}.get(mode, mode)
+
+
+# weight types, told apart by the block size of the stacked array's last axis
+Q8_0, MXFP4 = 0, 1
+_BLOCK_BYTES = {34: Q8_0, 17: MXFP4}
+
+
+def wtype(W: np.ndarray) -> int:
+    """Q8_0 (34-byte blocks) or MXFP4 (17-byte blocks) of a stacked weight
+    array [E][n_out][n_in/32][block bytes]."""
+    try:
+        return _BLOCK_BYTES[W.shape[-1]]
+    except KeyError:
+        raise ValueError(f"unknown weight block size {W.shape[-1]}") from None
 
 
 class OracleError(RuntimeError):
@@ -98,10 +112,10 @@ def row_ids(ids: np.ndarray, n_experts: int, mode="broadcast"):
 
 
 def dequant(W: np.ndarray, e: int) -> np.ndarray:
-    """fp64 weights of expert e, [n_out][n_in], from Q8_0 blocks."""
+    """fp64 weights of expert e, [n_out][n_in], from Q8_0 or MXFP4 blocks."""
     E, n_out, nb, _ = W.shape
     out = np.empty((n_out, nb * 32), np.float64)
-    _L().oracle_dequant(_p(W), n_out, nb * 32, e, _p(out))
+    _L().oracle_dequant(_p(W), n_out, nb * 32, e, _p(out), wtype(W))
     return out
 
 
@@ -113,7 +127,7 @@ def mul_mat_id(W, x, x_type, ids, mode="broadcast", grouped=False):
     dst = np.zeros((T, k, n_out), np.float64)
     tol = np.zeros((T, k, n_out), np.float64)
     f = _L().oracle_mul_mat_id_grouped if grouped else _L().oracle_mul_mat_id_brute
-    _chk(f(_p(W), E, n_out, nb * 32, _p(x), DTYPES[x_type], _p(ids), T, k, _mode(mode), _p(dst), _p(tol)))
+    _chk(f(_p(W), E, n_out, nb * 32, _p(x), DTYPES[x_type], _p(ids), T, k, _mode(mode), _p(dst), _p(tol), wtype(W)))
     return dst, tol
 
 
@@ -126,8 +140,15 @@ def mul_mat_id_rows(W, x, x_type, ids, slots, mode="broadcast"):
     out = np.zeros((len(slots), n_out), np.float64)
     tol = np.zeros_like(out)
     _chk(_L().oracle_mul_mat_id_rows(_p(W), E, n_out, nb * 32, _p(x), DTYPES[x_type], _p(ids), T, k,
-                                     _mode(mode), _p(slots), len(slots), _p(out), _p(tol)))
+                                     _mode(mode), _p(slots), len(slots), _p(out), _p(tol), wtype(W)))
     return out, tol
+
+
+def _same_wtype(*Ws):
+    t = {wtype(W) for W in Ws}
+    if len(t) != 1:
+        raise ValueError("the FFN's matrices must share one weight type")
+    return t.pop()
 
 
 def ffn(Wg, Wu, Wd, x, x_type, ids, slots=None):
@@ -146,7 +167,7 @@ def ffn(Wg, Wu, Wd, x, x_type, ids, slots=None):
     y = np.zeros((n, n_embd), np.float64)
     tol = np.zeros_like(y)
     _chk(_L().oracle_ffn_rows(_p(Wg), _p(Wu), _p(Wd), E, n_embd, n_ff, _p(x), DTYPES[x_type], _p(ids), T, k,
-                              sp, n, _p(y), _p(tol)))
+                              sp, n, _p(y), _p(tol), _same_wtype(Wg, Wu, Wd)))
     return y, tol
 
 
@@ -159,7 +180,7 @@ def shared_ffn(Sg, Su, Sd, x, x_type, tokens=None):
     y = np.zeros((len(tokens), n_embd), np.float64)
     tol = np.zeros_like(y)
     _chk(_L().oracle_shared_rows(_p(Sg), _p(Su), _p(Sd), n_embd, n_ff, _p(x), DTYPES[x_type], _p(tokens),
-                                 len(tokens), _p(y), _p(tol)))
+                                 len(tokens), _p(y), _p(tol), _same_wtype(Sg, Su, Sd)))
     return y, tol
 
 
@@ -173,7 +194,7 @@ def ffn_hidden(Wg, Wu, x, x_type, ids, slots):
     g = np.zeros_like(h)
     u = np.zeros_like(h)
     _chk(_L().oracle_ffn_hidden(_p(Wg), _p(Wu), E, nb * 32, n_ff, _p(x), DTYPES[x_type], _p(ids), T, k,
-                                _p(slots), len(slots), _p(h), _p(g), _p(u)))
+                                _p(slots), len(slots), _p(h), _p(g), _p(u), _same_wtype(Wg, Wu)))
     return h, g, u
 
 

@@ -20,9 +20,17 @@
  *   [cmoe]  "Optimalizace MoE modelů na slabém GPU: spuštění GPT-OSS-120B s 6 GB
  *           VRAM až 30 t/s", section "Architektura Mixture of Experts" (a router
  *           picks a few experts per token in every layer).
+ *   [TS]    the TensorSharp vs llama.cpp MoE CPU-offload benchmark page
+ *           (DeepSeek V4 / Gemma 4 / Qwen / GPT-OSS), per-model results: the
+ *           benchmarked weight types include GPT-OSS "Q8_0/MXFP4".
  *
  * Readings where the pages are silent (each also listed in the design notes):
  *   - Q8_0 block = fp16 scale d, then 32 int8 q; weight = d*q.
+ *   - MXFP4 block (the OCP microscaling FP4 type; the pages list MXFP4 among
+ *     the benchmarked weight types but print no bytes) = one E8M0 scale byte
+ *     X, then 16 bytes of 4-bit E2M1 codes, element i of the block in the low
+ *     nibble of byte i and element 16+i in its high nibble (the GGUF order
+ *     of 4-bit blocks); weight = 2^(X-127) * e2m1(code).
  *   - x is [T][n_in] (broadcast) or [T][k][n_in] (per_slot); dst is
  *     [T][k][n_out]; W is [E][n_out][n_in] (the page's ne-order
  *     [n_embd, n_embd_gate, n_experts] read innermost-first).
@@ -51,6 +59,7 @@
 enum { OR_OK = 0, OR_ERR_INVALID = -1, OR_ERR_RANGE = -2, OR_ERR_BAD_ID = -3 };
 enum { OR_BROADCAST = 0, OR_PER_SLOT = 1 };
 enum { OR_BF16 = 0, OR_F16 = 1, OR_F32 = 2 };
+enum { OR_Q8_0 = 0, OR_MXFP4 = 1 }; /* weight types */
 
 #define REL_TOL 2e-3
 #define ABS_TOL 1e-5
@@ -85,9 +94,30 @@ static double x_value(const void *x, int x_type, int64_t i) {
     }
 }
 
-/* Dequantised weight W[e][n][j] = d * q of a Q8_0 block ([PR283] 2.1 names
- * Q8_0 among the quantised types of the mmq_id path).  Exact in double. */
-static double w_value(const uint8_t *W, int64_t n_out, int64_t n_in, int64_t e, int64_t n, int64_t j) {
+/* E2M1 (OCP microscaling FP4 element): bit 3 sign, bits 2-1 exponent (bias 1),
+ * bit 0 mantissa.  Exponent 0 is the subnormal 0.5*m; otherwise
+ * 2^(exponent-1) * (1 + m/2).  Codes 0..7: 0, 0.5, 1, 1.5, 2, 3, 4, 6. */
+static double e2m1_value(int code) {
+    const int ex = (code >> 1) & 3, m = code & 1;
+    const double mag = ex == 0 ? 0.5 * m : ldexp(1.0 + 0.5 * m, ex - 1);
+    return (code & 8) ? -mag : mag;
+}
+
+/* E8M0 (OCP microscaling scale): 2^(X-127); X = 255 encodes NaN. */
+static double e8m0_value(uint8_t x) { return x == 255 ? NAN : ldexp(1.0, (int)x - 127); }
+
+/* Dequantised weight W[e][n][j], exact in double:
+ *   Q8_0  = d * q of its 34-byte block ([PR283] 2.1 names Q8_0 among the
+ *           quantised types of the mmq_id path);
+ *   MXFP4 = 2^(X-127) * e2m1(code) of its 17-byte block ([TS]'s GPT-OSS
+ *           weights are "Q8_0/MXFP4"). */
+static double w_value(const uint8_t *W, int wtype, int64_t n_out, int64_t n_in, int64_t e, int64_t n, int64_t j) {
+    if (wtype == OR_MXFP4) {
+        const uint8_t *blk = W + (((e * n_out + n) * (n_in / 32)) + j / 32) * 17;
+        const int i = (int)(j % 32);
+        const int code = i < 16 ? (blk[1 + i] & 15) : (blk[1 + i - 16] >> 4);
+        return e8m0_value(blk[0]) * e2m1_value(code);
+    }
     const uint8_t *blk = W + (((e * n_out + n) * (n_in / 32)) + j / 32) * 34;
     uint16_t d = (uint16_t)(blk[0] | (blk[1] << 8));
     int8_t q = (int8_t)blk[2 + (j % 32)];
@@ -147,12 +177,12 @@ int oracle_row_ids(const int32_t *ids, int64_t n_tokens, int k, int n_experts, i
 
 /* One output row: out[n] = sum_j W[e][n][j] * x[r][j] (ascending j, fp64), and
  * tol[n] = 2e-3 * sum_j |W[e][n][j] * x[r][j]| + 1e-5. */
-static void dot_row(const uint8_t *W, int64_t n_out, int64_t n_in, int64_t e, const void *x, int x_type,
+static void dot_row(const uint8_t *W, int wtype, int64_t n_out, int64_t n_in, int64_t e, const void *x, int x_type,
                     int64_t r, double *out, double *tol) {
     for (int64_t n = 0; n < n_out; ++n) {
         double acc = 0.0, mag = 0.0;
         for (int64_t j = 0; j < n_in; ++j) {
-            double prod = w_value(W, n_out, n_in, e, n, j) * x_value(x, x_type, r * n_in + j);
+            double prod = w_value(W, wtype, n_out, n_in, e, n, j) * x_value(x, x_type, r * n_in + j);
             acc += prod;
             mag += fabs(prod);
         }
@@ -167,7 +197,8 @@ static void dot_row(const uint8_t *W, int64_t n_out, int64_t n_in, int64_t e, co
  * of (t, s):  dst[t][s][:] = W[e] . x[r],  r = t (broadcast) or t*k+s.
  */
 int oracle_mul_mat_id_brute(const uint8_t *W, int n_experts, int n_out, int n_in, const void *x, int x_type,
-                            const int32_t *ids, int64_t n_tokens, int k, int mode, double *dst, double *tol) {
+                            const int32_t *ids, int64_t n_tokens, int k, int mode, double *dst, double *tol,
+                            int wtype) {
     int rc = oracle_check_args(n_tokens, k, n_experts);
     if (rc) return rc;
     if (n_in % 32) return OR_ERR_INVALID;
@@ -178,7 +209,7 @@ int oracle_mul_mat_id_brute(const uint8_t *W, int n_experts, int n_out, int n_in
     for (int64_t i = 0; i < S; ++i) {
         int64_t t = i / k;
         int64_t r = (mode == OR_BROADCAST) ? t : i;
-        dot_row(W, n_out, n_in, ids[i], x, x_type, r, dst + i * n_out, tol ? tol + i * n_out : NULL);
+        dot_row(W, wtype, n_out, n_in, ids[i], x, x_type, r, dst + i * n_out, tol ? tol + i * n_out : NULL);
     }
     return OR_OK;
 }
@@ -191,7 +222,8 @@ int oracle_mul_mat_id_brute(const uint8_t *W, int n_experts, int n_out, int n_in
  * force, so both must agree bit for bit.
  */
 int oracle_mul_mat_id_grouped(const uint8_t *W, int n_experts, int n_out, int n_in, const void *x, int x_type,
-                              const int32_t *ids, int64_t n_tokens, int k, int mode, double *dst, double *tol) {
+                              const int32_t *ids, int64_t n_tokens, int k, int mode, double *dst, double *tol,
+                              int wtype) {
     int rc = oracle_check_args(n_tokens, k, n_experts);
     if (rc) return rc;
     if (n_in % 32) return OR_ERR_INVALID;
@@ -203,7 +235,7 @@ int oracle_mul_mat_id_grouped(const uint8_t *W, int n_experts, int n_out, int n_
         for (int e = 0; e < n_experts; ++e) {
 #pragma omp parallel for schedule(dynamic, 1)
             for (int64_t p = bounds[e]; p < bounds[e + 1]; ++p)
-                dot_row(W, n_out, n_in, e, x, x_type, src1[p], dst + (int64_t)dstrow[p] * n_out,
+                dot_row(W, wtype, n_out, n_in, e, x, x_type, src1[p], dst + (int64_t)dstrow[p] * n_out,
                         tol ? tol + (int64_t)dstrow[p] * n_out : NULL);
         }
     }
@@ -216,14 +248,14 @@ int oracle_mul_mat_id_grouped(const uint8_t *W, int n_experts, int n_out, int n_
 /* Rows i of slot list `slots` only (for sampled checks at full size). */
 int oracle_mul_mat_id_rows(const uint8_t *W, int n_experts, int n_out, int n_in, const void *x, int x_type,
                            const int32_t *ids, int64_t n_tokens, int k, int mode, const int64_t *slots,
-                           int64_t n_slots, double *out, double *tol) {
+                           int64_t n_slots, double *out, double *tol, int wtype) {
     int rc = oracle_check_args(n_tokens, k, n_experts);
     if (rc) return rc;
 #pragma omp parallel for schedule(dynamic, 1)
     for (int64_t i = 0; i < n_slots; ++i) {
         int64_t sl = slots[i];
         int64_t r = (mode == OR_BROADCAST) ? sl / k : sl;
-        dot_row(W, n_out, n_in, ids[sl], x, x_type, r, out + i * n_out, tol ? tol + i * n_out : NULL);
+        dot_row(W, wtype, n_out, n_in, ids[sl], x, x_type, r, out + i * n_out, tol ? tol + i * n_out : NULL);
     }
     return OR_OK;
 }
@@ -246,15 +278,15 @@ static double silu(double z) { return z / (1.0 + exp(-z)); }
  *                   as bfloat16: relative rounding <= 2^-9)
  *   tol_y         = 2e-3 * sum|wd| (|h| + tol_h) + sum|wd| * tol_h + 1e-5
  */
-static void ffn_row(const uint8_t *Wg, const uint8_t *Wu, const uint8_t *Wd, int64_t e, int64_t n_embd,
+static void ffn_row(const uint8_t *Wg, const uint8_t *Wu, const uint8_t *Wd, int wtype, int64_t e, int64_t n_embd,
                     int64_t n_ff, const void *x, int x_type, int64_t r, double *y, double *tol_y, double *h,
                     double *th) {
     for (int64_t f = 0; f < n_ff; ++f) {
         double g = 0, u = 0, mg = 0, mu = 0;
         for (int64_t j = 0; j < n_embd; ++j) {
             double xv = x_value(x, x_type, r * n_embd + j);
-            double pg = w_value(Wg, n_ff, n_embd, e, f, j) * xv;
-            double pu = w_value(Wu, n_ff, n_embd, e, f, j) * xv;
+            double pg = w_value(Wg, wtype, n_ff, n_embd, e, f, j) * xv;
+            double pu = w_value(Wu, wtype, n_ff, n_embd, e, f, j) * xv;
             g += pg; u += pu; mg += fabs(pg); mu += fabs(pu);
         }
         double tg = REL_TOL * mg + ABS_TOL, tu = REL_TOL * mu + ABS_TOL;
@@ -266,7 +298,7 @@ static void ffn_row(const uint8_t *Wg, const uint8_t *Wu, const uint8_t *Wd, int
     for (int64_t n = 0; n < n_embd; ++n) {
         double acc = 0, m1 = 0, m2 = 0;
         for (int64_t f = 0; f < n_ff; ++f) {
-            double w = w_value(Wd, n_embd, n_ff, e, n, f);
+            double w = w_value(Wd, wtype, n_embd, n_ff, e, n, f);
             acc += w * h[f];
             m1 += fabs(w) * (fabs(h[f]) + th[f]);
             m2 += fabs(w) * th[f];
@@ -284,7 +316,7 @@ static void ffn_row(const uint8_t *Wg, const uint8_t *Wu, const uint8_t *Wd, int
  */
 int oracle_ffn_rows(const uint8_t *Wg, const uint8_t *Wu, const uint8_t *Wd, int n_experts, int n_embd, int n_ff,
                     const void *x, int x_type, const int32_t *ids, int64_t n_tokens, int k,
-                    const int64_t *slots, int64_t n_slots, double *y, double *tol_y) {
+                    const int64_t *slots, int64_t n_slots, double *y, double *tol_y, int wtype) {
     int rc = oracle_check_args(n_tokens, k, n_experts);
     if (rc) return rc;
     if (n_embd % 32 || n_ff % 32) return OR_ERR_INVALID;
@@ -299,7 +331,7 @@ int oracle_ffn_rows(const uint8_t *Wg, const uint8_t *Wu, const uint8_t *Wd, int
 #pragma omp for schedule(dynamic, 1)
         for (int64_t i = 0; i < count; ++i) {
             int64_t sl = slots ? slots[i] : i;
-            ffn_row(Wg, Wu, Wd, ids[sl], n_embd, n_ff, x, x_type, sl / k, y + i * n_embd,
+            ffn_row(Wg, Wu, Wd, wtype, ids[sl], n_embd, n_ff, x, x_type, sl / k, y + i * n_embd,
                     tol_y ? tol_y + i * n_embd : NULL, h, th);
         }
         free(h);
@@ -309,14 +341,15 @@ int oracle_ffn_rows(const uint8_t *Wg, const uint8_t *Wu, const uint8_t *Wd, int
 }
 
 int oracle_shared_rows(const uint8_t *Sg, const uint8_t *Su, const uint8_t *Sd, int n_embd, int n_ff_shared,
-                       const void *x, int x_type, const int64_t *tokens, int64_t n_tok, double *y, double *tol_y) {
+                       const void *x, int x_type, const int64_t *tokens, int64_t n_tok, double *y, double *tol_y,
+                       int wtype) {
     if (n_embd % 32 || n_ff_shared % 32) return OR_ERR_INVALID;
 #pragma omp parallel
     {
         double *h = malloc((size_t)n_ff_shared * sizeof(double)), *th = malloc((size_t)n_ff_shared * sizeof(double));
 #pragma omp for schedule(dynamic, 1)
         for (int64_t i = 0; i < n_tok; ++i)
-            ffn_row(Sg, Su, Sd, 0, n_embd, n_ff_shared, x, x_type, tokens[i], y + i * n_embd,
+            ffn_row(Sg, Su, Sd, wtype, 0, n_embd, n_ff_shared, x, x_type, tokens[i], y + i * n_embd,
                     tol_y ? tol_y + i * n_embd : NULL, h, th);
         free(h);
         free(th);
@@ -327,7 +360,7 @@ int oracle_shared_rows(const uint8_t *Sg, const uint8_t *Su, const uint8_t *Sd, 
 /* Hidden activations h = silu(g)*u of the listed slots (for pins on SwiGLU). */
 int oracle_ffn_hidden(const uint8_t *Wg, const uint8_t *Wu, int n_experts, int n_embd, int n_ff, const void *x,
                       int x_type, const int32_t *ids, int64_t n_tokens, int k, const int64_t *slots,
-                      int64_t n_slots, double *h_out, double *g_out, double *u_out) {
+                      int64_t n_slots, double *h_out, double *g_out, double *u_out, int wtype) {
     int rc = oracle_check_args(n_tokens, k, n_experts);
     if (rc) return rc;
 #pragma omp parallel for schedule(dynamic, 1)
@@ -337,8 +370,8 @@ int oracle_ffn_hidden(const uint8_t *Wg, const uint8_t *Wu, int n_experts, int n
             double g = 0, u = 0;
             for (int64_t j = 0; j < n_embd; ++j) {
                 double xv = x_value(x, x_type, r * n_embd + j);
-                g += w_value(Wg, n_ff, n_embd, e, f, j) * xv;
-                u += w_value(Wu, n_ff, n_embd, e, f, j) * xv;
+                g += w_value(Wg, wtype, n_ff, n_embd, e, f, j) * xv;
+                u += w_value(Wu, wtype, n_ff, n_embd, e, f, j) * xv;
             }
             g_out[i * n_ff + f] = g;
             u_out[i * n_ff + f] = u;
@@ -349,9 +382,9 @@ int oracle_ffn_hidden(const uint8_t *Wg, const uint8_t *Wu, int n_experts, int n
 }
 
 /* Dequantised weights of one expert as fp64 [n_out][n_in] (test helper). */
-void oracle_dequant(const uint8_t *W, int n_out, int n_in, int e, double *out) {
+void oracle_dequant(const uint8_t *W, int n_out, int n_in, int e, double *out, int wtype) {
     for (int64_t n = 0; n < n_out; ++n)
-        for (int64_t j = 0; j < n_in; ++j) out[n * n_in + j] = w_value(W, n_out, n_in, e, n, j);
+        for (int64_t j = 0; j < n_in; ++j) out[n * n_in + j] = w_value(W, wtype, n_out, n_in, e, n, j);
 }
 
 /*

@@ -7,13 +7,15 @@ hold exactly, and SwiGLU special values.  A dropped term, a wrong sign or
 index, or a transposed operand in the oracle fails at least one of them.
 """
 import itertools
+import json
+import os
 
 import numpy as np
 import pytest
 
 import oracle
 import workloads
-from tests.fixtures import hand_example, pack_q8_0, unpack_q8_0
+from tests.fixtures import GOLDEN, hand_example, pack_q8_0, unpack_q8_0
 
 
 def rand_q8(rng, E, n_out, n_in):
@@ -485,3 +487,84 @@ def test_float32_bounds_are_tight_enough_to_mean_something():
     assert np.all(tol_w <= 1e-4 * w)
     _, w_un, _ = oracle.route(logits, 8, normalize=False)  # forgetting the renormalisation
     assert np.all(np.abs(w_un - w) > tol_w)
+
+
+# ------------------------------------------------------------------- MXFP4
+def _golden_mxfp4():
+    with open(os.path.join(GOLDEN, "mxfp4_blocks.json")) as f:
+        return json.load(f)["blocks"]
+
+
+def _np_decode_mxfp4(W):
+    # independent restatement: the E2M1 magnitude table as the OCP MX
+    # specification lists it, sign from bit 3, nibbles split low/high
+    mag = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+    X = W[..., 0].astype(np.int64)
+    codes = np.concatenate([W[..., 1:] & 15, W[..., 1:] >> 4], axis=-1).astype(np.int64)
+    v = np.where(codes & 8, -1.0, 1.0) * mag[codes & 7]
+    scale = np.where(X == 255, np.nan, np.ldexp(1.0, X - 127))
+    out = v * scale[..., None]
+    return out.reshape(W.shape[:-2] + (W.shape[-2] * 32,))
+
+
+def test_mxfp4_hand_worked_blocks():
+    for blk in _golden_mxfp4():
+        W = np.array(blk["bytes"], np.uint8).reshape(1, 1, 1, 17)
+        got = oracle.dequant(W, 0)[0]
+        if blk.get("nan"):
+            assert np.isnan(got).all()
+            continue
+        if "values" in blk:
+            want = np.array(blk["values"], np.float64)
+        elif "values_pow2" in blk:
+            m, e = blk["values_pow2"][0]
+            want = np.full(32, np.ldexp(float(m), e))
+        elif "values_pow2_halves" in blk:
+            (m0, e0), (m1, e1) = blk["values_pow2_halves"]
+            want = np.concatenate([np.full(16, np.ldexp(float(m0), e0)), np.full(16, np.ldexp(float(m1), e1))])
+        else:
+            a, b = blk["values_halves"]
+            want = np.concatenate([np.full(16, float(a)), np.full(16, float(b))])
+        assert np.array_equal(got, want), blk["note"]
+        assert np.array_equal(np.signbit(got), np.signbit(want)), blk["note"]  # -0 stays -0
+
+
+def test_mxfp4_decoder_matches_numpy_on_random_blocks():
+    W = workloads.mxfp4_weights(3, 24, 96, 5, 9)
+    for e in range(3):
+        assert np.array_equal(oracle.dequant(W, e), _np_decode_mxfp4(W)[e])
+    # the generator's scales put the weights in a plausible range, every code occurs
+    w = _np_decode_mxfp4(W)
+    assert 0.7 < np.abs(w).max() <= 6 * 2.0 ** -3 and np.unique(np.concatenate([W[..., 1:] & 15, W[..., 1:] >> 4])).size == 16
+
+
+def test_mxfp4_mul_mat_id_is_a_dense_gemm_for_one_expert():
+    W = workloads.mxfp4_weights(1, 40, 128, 6, 1)
+    x = workloads.activations(7, 128, "f32", 6, 2)
+    ids = np.zeros((7, 1), np.int32)
+    dst, tol = oracle.mul_mat_id(W, x, "f32", ids)
+    want = x.astype(np.float64) @ _np_decode_mxfp4(W)[0].T
+    assert np.allclose(dst[:, 0, :], want, rtol=1e-13, atol=1e-13)
+    assert np.all(tol > 1e-5)
+
+
+def test_mxfp4_grouped_equals_brute_and_ffn_matches_numpy():
+    E, k, T, n_embd, n_ff = 6, 2, 9, 64, 96
+    ids = workloads.routing("uniform", T, E, k, 4)
+    W = workloads.mxfp4_weights(E, n_ff, n_embd, 4, 3)
+    x = workloads.activations(T, n_embd, "bf16", 4, 5)
+    a, _ = oracle.mul_mat_id(W, x, "bf16", ids)
+    b, _ = oracle.mul_mat_id(W, x, "bf16", ids, grouped=True)
+    assert np.array_equal(a, b)
+    Wg, Wu = W, workloads.mxfp4_weights(E, n_ff, n_embd, 4, 6)
+    Wd = workloads.mxfp4_weights(E, n_embd, n_ff, 4, 7)
+    y, _ = oracle.ffn(Wg, Wu, Wd, x, "bf16", ids)
+    xf = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    dg, du, dd = _np_decode_mxfp4(Wg), _np_decode_mxfp4(Wu), _np_decode_mxfp4(Wd)
+    for i in range(T * k):
+        t, e = i // k, ids.reshape(-1)[i]
+        g, u = dg[e] @ xf[t], du[e] @ xf[t]
+        h = g / (1.0 + np.exp(-g)) * u
+        assert np.allclose(y[i], dd[e] @ h, rtol=1e-12, atol=1e-12)
+    with pytest.raises(ValueError):
+        oracle.ffn(Wg, workloads.q8_0_weights(E, n_ff, n_embd, 4, 6), Wd, x, "bf16", ids)

@@ -55,6 +55,7 @@ def _L():
         _lib = ctypes.CDLL(build())
         i64, u64, dbl, vp, i32 = ctypes.c_int64, ctypes.c_uint64, ctypes.c_double, ctypes.c_void_p, ctypes.c_int
         _lib.wl_fill_q8_0.argtypes = [vp, i64, i64, i64, u64, u64, dbl, dbl]
+        _lib.wl_fill_mxfp4.argtypes = [vp, i64, i64, i64, u64, u64, i32, i32]
         for f in (_lib.wl_fill_normal_f32, _lib.wl_fill_normal_bf16, _lib.wl_fill_normal_f16):
             f.argtypes = [vp, i64, i64, u64, u64]
         _lib.wl_fill_uniform_f32.argtypes = [vp, i64, i64, dbl, dbl, u64, u64]
@@ -92,6 +93,23 @@ def q8_0_weights_experts(e0: int, n_e: int, n_out: int, n_in: int, seed: int, te
         raise ValueError("n_in must be a multiple of 32 for Q8_0")
     out = np.empty((n_e, n_out, n_in // 32, 34), dtype=np.uint8)
     _L().wl_fill_q8_0(_ptr(out), e0 * n_out, n_e * n_out, n_in, seed, tensor, D_LO, D_HI)
+    return out
+
+
+# MXFP4 scale bytes: 2^(X - 127) for X in [X_LO, X_HI], i.e. block scales 2^-9 .. 2^-3,
+# so the weights (element values up to 6 times the scale) span about 0.001 .. 0.75
+X_LO, X_HI = 118, 124
+
+
+def mxfp4_weights(n_experts: int, n_out: int, n_in: int, seed: int, tensor: int, e0: int = 0) -> np.ndarray:
+    """Stacked MXFP4 weights, uint8 array [n_experts][n_out][n_in/32][17]: per
+    block the scale byte, then 16 bytes of 4-bit codes (random bytes only).
+    Experts are numbered from e0 (counter-based: a slice equals the same
+    experts of a larger matrix)."""
+    if n_in % 32:
+        raise ValueError("n_in must be a multiple of 32 for MXFP4")
+    out = np.empty((n_experts, n_out, n_in // 32, 17), dtype=np.uint8)
+    _L().wl_fill_mxfp4(_ptr(out), e0 * n_out, n_experts * n_out, n_in, seed, tensor, X_LO, X_HI)
     return out
 
 

@@ -107,6 +107,35 @@ void wl_fill_q8_0(uint8_t *blocks, int64_t row0, int64_t n_rows_here, int64_t n_
     }
 }
 
+/*
+ * MXFP4 blocks (the OCP microscaling FP4 type, E2M1 elements sharing one E8M0
+ * scale per 32; the pages name "MXFP4" among the weight types of their
+ * benchmarks but do not print its bytes): 17 bytes per 32 weights along a
+ * row, the scale byte first, then 16 bytes of 4-bit element codes.  Only
+ * random bytes are drawn here: the scale byte uniform in [x_lo, x_hi], each
+ * 4-bit code uniform in [0, 15].  How a code and a scale give a weight is the
+ * consumer's business.
+ */
+void wl_fill_mxfp4(uint8_t *blocks, int64_t row0, int64_t n_rows_here, int64_t n_in,
+                   uint64_t seed, uint64_t tensor, int x_lo, int x_hi) {
+    const uint64_t kq = stream_key(seed, 2 * tensor);
+    const uint64_t kx = stream_key(seed, 2 * tensor + 1);
+    const int64_t nb = n_in / 32;
+    const uint64_t span = (uint64_t)(x_hi - x_lo + 1);
+#pragma omp parallel for schedule(static)
+    for (int64_t rr = 0; rr < n_rows_here; ++rr) {
+        const int64_t row = row0 + rr;
+        uint8_t *dst = blocks + rr * nb * 17;
+        for (int64_t b = 0; b < nb; ++b) {
+            dst[b * 17] = (uint8_t)(x_lo + (int)((draw(kx, (uint64_t)(row * nb + b)) >> 32) % span));
+            for (int j = 0; j < 16; ++j) {
+                uint64_t g = (uint64_t)(row * (n_in / 2) + b * 16 + j);
+                dst[b * 17 + 1 + j] = (uint8_t)(draw(kq, g) >> 56);
+            }
+        }
+    }
+}
+
 /* N(0,1) samples i0 .. i0+n-1 of a tensor, stored as float. */
 void wl_fill_normal_f32(float *out, int64_t i0, int64_t n, uint64_t seed, uint64_t tensor) {
     const uint64_t key = stream_key(seed, tensor);
