@@ -467,6 +467,10 @@ def run_ours(args):
     torch.cuda.empty_cache()
     if not args.no_decode:
         result["decode"] = run_decode(moe, torch, args, hbm_peak)
+        result["decode_noalloc"] = run_decode(moe, torch, args, hbm_peak, noalloc=True)
+    if not args.no_report:
+        result["lite"] = run_lite(moe, torch, hbm_peak, tc_peak)
+        result["skew"] = run_skew(moe, torch, hbm_peak, tc_peak)
 
     if rank == 0 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
@@ -477,9 +481,113 @@ def run_ours(args):
         print(json.dumps(result), flush=True)
 
 
-def run_decode(moe, torch, args, hbm_peak):
+def _roof(bytes_, flops, ms, hbm_peak, tc_peak):
+    """Roofline of one timed unit: the slower of its algorithmic bytes at the
+    HBM peak and its flops at the tensor peak, against the measured time."""
+    t_b, t_f = bytes_ / (hbm_peak * 1e9), flops / (tc_peak * 1e12)
+    return {"bound": "hbm" if t_b >= t_f else "tensor", "roofline_ms": round(max(t_b, t_f) * 1e3, 4),
+            "frac": round(max(t_b, t_f) * 1e3 / ms, 4), "GB/s": round(bytes_ / (ms * 1e-3) / 1e9, 1),
+            "TFLOP/s": round(flops / (ms * 1e-3) / 1e12, 1), "algorithmic_bytes": int(bytes_), "flops": flops}
+
+
+def _time_calls(torch, fn, reps=20, warm=3):
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def run_lite(moe, torch, hbm_peak, tc_peak):
+    """DeepSeek-Lite-shaped expert FFN: one moe_ffn on 512 tokens (64 experts,
+    top-6, 2048 -> 1408 -> 2048, uniform routing); weights 588 MB, beyond L2."""
+    wl = workloads.WORKLOADS["lite"]
+    E, k, n_embd, n_ff, T = wl.n_experts, wl.k, wl.n_in, wl.n_out, wl.n_tokens[0]
+    Wg = upload_prepared(moe, torch, E, n_ff, n_embd, workloads.T_WG)
+    Wu = upload_prepared(moe, torch, E, n_ff, n_embd, workloads.T_WU)
+    Wd = upload_prepared(moe, torch, E, n_embd, n_ff, workloads.T_WD)
+    ids_np = wl.ids(T)
+    x, ids = bf16_dev(torch, wl.x(T)), torch.from_numpy(ids_np).cuda()
+    ws = moe.workspace(T, k, E, n_embd, n_ff, 0, torch.bfloat16)
+    dst = torch.empty((T, k, n_embd), dtype=torch.float32, device="cuda")
+    ms = _time_calls(torch, lambda: moe.ffn(Wg, Wu, Wd, E, n_embd, n_ff, x, ids, ws=ws, out=dst))
+    if moe.get_status(ws) != moe.OK:
+        raise RuntimeError("lite: device status")
+    used, w_bytes = touched_ffn_bytes(ids_np, E, n_embd, n_ff)
+    S = T * k
+    b = w_bytes + T * n_embd * 2 + 2 * S * n_ff * 2 + S * n_embd * 4
+    out = {"ms": round(ms, 4), "tokens/s": round(T / (ms * 1e-3), 1), "experts_touched": int(used),
+           **_roof(b, 2.0 * S * n_embd * n_ff * 3, ms, hbm_peak, tc_peak),
+           "config": "moe_ffn, 64 experts top-6, 2048 -> 1408 -> 2048, Q8_0, bf16 x, 512 tokens, uniform routing; "
+                     "20 calls between CUDA events after 3 warm-up calls; weights beyond L2"}
+    del Wg, Wu, Wd
+    torch.cuda.empty_cache()
+    return out
+
+
+def _gemm_balance(counts, n_out, sms, bn=192, tile_m=128):
+    """The persistent GEMM's schedule for one mul_mat_id (tiles walked in (expert,
+    column tile, row unit) order, tile t on CTA t mod grid): per CTA the tiles and
+    the token columns (rounded to 16) it multiplies - where the 0-token and the
+    heavy experts of the skewed routing land."""
+    cols = []
+    for c in counts:
+        while c > 0:
+            cols.append(min(c, bn))
+            c -= bn
+    units = ((n_out + 15) // 16 * 16 + tile_m - 1) // tile_m
+    units = (units + 1) // 2  # two 128-row tiles per row unit (single matrix)
+    work = [int((n + 15) // 16 * 16) for n in cols for _ in range(units)]
+    grid = min(sms, len(work)) if work else 1
+    per_tiles = [len(work[i::grid]) for i in range(grid)]
+    per_cols = [sum(work[i::grid]) for i in range(grid)]
+    mean = sum(per_cols) / grid
+    return {"tiles": len(work), "grid": grid, "tiles_per_cta": [int(min(per_tiles)), int(max(per_tiles))],
+            "columns_per_cta": {"min": int(min(per_cols)), "max": int(max(per_cols)), "mean": round(float(mean), 1)},
+            "max_over_mean": round(float(max(per_cols) / mean), 4) if mean else None,
+            "experts_empty": int(sum(1 for c in counts if c == 0)), "largest_expert_tokens": int(max(counts))}
+
+
+def run_skew(moe, torch, hbm_peak, tc_peak):
+    """Skewed-load stress: moe_mul_mat_id on 8192 tokens (128 experts, top-4 Zipf
+    popularity with 8 empty experts, 2880 x 2880), broadcast and per_slot."""
+    wl = workloads.WORKLOADS["skew"]
+    E, k, n_in, n_out, T = wl.n_experts, wl.k, wl.n_in, wl.n_out, wl.n_tokens[0]
+    W = upload_prepared(moe, torch, E, n_out, n_in, workloads.T_W)
+    ids_np = wl.ids(T)
+    ids = torch.from_numpy(ids_np).cuda()
+    counts = np.bincount(ids_np.reshape(-1), minlength=E)
+    used = int((counts > 0).sum())
+    S = T * k
+    dst = torch.empty((T, k, n_out), dtype=torch.float32, device="cuda")
+    ws = moe.workspace(T, k, E, n_in, x_dtype=torch.bfloat16)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    out = {"balance": _gemm_balance(counts, n_out, sms)}
+    for mode in ("broadcast", "per_slot"):
+        x = bf16_dev(torch, wl.x(T, mode=mode))
+        ms = _time_calls(torch, lambda: moe.mul_mat_id(W, E, n_out, n_in, x, ids, mode, ws=ws, out=dst))
+        if moe.get_status(ws) != moe.OK:
+            raise RuntimeError("skew: device status")
+        b = used * n_out * n_in * Q8_BYTES_PER_W + x.numel() * 2 + S * n_out * 4
+        out[mode] = {"ms": round(ms, 4), "tokens/s": round(T / (ms * 1e-3), 1),
+                     **_roof(b, 2.0 * S * n_in * n_out, ms, hbm_peak, tc_peak)}
+        del x
+    out["config"] = ("moe_mul_mat_id, 128 experts top-4, Zipf(1.2) popularity (8 experts empty), 2880 x 2880, "
+                     "Q8_0, bf16 x, 8192 tokens; 20 calls between CUDA events after 3 warm-up calls")
+    del W
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_decode(moe, torch, args, hbm_peak, noalloc=False):
     """Decode step: n_layers distinct layer copies (beyond L2), fresh routing per
-    layer, replayed as one CUDA graph per token count."""
+    layer, replayed as one CUDA graph per token count; through moe_ffn with a
+    workspace per layer, or (noalloc) through the entry point without one."""
     E, k, n_embd, n_ff, n_sh = DEC.n_experts, DEC.k, DEC.n_in, DEC.n_out, DEC.n_ff_shared
     L = args.decode_layers
     base_g = upload_prepared(moe, torch, E, n_ff, n_embd, workloads.T_WG)
@@ -501,11 +609,17 @@ def run_decode(moe, torch, args, hbm_peak):
         dst = [torch.empty((T, k, n_embd), dtype=torch.float32, device="cuda") for _ in range(L)]
         dsh = [torch.empty((T, n_embd), dtype=torch.float32, device="cuda") for _ in range(L)]
 
+        status = torch.zeros(1, dtype=torch.int32, device="cuda")
+
         def all_layers():
             for l in range(L):
                 g, u, d = layers[l]
-                moe.ffn(g, u, d, E, n_embd, n_ff, x, ids[l], shared=(*shared[l], n_sh), ws=ws[l], out=dst[l],
-                        out_shared=dsh[l])
+                if noalloc:
+                    moe.ffn_decode_noalloc(g, u, d, E, n_embd, n_ff, x, ids[l], shared=(*shared[l], n_sh),
+                                           out=dst[l], out_shared=dsh[l], status=status)
+                else:
+                    moe.ffn(g, u, d, E, n_embd, n_ff, x, ids[l], shared=(*shared[l], n_sh), ws=ws[l], out=dst[l],
+                            out_shared=dsh[l])
 
         all_layers()
         torch.cuda.synchronize()
@@ -531,6 +645,8 @@ def run_decode(moe, torch, args, hbm_peak):
             st = moe.get_status(w)
             if st != moe.OK:
                 raise RuntimeError(f"decode T={T}: {moe.status_string(st)}")
+        if noalloc and int(status.item()) != moe.OK:
+            raise RuntimeError(f"decode (no workspace) T={T}: {moe.status_string(int(status.item()))}")
         bytes_step = touched * per_expert + L * per_shared
         gbs = bytes_step / (ms * 1e-3) / 1e9
         out[f"T={T}"] = {"us_per_layer": round(ms * 1e3 / L, 2), "GB/s": round(gbs, 1),
@@ -577,6 +693,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-combine", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-report", action="store_true", help="skip the Lite and skewed-load report keys")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--decode-layers", type=int, default=16)
     ap.add_argument("--decode-only", action="store_true", help="profiling only: the decode measurement alone")
@@ -591,7 +708,8 @@ def main():
 
         import indirect_expert_matmul_b200 as moe
         hbm_peak = load_peaks()[0]
-        print(json.dumps({"decode": run_decode(moe, torch, args, hbm_peak)}), flush=True)
+        print(json.dumps({"decode": run_decode(moe, torch, args, hbm_peak),
+                          "decode_noalloc": run_decode(moe, torch, args, hbm_peak, noalloc=True)}), flush=True)
     else:
         run_ours(args)
 

@@ -71,6 +71,15 @@ typedef enum {
 
 typedef enum { MOE_BROADCAST = 0, MOE_PER_SLOT = 1 } moe_mode;
 typedef enum { MOE_BF16 = 0, MOE_F16 = 1, MOE_F32 = 2 } moe_dtype;
+/* Expert weight types.  Q8_0: 34-byte blocks (fp16 d, 32 int8 q; w = d*q).
+ * MXFP4: 17-byte blocks of 32 weights (the OCP microscaling FP4 type that the
+ * TensorSharp benchmark page lists for GPT-OSS, "Q8_0/MXFP4"): an E8M0 scale
+ * byte X, then 16 bytes of 4-bit E2M1 codes, element i of the block in the low
+ * nibble of byte i and element 16+i in its high nibble; w = 2^(X-127) * e2m1,
+ * with E2M1 = sign, 2 exponent bits (bias 1), 1 mantissa bit (codes 0..7 are
+ * 0, 0.5, 1, 1.5, 2, 3, 4, 6).  X = 255 (NaN) and weights beyond the float
+ * range give unspecified results. */
+typedef enum { MOE_Q8_0 = 0, MOE_MXFP4 = 1 } moe_wtype;
 
 typedef void *moe_stream; /* cudaStream_t */
 
@@ -120,6 +129,17 @@ MOE_API size_t moe_weights_prepared_size(int n_experts, int n_out, int n_in);
  */
 MOE_API moe_status moe_weights_prepare(const void *q8_0_blocks, int n_experts, int n_out, int n_in, void *prepared,
                                moe_stream stream);
+
+/*
+ * The same two calls for a given weight type: moe_weights_prepared_size(...)
+ * and moe_weights_prepare(...) are these with MOE_Q8_0.  MOE_MXFP4 takes the
+ * 17-byte blocks described at moe_wtype (any 1-byte alignment) and repacks
+ * them the same tile-major way (0.53125 bytes per weight when n_out % 16 == 0
+ * and n_in % 64 == 0).  MOE_ERR_INVALID for an unknown type.
+ */
+MOE_API size_t moe_weights_prepared_size_w(moe_wtype w_type, int n_experts, int n_out, int n_in);
+MOE_API moe_status moe_weights_prepare_w(moe_wtype w_type, const void *blocks, int n_experts, int n_out, int n_in,
+                                         void *prepared, moe_stream stream);
 
 /* ------------------------------------------------------------------ row ids */
 
@@ -172,6 +192,23 @@ MOE_API moe_status moe_ffn(const void *Wg, const void *Wu, const void *Wd, int n
                    const void *Sg, const void *Su, const void *Sd, int n_ff_shared, const void *x, moe_dtype x_type,
                    const int32_t *ids, int64_t n_tokens, int k, float *dst, float *dst_shared, void *workspace,
                    moe_stream stream);
+
+/*
+ * moe_mul_mat_id and moe_ffn for a given weight type (the plain entry points
+ * are these with MOE_Q8_0); every weight pointer must hold that type's
+ * prepared form.  MXFP4 weights decode exactly to float (and to bf16: an E2M1
+ * value times a power of two has at most 2 significant bits), so the
+ * tensor-core path multiplies bf16 operands: x is used as bf16 (exact for bf16
+ * input, one rounding for fp16 / fp32 input).  The mat-vec path accumulates
+ * exact fp32 products.  MOE_ERR_INVALID for an unknown type.
+ */
+MOE_API moe_status moe_mul_mat_id_w(moe_wtype w_type, const void *W_prepared, int n_experts, int n_out, int n_in,
+                                    const void *x, moe_dtype x_type, const int32_t *ids, int64_t n_tokens, int k,
+                                    moe_mode mode, float *dst, void *workspace, moe_stream stream);
+MOE_API moe_status moe_ffn_w(moe_wtype w_type, const void *Wg, const void *Wu, const void *Wd, int n_experts,
+                             int n_embd, int n_ff, const void *Sg, const void *Su, const void *Sd, int n_ff_shared,
+                             const void *x, moe_dtype x_type, const int32_t *ids, int64_t n_tokens, int k, float *dst,
+                             float *dst_shared, void *workspace, moe_stream stream);
 
 /*
  * Decode-size moe_ffn that allocates nothing and takes no workspace.  The

@@ -19,12 +19,16 @@ LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 OK, ERR_INVALID, ERR_RANGE, ERR_BAD_ID, ERR_CUDA, ERR_TIMEOUT, ERR_UNSUPPORTED = 0, -1, -2, -3, -4, -5, -6
 BROADCAST, PER_SLOT = 0, 1
 BF16, F16, F32 = 0, 1, 2
+Q8_0, MXFP4 = 0, 1
+_WTYPE = {"q8_0": Q8_0, "mxfp4": MXFP4, Q8_0: Q8_0, MXFP4: MXFP4}
 
 # every symbol declared in include/moe.h
 ABI_SYMBOLS = (
     "moe_status_string", "moe_workspace_size", "moe_workspace_init", "moe_get_status",
     "moe_weights_prepared_size", "moe_weights_prepare", "moe_row_ids", "moe_mul_mat_id", "moe_ffn",
-    "moe_ffn_decode_noalloc", "moe_route", "moe_combine", "moe_set_gemv_threshold", "moe_get_gemv_threshold", "moe_set_path", "moe_profile_enable", "moe_profile_read",
+    "moe_ffn_decode_noalloc", "moe_route", "moe_combine", "moe_set_gemv_threshold", "moe_get_gemv_threshold",
+    "moe_set_path", "moe_profile_enable", "moe_profile_read", "moe_weights_prepared_size_w", "moe_weights_prepare_w",
+    "moe_mul_mat_id_w", "moe_ffn_w", "moe_testing_stall",
 )
 
 _lib = None
@@ -48,6 +52,12 @@ def _L() -> ctypes.CDLL:
     L.moe_weights_prepared_size.argtypes = [_i32, _i32, _i32]
     L.moe_weights_prepared_size.restype = _sz
     L.moe_weights_prepare.argtypes = [_vp, _i32, _i32, _i32, _vp, _vp]
+    L.moe_weights_prepared_size_w.argtypes = [_i32, _i32, _i32, _i32]
+    L.moe_weights_prepared_size_w.restype = _sz
+    L.moe_weights_prepare_w.argtypes = [_i32, _vp, _i32, _i32, _i32, _vp, _vp]
+    L.moe_mul_mat_id_w.argtypes = [_i32, _vp, _i32, _i32, _i32, _vp, _i32, _vp, _i64, _i32, _i32, _vp, _vp, _vp]
+    L.moe_ffn_w.argtypes = [_i32, _vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _i32, _vp, _i64, _i32,
+                            _vp, _vp, _vp, _vp]
     L.moe_row_ids.argtypes = [_vp, _i64, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp]
     L.moe_mul_mat_id.argtypes = [_vp, _i32, _i32, _i32, _vp, _i32, _vp, _i64, _i32, _i32, _vp, _vp, _vp]
     L.moe_ffn.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _i32, _vp, _i64, _i32,
@@ -61,6 +71,8 @@ def _L() -> ctypes.CDLL:
     L.moe_get_gemv_threshold.argtypes = []
     L.moe_set_path.argtypes = [_i32]
     L.moe_set_path.restype = None
+    L.moe_testing_stall.argtypes = [_i32, _i32, _i32]
+    L.moe_testing_stall.restype = None
     L.moe_profile_enable.argtypes = [_i32]
     L.moe_profile_enable.restype = None
     L.moe_profile_read.argtypes = [ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(_i32),
@@ -148,18 +160,23 @@ def get_status(ws) -> int:
 
 
 # ---------------------------------------------------------------- weights
-def weights_prepared_size(n_experts, n_out, n_in) -> int:
-    return _L().moe_weights_prepared_size(n_experts, n_out, n_in)
+def weights_prepared_size(n_experts, n_out, n_in, wtype="q8_0") -> int:
+    return _L().moe_weights_prepared_size_w(_WTYPE[wtype], n_experts, n_out, n_in)
 
 
-def weights_prepare(q8_0, n_experts, n_out, n_in, out=None):
-    """Repack Q8_0 blocks (uint8 [E][n_out][n_in/32][34], on the GPU)."""
-    _cuda(q8_0, "q8_0", torch.uint8)
-    n = weights_prepared_size(n_experts, n_out, n_in)
+_BLOCK_BYTES = {Q8_0: 34, MXFP4: 17}
+
+
+def weights_prepare(blocks, n_experts, n_out, n_in, out=None, wtype="q8_0"):
+    """Repack Q8_0 blocks (uint8 [E][n_out][n_in/32][34]) or MXFP4 blocks
+    (uint8 [E][n_out][n_in/32][17]), on the GPU, into the form the kernels read."""
+    w = _WTYPE[wtype]
+    _need(blocks, "blocks", torch.uint8, n_experts * n_out * (n_in // 32) * _BLOCK_BYTES[w])
+    n = weights_prepared_size(n_experts, n_out, n_in, w)
     if out is None:
-        out = torch.empty(n, dtype=torch.uint8, device=q8_0.device)
-    _need(out, "out", torch.uint8, n, q8_0.device)
-    _chk(_L().moe_weights_prepare(_ptr(q8_0), n_experts, n_out, n_in, _ptr(out), _stream(q8_0.device)),
+        out = torch.empty(n, dtype=torch.uint8, device=blocks.device)
+    _need(out, "out", torch.uint8, n, blocks.device)
+    _chk(_L().moe_weights_prepare_w(w, _ptr(blocks), n_experts, n_out, n_in, _ptr(out), _stream(blocks.device)),
          "moe_weights_prepare")
     return out
 
@@ -183,16 +200,18 @@ def row_ids(ids, n_experts, mode="broadcast", ws=None):
 
 
 # --------------------------------------------------------------- operators
-def mul_mat_id(W, n_experts, n_out, n_in, x, ids, mode="broadcast", ws=None, out=None):
+def mul_mat_id(W, n_experts, n_out, n_in, x, ids, mode="broadcast", ws=None, out=None, wtype="q8_0"):
     """dst float32 [T][k][n_out] = W[ids[t][s]] . x[t or (t, s)].
 
-    Without `ws` the call makes its own workspace, synchronises and raises
-    MoeError on a device-side error; with `ws` the caller reads get_status."""
+    W: prepared weights of type `wtype` ("q8_0" or "mxfp4").  Without `ws` the
+    call makes its own workspace, synchronises and raises MoeError on a
+    device-side error; with `ws` the caller reads get_status."""
+    w = _WTYPE[wtype]
     _cuda(x, "x")
     dev = x.device
     _cuda(ids, "ids", torch.int32, dev)
     T, k = ids.shape
-    _need(W, "W", torch.uint8, weights_prepared_size(n_experts, n_out, n_in), dev)
+    _need(W, "W", torch.uint8, weights_prepared_size(n_experts, n_out, n_in, w), dev)
     _need(x, "x", x.dtype, (T if _MODE[mode] == BROADCAST else T * k) * n_in)
     own_ws = ws is None
     if own_ws:
@@ -201,29 +220,31 @@ def mul_mat_id(W, n_experts, n_out, n_in, x, ids, mode="broadcast", ws=None, out
     if out is None:
         out = torch.empty((T, k, n_out), dtype=torch.float32, device=dev)
     _need(out, "out", torch.float32, T * k * n_out, dev)
-    _chk(_L().moe_mul_mat_id(_ptr(W), n_experts, n_out, n_in, _ptr(x), _XTYPE[x.dtype], _ptr(ids), T, k,
-                             _MODE[mode], _ptr(out), _ptr(ws), _stream(x.device)), "moe_mul_mat_id")
+    _chk(_L().moe_mul_mat_id_w(w, _ptr(W), n_experts, n_out, n_in, _ptr(x), _XTYPE[x.dtype], _ptr(ids), T, k,
+                               _MODE[mode], _ptr(out), _ptr(ws), _stream(x.device)), "moe_mul_mat_id")
     if own_ws:
         _chk(get_status(ws), "moe_mul_mat_id (device status)")
     return out
 
 
-def _check_ffn_inputs(Wg, Wu, Wd, Sg, Su, Sd, n_experts, n_embd, n_ff, n_ff_sh, x, T):
+def _check_ffn_inputs(Wg, Wu, Wd, Sg, Su, Sd, n_experts, n_embd, n_ff, n_ff_sh, x, T, w=Q8_0):
     dev = x.device
-    _need(Wg, "Wg", torch.uint8, weights_prepared_size(n_experts, n_ff, n_embd), dev)
-    _need(Wu, "Wu", torch.uint8, weights_prepared_size(n_experts, n_ff, n_embd), dev)
-    _need(Wd, "Wd", torch.uint8, weights_prepared_size(n_experts, n_embd, n_ff), dev)
+    _need(Wg, "Wg", torch.uint8, weights_prepared_size(n_experts, n_ff, n_embd, w), dev)
+    _need(Wu, "Wu", torch.uint8, weights_prepared_size(n_experts, n_ff, n_embd, w), dev)
+    _need(Wd, "Wd", torch.uint8, weights_prepared_size(n_experts, n_embd, n_ff, w), dev)
     if n_ff_sh:
-        _need(Sg, "Sg", torch.uint8, weights_prepared_size(1, n_ff_sh, n_embd), dev)
-        _need(Su, "Su", torch.uint8, weights_prepared_size(1, n_ff_sh, n_embd), dev)
-        _need(Sd, "Sd", torch.uint8, weights_prepared_size(1, n_embd, n_ff_sh), dev)
+        _need(Sg, "Sg", torch.uint8, weights_prepared_size(1, n_ff_sh, n_embd, w), dev)
+        _need(Su, "Su", torch.uint8, weights_prepared_size(1, n_ff_sh, n_embd, w), dev)
+        _need(Sd, "Sd", torch.uint8, weights_prepared_size(1, n_embd, n_ff_sh, w), dev)
     _need(x, "x", x.dtype, T * n_embd)
 
 
-def ffn(Wg, Wu, Wd, n_experts, n_embd, n_ff, x, ids, shared=None, ws=None, out=None, out_shared=None):
-    """Routed SwiGLU expert FFN (+ optional shared expert (Sg, Su, Sd, n_ff_shared)).
+def ffn(Wg, Wu, Wd, n_experts, n_embd, n_ff, x, ids, shared=None, ws=None, out=None, out_shared=None, wtype="q8_0"):
+    """Routed SwiGLU expert FFN (+ optional shared expert (Sg, Su, Sd, n_ff_shared)),
+    every matrix prepared as `wtype` ("q8_0" or "mxfp4").
 
     Returns (dst [T][k][n_embd], dst_shared [T][n_embd] or None), float32."""
+    w = _WTYPE[wtype]
     _cuda(x, "x")
     dev = x.device
     _cuda(ids, "ids", torch.int32, dev)
@@ -232,7 +253,7 @@ def ffn(Wg, Wu, Wd, n_experts, n_embd, n_ff, x, ids, shared=None, ws=None, out=N
     n_ff_sh = 0
     if shared is not None:
         Sg, Su, Sd, n_ff_sh = shared
-    _check_ffn_inputs(Wg, Wu, Wd, Sg, Su, Sd, n_experts, n_embd, n_ff, n_ff_sh, x, T)
+    _check_ffn_inputs(Wg, Wu, Wd, Sg, Su, Sd, n_experts, n_embd, n_ff, n_ff_sh, x, T, w)
     own_ws = ws is None
     if own_ws:
         ws = workspace(T, k, n_experts, n_embd, n_ff, n_ff_sh, x.dtype, device=dev)
@@ -244,9 +265,9 @@ def ffn(Wg, Wu, Wd, n_experts, n_embd, n_ff, x, ids, shared=None, ws=None, out=N
         out_shared = torch.empty((T, n_embd), dtype=torch.float32, device=dev)
     if shared is not None:
         _need(out_shared, "out_shared", torch.float32, T * n_embd, dev)
-    _chk(_L().moe_ffn(_ptr(Wg), _ptr(Wu), _ptr(Wd), n_experts, n_embd, n_ff, _ptr(Sg), _ptr(Su), _ptr(Sd), n_ff_sh,
-                      _ptr(x), _XTYPE[x.dtype], _ptr(ids), T, k, _ptr(out), _ptr(out_shared), _ptr(ws),
-                      _stream(x.device)), "moe_ffn")
+    _chk(_L().moe_ffn_w(w, _ptr(Wg), _ptr(Wu), _ptr(Wd), n_experts, n_embd, n_ff, _ptr(Sg), _ptr(Su), _ptr(Sd),
+                        n_ff_sh, _ptr(x), _XTYPE[x.dtype], _ptr(ids), T, k, _ptr(out), _ptr(out_shared), _ptr(ws),
+                        _stream(x.device)), "moe_ffn")
     if own_ws:
         _chk(get_status(ws), "moe_ffn (device status)")
     return out, out_shared

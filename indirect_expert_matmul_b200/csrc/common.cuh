@@ -23,23 +23,34 @@ __device__ __forceinline__ int read_status(const int* status) { return *(volatil
 
 // ------------------------------------------------------------ repacked weights
 // Tile-major form: per expert, per 128-row tile mt, per 64-column tile kt, one
-// block of rows(mt) rows: rows*32 bytes of u = q + 128 for columns [0, 32) of
-// each row (32 bytes per row), then rows*32 bytes for columns [32, 64), then
-// rows*4 bytes of scales (two fp16 per row, one per 32-column half).
+// block of rows(mt) rows, itself cut into sub-blocks of 32 rows (the last one
+// 16 rows when rows(mt) is not a multiple of 32).  Any run of consecutive
+// 32-row sub-blocks of one k-step is contiguous, so a row sub-tile of 32, 64
+// or 128 rows is one copy per k-step.  A sub-block of nr rows holds, per type:
+//  Q8_0  (68 bytes a row): nr*32 bytes of u = q + 128 for columns [0, 32) of
+//        each row (32 bytes per row), then nr*32 bytes for columns [32, 64),
+//        then nr*4 bytes of scales (two fp16 per row, one per 32-column half);
+//  MXFP4 (34 bytes a row): nr*32 bytes of 4-bit E2M1 codes (32 bytes per row:
+//        byte j holds column 2j in its low nibble and 2j+1 in its high
+//        nibble), then nr*2 bytes of E8M0 scales (one per 32-column half).
 // rows(mt) = min(128, n_out_pad - 128*mt), n_out_pad = round_up(n_out, 16).
 constexpr int kTileM = 128;
 constexpr int kTileK = 64;
-constexpr int kRowBytes = kTileK + 4;  // 64 q bytes + 2 fp16 scales
+constexpr int kRowBytes = kTileK + 4;  // Q8_0: 64 q bytes + 2 fp16 scales
+constexpr int kRowBytesMx = 32 + 2;    // MXFP4: 64 codes + 2 scale bytes
+constexpr int kSubRows = 32;           // rows of a sub-block
 
 struct WLayout {
     int n_out, n_in, n_out_pad, kt_count, mt_count;
+    int rb;  // bytes of one row of one k-step: kRowBytes (Q8_0) or kRowBytesMx (MXFP4)
     int64_t expert_bytes;
     __host__ __device__ WLayout() {}
-    __host__ __device__ WLayout(int n_out_, int n_in_) : n_out(n_out_), n_in(n_in_) {
+    __host__ __device__ WLayout(int n_out_, int n_in_, int wtype = MOE_Q8_0) : n_out(n_out_), n_in(n_in_) {
+        rb = wtype == MOE_MXFP4 ? kRowBytesMx : kRowBytes;
         n_out_pad = (n_out + 15) / 16 * 16;
         kt_count = (n_in + kTileK - 1) / kTileK;
         mt_count = (n_out_pad + kTileM - 1) / kTileM;
-        expert_bytes = (int64_t)n_out_pad * kt_count * kRowBytes;
+        expert_bytes = (int64_t)n_out_pad * kt_count * rb;
     }
     __host__ __device__ int rows(int mt) const {
         int r = n_out_pad - mt * kTileM;
@@ -47,9 +58,18 @@ struct WLayout {
     }
     // byte offset of block (e, mt, kt)
     __host__ __device__ int64_t block(int e, int mt, int kt) const {
-        return e * expert_bytes + (int64_t)mt * kTileM * kt_count * kRowBytes + (int64_t)rows(mt) * kt * kRowBytes;
+        return e * expert_bytes + (int64_t)mt * kTileM * kt_count * rb + (int64_t)rows(mt) * kt * rb;
     }
+    __host__ __device__ int sub_bytes() const { return kSubRows * rb; }  // one full sub-block
 };
+
+// Inside a k-step block of `rows` rows: row r lies in sub-block r / 32, which
+// starts (r / 32) * sub_bytes() into the block and holds sub_rows(rows, r / 32) rows.
+__host__ __device__ __forceinline__ int sub_rows(int rows, int sb) {
+    const int r = rows - sb * kSubRows;
+    return r < kSubRows ? r : kSubRows;
+}
+
 
 // ------------------------------------------------------------------ workspace
 // Rows of the tile-major activation buffers of the grouped GEMM: every
@@ -59,14 +79,9 @@ struct WLayout {
 inline int64_t tiled_rows(int64_t S, int n_groups) {
     return S + 8 * (S < n_groups ? S : n_groups) + 32;
 }
-// Split-K of the mat-vec kernel (decode FFN gate/up): at most kGvMaxChunks
-// K-chunks per (expert, row tile), only for n_tokens*k <= kGvSplitSlots; the
-// chunks' fp32 partial sums live in the workspace.
-constexpr int kGvSplitSlots = 64;
-constexpr int kGvMaxChunks = 8;
 struct WsLayout {
     int64_t S, rows_pad, rows_pad_sh;
-    size_t hdr, src1, dst, sprow, bounds, active, tiles, pad, h, h_sh, xt, xt_sh, xs, xs_sh, gv_part, gv_part_sh, total;
+    size_t hdr, src1, dst, sprow, bounds, active, tiles, pad, h, h_sh, xt, xt_sh, xs, xs_sh, total;
     static size_t up(size_t v) { return (v + 255) / 256 * 256; }
     WsLayout(int64_t n_tokens, int k, int n_experts, int n_in, int n_hidden, int n_hidden_sh, int x_type) {
         (void)x_type;
@@ -91,9 +106,6 @@ struct WsLayout {
         xt_sh = o; o += n_hidden_sh > 0 ? up((size_t)rows_pad_sh * kin * 128) : 0;
         xs = o; o += up((size_t)rows_pad * 4);  // power-of-two scale of each tiled activation row
         xs_sh = o; o += n_hidden_sh > 0 ? up((size_t)rows_pad_sh * 4) : 0;
-        const bool split = S <= kGvSplitSlots;
-        gv_part = o; o += split ? up((size_t)kGvMaxChunks * S * ((n_hidden + 15) / 16 * 16) * 2 * 4) : 0;
-        gv_part_sh = o; o += split ? up((size_t)kGvMaxChunks * n_tokens * ((n_hidden_sh + 15) / 16 * 16) * 2 * 4) : 0;
         total = o;
     }
 };

@@ -92,6 +92,7 @@ struct GemmParams {
     int out_ld;
     int* hdr;
     int bf16;                   // operand type: 1 bf16, 0 fp16
+    int wtype;                  // A operand: MOE_Q8_0, or MOE_MXFP4 (bf16 operands)
     const float* col_scale;     // per tiled row of B (a tile column): factor the accumulator takes (null: 1)
 };
 
@@ -226,7 +227,37 @@ __device__ __forceinline__ void dequant16_sts(uint4 x, uint32_t d2, float dsc, u
     ptx::sts128(dst1, make_uint4(pk[4], pk[5], pk[6], pk[7]));
 }
 
-template <int DUAL, int BF16>
+// E8M0 scale byte -> 2^(x - 127) as a float (x = 0: 2^-127; x = 255: NaN).
+__device__ __forceinline__ float e8m0_scale(uint32_t x) {
+    return x == 0u ? __uint_as_float(0x00400000u) : x == 255u ? __uint_as_float(0x7fc00000u) : __uint_as_float(x << 23);
+}
+
+// 8 MXFP4 codes (one 32-bit word, code i in bits 4i..4i+3; consecutive
+// columns) -> one 16-byte chunk of bf16 operand values, exact: the pair
+// conversion to f16 is exact (two significant bits), the power-of-two scale
+// is exact in float, and the product has at most two significant bits.
+__device__ __forceinline__ void dequant_mx8_sts(uint32_t w, float s, uint32_t dst) {
+    uint32_t h[4];
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+        : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+        : "r"(w));
+    uint32_t pk[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __half2 v = *(const __half2*)&h[i];
+        const __nv_bfloat162 b = __floats2bfloat162_rn(__low2float(v) * s, __high2float(v) * s);
+        pk[i] = *(const uint32_t*)&b;
+    }
+    ptx::sts128(dst, make_uint4(pk[0], pk[1], pk[2], pk[3]));
+}
+
+// WT: weight type of the A operand (MOE_Q8_0, or MOE_MXFP4 with BF16 = 1).
+template <int DUAL, int BF16, int WT>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 grouped_gemm_kernel(const GemmParams p) {
     extern __shared__ uint8_t smem_dyn[];
@@ -326,7 +357,7 @@ grouped_gemm_kernel(const GemmParams p) {
                     for (int i = 0; i < 2; ++i) {
                         int rows, mt;
                         source(tl, i, pf_a[i], rows, mt);
-                        pf_b[i] = (uint32_t)rows * kRowBytes;
+                        pf_b[i] = (uint32_t)rows * L.rb;
                     }
                     pf_tile = pf_t;
                 }
@@ -343,7 +374,7 @@ grouped_gemm_kernel(const GemmParams p) {
                 for (int i = 0; i < 2; ++i) {
                     int rows, mt;
                     source(tl, i, a[i], rows, mt);
-                    nb[i] = (uint32_t)rows * kRowBytes;
+                    nb[i] = (uint32_t)rows * L.rb;
                 }
                 for (int kt = 0; kt < KT; ++kt) {
                     prefetch_one();
@@ -482,7 +513,32 @@ grouped_gemm_kernel(const GemmParams p) {
                         ok = warp_wait(&raw_full[rs], rph, abort_flag, status) &&
                              warp_wait(&a_empty[as], aph ^ 1, abort_flag, status);
                         if (!ok) break;
-                        if (nr > 0) {
+                        if (nr > 0 && WT == MOE_MXFP4) {
+                            // this warp's rows are sub-block di & 3 (nsr rows): 32 code bytes a row at
+                            // sub + lane*32 (two 16-byte halves, read in alternating order), then two
+                            // scale bytes a row at sub + nsr*32 + lane*2
+                            const uint32_t raw = raw_sa + (uint32_t)(rs * 2 + mat) * kRawBytes;
+                            const uint32_t dst = a_sa + (uint32_t)as * 2u * kATileBytes + a_row;
+                            uint4 h0 = make_uint4(0u, 0u, 0u, 0u), h1 = h0;
+                            uint32_t xs = 0x7f7fu;  // padding rows: codes 0, scale 1
+                            if (r < nr) {
+                                const int nsr = sub_rows(nr, di & 3);
+                                const uint32_t sub = raw + (uint32_t)(di & 3) * (uint32_t)L.sub_bytes();
+                                const uint32_t q = sub + (uint32_t)lane * 32u;
+                                const uint4 ca = ptx::lds128(q + first * 16), cb = ptx::lds128(q + (first ^ 1) * 16);
+                                h0 = first ? cb : ca;
+                                h1 = first ? ca : cb;
+                                xs = ptx::lds16(sub + (uint32_t)nsr * 32u + (uint32_t)lane * 2u);
+                            }
+                            const float s0 = e8m0_scale(xs & 0xffu), s1 = e8m0_scale(xs >> 8);
+                            const uint32_t w0[4] = {h0.x, h0.y, h0.z, h0.w}, w1[4] = {h1.x, h1.y, h1.z, h1.w};
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {  // word i of half h holds operand chunk 4h + i
+                                dequant_mx8_sts(w0[i], s0, dst + ((((uint32_t)i) ^ rx) << 4));
+                                dequant_mx8_sts(w1[i], s1, dst + (((4u + (uint32_t)i) ^ rx) << 4));
+                            }
+                            ptx::fence_proxy_async_smem();  // generic writes -> tensor-core reads
+                        } else if (nr > 0) {
                             const uint32_t raw = raw_sa + (uint32_t)(rs * 2 + mat) * kRawBytes;
                             const uint32_t dst = a_sa + (uint32_t)as * 2u * kATileBytes + a_row;
                             uint4 x[4];
@@ -490,15 +546,18 @@ grouped_gemm_kernel(const GemmParams p) {
 #pragma unroll
                             for (int i = 0; i < 4; ++i) x[i] = make_uint4(0x80808080u, 0x80808080u, 0x80808080u, 0x80808080u);
                             if (r < nr) {
-                                // half h, 16-byte chunk c at raw + h*nr*32 + r*32 + c*16; lanes alternate
-                                // the chunk order so that the 16-byte loads are conflict-free
-                                const uint32_t q = raw + (uint32_t)r * 32u;
-                                const uint32_t h1 = (uint32_t)nr * 32u;
+                                // this warp's rows are sub-block di & 3 (nsr rows); half h, 16-byte chunk
+                                // c at sub + h*nsr*32 + lane*32 + c*16; lanes alternate the chunk order so
+                                // that the 16-byte loads are conflict-free
+                                const int nsr = sub_rows(nr, di & 3);
+                                const uint32_t sub = raw + (uint32_t)(di & 3) * (uint32_t)L.sub_bytes();
+                                const uint32_t q = sub + (uint32_t)lane * 32u;
+                                const uint32_t h1 = (uint32_t)nsr * 32u;
                                 x[0] = ptx::lds128(q + first * 16);
                                 x[1] = ptx::lds128(q + (first ^ 1) * 16);
                                 x[2] = ptx::lds128(q + h1 + first * 16);
                                 x[3] = ptx::lds128(q + h1 + (first ^ 1) * 16);
-                                sc = ptx::lds32(raw + (uint32_t)nr * kTileK + (uint32_t)r * 4u);
+                                sc = ptx::lds32(sub + (uint32_t)nsr * kTileK + (uint32_t)lane * 4u);
                             }
                             uint32_t d0, d1;
                             asm("prmt.b32 %0, %1, %1, 0x1010;" : "=r"(d0) : "r"(sc));
@@ -633,6 +692,18 @@ __device__ __forceinline__ void load8(const void* x, int x_type, int64_t row, in
 // power of two 2^-e that puts its largest magnitude in [2^14, 2^15) - exact,
 // and inside the fp16 range whatever the input type - and xs[row] = 2^e is what
 // the GEMM epilogue multiplies that token's results by.
+// OUT_BF16: write the rows as bf16 without scaling (xs = 1), the operand type
+// of the MXFP4 GEMM.
+__device__ __forceinline__ uint32_t pack_out(float a, float b, float sc, int out_bf16) {
+    if (out_bf16) {
+        const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+        return *(const uint32_t*)&v;
+    }
+    const __half2 v = __floats2half2_rn(a * sc, b * sc);
+    return *(const uint32_t*)&v;
+}
+
+template <int OUT_BF16>
 __global__ void __launch_bounds__(256)
 gather_tiled_kernel(const void* __restrict__ x, int x_type, int n_in, int KT, const int32_t* __restrict__ src_rows,
                     const int32_t* __restrict__ bounds, const int32_t* __restrict__ pad_start, int n_groups,
@@ -654,14 +725,16 @@ gather_tiled_kernel(const void* __restrict__ x, int x_type, int n_in, int KT, co
             srow = src_rows ? __ldg(src_rows + p) : p;
         }
         float mx = 0.f;
-        for (int seg = lane; seg < KT * 8; seg += 32) {
-            float e[8];
-            load8(x, x_type, srow, n_in, (seg >> 3) * 64 + (seg & 7) * 8, e);
+        if (!OUT_BF16) {
+            for (int seg = lane; seg < KT * 8; seg += 32) {
+                float e[8];
+                load8(x, x_type, srow, n_in, (seg >> 3) * 64 + (seg & 7) * 8, e);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(e[i]));
+                for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(e[i]));
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
         int ex = 0;
         if (mx > 0.f && mx <= 3.402823466e38f) {
             ex = ilogbf(mx) - 14;
@@ -675,10 +748,7 @@ gather_tiled_kernel(const void* __restrict__ x, int x_type, int n_in, int KT, co
             load8(x, x_type, srow, n_in, kt * 64 + c * 8, e);
             uint32_t h[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const __half2 v2 = __floats2half2_rn(e[2 * i] * sc, e[2 * i + 1] * sc);
-                h[i] = *(const uint32_t*)&v2;
-            }
+            for (int i = 0; i < 4; ++i) h[i] = pack_out(e[2 * i], e[2 * i + 1], sc, OUT_BF16);
             *(uint4*)(xt + ((size_t)kt * rows_pad + prow) * 128u + ((c ^ (int)(prow & 7)) << 4)) =
                 make_uint4(h[0], h[1], h[2], h[3]);
         }
@@ -687,6 +757,7 @@ gather_tiled_kernel(const void* __restrict__ x, int x_type, int n_in, int KT, co
 
 // Broadcast gather, one warp per token: the token's row is read (and its scale
 // found) once and written to the tiled rows of all k of its slots.
+template <int OUT_BF16>
 __global__ void __launch_bounds__(256)
 gather_tokens_kernel(const void* __restrict__ x, int x_type, int n_in, int KT, const int32_t* __restrict__ slot_prow,
                      int k, int64_t n_tokens, int64_t rows_pad, uint8_t* __restrict__ xt, float* __restrict__ xs,
@@ -697,15 +768,17 @@ gather_tokens_kernel(const void* __restrict__ x, int x_type, int n_in, int KT, c
     for (int64_t t = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); t < n_tokens; t += nw) {
         const int32_t* pr = slot_prow + t * k;
         float mx = 0.f;
+        if (!OUT_BF16) {
 #pragma unroll 4
-        for (int seg = lane; seg < KT * 8; seg += 32) {
-            float e[8];
-            load8(x, x_type, t, n_in, (seg >> 3) * 64 + (seg & 7) * 8, e);
+            for (int seg = lane; seg < KT * 8; seg += 32) {
+                float e[8];
+                load8(x, x_type, t, n_in, (seg >> 3) * 64 + (seg & 7) * 8, e);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(e[i]));
+                for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(e[i]));
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
         int ex = 0;
         if (mx > 0.f && mx <= 3.402823466e38f) {
             ex = ilogbf(mx) - 14;
@@ -720,10 +793,7 @@ gather_tokens_kernel(const void* __restrict__ x, int x_type, int n_in, int KT, c
             load8(x, x_type, t, n_in, kt * 64 + c * 8, e);
             uint32_t h[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const __half2 v2 = __floats2half2_rn(e[2 * i] * sc, e[2 * i + 1] * sc);
-                h[i] = *(const uint32_t*)&v2;
-            }
+            for (int i = 0; i < 4; ++i) h[i] = pack_out(e[2 * i], e[2 * i + 1], sc, OUT_BF16);
             const uint4 v = make_uint4(h[0], h[1], h[2], h[3]);
             uint8_t* plane = xt + (size_t)kt * rows_pad * 128u;
             for (int j = 0; j < k; ++j) {
@@ -746,67 +816,79 @@ static int sm_count() {
     return n > 0 ? n : 148;
 }
 
-template <int DUAL>
-static moe_status run_gemm(const GemmParams& p, int64_t max_coltiles, cudaStream_t stream) {
+template <int DUAL, int BF16, int WT>
+static moe_status launch_grouped(const GemmParams& p, int grid, cudaStream_t stream) {
     static int attr_dev = -1;
     int dev = 0;
     cudaGetDevice(&dev);
     if (attr_dev != dev) {
-        if (cudaFuncSetAttribute(grouped_gemm_kernel<DUAL, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)Cfg::smem_bytes) != cudaSuccess ||
-            cudaFuncSetAttribute(grouped_gemm_kernel<DUAL, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(grouped_gemm_kernel<DUAL, BF16, WT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)Cfg::smem_bytes) != cudaSuccess)
             return MOE_ERR_CUDA;
         attr_dev = dev;
     }
+    grouped_gemm_kernel<DUAL, BF16, WT><<<grid, kGemmThreads, Cfg::smem_bytes, stream>>>(p);
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+template <int DUAL>
+static moe_status run_gemm(const GemmParams& p, int64_t max_coltiles, cudaStream_t stream) {
     const int64_t units = DUAL ? p.L.mt_count : (p.L.mt_count + 1) / 2;
     int64_t tiles = max_coltiles * units;
     if (tiles <= 0) return MOE_OK;
-    int grid = (int)(tiles < sm_count() ? tiles : sm_count());
-    if (p.bf16)
-        grouped_gemm_kernel<DUAL, 1><<<grid, kGemmThreads, Cfg::smem_bytes, stream>>>(p);
-    else
-        grouped_gemm_kernel<DUAL, 0><<<grid, kGemmThreads, Cfg::smem_bytes, stream>>>(p);
-    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
+    if (p.wtype == MOE_MXFP4) return launch_grouped<DUAL, 1, MOE_MXFP4>(p, grid, stream);  // bf16 operands
+    if (p.bf16) return launch_grouped<DUAL, 1, MOE_Q8_0>(p, grid, stream);
+    return launch_grouped<DUAL, 0, MOE_Q8_0>(p, grid, stream);
 }
 
 static int64_t coltile_bound(int64_t S, int E) { return (S + kGemmBN - 1) / kGemmBN + (S < E ? S : E); }
 
 // Broadcast mode (every slot of a token reads the token's row): per token.
 static moe_status gather_tokens(const void* x, int x_type, int n_in, const int32_t* slot_prow, int k, int64_t n_tokens,
-                                int64_t rows_pad, void* xt, float* xs, int* hdr, cudaStream_t s) {
+                                int64_t rows_pad, void* xt, float* xs, int* hdr, int out_bf16, cudaStream_t s) {
     const int KT = (n_in + kTileK - 1) / kTileK;
     int64_t blocks = (n_tokens + 7) / 8;
     if (blocks > (int64_t)sm_count() * 8) blocks = (int64_t)sm_count() * 8;
     if (blocks < 1) blocks = 1;
-    gather_tokens_kernel<<<(unsigned)blocks, 256, 0, s>>>(x, x_type, n_in, KT, slot_prow, k, n_tokens, rows_pad,
-                                                          (uint8_t*)xt, xs, hdr);
+    if (out_bf16)
+        gather_tokens_kernel<1><<<(unsigned)blocks, 256, 0, s>>>(x, x_type, n_in, KT, slot_prow, k, n_tokens, rows_pad,
+                                                                 (uint8_t*)xt, xs, hdr);
+    else
+        gather_tokens_kernel<0><<<(unsigned)blocks, 256, 0, s>>>(x, x_type, n_in, KT, slot_prow, k, n_tokens, rows_pad,
+                                                                 (uint8_t*)xt, xs, hdr);
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 static moe_status gather(const void* x, int x_type, int n_in, const int32_t* src_rows, const int32_t* bounds,
                          const int32_t* pad_start, int n_groups, int64_t rows, int64_t rows_pad, void* xt, float* xs,
-                         int* hdr, cudaStream_t s) {
+                         int* hdr, int out_bf16, cudaStream_t s) {
     const int KT = (n_in + kTileK - 1) / kTileK;
     int64_t blocks = (rows + 7) / 8;
     if (blocks > (int64_t)sm_count() * 8) blocks = (int64_t)sm_count() * 8;
     if (blocks < 1) blocks = 1;
-    gather_tiled_kernel<<<(unsigned)blocks, 256, 0, s>>>(x, x_type, n_in, KT, src_rows, bounds, pad_start, n_groups,
-                                                         rows, rows_pad, (uint8_t*)xt, xs, hdr);
+    if (out_bf16)
+        gather_tiled_kernel<1><<<(unsigned)blocks, 256, 0, s>>>(x, x_type, n_in, KT, src_rows, bounds, pad_start,
+                                                                n_groups, rows, rows_pad, (uint8_t*)xt, xs, hdr);
+    else
+        gather_tiled_kernel<0><<<(unsigned)blocks, 256, 0, s>>>(x, x_type, n_in, KT, src_rows, bounds, pad_start,
+                                                                n_groups, rows, rows_pad, (uint8_t*)xt, xs, hdr);
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 moe_status launch_gemm_mul_mat_id(const GemmMulMatId& g, cudaStream_t stream) {
+    const int mx = g.wtype == MOE_MXFP4;  // bf16 operands, unscaled activation rows
     moe_status st = g.x_rows * g.k == g.S
                         ? gather_tokens(g.x, g.x_type, g.n_in, g.slot_prow, g.k, g.x_rows, g.rows_pad, g.xt, g.xs,
-                                        g.hdr, stream)
+                                        g.hdr, mx, stream)
                         : gather(g.x, g.x_type, g.n_in, g.ids_src1, g.bounds, g.pad_start, g.E, g.S, g.rows_pad, g.xt,
-                                 g.xs, g.hdr, stream);
+                                 g.xs, g.hdr, mx, stream);
     if (st) return st;
     prof_mark(stream, "gather");
     GemmParams p = {};
     p.A0 = g.W;
-    p.L = WLayout(g.n_out, g.n_in);
+    p.L = WLayout(g.n_out, g.n_in, g.wtype);
+    p.wtype = g.wtype;
     p.n_groups = g.E;
     p.bounds = g.bounds;
     p.ntile_prefix = g.ntile_prefix;
@@ -817,17 +899,18 @@ moe_status launch_gemm_mul_mat_id(const GemmMulMatId& g, cudaStream_t stream) {
     p.out = g.dst;
     p.out_ld = g.n_out;
     p.hdr = g.hdr;
-    p.bf16 = 0;  // fp16 activation tiles (scaled rows)
-    p.col_scale = g.xs;
+    p.bf16 = mx;  // Q8_0: fp16 activation tiles (scaled rows); MXFP4: bf16
+    p.col_scale = mx ? nullptr : g.xs;
     st = run_gemm<0>(p, coltile_bound(g.S, g.E), stream);
     prof_mark(stream, "gemm");
     return st;
 }
 
 moe_status launch_gemm_ffn(const GemmFfn& g, cudaStream_t stream) {
+    const int mx = g.wtype == MOE_MXFP4;  // bf16 operands, unscaled activation rows
     const int kt_ff = (g.n_ff + kTileK - 1) / kTileK;
     moe_status st =
-        gather_tokens(g.x, g.x_type, g.n_embd, g.slot_prow, g.k, g.T, g.rows_pad, g.xt, g.xs, g.hdr, stream);
+        gather_tokens(g.x, g.x_type, g.n_embd, g.slot_prow, g.k, g.T, g.rows_pad, g.xt, g.xs, g.hdr, mx, stream);
     if (st) return st;
     prof_mark(stream, "gather");
     if (g.n_ff % kTileK) {  // columns past n_ff of the last k-plane of h are read by the down GEMM: keep them 0
@@ -839,7 +922,8 @@ moe_status launch_gemm_ffn(const GemmFfn& g, cudaStream_t stream) {
     GemmParams p = {};
     p.A0 = g.Wg;
     p.A1 = g.Wu;
-    p.L = WLayout(g.n_ff, g.n_embd);
+    p.L = WLayout(g.n_ff, g.n_embd, g.wtype);
+    p.wtype = g.wtype;
     p.n_groups = g.E;
     p.bounds = g.bounds;
     p.ntile_prefix = g.ntile_prefix;
@@ -850,15 +934,15 @@ moe_status launch_gemm_ffn(const GemmFfn& g, cudaStream_t stream) {
     p.h_rows = g.rows_pad;
     p.out_ld = g.n_ff;
     p.hdr = g.hdr;
-    p.bf16 = 0;  // fp16 activation tiles (scaled rows)
-    p.col_scale = g.xs;
+    p.bf16 = mx;  // Q8_0: fp16 activation tiles (scaled rows); MXFP4: bf16
+    p.col_scale = mx ? nullptr : g.xs;
     st = run_gemm<1>(p, coltile_bound(g.S, g.E), stream);
     if (st) return st;
     prof_mark(stream, "gemm_gate_up");
     const int kt_sh = (g.n_ff_shared + kTileK - 1) / kTileK;
     if (g.n_ff_shared > 0) {
         st = gather(g.x, g.x_type, g.n_embd, nullptr, nullptr, nullptr, 0, g.T, g.rows_pad_sh, g.xt_sh, g.xs_sh,
-                    g.hdr, stream);
+                    g.hdr, mx, stream);
         if (st) return st;
         if (g.n_ff_shared % kTileK) {
             if (cudaMemsetAsync((uint8_t*)g.h_sh + (size_t)(kt_sh - 1) * g.rows_pad_sh * 128u, 0,
@@ -868,7 +952,8 @@ moe_status launch_gemm_ffn(const GemmFfn& g, cudaStream_t stream) {
         GemmParams q = {};
         q.A0 = g.Sg;
         q.A1 = g.Su;
-        q.L = WLayout(g.n_ff_shared, g.n_embd);
+        q.L = WLayout(g.n_ff_shared, g.n_embd, g.wtype);
+        q.wtype = g.wtype;
         q.n_rows = (int)g.T;
         q.B = (const uint8_t*)g.xt_sh;
         q.b_rows = g.rows_pad_sh;
@@ -876,8 +961,8 @@ moe_status launch_gemm_ffn(const GemmFfn& g, cudaStream_t stream) {
         q.h_rows = g.rows_pad_sh;
         q.out_ld = g.n_ff_shared;
         q.hdr = g.hdr;
-        q.bf16 = 0;
-        q.col_scale = g.xs_sh;
+        q.bf16 = mx;
+        q.col_scale = mx ? nullptr : g.xs_sh;
         st = run_gemm<1>(q, (g.T + kGemmBN - 1) / kGemmBN, stream);
         if (st) return st;
         prof_mark(stream, "gemm_shared_gate_up");
@@ -885,7 +970,8 @@ moe_status launch_gemm_ffn(const GemmFfn& g, cudaStream_t stream) {
     // down: B = h, contiguous per expert; the epilogue scatters rows to dst by ids_dst
     GemmParams d = {};
     d.A0 = g.Wd;
-    d.L = WLayout(g.n_embd, g.n_ff);
+    d.L = WLayout(g.n_embd, g.n_ff, g.wtype);
+    d.wtype = g.wtype;
     d.n_groups = g.E;
     d.bounds = g.bounds;
     d.ntile_prefix = g.ntile_prefix;
@@ -903,7 +989,8 @@ moe_status launch_gemm_ffn(const GemmFfn& g, cudaStream_t stream) {
     if (g.n_ff_shared > 0) {
         GemmParams q = {};
         q.A0 = g.Sd;
-        q.L = WLayout(g.n_embd, g.n_ff_shared);
+        q.L = WLayout(g.n_embd, g.n_ff_shared, g.wtype);
+        q.wtype = g.wtype;
         q.n_rows = (int)g.T;
         q.B = (const uint8_t*)g.h_sh;
         q.b_rows = g.rows_pad_sh;

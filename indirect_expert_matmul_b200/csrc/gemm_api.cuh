@@ -5,6 +5,7 @@
 namespace moe {
 
 struct GemmMulMatId {
+    int wtype;        // MOE_Q8_0 / MOE_MXFP4
     const uint8_t* W;
     int E, n_out, n_in;
     const void* x;
@@ -26,6 +27,7 @@ struct GemmMulMatId {
 };
 
 struct GemmFfn {
+    int wtype;        // MOE_Q8_0 / MOE_MXFP4
     const uint8_t *Wg, *Wu, *Wd;
     int E, n_embd, n_ff;
     const uint8_t *Sg, *Su, *Sd;

@@ -3,98 +3,96 @@
 // llama.cpp PR #29184 ("CUDA: fuse shared experts into MMVQ", release b11370)
 // restated for this library.
 //
-// Decode is bound by the weight stream, so the kernel is built around moving
-// the repacked weights in large contiguous pieces:
-//  - a work item is (distinct routed expert, 128-row tile, K-chunk) or
-//    (shared expert, 128-row tile, K-chunk); every k-step block of one
-//    (expert, row tile) is contiguous in the repacked layout, so a stage of
-//    up to two (dual) or four (single) k-steps of one matrix is a single bulk
-//    copy of up to 34 KB;
-//  - one producer warp streams the stages of the CTA's items through a ring
-//    of shared-memory stages, ahead of the consumers and across items;
-//  - 512 consumer threads dequantise (exact fp32 q*d) and take the dot
-//    products with up to 8 tokens at a time: thread = (row, 16 columns);
-//  - when there are fewer (expert, row tile) groups than SMs (a single decode
-//    token), K is split into chunks; each chunk writes fp32 partial sums and
-//    the CTA that finishes a group last adds the chunks in chunk order and
-//    applies the epilogue.  Every sum has a fixed order, so results do not
-//    depend on timing.
-// A CTA finds the distinct experts and their slots from ids itself (bitmap +
-// a per-CTA slot table), so the decode path needs no row-id launch.
+// Decode is bound by the weight stream.  The kernel is built so that the two
+// launches of an expert FFN (gate/up, then down) stream their weights at the
+// same time:
+//  - each launch takes at most ~110 KB of shared memory and 288 threads of 112
+//    registers, so a CTA of the down launch fits on an SM beside a CTA of the
+//    gate/up launch; the down launch is a programmatic dependent of gate/up,
+//    its producer streams the down weights from the start and only its
+//    consumers wait for gate/up's h;
+//  - a work item is (routed expert, row sub-tile of 32, 64 or 128 rows) or
+//    (shared expert, row sub-tile), always over the whole K, so no item needs
+//    another's partial sums; the sub-tile height is chosen per launch so that
+//    the items cover the SMs;
+//  - one producer warp streams 17 KB stages (the sub-tile's rows for several
+//    k-steps of each matrix: one bulk copy per k-step and matrix, the rows of
+//    a sub-tile being contiguous in the repacked layout) through a ring,
+//    running ahead across items;
+//  - 256 consumer threads, thread = (row of the sub-tile, 32-column slice of a
+//    k-step): exact fp32 dequantisation (q*d) and fp32 dot products with up
+//    to 8 tokens at a time; the slices of a row are added in slice order.
+//    Every sum has a fixed order, so results do not depend on timing.
+// The distinct routed experts come from ids directly: for up to 64 slots every
+// warp finds them with ballots in its own registers (no block-wide pass before
+// the first copy); for more slots a block-wide pass builds tables in shared
+// memory.
 //
 // Modes: single matrix (mul_mat_id rows, or the down projection writing
 // dst[t][s]), or dual gate/up with a SwiGLU epilogue writing bf16 h[t][s].
-// The down launch is a programmatic dependent of the gate/up launch: its
-// producer streams weights while gate/up finishes; its consumers wait for
-// gate/up before reading h.
+#include <atomic>
+
 #include "common.cuh"
 #include "gemv_args.cuh"
+#include "moe_testing.h"
 #include "ptx.cuh"
 
 namespace moe {
 
-constexpr int kGvConsumers = 512;
+constexpr int kGvConsumers = 256;
 constexpr int kGvThreads = 32 + kGvConsumers;  // warp 0: producer
-constexpr uint32_t kGvBlock = kTileM * kRowBytes;  // 8704: one k-step of a full row tile
-constexpr uint32_t kGvSmemBudget = 200 * 1024;
-constexpr long long kGvWaitLimit = 1ll << 32;
+constexpr uint32_t kGvStage = 256 * kRowBytes;  // 17408 bytes: 256 (row, k-step) pieces of Q8_0
+constexpr uint32_t kGvSmemBudget = 110 * 1024;
+constexpr long long kGvWaitLimit = 1ll << 32;   // ~2 s
+constexpr int kGvFast = 64;                     // slots up to which the experts come from warp ballots
+constexpr uint32_t kGvXBytes = 16 * 1024;       // activation window (fp32)
+constexpr uint32_t kGvRedBytes = kGvConsumers * kGvNT * 2 * 4;
 
 struct GvLay {
-    uint32_t ring, x, red, bm, wp, tab, bars, misc, total;
+    uint32_t ring, x, red, tab, bars, misc, total;
 };
 
-__host__ __device__ inline GvLay gv_lay(const GemvArgs& a) {
+// Shared memory: ring | activation window | reduction | tables (slow path) | barriers | misc.
+__host__ __device__ inline GvLay gv_lay(int ns, int S, int n_experts) {
     GvLay m;
     uint32_t o = 0;
-    m.ring = o; o += (uint32_t)a.ns * a.stage_bytes;
-    m.x = o; o += a.x_bytes;
-    m.red = o; o += a.red_bytes;
-    m.bm = o; o += a.bm_words * 4u;
-    m.wp = o; o += (a.bm_words + 1u) * 4u;
-    m.tab = o; o += a.tab_words * 4u;
+    m.ring = o; o += (uint32_t)ns * kGvStage;
+    m.x = o; o += kGvXBytes;
+    m.red = o; o += kGvRedBytes;
+    m.tab = o;
+    if (S > kGvFast) o += (uint32_t)(((n_experts + 31) / 32) * 2 + 2 + 2 * (S + 1) + 2 * S) * 4u;
     o = (o + 15u) & ~15u;
-    m.bars = o; o += 2u * (uint32_t)a.ns * 8u;
-    m.misc = o; o += 16u * 4u;
+    m.bars = o; o += 2u * (uint32_t)ns * 8u;
+    m.misc = o; o += 16u;
     m.total = o;
     return m;
 }
 
-// Packed fp32 pairs (two lanes of one 64-bit register): fma.rn.f32x2 does two
-// independent round-to-nearest fp32 fmas, the same as two fmaf calls.
-__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-    return r;
-}
-__device__ __forceinline__ float f2sum(uint64_t v) {
-    float lo, hi;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-    return lo + hi;
-}
-__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
-    uint64_t r;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-    return r;
-}
-
-__device__ __forceinline__ float ld_x16(uint32_t bits16, int x_type) {
-    return x_type == MOE_BF16 ? __uint_as_float(bits16 << 16) : __half2float(__ushort_as_half((unsigned short)bits16));
-}
-
-// Bounded wait by one thread: false on expiry (status set, abort raised) or
-// when another thread has raised abort.
-__device__ __forceinline__ bool gv_wait(uint64_t* bar, uint32_t parity, int* status, volatile int* abort_flag) {
+// Bounded wait by one thread: false on expiry (status set, the wait's site
+// recorded, abort raised) or when another thread raised abort.
+__device__ __forceinline__ bool gv_wait(uint64_t* bar, uint32_t parity, int* status, volatile int* abort_flag,
+                                        long long limit) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (!ptx::mbar_try_wait_sleep(bar, parity, 20000)) {
         if (*abort_flag) return false;
-        if (clock64() - t0 > kGvWaitLimit) {
+        if (clock64() - t0 > limit) {
             *abort_flag = 1;
+            const int site = (1 << 30) | ((int)(threadIdx.x >> 5) << 20) | (int)(ptx::smem_u32(bar) & 0xfffffu);
+            atomicCAS(status + (kHdrWaitSite - kHdrStatus), 0, site);
             set_status(status, MOE_ERR_TIMEOUT);
             return false;
         }
     }
     return true;
+}
+
+// gv_wait by lane 0; every lane of the warp gets its outcome.
+__device__ __forceinline__ bool gv_warp_wait(uint64_t* bar, uint32_t parity, int* status, volatile int* abort_flag,
+                                             long long limit) {
+    int ok = 1;
+    if ((threadIdx.x & 31) == 0) ok = gv_wait(bar, parity, status, abort_flag, limit);
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
 // Named barrier 1 over the consumer warps; consumers_and also returns the AND
@@ -113,47 +111,230 @@ __device__ __forceinline__ bool consumers_and(bool v) {
     return r != 0;
 }
 
-// One work item.
-struct GvItem {
-    const GemvSide* sd;
-    int shared;   // 1: shared expert
-    int e;        // expert of the weights
-    int mt;       // 128-row tile
-    int c;        // K-chunk
-    int kt0, nk;  // first k-step and k-steps of the chunk
-    int rows;     // rows of the tile
-    int nsl;      // slots (routed) or tokens (shared)
-    int sbase;    // first entry of the expert's slots in the slot list
-    int group;    // split-K counter index
+__device__ __forceinline__ float f2sum(uint64_t v) {
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+    return lo + hi;
+}
+
+__device__ __forceinline__ float ld_x16(uint32_t bits16, int x_type) {
+    return x_type == MOE_BF16 ? __uint_as_float(bits16 << 16) : __half2float(__ushort_as_half((unsigned short)bits16));
+}
+
+// E8M0 scale byte -> 2^(x - 127) as a float (x = 0: 2^-127, a float subnormal;
+// x = 255: NaN).
+__device__ __forceinline__ float e8m0_float(uint32_t x) {
+    return x == 0u ? __uint_as_float(0x00400000u) : x == 255u ? __uint_as_float(0x7fc00000u) : __uint_as_float(x << 23);
+}
+
+// Eight E2M1 codes (a 32-bit word, code i in bits 4i..4i+3) -> their exact
+// values as floats, by the sm_100a pair conversion to f16 (exact: two
+// significant bits), then f16 -> float.
+__device__ __forceinline__ void e2m1x8_to_float(uint32_t w, float (&v)[8]) {
+    uint32_t h[4];
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+        : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+        : "r"(w));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __half2 p = *(const __half2*)&h[i];
+        v[2 * i] = __low2float(p);
+        v[2 * i + 1] = __high2float(p);
+    }
+}
+
+// n-th (0-based) set bit of a 64-bit mask given as two words.
+__device__ __forceinline__ int nth_bit(uint32_t m0, uint32_t m1, int n) {
+    const int c0 = __popc(m0);
+    return n < c0 ? (int)__fns(m0, 0, n + 1) : 32 + (int)__fns(m1, 0, n - c0 + 1);
+}
+
+// The distinct routed experts of this call, as one warp sees them.
+//  fast (slots <= 64): v0/v1 = ids of slots lane and lane + 32 (-1 past the
+//  end or out of range); fb0/fb1 = ballots of the slots that are the first
+//  occurrence of their expert; distinct expert j = the expert of the j-th
+//  first occurrence (slot order).
+//  slow: tables in shared memory, distinct experts in ascending id order.
+struct Routing {
+    int v0, v1;
+    uint32_t fb0, fb1;
+    int n;
+    const int* list_e;  // slow: [n] expert ids
+    const int* off;     // slow: [n + 1] slot list offsets
+    const int* slots;   // slow: slot list
+    bool fast;
+
+    // warp-collective in fast mode
+    __device__ __forceinline__ int expert(int j) const {
+        if (!fast) return list_e[j];
+        const int s = nth_bit(fb0, fb1, j);
+        const int a = __shfl_sync(0xffffffffu, v0, s & 31), b = __shfl_sync(0xffffffffu, v1, s & 31);
+        return s < 32 ? a : b;
+    }
 };
 
-template <int DUAL, int XB>
-__global__ void __launch_bounds__(kGvThreads, 1)
+// Warp-level distinct-expert scan for up to 64 slots (every lane of the warp).
+__device__ __forceinline__ void routing_fast(Routing& R, const int32_t* ids, int S, int E, int* status) {
+    const int lane = threadIdx.x & 31;
+    const uint32_t lt = (1u << lane) - 1u;
+    int v0 = lane < S ? __ldg(ids + lane) : -1;
+    int v1 = lane + 32 < S ? __ldg(ids + lane + 32) : -1;
+    const bool bad = (lane < S && (v0 < 0 || v0 >= E)) || (lane + 32 < S && (v1 < 0 || v1 >= E));
+    if (__any_sync(0xffffffffu, bad) && lane == 0) set_status(status, MOE_ERR_BAD_ID);
+    if (v0 >= E) v0 = -1;
+    if (v1 >= E) v1 = -1;
+    if (v0 < 0) v0 = -1;
+    if (v1 < 0) v1 = -1;
+    const uint32_t m0 = __match_any_sync(0xffffffffu, v0), m1 = __match_any_sync(0xffffffffu, v1);
+    bool f0 = v0 >= 0 && (m0 & lt) == 0u;
+    bool f1 = v1 >= 0 && (m1 & lt) == 0u;
+    for (int i = 0; i < 32; ++i) {  // an expert of the second half seen in the first is not new
+        const int o = __shfl_sync(0xffffffffu, v0, i);
+        if (o == v1) f1 = false;
+    }
+    R.v0 = v0;
+    R.v1 = v1;
+    R.fb0 = __ballot_sync(0xffffffffu, f0);
+    R.fb1 = __ballot_sync(0xffffffffu, f1);
+    R.n = __popc(R.fb0) + __popc(R.fb1);
+    R.fast = true;
+}
+
+// Block-wide scan for more than 64 slots (every thread of the CTA): bitmap
+// of the experts, per-word prefix, then a stable slot list per expert.
+__device__ void routing_slow(Routing& R, const int32_t* ids, int S, int E, int* tab, int* status) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int nw = (E + 31) / 32;
+    uint32_t* bm = (uint32_t*)tab;        // [nw]
+    int* wp = tab + nw;                   // [nw + 1]: distinct experts before word w
+    int* nd = wp + nw + 1;                // [1]
+    int* cnt = nd + 1;                    // [S + 1]
+    int* off = cnt + S + 1;               // [S + 1]
+    int* list = off + S + 1;              // [S]: slots grouped by distinct expert
+    int* rank_sh = list + S;              // [S]: distinct index of each slot
+    for (int w = tid; w < nw; w += blockDim.x) bm[w] = 0u;
+    __syncthreads();
+    for (int i = tid; i < S; i += blockDim.x) {
+        const int v = __ldg(ids + i);
+        if (v >= 0 && v < E) atomicOr(&bm[v >> 5], 1u << (v & 31));
+        else set_status(status, MOE_ERR_BAD_ID);
+    }
+    __syncthreads();
+    if (warp == 0) {  // exclusive prefix of popcounts over the words
+        int run = 0;
+        for (int w0 = 0; w0 < nw; w0 += 32) {
+            const int w = w0 + lane;
+            const int c = w < nw ? __popc(bm[w]) : 0;
+            int incl = c;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int nn = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += nn;
+            }
+            if (w < nw) wp[w] = run + incl - c;
+            run += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) { wp[nw] = run; *nd = run; }
+    }
+    __syncthreads();
+    const int n = *nd;
+    for (int j = tid; j <= n; j += blockDim.x) cnt[j] = 0;
+    __syncthreads();
+    for (int i = tid; i < S; i += blockDim.x) {
+        const int v = __ldg(ids + i);
+        int r = -1;
+        if (v >= 0 && v < E) {
+            r = wp[v >> 5] + __popc(bm[v >> 5] & ((1u << (v & 31)) - 1u));
+            atomicAdd(&cnt[r], 1);
+        }
+        rank_sh[i] = r;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        int run = 0;
+        for (int j0 = 0; j0 < n; j0 += 32) {
+            const int j = j0 + lane;
+            const int c = j < n ? cnt[j] : 0;
+            int incl = c;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int nn = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += nn;
+            }
+            if (j < n) off[j] = run + incl - c;
+            run += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) off[n] = run;
+    }
+    __syncthreads();
+    // stable placement (ascending slot inside an expert), one warp per 32 slots in order
+    if (warp == 0) {
+        for (int base = 0; base < S; base += 32) {
+            const int i = base + lane;
+            const int r = i < S ? rank_sh[i] : -1;
+            const uint32_t m = __match_any_sync(0xffffffffu, r);
+            if (r >= 0) list[off[r] + __popc(m & ((1u << lane) - 1u))] = i;
+            __syncwarp();
+            if (r >= 0 && (m & ((1u << lane) - 1u)) == 0u) off[r] += __popc(m);
+            __syncwarp();
+        }
+        __syncwarp();
+        // restore the offsets (each was advanced by its count)
+        for (int j = lane; j < n; j += 32) off[j] -= cnt[j];
+    }
+    // the expert id of distinct index j: the j-th set bit of the bitmap
+    int* list_e = rank_sh;  // reuse: slot ranks are no longer needed after placement
+    __syncthreads();
+    for (int w = tid; w < nw; w += blockDim.x) {
+        uint32_t bits = bm[w];
+        int j = wp[w];
+        while (bits) {
+            const int b = __ffs(bits) - 1;
+            list_e[j++] = w * 32 + b;
+            bits &= bits - 1;
+        }
+    }
+    __syncthreads();
+    R.n = n;
+    R.list_e = list_e;
+    R.off = off;
+    R.slots = list;
+    R.fast = false;
+}
+
+// One work item.
+struct GvItem {
+    int side;    // 0 routed, 1 shared
+    int e;       // expert of the weights
+    int mt, r0;  // 128-row tile and first row of the sub-tile inside it
+    int nrow;    // rows of the sub-tile (<= rsub); 0 = empty item (tail of the last tile)
+    int nsl;     // slots (routed) or tokens (shared)
+};
+
+// At most 112 registers a thread: two CTAs of 288 threads (one of each launch
+// of an FFN) fit in the SM's 64 K registers.
+template <int DUAL, int XB, int WT>
+__global__ void __maxnreg__(112)
 gemv_kernel(const GemvArgs a) {
     extern __shared__ __align__(128) uint8_t sm[];
     constexpr int NMAT = DUAL + 1;
     int* status = a.hdr + kHdrStatus;
-    if (!a.pdl_secondary) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    if (read_status(status) != 0) return;
-
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const GvLay lay = gv_lay(a);
+    const int S = a.n_tokens * a.k;
+    const GvLay lay = gv_lay(a.ns, S, a.n_experts);
     uint8_t* ring = sm + lay.ring;
-    uint8_t* sx = sm + lay.x;
+    float* sx = (float*)(sm + lay.x);
     float* red = (float*)(sm + lay.red);
-    uint32_t* bm = (uint32_t*)(sm + lay.bm);
-    int* wp = (int*)(sm + lay.wp);
-    int* tab = (int*)(sm + lay.tab);
     uint64_t* full = (uint64_t*)(sm + lay.bars);
     uint64_t* empty = full + a.ns;
-    int* misc = (int*)(sm + lay.misc);
-    volatile int* abort_flag = misc;   // misc[0]
-    int* last_flag = misc + 1;
-    const int S = a.n_tokens * a.k;
-    const int nwords = (int)a.bm_words;
+    volatile int* abort_flag = (volatile int*)(sm + lay.misc);
+    int* st_copy = (int*)(sm + lay.misc + 4);
 
-    // ---- the distinct routed experts: bitmap + per-word prefix of popcounts
-    for (int w = tid; w < nwords; w += kGvThreads) bm[w] = 0u;
     if (tid == 0) {
         for (int s = 0; s < a.ns; ++s) {
             ptx::mbar_init(&full[s], 1);
@@ -162,189 +343,179 @@ gemv_kernel(const GemvArgs a) {
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
+    // Upstream dependency (this launch may start before the previous kernel of
+    // the stream finished): nothing the previous kernel may write - ids,
+    // activations, weights, the status - is read before this wait.
+    if (a.pdl_wait) asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (a.pdl_trigger) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    // a sticky error stops the launch; one read, shared, so that the exit is
+    // uniform (the other launch of the FFN may write the word meanwhile)
+    if (tid == 0) *st_copy = read_status(status);
     __syncthreads();
-    int* ids_sh = tab + 2 * (a.max_distinct + 1) + S;  // ids, read from global memory once
-    for (int i = tid; i < S; i += kGvThreads) {
-        const int v = __ldg(a.ids + i);
-        ids_sh[i] = v;
-        if (v >= 0 && v < a.n_experts) atomicOr(&bm[v >> 5], 1u << (v & 31));
-        else set_status(status, MOE_ERR_BAD_ID);
-    }
-    __syncthreads();
-    if (warp == 0) {  // exclusive prefix, 32 words per step
-        int run = 0;
-        for (int w0 = 0; w0 < nwords; w0 += 32) {
-            const int w = w0 + lane;
-            const int c = w < nwords ? __popc(bm[w]) : 0;
-            int incl = c;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int n = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += n;
-            }
-            if (w < nwords) wp[w] = run + incl - c;
-            run += __shfl_sync(0xffffffffu, incl, 31);
-        }
-        if (lane == 0) wp[nwords] = run;
-    }
-    __syncthreads();
-    const int n_distinct = wp[nwords];
-    // ---- slot table: the slots of distinct expert j are list[off[j] .. off[j+1])
-    int* cnt = tab;                      // [n_distinct + 1]
-    int* off = tab + (a.max_distinct + 1);
-    int* list = off + (a.max_distinct + 1);
-    auto rank_of = [&](int v) { return wp[v >> 5] + __popc(bm[v >> 5] & ((1u << (v & 31)) - 1u)); };
-    for (int j = tid; j <= n_distinct; j += kGvThreads) cnt[j] = 0;
-    __syncthreads();
-    for (int i = tid; i < S; i += kGvThreads) {
-        const int v = ids_sh[i];
-        if (v >= 0 && v < a.n_experts) atomicAdd(&cnt[rank_of(v)], 1);
-    }
-    __syncthreads();
-    if (warp == 0) {
-        int run = 0;
-        for (int j0 = 0; j0 < n_distinct; j0 += 32) {
-            const int j = j0 + lane;
-            const int c = j < n_distinct ? cnt[j] : 0;
-            int incl = c;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int n = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += n;
-            }
-            if (j < n_distinct) off[j] = run + incl - c;
-            run += __shfl_sync(0xffffffffu, incl, 31);
-        }
-        if (lane == 0) off[n_distinct] = run;
-    }
-    __syncthreads();
-    for (int j = tid; j < n_distinct; j += kGvThreads) cnt[j] = 0;
-    __syncthreads();
-    for (int i = tid; i < S; i += kGvThreads) {  // order inside an expert is free: slots are independent
-        const int v = ids_sh[i];
-        if (v >= 0 && v < a.n_experts) {
-            const int j = rank_of(v);
-            list[off[j] + atomicAdd(&cnt[j], 1)] = i;
-        }
-    }
-    __syncthreads();
+    if (*st_copy != 0) return;
 
-    const GemvSide& R = a.routed;
-    const GemvSide& Sh = a.shared;
-    const int per_e = R.L.mt_count * R.chunks;
-    const int n_items_r = n_distinct * per_e;
-    const int n_items = n_items_r + (a.has_shared ? Sh.L.mt_count * Sh.chunks : 0);
+    Routing R;
+    if (S <= kGvFast) routing_fast(R, a.ids, S, a.n_experts, status);
+    else routing_slow(R, a.ids, S, a.n_experts, (int*)(sm + lay.tab), status);
 
-    auto item_of = [&](int it) {
+    // A field of a side, read from the parameter space where it is used (taking
+    // a kernel parameter's address, or copying a side whole, would cost local
+    // memory or registers).
+#define GV_SIDE(sh, field) ((sh) ? a.shared.field : a.routed.field)
+    const int n_sh = a.has_shared ? a.shared.subs : 0;
+    const int n_items = n_sh + R.n * a.routed.subs;
+    // items: the shared expert's sub-tiles first, then each distinct routed expert's
+    auto item_of = [&](int it) {  // warp-collective in fast mode
         GvItem f;
-        if (it < n_items_r) {
-            const int j = it / per_e, rem = it - j * per_e;
-            f.sd = &R;
-            f.shared = 0;
-            f.mt = rem / R.chunks;
-            f.c = rem - f.mt * R.chunks;
-            int lo = 0, hi = nwords;  // wp[lo] <= j < wp[hi]
-            while (hi - lo > 1) {
-                const int mid = (lo + hi) >> 1;
-                if (wp[mid] <= j) lo = mid; else hi = mid;
-            }
-            uint32_t bits = bm[lo];
-            for (int q = j - wp[lo]; q > 0; --q) bits &= bits - 1;
-            f.e = lo * 32 + __ffs(bits) - 1;
-            f.sbase = off[j];
-            f.nsl = off[j + 1] - off[j];
-            f.group = R.group0 + j * R.L.mt_count + f.mt;
-        } else {
-            const int i2 = it - n_items_r;
-            f.sd = &Sh;
-            f.shared = 1;
-            f.mt = i2 / Sh.chunks;
-            f.c = i2 - f.mt * Sh.chunks;
+        int u;
+        if (it < n_sh) {
+            f.side = 1;
             f.e = 0;
-            f.sbase = 0;
+            u = it;
             f.nsl = a.n_tokens;
-            f.group = Sh.group0 + f.mt;
+        } else {
+            const int j = (it - n_sh) / a.routed.subs;
+            u = (it - n_sh) - j * a.routed.subs;
+            f.side = 0;
+            f.e = R.expert(j);
+            f.nsl = -1;  // counted by the consumers
         }
-        f.kt0 = f.c * f.sd->kc;
-        f.nk = min(f.sd->kc, f.sd->L.kt_count - f.kt0);
-        f.rows = f.sd->L.rows(f.mt);
+        const int rsub = f.side ? a.shared.rsub : a.routed.rsub;
+        const WLayout L = f.side ? a.shared.L : a.routed.L;
+        const int per_tile = kTileM / rsub;
+        f.mt = u / per_tile;
+        f.r0 = (u - f.mt * per_tile) * rsub;
+        const int rows = L.rows(f.mt);
+        f.nrow = rows - f.r0 < rsub ? rows - f.r0 : rsub;
+        if (f.nrow < 0) f.nrow = 0;
         return f;
     };
-    const int sk = a.sk, ns = a.ns;
 
     if (warp == 0) {
         // ------------------------------------------------------- producer
-        if (lane == 0) {
-            uint32_t sc = 0;
-            bool ok = true;
-            for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-                const GvItem f = item_of(it);
-                const GemvSide& sd = *f.sd;
-                const int G = (f.nsl + kGvNT - 1) / kGvNT;
-                for (int g = 0; g < G && ok; ++g)
-                    for (int ks = 0; ks < f.nk; ks += sk, ++sc) {
-                        const int nks = min(sk, f.nk - ks);
-                        const int s = (int)(sc % (uint32_t)ns);
-                        if (!gv_wait(&empty[s], ((sc / ns) & 1u) ^ 1u, status, abort_flag)) { ok = false; break; }
-                        const uint32_t bytes = (uint32_t)nks * f.rows * kRowBytes;
-                        ptx::mbar_arrive_expect_tx(&full[s], NMAT * bytes);
+        // Every lane runs the loop (the item decode is warp-collective); lane 0
+        // issues the copies.  A stage holds kps k-steps of the sub-tile's rows
+        // of each matrix: NMAT * kps copies of nrow * 68 bytes.
+        uint32_t sc = 0;
+        bool ok = true;
+        for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+            const GvItem f = item_of(it);
+            if (f.nrow == 0) continue;
+            int nsl = f.nsl;
+            if (nsl < 0) {  // routed: slots of this expert
+                if (R.fast)
+                    nsl = __popc(__ballot_sync(0xffffffffu, R.v0 == f.e)) + __popc(__ballot_sync(0xffffffffu, R.v1 == f.e));
+                else
+                    nsl = R.off[(it - n_sh) / a.routed.subs + 1] - R.off[(it - n_sh) / a.routed.subs];
+            }
+            const int G = (nsl + kGvNT - 1) / kGvNT;
+            const WLayout L = GV_SIDE(f.side, L);
+            const int KT = L.kt_count, kps = GV_SIDE(f.side, kps);
+            const uint8_t* W0 = GV_SIDE(f.side, W0);
+            const uint8_t* W1 = GV_SIDE(f.side, W1);
+            const uint32_t piece = (uint32_t)f.nrow * L.rb;
+            for (int g = 0; g < G && ok; ++g)
+                for (int k0 = 0; k0 < KT; k0 += kps, ++sc) {
+                    const int s = (int)(sc % (uint32_t)a.ns);
+                    if (!gv_warp_wait(&empty[s], ((sc / a.ns) & 1u) ^ 1u, status, abort_flag, a.wait_limit)) {
+                        ok = false;
+                        break;
+                    }
+                    const int nk = KT - k0 < kps ? KT - k0 : kps;
+                    const bool stall = (int)blockIdx.x == a.stall_cta && (int)sc == a.stall_stage;  // test only
+                    if (lane == 0 && !stall) {
+                        ptx::mbar_arrive_expect_tx(&full[s], (uint32_t)(NMAT * nk) * piece);
 #pragma unroll
                         for (int m = 0; m < NMAT; ++m)
-                            ptx::bulk_g2s(ring + (size_t)s * a.stage_bytes + (size_t)m * sk * kGvBlock,
-                                          (m ? sd.W1 : sd.W0) + sd.L.block(f.e, f.mt, f.kt0 + ks), bytes, &full[s]);
+                            for (int kk = 0; kk < nk; ++kk)
+                                ptx::bulk_g2s(ring + (size_t)s * kGvStage + (size_t)(m * kps + kk) * piece,
+                                              (m ? W1 : W0) + L.block(f.e, f.mt, k0 + kk) +
+                                                  (size_t)f.r0 * L.rb,
+                                              piece, &full[s]);
                     }
-            }
-            // every copy issued lands before the CTA can exit (bounded)
+                    __syncwarp();
+                }
+        }
+        // every copy issued lands before the CTA can exit (bounded; a stage the
+        // test-only stall skipped has no copy to wait for)
+        if (lane == 0) {
             volatile int never = 0;
-            const uint32_t first = sc > (uint32_t)ns ? sc - ns : 0u;
-            for (uint32_t q = first; q < sc; ++q) gv_wait(&full[q % ns], (q / ns) & 1u, status, &never);
+            const uint32_t first = sc > (uint32_t)a.ns ? sc - a.ns : 0u;
+            for (uint32_t q = first; q < sc; ++q)
+                if (!((int)blockIdx.x == a.stall_cta && (int)q == a.stall_stage))
+                    gv_wait(&full[q % a.ns], (q / a.ns) & 1u, status, &never, a.wait_limit);
         }
         return;
     }
 
     // ----------------------------------------------------------- consumers
-    // thread = (32-column half hh, row r, 16-column chunk c16): eight lanes read
-    // four rows' 128 contiguous bytes, so the 16-byte shared loads do not conflict
     const int ct = tid - 32;
-    const int c16 = ct & 1, r = (ct >> 1) & (kTileM - 1), hh = ct >> 8;
-    const uint32_t xrow = (uint32_t)a.xw * kTileK;  // activation window row, elements
     uint32_t sc = 0;
     bool waited_primary = !a.pdl_secondary;
 
     for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
         const GvItem f = item_of(it);
-        const GemvSide& sd = *f.sd;
-        const WLayout L = sd.L;
-        const int G = (f.nsl + kGvNT - 1) / kGvNT;
-        const int S_side = f.shared ? a.n_tokens : S;
-        auto slot_of = [&](int q) { return f.shared ? q : list[f.sbase + q]; };
+        if (f.nrow == 0) continue;
+        const WLayout L = GV_SIDE(f.side, L);
+        const int rsub = GV_SIDE(f.side, rsub), kps = GV_SIDE(f.side, kps), KT = L.kt_count;
+        // slot list of the item: routed fast = the ballot masks of its expert
+        uint32_t mk0 = 0u, mk1 = 0u;
+        int nsl = f.nsl, jrow = 0;
+        if (f.side == 0) {
+            if (R.fast) {
+                mk0 = __ballot_sync(0xffffffffu, R.v0 == f.e);
+                mk1 = __ballot_sync(0xffffffffu, R.v1 == f.e);
+                nsl = __popc(mk0) + __popc(mk1);
+            } else {
+                jrow = (it - n_sh) / a.routed.subs;
+                nsl = R.off[jrow + 1] - R.off[jrow];
+            }
+        }
+        auto slot_of = [&](int q) {
+            if (f.side == 1) return q;
+            return R.fast ? nth_bit(mk0, mk1, q) : R.slots[R.off[jrow] + q];
+        };
+        // thread = (row rho of the sub-tile, slice sig); a slice is (k-step kk, 32-column half hh)
+        const int rho = ct % rsub, sig = ct / rsub;
+        const int nsig = kGvConsumers / rsub;  // slices processed at once
+        const int G = (nsl + kGvNT - 1) / kGvNT;
+        // this row's place in the stage pieces: sub-block rho / 32 of the sub-tile
+        const int sb = (f.r0 + rho) / kSubRows;
+        const int nr = sub_rows(L.rows(f.mt), sb);
+        const uint32_t roff = (uint32_t)((rho / kSubRows) * L.sub_bytes());
+        const int rr = rho % kSubRows;
+        const int first = (lane >> 2) & 1;  // alternate 16-byte chunk order: conflict-free loads
         for (int g = 0; g < G; ++g) {
-            const int nt = min(kGvNT, f.nsl - g * kGvNT);
+            const int nt = nsl - g * kGvNT < kGvNT ? nsl - g * kGvNT : kGvNT;
             float acc[NMAT][kGvNT];
 #pragma unroll
             for (int m = 0; m < NMAT; ++m)
 #pragma unroll
                 for (int q = 0; q < kGvNT; ++q) acc[m][q] = 0.f;
+            // activation window: as many k-steps as fit kGvXBytes for nt tokens, a multiple of kps
+            int xw = (int)(kGvXBytes / ((uint32_t)nt * kTileK * 4u));
+            xw = xw / kps * kps;
+            if (xw < kps) xw = kps;
             bool ok = true;
-            for (int w0 = 0; w0 < f.nk; w0 += a.xw) {
-                const int nw = min(a.xw, f.nk - w0);
-                // the previous window's activations are no longer read; stop together on abort
-                ok = consumers_and(ok && !*abort_flag);
+            for (int w0 = 0; w0 < KT; w0 += xw) {
+                const int nw = KT - w0 < xw ? KT - w0 : xw;
+                ok = consumers_and(ok && !*abort_flag);  // the previous window is no longer read
                 if (!ok) break;
                 if (!waited_primary) {
                     asm volatile("griddepcontrol.wait;" ::: "memory");
                     waited_primary = true;
                 }
-                // stage the activations of the nt tokens for this window, as fp32
-                const int cols = nw * kTileK, col0 = (f.kt0 + w0) * kTileK;
+                // stage the nt tokens' activations of this window as fp32: sx[q][col]
+                const int cols = nw * kTileK, col0 = w0 * kTileK;
                 constexpr int VE = 16 / XB;  // elements per 16-byte vector
                 for (int idx = ct; idx < nt * cols / VE; idx += kGvConsumers) {
                     const int q = idx / (cols / VE), cc = (idx - q * (cols / VE)) * VE, col = col0 + cc;
                     const int sl = slot_of(g * kGvNT + q);
-                    const int row = f.shared ? sl : (sd.x_per_slot ? sl : sl / a.k);
+                    const int row = f.side == 1 ? sl : (a.routed.x_per_slot ? sl : sl / a.k);
                     uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                    if (col < L.n_in) v = __ldg((const uint4*)((const uint8_t*)sd.x + ((size_t)row * L.n_in + col) * XB));
-                    float* dst = (float*)sx + (size_t)q * xrow + cc;
+                    if (col < L.n_in)
+                        v = __ldg((const uint4*)((const uint8_t*)GV_SIDE(f.side, x) + ((size_t)row * L.n_in + col) * XB));
+                    float* dst = sx + (size_t)q * cols + cc;
                     if (XB == 4) {
                         *(uint4*)dst = v;
                     } else {
@@ -352,60 +523,104 @@ gemv_kernel(const GemvArgs a) {
                         float e[8];
 #pragma unroll
                         for (int b = 0; b < 4; ++b) {
-                            e[2 * b] = ld_x16(uw[b] & 0xffffu, sd.x_type);
-                            e[2 * b + 1] = ld_x16(uw[b] >> 16, sd.x_type);
+                            e[2 * b] = ld_x16(uw[b] & 0xffffu, GV_SIDE(f.side, x_type));
+                            e[2 * b + 1] = ld_x16(uw[b] >> 16, GV_SIDE(f.side, x_type));
                         }
                         *(float4*)dst = make_float4(e[0], e[1], e[2], e[3]);
                         *(float4*)(dst + 4) = make_float4(e[4], e[5], e[6], e[7]);
                     }
                 }
                 consumers_sync();
-                for (int ks = w0; ks < w0 + nw; ks += sk, ++sc) {
-                    const int nks = min(sk, f.nk - ks);
-                    const int s = (int)(sc % (uint32_t)ns);
-                    int okw = 1;
-                    if (lane == 0) okw = gv_wait(&full[s], (sc / ns) & 1u, status, abort_flag);
-                    if (!__shfl_sync(0xffffffffu, okw, 0)) { ok = false; break; }
-                    if (r < f.rows) {
-                        for (int kk = 0; kk < nks; ++kk) {
-                            // w = q*d for this thread's 16 columns of each matrix, as 8 packed pairs
-                            uint64_t w2[NMAT][8];
+                for (int k0 = w0; k0 < w0 + nw; k0 += kps, ++sc) {
+                    const int nk = KT - k0 < kps ? KT - k0 : kps;
+                    const int s = (int)(sc % (uint32_t)a.ns);
+                    if (!gv_warp_wait(&full[s], (sc / a.ns) & 1u, status, abort_flag, a.wait_limit)) {
+                        ok = false;
+                        break;
+                    }
+                    if (rho < f.nrow) {
+                        // single: two slices per thread (sig, sig + nsig); dual: one slice, both matrices
+                        for (int sl2 = sig; sl2 < 2 * nk; sl2 += nsig) {
+                            const int kk = sl2 >> 1, hh = sl2 & 1;
+                            const float* xk = sx + (size_t)(k0 - w0 + kk) * kTileK + hh * 32;
+                            if (WT == MOE_MXFP4) {
+                                // 32 E2M1 codes of this row's half (16 bytes) and its E8M0 scale: the dot
+                                // runs on the codes' exact values; the slice's sum is then multiplied by
+                                // the power-of-two scale (each product differs from the scaled one by that
+                                // exact factor, so the roundings are the same)
 #pragma unroll
-                            for (int m = 0; m < NMAT; ++m) {
-                                const uint8_t* blk = ring + (size_t)s * a.stage_bytes + (size_t)m * sk * kGvBlock +
-                                                     (size_t)kk * f.rows * kRowBytes;
-                                const uint4 qv = *(const uint4*)(blk + (size_t)hh * f.rows * 32 + r * 32 + c16 * 16);
-                                const float d =
-                                    __half2float(*(const __half*)(blk + (size_t)f.rows * kTileK + r * 4 + hh * 2));
-                                const uint64_t dd = f2pack(d, d), nd = f2pack(-32896.0f * d, -32896.0f * d);
-                                const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
+                                for (int m = 0; m < NMAT; ++m) {
+                                    const uint8_t* pc = ring + (size_t)s * kGvStage + (size_t)(m * kps + kk) * f.nrow * L.rb + roff;
+                                    const uint4 cv = *(const uint4*)(pc + (size_t)rr * 32 + hh * 16);
+                                    const float ssc = e8m0_float(pc[(size_t)nr * 32 + rr * 2 + hh]);
+                                    const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};
 #pragma unroll
-                                for (int i = 0; i < 8; ++i) {
-                                    const uint32_t wd = qw[i >> 1];
-                                    const int b0 = (2 * i) & 3;
-                                    w2[m][i] = fma2(f2pack(magic_byte(wd, b0), magic_byte(wd, b0 + 1)), dd, nd);
-                                }
-                            }
-                            const float* xk = (const float*)sx + (size_t)(ks - w0 + kk) * kTileK + hh * 32 + c16 * 16;
+                                    for (int q = 0; q < kGvNT; ++q) {
+                                        if (q >= nt) break;
+                                        const float4* xq = (const float4*)(xk + (size_t)q * cols);
+                                        float t = 0.f;
 #pragma unroll
-                            for (int q = 0; q < kGvNT; ++q) {
-                                if (q >= nt) break;
-                                const ulonglong2* xv = (const ulonglong2*)(xk + (size_t)q * xrow);
-                                // two independent packed chains per matrix, added in a fixed order
-                                uint64_t t0[NMAT], t1[NMAT];
-#pragma unroll
-                                for (int m = 0; m < NMAT; ++m) t0[m] = t1[m] = 0ull;
-#pragma unroll
-                                for (int v4 = 0; v4 < 4; ++v4) {
-                                    const ulonglong2 u = xv[v4];
-#pragma unroll
-                                    for (int m = 0; m < NMAT; ++m) {
-                                        t0[m] = fma2(w2[m][2 * v4], u.x, t0[m]);
-                                        t1[m] = fma2(w2[m][2 * v4 + 1], u.y, t1[m]);
+                                        for (int w4 = 0; w4 < 4; ++w4) {  // 8 codes a word: columns 8*w4 .. 8*w4+7
+                                            const float4 xa = xq[2 * w4], xb = xq[2 * w4 + 1];
+                                            float v[8];
+                                            e2m1x8_to_float(cw[w4], v);
+                                            t = fmaf(v[0], xa.x, t); t = fmaf(v[1], xa.y, t);
+                                            t = fmaf(v[2], xa.z, t); t = fmaf(v[3], xa.w, t);
+                                            t = fmaf(v[4], xb.x, t); t = fmaf(v[5], xb.y, t);
+                                            t = fmaf(v[6], xb.z, t); t = fmaf(v[7], xb.w, t);
+                                        }
+                                        acc[m][q] += t * ssc;
                                     }
                                 }
-#pragma unroll
-                                for (int m = 0; m < NMAT; ++m) acc[m][q] += f2sum(t0[m]) + f2sum(t1[m]);
+                            } else {
+                                const uint8_t* qp[NMAT];
+                                float dsc[NMAT];
+    #pragma unroll
+                                for (int m = 0; m < NMAT; ++m) {
+                                    const uint8_t* pc = ring + (size_t)s * kGvStage + (size_t)(m * kps + kk) * f.nrow * L.rb + roff;
+                                    qp[m] = pc + (size_t)hh * nr * 32 + (size_t)rr * 32;
+                                    dsc[m] = __half2float(*(const __half*)(pc + (size_t)nr * kTileK + rr * 4 + hh * 2));
+                                }
+                                // two chunks of 16 columns, in an order that alternates between groups of
+                                // four lanes (conflict-free 16-byte loads): dequantise (exact q*d), then the
+                                // dot with each token; the order is fixed per row, so runs agree bit for bit
+    #pragma unroll
+                                for (int ci = 0; ci < 2; ++ci) {
+                                    const int c2 = ci ^ first;
+                                    uint64_t w2[NMAT][8];
+    #pragma unroll
+                                    for (int m = 0; m < NMAT; ++m) {
+                                        const uint64_t dd = ptx::f2pack(dsc[m], dsc[m]);
+                                        const uint64_t nd = ptx::f2pack(-32896.0f * dsc[m], -32896.0f * dsc[m]);
+                                        const uint4 qv = *(const uint4*)(qp[m] + c2 * 16);
+                                        const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
+    #pragma unroll
+                                        for (int i = 0; i < 8; ++i) {
+                                            const uint32_t wd = qw[i >> 1];
+                                            const int b0 = (2 * i) & 3;
+                                            w2[m][i] = ptx::fma2(ptx::f2pack(magic_byte(wd, b0), magic_byte(wd, b0 + 1)), dd, nd);
+                                        }
+                                    }
+    #pragma unroll
+                                    for (int q = 0; q < kGvNT; ++q) {
+                                        if (q >= nt) break;
+                                        const ulonglong2* xv = (const ulonglong2*)(xk + (size_t)q * cols + c2 * 16);
+                                        uint64_t t0[NMAT], t1[NMAT];
+    #pragma unroll
+                                        for (int m = 0; m < NMAT; ++m) t0[m] = t1[m] = 0ull;
+    #pragma unroll
+                                        for (int v8 = 0; v8 < 4; ++v8) {
+                                            const ulonglong2 u = xv[v8];
+    #pragma unroll
+                                            for (int m = 0; m < NMAT; ++m) {
+                                                t0[m] = ptx::fma2(w2[m][2 * v8], u.x, t0[m]);
+                                                t1[m] = ptx::fma2(w2[m][2 * v8 + 1], u.y, t1[m]);
+                                            }
+                                        }
+    #pragma unroll
+                                        for (int m = 0; m < NMAT; ++m) acc[m][q] += f2sum(t0[m]) + f2sum(t1[m]);
+                                    }
+                                }
                             }
                         }
                     }
@@ -413,90 +628,73 @@ gemv_kernel(const GemvArgs a) {
                     if (lane == 0) ptx::mbar_arrive(&empty[s]);
                 }
             }
-            // the two 16-column chunks (adjacent lanes; a + b == b + a), then the
-            // two 32-column halves of each row, in a fixed order
+            // slice partial sums, then each (row, token) adds its slices in slice order
 #pragma unroll
             for (int m = 0; m < NMAT; ++m)
 #pragma unroll
-                for (int q = 0; q < kGvNT; ++q) {
-                    const float v = acc[m][q] + __shfl_xor_sync(0xffffffffu, acc[m][q], 1);
-                    if (c16 == 0 && q < nt) red[((hh * kTileM + r) * kGvNT + q) * NMAT + m] = v;
-                }
+                for (int q = 0; q < kGvNT; ++q) red[(ct * kGvNT + q) * NMAT + m] = acc[m][q];
             if (!consumers_and(ok && !*abort_flag)) return;  // uniform
-            if (hh == 0 && c16 == 0 && r < f.rows) {
-                const int n = f.mt * kTileM + r;
-                if (n < L.n_out)
-                    for (int q = 0; q < nt; ++q) {
-                        const int sl = slot_of(g * kGvNT + q);
-                        float v[NMAT];
+            for (int idx = ct; idx < rsub * nt; idx += kGvConsumers) {
+                const int r = idx % rsub, q = idx / rsub;
+                const int n = f.mt * kTileM + f.r0 + r;
+                if (r >= f.nrow || n >= L.n_out) continue;
+                float v[NMAT];
 #pragma unroll
-                        for (int m = 0; m < NMAT; ++m)
-                            v[m] = red[((0 * kTileM + r) * kGvNT + q) * NMAT + m] +
-                                   red[((1 * kTileM + r) * kGvNT + q) * NMAT + m];
-                        if (sd.chunks > 1) {
-                            float* pp = sd.part + (((size_t)f.c * S_side + sl) * L.n_out_pad + n) * NMAT;
-#pragma unroll
-                            for (int m = 0; m < NMAT; ++m) pp[m] = v[m];
-                        } else if (DUAL) {
-                            const float gt = v[0], up = v[NMAT - 1];
-                            sd.h[(int64_t)sl * L.n_out + n] = __float2bfloat16_rn(gt / (1.0f + expf(-gt)) * up);
-                        } else {
-                            sd.out[(int64_t)sl * L.n_out + n] = v[0];
-                        }
-                    }
+                for (int m = 0; m < NMAT; ++m) {
+                    float t = 0.f;
+                    for (int s2 = 0; s2 < nsig; ++s2) t += red[((s2 * rsub + r) * kGvNT + q) * NMAT + m];
+                    v[m] = t;
+                }
+                const int sl = slot_of(g * kGvNT + q);
+                if (DUAL) {
+                    const float gt = v[0], up = v[NMAT - 1];
+                    GV_SIDE(f.side, h)[(int64_t)sl * L.n_out + n] = __float2bfloat16_rn(gt / (1.0f + expf(-gt)) * up);
+                } else {
+                    GV_SIDE(f.side, out)[(int64_t)sl * L.n_out + n] = v[0];
+                }
             }
             consumers_sync();  // red is free again
         }
-        if (sd.chunks > 1) {
-            // the last chunk of this (expert, row tile) to finish adds all chunks in order
-            __threadfence();
-            consumers_sync();
-            if (ct == 0) *last_flag = atomicAdd(a.hdr + kHdrCnt0 + f.group, 1) == sd.chunks - 1;
-            consumers_sync();
-            if (*last_flag) {
-                __threadfence();
-                for (int idx = ct; idx < f.nsl * f.rows; idx += kGvConsumers) {
-                    const int q = idx / f.rows, rr = idx - q * f.rows;
-                    const int n = f.mt * kTileM + rr;
-                    if (n >= L.n_out) continue;
-                    const int sl = slot_of(q);
-                    float v[NMAT];
-#pragma unroll
-                    for (int m = 0; m < NMAT; ++m) v[m] = 0.f;
-                    for (int c = 0; c < sd.chunks; ++c) {
-                        const volatile float* pp = sd.part + (((size_t)c * S_side + sl) * L.n_out_pad + n) * NMAT;
-#pragma unroll
-                        for (int m = 0; m < NMAT; ++m) v[m] += pp[m];
-                    }
-                    if (DUAL) {
-                        const float gt = v[0], up = v[NMAT - 1];
-                        sd.h[(int64_t)sl * L.n_out + n] = __float2bfloat16_rn(gt / (1.0f + expf(-gt)) * up);
-                    } else {
-                        sd.out[(int64_t)sl * L.n_out + n] = v[0];
-                    }
-                }
-                if (ct == 0) atomicExch(a.hdr + kHdrCnt0 + f.group, 0);
-            }
-            consumers_sync();  // last_flag is free again
-        }
     }
+#undef GV_SIDE
+}
+
+// Rows per item of the routed side: the largest of 128, 64, 32 whose items
+// (over at most `experts` experts, plus the shared side's) come to at least
+// 0.9 of the SMs, else 32.
+static int pick_rsub(const WLayout& L, int64_t experts, int64_t other_items, int sms) {
+    for (int r : {128, 64}) {
+        const int64_t items = experts * L.mt_count * (kTileM / r) + other_items;
+        if (items * 10 >= (int64_t)sms * 9) return r;
+    }
+    return 32;
+}
+
+// k-steps per ring stage: as many as fill kGvStage bytes with the sub-tile's
+// rows of every matrix, at most 8 (the activation window of 8 tokens holds 8).
+static int stage_ksteps(const WLayout& L, int rsub, int nmat) {
+    const int k = (int)(kGvStage / ((uint32_t)L.rb * rsub * nmat));
+    return k < 1 ? 1 : k > 8 ? 8 : k;
 }
 
 void gemv_plan_side(GemvSide& s, int dual) {
-    (void)dual;
-    s.kc = s.L.kt_count;
-    s.chunks = 1;
-    s.group0 = 0;
+    s.rsub = kTileM;
+    s.subs = s.L.mt_count;
+    s.kps = stage_ksteps(s.L, kTileM, dual + 1);
 }
 
-template <int DUAL, int XB>
-static moe_status launch_t(const GemvArgs& a, size_t smem, unsigned grid, cudaStream_t stream) {
+template <int DUAL, int XB, int WT>
+static moe_status launch_t(const GemvArgs& a, size_t smem, unsigned grid, int pdl_attr, cudaStream_t stream) {
     static int attr_dev = -1;
     int dev = 0;
     cudaGetDevice(&dev);
     if (attr_dev != dev) {
-        if (cudaFuncSetAttribute(gemv_kernel<DUAL, XB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)kGvSmemBudget + 16 * 1024) != cudaSuccess)
+        // the largest shared-memory carveout: an SM configured for one launch's
+        // CTA alone would have no room left for a CTA of the other launch
+        if (cudaFuncSetAttribute(gemv_kernel<DUAL, XB, WT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kGvSmemBudget) != cudaSuccess ||
+            cudaFuncSetAttribute(gemv_kernel<DUAL, XB, WT>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 (int)cudaSharedmemCarveoutMaxShared) != cudaSuccess)
             return MOE_ERR_CUDA;
         attr_dev = dev;
     }
@@ -509,8 +707,8 @@ static moe_status launch_t(const GemvArgs& a, size_t smem, unsigned grid, cudaSt
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = a.pdl_secondary ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, gemv_kernel<DUAL, XB>, a) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    cfg.numAttrs = pdl_attr ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, gemv_kernel<DUAL, XB, WT>, a) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 static int gv_sm_count() {
@@ -524,70 +722,71 @@ static int gv_sm_count() {
     return n > 0 ? n : 148;
 }
 
+// test-only stall (moe_testing_stall): CTA, stage, wait limit in microseconds
+static std::atomic<int> g_stall_cta{-1}, g_stall_stage{0}, g_stall_wait_us{0};
+
 moe_status launch_gemv(const GemvArgs& in, cudaStream_t stream) {
     GemvArgs a = in;
+    a.stall_cta = g_stall_cta.load();
+    a.stall_stage = g_stall_stage.load();
+    if (a.stall_cta >= 0) {
+        int dev = 0, khz = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&khz, cudaDevAttrClockRate, dev);
+        a.wait_limit = (long long)g_stall_wait_us.load() * (khz > 0 ? khz : 2000000) / 1000;
+    }
     const int S = a.n_tokens * a.k;
-    if (S > kGvMaxSlots) return MOE_ERR_UNSUPPORTED;
-    const int64_t groups_r = (int64_t)a.max_distinct * a.routed.L.mt_count;
-    const int64_t groups_s = a.has_shared ? a.shared.L.mt_count : 0;
-    if (groups_r + groups_s == 0) return MOE_OK;
+    if (S > kGvMaxSlots || (a.wtype != MOE_Q8_0 && a.wtype != MOE_MXFP4)) return MOE_ERR_UNSUPPORTED;
     const bool f32 = a.routed.x_type == MOE_F32 || (a.has_shared && a.shared.x_type == MOE_F32);
     if (f32 && a.has_shared && a.routed.x_type != a.shared.x_type) return MOE_ERR_UNSUPPORTED;
     const int nmat = a.dual + 1;
     const int sms = gv_sm_count();
-
-    // Split K when the (expert, row tile) groups alone cannot cover the SMs.
-    // Shared-expert items carry every token, so that side is split further.
-    // Split groups count arrivals in the header (kGvMaxGroups counters).
-    GemvSide* sides[2] = {&a.routed, a.has_shared ? &a.shared : nullptr};
-    for (GemvSide* s : sides)
-        if (s) s->kc = s->L.kt_count, s->chunks = 1;
-    const bool small = S <= kGvSplitSlots;
-    int chunks_r = 1, chunks_s = 1;
-    if (small) {
-        // as many chunks as fit in one wave of CTAs (a second, partial wave would
-        // double the time of the CTAs that run it)
-        chunks_r = (int)(sms / (groups_r + groups_s));
-        if (chunks_r < 1) chunks_r = 1;
-        chunks_s = chunks_r > 2 * a.n_tokens ? chunks_r : 2 * a.n_tokens;
+    // rows per item: 32 for the shared side (its items carry every token, so
+    // they are the slowest per byte), then the routed side given those items
+    int64_t sh_items = 0;
+    if (a.has_shared) {
+        a.shared.rsub = 32;
+        a.shared.subs = a.shared.L.mt_count * (kTileM / a.shared.rsub);
+        a.shared.kps = stage_ksteps(a.shared.L, a.shared.rsub, nmat);
+        sh_items = a.shared.subs;
     }
-    int counters = 0;
-    auto split = [&](GemvSide* s, int64_t groups, int want) {
-        if (!s || !s->part || want <= 1 || counters + groups > kGvMaxGroups) return;
-        const int KT = s->L.kt_count;
-        if (want > kGvMaxChunks) want = kGvMaxChunks;
-        if (want > KT) want = KT;
-        s->kc = (KT + want - 1) / want;
-        s->chunks = (KT + s->kc - 1) / s->kc;
-        s->group0 = counters;
-        counters += (int)groups;
-    };
-    split(&a.routed, groups_r, chunks_r);
-    if (a.has_shared) split(&a.shared, groups_s, chunks_s);
+    a.routed.rsub = pick_rsub(a.routed.L, a.max_distinct, sh_items, sms);
+    a.routed.subs = a.routed.L.mt_count * (kTileM / a.routed.rsub);
+    a.routed.kps = stage_ksteps(a.routed.L, a.routed.rsub, nmat);
+    if (a.wait_limit <= 0) a.wait_limit = kGvWaitLimit;
 
-    // A stage carries ~34 KB whatever the mode (per-stage costs are fixed): two
-    // k-steps of both matrices, or four of one.
-    a.sk = a.dual ? 2 : 4;
-    a.xw = 16;
-    a.stage_bytes = (uint32_t)nmat * a.sk * kGvBlock;
-    a.x_bytes = (uint32_t)kGvNT * a.xw * kTileK * 4;  // fp32 after staging
-    a.red_bytes = (uint32_t)2 * kTileM * kGvNT * nmat * 4;
-    a.bm_words = (uint32_t)((a.n_experts + 31) / 32);
-    a.tab_words = (uint32_t)(2 * (a.max_distinct + 1) + 2 * S);  // cnt, off, slot list, ids
-    a.ns = 1;
-    const uint32_t fixed = gv_lay(a).total - a.stage_bytes;
-    int ns = (int)((kGvSmemBudget - fixed) / a.stage_bytes);
+    const uint32_t fixed = gv_lay(0, S, a.n_experts).total;
+    int ns = (int)((kGvSmemBudget - fixed - 2 * 8 * 8) / kGvStage);
     if (ns > 8) ns = 8;
     if (ns < 2) return MOE_ERR_UNSUPPORTED;
     a.ns = ns;
-    const size_t smem = gv_lay(a).total;
+    const size_t smem = gv_lay(ns, S, a.n_experts).total;
+    if (smem > kGvSmemBudget) return MOE_ERR_UNSUPPORTED;
 
-    const int64_t items_max = groups_r * a.routed.chunks + groups_s * (a.has_shared ? a.shared.chunks : 0);
+    const int64_t items_max = (int64_t)a.max_distinct * a.routed.subs + sh_items;
+    if (items_max == 0) return MOE_OK;
     int64_t grid = sms;
     if (grid > items_max) grid = items_max;
+    const int pdl_attr = a.pdl_wait || a.pdl_secondary;
+    const unsigned g = (unsigned)grid;
+    if (a.wtype == MOE_MXFP4) {
+        if (a.dual)
+            return f32 ? launch_t<1, 4, MOE_MXFP4>(a, smem, g, pdl_attr, stream)
+                       : launch_t<1, 2, MOE_MXFP4>(a, smem, g, pdl_attr, stream);
+        return f32 ? launch_t<0, 4, MOE_MXFP4>(a, smem, g, pdl_attr, stream)
+                   : launch_t<0, 2, MOE_MXFP4>(a, smem, g, pdl_attr, stream);
+    }
     if (a.dual)
-        return f32 ? launch_t<1, 4>(a, smem, (unsigned)grid, stream) : launch_t<1, 2>(a, smem, (unsigned)grid, stream);
-    return f32 ? launch_t<0, 4>(a, smem, (unsigned)grid, stream) : launch_t<0, 2>(a, smem, (unsigned)grid, stream);
+        return f32 ? launch_t<1, 4, MOE_Q8_0>(a, smem, g, pdl_attr, stream)
+                   : launch_t<1, 2, MOE_Q8_0>(a, smem, g, pdl_attr, stream);
+    return f32 ? launch_t<0, 4, MOE_Q8_0>(a, smem, g, pdl_attr, stream)
+               : launch_t<0, 2, MOE_Q8_0>(a, smem, g, pdl_attr, stream);
 }
 
 }  // namespace moe
+
+extern "C" void moe_testing_stall(int cta, int stage, int wait_us) {
+    moe::g_stall_stage.store(stage < 0 ? 0 : stage);
+    moe::g_stall_wait_us.store(wait_us < 1 ? 1 : wait_us);
+    moe::g_stall_cta.store(cta < 0 ? -1 : cta);
+}

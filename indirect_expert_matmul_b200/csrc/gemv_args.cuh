@@ -5,9 +5,7 @@
 namespace moe {
 
 constexpr int kGvMaxSlots = 1024;   // the mat-vec path handles n_tokens*k up to this
-constexpr int kGvNT = 8;            // tokens per pass over a weight chunk
-constexpr int kHdrCnt0 = 16;        // header words [16, 64): split-K arrival counters
-constexpr int kGvMaxGroups = 48;    // (expert, row tile) groups that may be split
+constexpr int kGvNT = 8;            // tokens per pass over a weight stage
 
 struct GemvSide {
     const uint8_t* W0;  // prepared weights (single, or gate)
@@ -18,30 +16,31 @@ struct GemvSide {
     int x_per_slot;     // routed x row: 1 -> slot t*k+s, 0 -> token t
     float* out;         // single: out[slot][n] (routed) or out[t][n] (shared)
     __nv_bfloat16* h;   // dual: h[slot][n] (routed) or h[t][n] (shared)
-    float* part;        // split-K partial sums [chunk][slot][n_out_pad][1 + dual], or null (no split)
-    int kc;             // k-steps per chunk (filled by launch_gemv)
-    int chunks;         // ceil(kt_count / kc)
-    int group0;         // first counter index of this side's (expert, row tile) groups
+    // launch plan (filled by launch_gemv)
+    int rsub;           // rows per work item: 32, 64 or 128
+    int subs;           // work items per expert (row sub-tiles, counting empty ones of a tail tile)
+    int kps;            // k-steps per ring stage
 };
 
 struct GemvArgs {
     GemvSide routed, shared;
     int has_shared;
     int dual;
+    int wtype;           // MOE_Q8_0 / MOE_MXFP4 (both sides)
     const int32_t* ids;  // [n_tokens][k]
     int n_tokens, k, n_experts;
     int max_distinct;    // min(n_tokens*k, n_experts)
-    int pdl_secondary;   // launched as a programmatic dependent: wait before reading activations
+    int pdl_wait;        // may start before the previous kernel of the stream ends: wait first
+    int pdl_trigger;     // has a programmatic dependent: let it start once ids are valid
+    int pdl_secondary;   // programmatic dependent: consumers wait before reading activations
     int* hdr;
-    // launch plan (filled by launch_gemv)
-    int sk;              // k-steps per ring stage
-    int ns;              // ring stages
-    int xw;              // activation window, in k-steps (a multiple of sk)
-    uint32_t stage_bytes, x_bytes, red_bytes, tab_words, bm_words;
+    long long wait_limit;  // cycles a bounded wait may take (0: the default, ~2 s)
+    int stall_cta, stall_stage;  // test-only: this CTA's producer skips this ring stage (-1: none)
+    int ns;              // ring stages (filled by launch_gemv)
 };
 
 moe_status launch_gemv(const GemvArgs& a, cudaStream_t stream);
-// Reset the split fields of a side (no split); launch_gemv chooses the split.
+// Default plan of a side (128-row items); launch_gemv chooses the final plan.
 void gemv_plan_side(GemvSide& s, int dual);
 
 }  // namespace moe

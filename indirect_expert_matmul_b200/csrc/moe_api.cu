@@ -9,7 +9,7 @@ namespace moe {
 moe_status launch_row_ids(const int32_t* ids, int64_t S, int k, int E, int mode, int32_t* ids_src1,
                           int32_t* ids_dst, int32_t* bounds, int32_t* active, int32_t* ntile_prefix,
                           int32_t* pad_start, int32_t* slot_prow, int bn, int* hdr, cudaStream_t stream);
-moe_status launch_prepare(const void* src, int E, int n_out, int n_in, void* dst, cudaStream_t stream);
+moe_status launch_prepare(int wtype, const void* src, int E, int n_out, int n_in, void* dst, cudaStream_t stream);
 }  // namespace moe
 
 #include "gemv_args.cuh"
@@ -73,17 +73,29 @@ moe_status moe_get_status(void* workspace, moe_stream stream) {
     return (moe_status)st;
 }
 
+static bool valid_wtype(int w) { return w == MOE_Q8_0 || w == MOE_MXFP4; }
+
+size_t moe_weights_prepared_size_w(moe_wtype w_type, int n_experts, int n_out, int n_in) {
+    if (!valid_wtype(w_type) || n_experts <= 0 || n_out <= 0 || n_in <= 0) return 0;
+    return (size_t)(n_experts * WLayout(n_out, n_in, w_type).expert_bytes);
+}
+
 size_t moe_weights_prepared_size(int n_experts, int n_out, int n_in) {
-    if (n_experts <= 0 || n_out <= 0 || n_in <= 0) return 0;
-    return (size_t)(n_experts * WLayout(n_out, n_in).expert_bytes);
+    return moe_weights_prepared_size_w(MOE_Q8_0, n_experts, n_out, n_in);
+}
+
+moe_status moe_weights_prepare_w(moe_wtype w_type, const void* blocks, int n_experts, int n_out, int n_in,
+                                 void* prepared, moe_stream stream) {
+    if (!valid_wtype(w_type)) return MOE_ERR_INVALID;
+    if (!blocks || !prepared || n_experts <= 0 || n_out <= 0 || n_in <= 0) return MOE_ERR_INVALID;
+    if (n_in % 32 || !aligned(prepared, 16) || (w_type == MOE_Q8_0 && !aligned(blocks, 2))) return MOE_ERR_INVALID;
+    if (n_experts > kMaxExperts) return MOE_ERR_RANGE;
+    return launch_prepare(w_type, blocks, n_experts, n_out, n_in, prepared, (cudaStream_t)stream);
 }
 
 moe_status moe_weights_prepare(const void* q8_0_blocks, int n_experts, int n_out, int n_in, void* prepared,
                                moe_stream stream) {
-    if (!q8_0_blocks || !prepared || n_experts <= 0 || n_out <= 0 || n_in <= 0) return MOE_ERR_INVALID;
-    if (n_in % 32 || !aligned(prepared, 16) || !aligned(q8_0_blocks, 2)) return MOE_ERR_INVALID;
-    if (n_experts > kMaxExperts) return MOE_ERR_RANGE;
-    return launch_prepare(q8_0_blocks, n_experts, n_out, n_in, prepared, (cudaStream_t)stream);
+    return moe_weights_prepare_w(MOE_Q8_0, q8_0_blocks, n_experts, n_out, n_in, prepared, stream);
 }
 
 moe_status moe_row_ids(const int32_t* ids, int64_t n_tokens, int k, int n_experts, moe_mode mode,
@@ -107,6 +119,14 @@ moe_status moe_row_ids(const int32_t* ids, int64_t n_tokens, int k, int n_expert
 moe_status moe_mul_mat_id(const void* W_prepared, int n_experts, int n_out, int n_in, const void* x,
                           moe_dtype x_type, const int32_t* ids, int64_t n_tokens, int k, moe_mode mode,
                           float* dst, void* workspace, moe_stream stream) {
+    return moe_mul_mat_id_w(MOE_Q8_0, W_prepared, n_experts, n_out, n_in, x, x_type, ids, n_tokens, k, mode, dst,
+                            workspace, stream);
+}
+
+moe_status moe_mul_mat_id_w(moe_wtype w_type, const void* W_prepared, int n_experts, int n_out, int n_in,
+                            const void* x, moe_dtype x_type, const int32_t* ids, int64_t n_tokens, int k,
+                            moe_mode mode, float* dst, void* workspace, moe_stream stream) {
+    if (!valid_wtype(w_type)) return MOE_ERR_INVALID;
     moe_status st = check_sizes(n_tokens, k, n_experts);
     if (st) return st;
     if (mode != MOE_BROADCAST && mode != MOE_PER_SLOT) return MOE_ERR_INVALID;
@@ -128,19 +148,21 @@ moe_status moe_mul_mat_id(const void* W_prepared, int n_experts, int n_out, int 
     if (use_gemv(n_tokens, S)) {
         GemvArgs a = {};
         a.routed.W0 = (const uint8_t*)W_prepared;
-        a.routed.L = WLayout(n_out, n_in);
+        a.routed.L = WLayout(n_out, n_in, w_type);
         a.routed.x = x;
         a.routed.x_type = x_type;
         a.routed.x_per_slot = mode == MOE_PER_SLOT;
         a.routed.out = dst;
         gemv_plan_side(a.routed, 0);
         a.dual = 0;
+        a.wtype = w_type;
         a.ids = ids;
         a.n_tokens = (int)n_tokens;
         a.k = k;
         a.n_experts = n_experts;
         a.max_distinct = (int)(S < n_experts ? S : n_experts);
         a.hdr = hdr;
+        a.pdl_wait = 1;
         st = launch_gemv(a, s);
         prof_mark(s, "gemv");
         return st;
@@ -150,6 +172,7 @@ moe_status moe_mul_mat_id(const void* W_prepared, int n_experts, int n_out, int 
     if (st) return st;
     prof_mark(s, "row_ids");
     GemmMulMatId g = {};
+    g.wtype = w_type;
     g.W = (const uint8_t*)W_prepared;
     g.E = n_experts;
     g.n_out = n_out;
@@ -177,6 +200,15 @@ moe_status moe_ffn(const void* Wg, const void* Wu, const void* Wd, int n_experts
                    const void* Sg, const void* Su, const void* Sd, int n_ff_shared, const void* x, moe_dtype x_type,
                    const int32_t* ids, int64_t n_tokens, int k, float* dst, float* dst_shared, void* workspace,
                    moe_stream stream) {
+    return moe_ffn_w(MOE_Q8_0, Wg, Wu, Wd, n_experts, n_embd, n_ff, Sg, Su, Sd, n_ff_shared, x, x_type, ids, n_tokens,
+                     k, dst, dst_shared, workspace, stream);
+}
+
+moe_status moe_ffn_w(moe_wtype w_type, const void* Wg, const void* Wu, const void* Wd, int n_experts, int n_embd,
+                     int n_ff, const void* Sg, const void* Su, const void* Sd, int n_ff_shared, const void* x,
+                     moe_dtype x_type, const int32_t* ids, int64_t n_tokens, int k, float* dst, float* dst_shared,
+                     void* workspace, moe_stream stream) {
+    if (!valid_wtype(w_type)) return MOE_ERR_INVALID;
     moe_status st = check_sizes(n_tokens, k, n_experts);
     if (st) return st;
     if (x_type != MOE_BF16 && x_type != MOE_F16 && x_type != MOE_F32) return MOE_ERR_INVALID;
@@ -213,28 +245,30 @@ moe_status moe_ffn(const void* Wg, const void* Wu, const void* Wd, int n_experts
         a.hdr = hdr;
         // gate/up -> h[t][s] (SwiGLU), shared -> h_sh[t]
         a.dual = 1;
+        a.wtype = w_type;
         a.routed.W0 = (const uint8_t*)Wg;
         a.routed.W1 = (const uint8_t*)Wu;
-        a.routed.L = WLayout(n_ff, n_embd);
+        a.routed.L = WLayout(n_ff, n_embd, w_type);
         a.routed.x = x;
         a.routed.x_type = x_type;
         a.routed.h = h;
         gemv_plan_side(a.routed, 1);
-        a.routed.part = S <= kGvSplitSlots ? (float*)(ws + W.gv_part) : nullptr;  // split-K partial sums
+        a.pdl_wait = 1;     // may start during the previous kernel's tail; reads nothing before its wait
+        a.pdl_trigger = 1;  // the down launch below may start once ids are valid
         if (has_shared) {
             a.shared.W0 = (const uint8_t*)Sg;
             a.shared.W1 = (const uint8_t*)Su;
-            a.shared.L = WLayout(n_ff_shared, n_embd);
+            a.shared.L = WLayout(n_ff_shared, n_embd, w_type);
             a.shared.x = x;
             a.shared.x_type = x_type;
             a.shared.h = h_sh;
             gemv_plan_side(a.shared, 1);
-            a.shared.part = S <= kGvSplitSlots ? (float*)(ws + W.gv_part_sh) : nullptr;
         }
         st = launch_gemv(a, s);
         if (st) return st;
         prof_mark(s, "gemv_gate_up");
-        // down -> dst[t][s], dst_shared[t]; a programmatic dependent of gate/up
+        // down -> dst[t][s], dst_shared[t]; a programmatic dependent of gate/up: its
+        // producer streams the down weights while gate/up runs
         GemvArgs b = {};
         b.has_shared = has_shared;
         b.ids = ids;
@@ -244,9 +278,10 @@ moe_status moe_ffn(const void* Wg, const void* Wu, const void* Wd, int n_experts
         b.max_distinct = a.max_distinct;
         b.hdr = hdr;
         b.dual = 0;
+        b.wtype = w_type;
         b.pdl_secondary = 1;
         b.routed.W0 = (const uint8_t*)Wd;
-        b.routed.L = WLayout(n_embd, n_ff);
+        b.routed.L = WLayout(n_embd, n_ff, w_type);
         b.routed.x = h;
         b.routed.x_type = MOE_BF16;
         b.routed.x_per_slot = 1;
@@ -254,7 +289,7 @@ moe_status moe_ffn(const void* Wg, const void* Wu, const void* Wd, int n_experts
         gemv_plan_side(b.routed, 0);
         if (has_shared) {
             b.shared.W0 = (const uint8_t*)Sd;
-            b.shared.L = WLayout(n_embd, n_ff_shared);
+            b.shared.L = WLayout(n_embd, n_ff_shared, w_type);
             b.shared.x = h_sh;
             b.shared.x_type = MOE_BF16;
             b.shared.out = dst_shared;
@@ -269,6 +304,7 @@ moe_status moe_ffn(const void* Wg, const void* Wu, const void* Wd, int n_experts
     if (st) return st;
     prof_mark(s, "row_ids");
     GemmFfn g = {};
+    g.wtype = w_type;
     g.Wg = (const uint8_t*)Wg;
     g.Wu = (const uint8_t*)Wu;
     g.Wd = (const uint8_t*)Wd;

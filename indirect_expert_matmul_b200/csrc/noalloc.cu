@@ -104,6 +104,7 @@ extern "C" moe_status moe_ffn_decode_noalloc(const void* Wg, const void* Wu, con
         a.routed.x_type = x_type;
         a.routed.h = h;
         gemv_plan_side(a.routed, 1);
+        a.pdl_trigger = 1;  // the down launch may start once ids are valid (after the header memset)
         if (has_shared) {
             a.shared.W0 = (const uint8_t*)Sg;
             a.shared.W1 = (const uint8_t*)Su;

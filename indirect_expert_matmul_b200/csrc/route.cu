@@ -62,7 +62,7 @@ route_kernel(const float* __restrict__ logits, const float* __restrict__ bias, i
     }
 
     uint32_t taken = 0u;  // bit j: expert j*32 + lane chosen
-    float mc = -INFINITY; // lane 0: largest chosen logit (renormalised weights)
+    float mine = -INFINITY;  // lane i (k <= 32): the logit chosen in round i
     int32_t* it = ids + t * k;
     float* wt = weights + t * k;
     for (int i = 0; i < k; ++i) {
@@ -101,21 +101,35 @@ route_kernel(const float* __restrict__ logits, const float* __restrict__ bias, i
             }
         }
         if ((be & 31) == lane) taken |= 1u << (be >> 5);
+        if (lane == (i & 31)) mine = bl;
         if (lane == 0) {
             it[i] = be;
-            if (normalize) {
-                wt[i] = bl;  // the chosen logit, turned into its weight below
-                mc = fmaxf(mc, bl);
-            } else {
-                wt[i] = __fdiv_rn(expf(__fsub_rn(bl, mx)), z);
-            }
+            // unnormalised: the probability itself; normalised, k > 32: the chosen
+            // logit, turned into its weight below
+            wt[i] = normalize ? bl : __fdiv_rn(expf(__fsub_rn(bl, mx)), z);
         }
     }
+    if (!normalize) return;
     // Renormalised weights p_i / sum_chosen p_j are the softmax over the chosen
     // logits alone; taken relative to the largest chosen logit, the sum is at
     // least 1, so it cannot underflow to zero however far the chosen logits sit
-    // below the row's maximum.  Lane 0, in choice order.
-    if (normalize && lane == 0) {
+    // below the row's maximum.
+    if (k <= 32) {
+        // one chosen logit per lane; the sums run in a fixed butterfly order
+        float mc = mine;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mc = fmaxf(mc, __shfl_xor_sync(0xffffffffu, mc, o));
+        const float e = lane < k ? expf(__fsub_rn(mine, mc)) : 0.f;
+        float sel = e;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sel = __fadd_rn(sel, __shfl_xor_sync(0xffffffffu, sel, o));
+        if (lane < k) wt[lane] = __fdiv_rn(e, sel);
+        return;
+    }
+    __syncwarp();
+    if (lane == 0) {  // k > 32: lane 0, in choice order
+        float mc = -INFINITY;
+        for (int i = 0; i < k; ++i) mc = fmaxf(mc, wt[i]);
         float sel = 0.f;
         for (int i = 0; i < k; ++i) {
             const float e = expf(__fsub_rn(wt[i], mc));

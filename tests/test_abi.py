@@ -133,7 +133,7 @@ def test_tensors_on_another_device_are_refused(monkeypatch):
 
     class SizesOnly:  # the library's size queries run; any other entry point is recorded
         def __getattr__(self, name):
-            if name.endswith("_size") or name == "moe_status_string":
+            if "_size" in name or name == "moe_status_string":
                 return getattr(real, name)
             return lambda *a: called.append(name) or 0
 
@@ -156,3 +156,17 @@ def test_tensors_on_another_device_are_refused(monkeypatch):
 
 def moe_prepared_bytes(E, n_out, n_in):
     return E * ((n_out + 15) // 16 * 16) * ((n_in + 63) // 64) * 68
+
+
+def test_unknown_weight_type_is_refused():
+    lib = moe.lib()
+    with pytest.raises(KeyError):
+        moe.weights_prepared_size(1, 16, 32, "q4_k")
+    assert lib.moe_weights_prepared_size_w(7, 1, 16, 32) == 0
+    assert lib.moe_weights_prepare_w(7, 16, 1, 16, 32, 16, None) == moe.ERR_INVALID
+    assert lib.moe_mul_mat_id_w(7, None, 4, 8, 64, None, 0, None, 1, 1, 0, None, None, None) == moe.ERR_INVALID
+    assert lib.moe_ffn_w(7, None, None, None, 4, 64, 64, None, None, None, 0, None, 0, None, 1, 1, None, None, None,
+                         None) == moe.ERR_INVALID
+    # MXFP4 sizes: 17 bytes per 32 weights
+    assert moe.weights_prepared_size(256, 2048, 7168, "mxfp4") == 256 * 2048 * 7168 // 32 * 17
+    assert moe.weights_prepared_size(1, 17, 32, "mxfp4") == 32 * 1 * 34
