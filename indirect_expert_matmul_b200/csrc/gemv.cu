@@ -3,26 +3,26 @@
 // llama.cpp PR #29184 ("CUDA: fuse shared experts into MMVQ", release b11370)
 // restated for this library.
 //
-// Decode is bound by the weight stream.  The kernel is built so that the two
-// launches of an expert FFN (gate/up, then down) stream their weights at the
-// same time:
-//  - each launch takes at most ~110 KB of shared memory and 288 threads of 112
-//    registers, so a CTA of the down launch fits on an SM beside a CTA of the
-//    gate/up launch; the down launch is a programmatic dependent of gate/up,
-//    its producer streams the down weights from the start and only its
-//    consumers wait for gate/up's h;
+// Decode is bound by the weight stream; the kernel is built around keeping it
+// moving:
+//  - the down launch is a programmatic dependent of gate/up: its CTAs start as
+//    gate/up's leave the SMs, their producers stream the down weights at once
+//    and only their consumers wait for gate/up's h;
 //  - a work item is (routed expert, row sub-tile of 32, 64 or 128 rows) or
 //    (shared expert, row sub-tile), always over the whole K, so no item needs
 //    another's partial sums; the sub-tile height is chosen per launch so that
 //    the items cover the SMs;
-//  - one producer warp streams 17 KB stages (the sub-tile's rows for several
+//  - one producer warp streams 34 KB stages (the sub-tile's rows for several
 //    k-steps of each matrix: one bulk copy per k-step and matrix, the rows of
 //    a sub-tile being contiguous in the repacked layout) through a ring,
 //    running ahead across items;
-//  - 256 consumer threads, thread = (row of the sub-tile, 32-column slice of a
-//    k-step): exact fp32 dequantisation (q*d) and fp32 dot products with up
-//    to 8 tokens at a time; the slices of a row are added in slice order.
-//    Every sum has a fixed order, so results do not depend on timing.
+//  - 16 consumer warps on the tensor cores (mma.sync m16n8k16, fp16 in, fp32
+//    out): A = 16 weight rows of quantised values, exact in fp16; B = up to 8
+//    tokens' activations, each token scaled by a power of two into the fp16
+//    range; each 32-column block's product is multiplied by its block scales
+//    in fp32.  A warp owns one (matrix, 16-row group) and every W-th k-step;
+//    the warps of a group are added in a fixed order, so results do not
+//    depend on timing.
 // The distinct routed experts come from ids directly: for up to 64 slots every
 // warp finds them with ballots in its own registers (no block-wide pass before
 // the first copy); for more slots a block-wide pass builds tables in shared
@@ -39,14 +39,16 @@
 
 namespace moe {
 
-constexpr int kGvConsumers = 256;
+constexpr int kGvConsumers = 512;
 constexpr int kGvThreads = 32 + kGvConsumers;  // warp 0: producer
-constexpr uint32_t kGvStage = 256 * kRowBytes;  // 17408 bytes: 256 (row, k-step) pieces of Q8_0
-constexpr uint32_t kGvSmemBudget = 110 * 1024;
+constexpr uint32_t kGvStage = 512 * kRowBytes;  // 34816 bytes: 512 (row, k-step) pieces of Q8_0
+constexpr uint32_t kGvSmemBudget = 216 * 1024;
 constexpr long long kGvWaitLimit = 1ll << 32;   // ~2 s
 constexpr int kGvFast = 64;                     // slots up to which the experts come from warp ballots
-constexpr uint32_t kGvXBytes = 16 * 1024;       // activation window (fp32)
-constexpr uint32_t kGvRedBytes = kGvConsumers * kGvNT * 2 * 4;
+constexpr int kGvXSteps = 32;                   // k-steps of the activation window (2048 columns)
+constexpr uint32_t kGvXRow = kGvXSteps * kTileK * 2 + 16;  // bytes of one token's fp16 window row (+16: banks)
+constexpr uint32_t kGvXBytes = kGvNT * kGvXRow + 2 * kGvNT * 4;  // window + per-token max and factor
+constexpr uint32_t kGvRedBytes = (kGvConsumers / 32) * 32 * 4 * 4;  // 4 fp32 results a consumer thread
 
 struct GvLay {
     uint32_t ring, x, red, tab, bars, misc, total;
@@ -146,6 +148,46 @@ __device__ __forceinline__ void e2m1x8_to_float(uint32_t w, float (&v)[8]) {
         v[2 * i] = __low2float(p);
         v[2 * i + 1] = __high2float(p);
     }
+}
+
+// Exponent e such that m * 2^-e lies in [2^14, 2^15): the power of two that
+// brings a token's largest magnitude to the top of the fp16 range (0 for zero
+// or non-finite m; at least -100, so that 2^-e stays a finite float).
+__device__ __forceinline__ int scale_exp(float m) {
+    if (!(m > 0.f) || !(m <= 3.402823466e38f)) return 0;
+    const int e = ilogbf(m) - 14;
+    return e < -100 ? -100 : e;
+}
+
+// D += A * B on the tensor cores: A 16 x 16 fp16 (row major, four registers
+// of two), B 16 x 8 fp16 (column major, two registers), D 16 x 8 fp32.
+__device__ __forceinline__ void mma_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Two stored Q8_0 bytes u = q + 128 (picked by the byte-permute selector:
+// 0x7170 bytes 0 and 1, 0x7372 bytes 2 and 3) -> {q, q'} as fp16, exactly:
+// the fp16 pattern {0x64, u} is 1024 + u, and 1024 + u - 1152 = q.
+__device__ __forceinline__ uint32_t q8_h2(uint32_t w, uint32_t sel) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(w), "r"(0x64646464u), "r"(sel));
+    const __half2 v = __hsub2(*(const __half2*)&r, __float2half2_rn(1152.0f));
+    return *(const uint32_t*)&v;
+}
+
+// The two E2M1 codes of the low byte of w (low nibble first) -> fp16x2, exact.
+__device__ __forceinline__ uint32_t e2m1x2_h2(uint32_t w) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "mov.b32 {b0, b1, b2, b3}, %1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t}"
+        : "=r"(r)
+        : "r"(w));
+    return r;
 }
 
 // n-th (0-based) set bit of a 64-bit mask given as two words.
@@ -316,10 +358,9 @@ struct GvItem {
     int nsl;     // slots (routed) or tokens (shared)
 };
 
-// At most 112 registers a thread: two CTAs of 288 threads (one of each launch
-// of an FFN) fit in the SM's 64 K registers.
+// One CTA of 544 threads an SM.
 template <int DUAL, int XB, int WT>
-__global__ void __maxnreg__(112)
+__global__ void __launch_bounds__(kGvThreads, 1)
 gemv_kernel(const GemvArgs a) {
     extern __shared__ __align__(128) uint8_t sm[];
     constexpr int NMAT = DUAL + 1;
@@ -328,7 +369,6 @@ gemv_kernel(const GemvArgs a) {
     const int S = a.n_tokens * a.k;
     const GvLay lay = gv_lay(a.ns, S, a.n_experts);
     uint8_t* ring = sm + lay.ring;
-    float* sx = (float*)(sm + lay.x);
     float* red = (float*)(sm + lay.red);
     uint64_t* full = (uint64_t*)(sm + lay.bars);
     uint64_t* empty = full + a.ns;
@@ -449,7 +489,22 @@ gemv_kernel(const GemvArgs a) {
     }
 
     // ----------------------------------------------------------- consumers
-    const int ct = tid - 32;
+    // Warp cw owns one (matrix, 16-row group) pair of the item and every W-th
+    // k-step of each stage.  Per k-step it runs four m16n8k16 tensor-core
+    // products: A = 16 weight rows x 16 columns (the quantised values
+    // themselves, exact in fp16), B = the same 16 columns of the 8 token
+    // columns (fp16, each token's window scaled by a power of two).  The
+    // 16 columns of a product lie in one 32-column block, and thread t of a
+    // fragment holds columns 8t .. 8t+3 (first product) or 8t+4 .. 8t+7
+    // (second) of the block: the same permutation of K in A and B, so that a
+    // thread's A values are one 8-byte load per row.  Each block's fp32 result
+    // is multiplied by the rows' block scales and added in block order.
+    const int ct = tid - 32, cw = ct >> 5;
+    const int gq = lane >> 2, tq = lane & 3;  // fragment row group / token, thread in group
+    uint8_t* sxb = sm + lay.x;                // [kGvNT][kGvXRow] fp16 activation window
+    int* xmax = (int*)(sm + lay.x + kGvNT * kGvXRow);  // [kGvNT]: max |x| of the window (float bits)
+    float* xsc = (float*)(xmax + kGvNT);               // [kGvNT]: the factor that undoes the scaling
+    if (ct < kGvNT) xmax[ct] = 0;             // ordered before first use by the window barrier
     uint32_t sc = 0;
     bool waited_primary = !a.pdl_secondary;
 
@@ -475,62 +530,104 @@ gemv_kernel(const GemvArgs a) {
             if (f.side == 1) return q;
             return R.fast ? nth_bit(mk0, mk1, q) : R.slots[R.off[jrow] + q];
         };
-        // thread = (row rho of the sub-tile, slice sig); a slice is (k-step kk, 32-column half hh)
-        const int rho = ct % rsub, sig = ct / rsub;
-        const int nsig = kGvConsumers / rsub;  // slices processed at once
+        // this warp's (matrix, row group) pair and k-step residue
+        const int nrg = rsub / 16, P = nrg * NMAT, W = (kGvConsumers / 32) / P;
+        const int pr = cw % P, kr = cw / P;
+        const int mw = pr / nrg, rg = pr - mw * nrg;
+        const bool live = 16 * rg < f.nrow;
+        // the row group inside the stage piece: sub-block (r0 + 16 rg) / 32 of the tile
+        const int sbk = (f.r0 + 16 * rg) / kSubRows;
+        const int nr = sub_rows(L.rows(f.mt), sbk);
+        const uint32_t roff = (uint32_t)((16 * rg / kSubRows) * L.sub_bytes());
+        const int rra = (16 * rg) % kSubRows + gq;  // rows rra and rra + 8 of the sub-block
+        const uint32_t piece = (uint32_t)f.nrow * L.rb;
         const int G = (nsl + kGvNT - 1) / kGvNT;
-        // this row's place in the stage pieces: sub-block rho / 32 of the sub-tile
-        const int sb = (f.r0 + rho) / kSubRows;
-        const int nr = sub_rows(L.rows(f.mt), sb);
-        const uint32_t roff = (uint32_t)((rho / kSubRows) * L.sub_bytes());
-        const int rr = rho % kSubRows;
-        const int first = (lane >> 2) & 1;  // alternate 16-byte chunk order: conflict-free loads
         for (int g = 0; g < G; ++g) {
             const int nt = nsl - g * kGvNT < kGvNT ? nsl - g * kGvNT : kGvNT;
-            float acc[NMAT][kGvNT];
-#pragma unroll
-            for (int m = 0; m < NMAT; ++m)
-#pragma unroll
-                for (int q = 0; q < kGvNT; ++q) acc[m][q] = 0.f;
-            // activation window: as many k-steps as fit kGvXBytes for nt tokens, a multiple of kps
-            int xw = (int)(kGvXBytes / ((uint32_t)nt * kTileK * 4u));
-            xw = xw / kps * kps;
-            if (xw < kps) xw = kps;
+            float tot[4] = {0.f, 0.f, 0.f, 0.f};  // rows rra, rra+8 x tokens 2tq, 2tq+1
             bool ok = true;
-            for (int w0 = 0; w0 < KT; w0 += xw) {
-                const int nw = KT - w0 < xw ? KT - w0 : xw;
+            for (int w0 = 0; w0 < KT; w0 += kGvXSteps) {
+                const int nw = KT - w0 < kGvXSteps ? KT - w0 : kGvXSteps;
                 ok = consumers_and(ok && !*abort_flag);  // the previous window is no longer read
                 if (!ok) break;
                 if (!waited_primary) {
                     asm volatile("griddepcontrol.wait;" ::: "memory");
                     waited_primary = true;
                 }
-                // stage the nt tokens' activations of this window as fp32: sx[q][col]
+                // stage the nt tokens' activations of this window: each token's largest
+                // magnitude first, then the values times the power of two that puts it in
+                // [2^14, 2^15), rounded to fp16 (exact for 16-bit inputs in range)
                 const int cols = nw * kTileK, col0 = w0 * kTileK;
                 constexpr int VE = 16 / XB;  // elements per 16-byte vector
-                for (int idx = ct; idx < nt * cols / VE; idx += kGvConsumers) {
-                    const int q = idx / (cols / VE), cc = (idx - q * (cols / VE)) * VE, col = col0 + cc;
-                    const int sl = slot_of(g * kGvNT + q);
-                    const int row = f.side == 1 ? sl : (a.routed.x_per_slot ? sl : sl / a.k);
-                    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                    if (col < L.n_in)
-                        v = __ldg((const uint4*)((const uint8_t*)GV_SIDE(f.side, x) + ((size_t)row * L.n_in + col) * XB));
-                    float* dst = sx + (size_t)q * cols + cc;
-                    if (XB == 4) {
-                        *(uint4*)dst = v;
-                    } else {
-                        const uint32_t uw[4] = {v.x, v.y, v.z, v.w};
-                        float e[8];
+                const int vpr = cols / VE;   // vectors per token row
+                const void* xg = GV_SIDE(f.side, x);
+                const int xt = GV_SIDE(f.side, x_type);
+                // every vector of the window is loaded once, into registers (at most 8
+                // tokens x 2048 columns: RV vectors a thread), then converted from there
+                constexpr int RV = XB == 4 ? 8 : 4;
+                uint4 v[RV];
+                int qv[RV];
 #pragma unroll
-                        for (int b = 0; b < 4; ++b) {
-                            e[2 * b] = ld_x16(uw[b] & 0xffffu, GV_SIDE(f.side, x_type));
-                            e[2 * b + 1] = ld_x16(uw[b] >> 16, GV_SIDE(f.side, x_type));
-                        }
-                        *(float4*)dst = make_float4(e[0], e[1], e[2], e[3]);
-                        *(float4*)(dst + 4) = make_float4(e[4], e[5], e[6], e[7]);
+                for (int r = 0; r < RV; ++r) {
+                    const int idx = ct + r * kGvConsumers;
+                    qv[r] = -1;
+                    v[r] = make_uint4(0u, 0u, 0u, 0u);
+                    if (idx < nt * vpr) {
+                        const int q = idx / vpr, cc = (idx - q * vpr) * VE, col = col0 + cc;
+                        const int sl = slot_of(g * kGvNT + q);
+                        const int row = f.side == 1 ? sl : (a.routed.x_per_slot ? sl : sl / a.k);
+                        qv[r] = q;
+                        if (col < L.n_in)
+                            v[r] = __ldg((const uint4*)((const uint8_t*)xg + ((size_t)row * L.n_in + col) * XB));
                     }
                 }
+                auto unpack = [&](const uint4& u, float (&e)[8]) {
+                    if (XB == 4) {
+                        e[0] = __uint_as_float(u.x); e[1] = __uint_as_float(u.y);
+                        e[2] = __uint_as_float(u.z); e[3] = __uint_as_float(u.w);
+                    } else {
+                        const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                        for (int b = 0; b < 4; ++b) {
+                            e[2 * b] = ld_x16(uw[b] & 0xffffu, xt);
+                            e[2 * b + 1] = ld_x16(uw[b] >> 16, xt);
+                        }
+                    }
+                };
+#pragma unroll
+                for (int r = 0; r < RV; ++r) {
+                    if (qv[r] < 0) continue;
+                    float e[8];
+                    unpack(v[r], e);
+                    float mx = 0.f;
+#pragma unroll
+                    for (int i = 0; i < VE; ++i) mx = fmaxf(mx, fabsf(e[i]));
+                    if (mx > 0.f) atomicMax(&xmax[qv[r]], __float_as_int(mx));
+                }
                 consumers_sync();
+#pragma unroll
+                for (int r = 0; r < RV; ++r) {
+                    if (qv[r] < 0) continue;
+                    const int q = qv[r], idx = ct + r * kGvConsumers;
+                    float e[8];
+                    unpack(v[r], e);
+                    const float sinv = ldexpf(1.0f, -scale_exp(__int_as_float(xmax[q])));
+                    uint32_t hv[4];
+#pragma unroll
+                    for (int i = 0; i < VE / 2; ++i) {
+                        const __half2 hh = __floats2half2_rn(e[2 * i] * sinv, e[2 * i + 1] * sinv);
+                        hv[i] = *(const uint32_t*)&hh;
+                    }
+                    uint8_t* dstx = sxb + (size_t)q * kGvXRow + (size_t)(idx - q * vpr) * VE * 2;
+                    if (XB == 4) *(uint2*)dstx = make_uint2(hv[0], hv[1]);
+                    else *(uint4*)dstx = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+                }
+                if (ct < kGvNT) xsc[ct] = ldexpf(1.0f, scale_exp(__int_as_float(xmax[ct])));
+                consumers_sync();
+                if (ct < kGvNT) xmax[ct] = 0;  // next written after the next window's first barrier
+                const float s0 = xsc[2 * tq], s1 = xsc[2 * tq + 1];  // tokens 2tq, 2tq + 1
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                const uint8_t* xrow = sxb + (size_t)gq * kGvXRow + 16 * tq;  // token gq, columns 8tq..
                 for (int k0 = w0; k0 < w0 + nw; k0 += kps, ++sc) {
                     const int nk = KT - k0 < kps ? KT - k0 : kps;
                     const int s = (int)(sc % (uint32_t)a.ns);
@@ -538,88 +635,58 @@ gemv_kernel(const GemvArgs a) {
                         ok = false;
                         break;
                     }
-                    if (rho < f.nrow) {
-                        // single: two slices per thread (sig, sig + nsig); dual: one slice, both matrices
-                        for (int sl2 = sig; sl2 < 2 * nk; sl2 += nsig) {
-                            const int kk = sl2 >> 1, hh = sl2 & 1;
-                            const float* xk = sx + (size_t)(k0 - w0 + kk) * kTileK + hh * 32;
+                    if (live) {
+                        for (int kk = kr; kk < nk; kk += W) {
+                            const uint8_t* pc = ring + (size_t)s * kGvStage + (size_t)(mw * kps + kk) * piece + roff;
+                            const uint8_t* xk = xrow + (size_t)(k0 - w0 + kk) * kTileK * 2;
+                            const uint4 xb[2] = {*(const uint4*)xk, *(const uint4*)(xk + 64)};
                             if (WT == MOE_MXFP4) {
-                                // 32 E2M1 codes of this row's half (16 bytes) and its E8M0 scale: the dot
-                                // runs on the codes' exact values; the slice's sum is then multiplied by
-                                // the power-of-two scale (each product differs from the scaled one by that
-                                // exact factor, so the roundings are the same)
+                                // block b: bytes 16b + 4tq .. of the row (columns 32b + 8tq .. 32b + 8tq + 7)
+                                const uint8_t* ca = pc + (size_t)rra * 32 + 4 * tq;
+                                const uint32_t wa[2] = {*(const uint32_t*)ca, *(const uint32_t*)(ca + 16)};
+                                const uint32_t wb[2] = {*(const uint32_t*)(ca + 256), *(const uint32_t*)(ca + 256 + 16)};
+                                const uint32_t sa = *(const uint16_t*)(pc + (size_t)nr * 32 + rra * 2);
+                                const uint32_t sb2 = *(const uint16_t*)(pc + (size_t)nr * 32 + (rra + 8) * 2);
 #pragma unroll
-                                for (int m = 0; m < NMAT; ++m) {
-                                    const uint8_t* pc = ring + (size_t)s * kGvStage + (size_t)(m * kps + kk) * f.nrow * L.rb + roff;
-                                    const uint4 cv = *(const uint4*)(pc + (size_t)rr * 32 + hh * 16);
-                                    const float ssc = e8m0_float(pc[(size_t)nr * 32 + rr * 2 + hh]);
-                                    const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};
+                                for (int b = 0; b < 2; ++b) {
+                                    float c[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                                    for (int q = 0; q < kGvNT; ++q) {
-                                        if (q >= nt) break;
-                                        const float4* xq = (const float4*)(xk + (size_t)q * cols);
-                                        float t = 0.f;
-#pragma unroll
-                                        for (int w4 = 0; w4 < 4; ++w4) {  // 8 codes a word: columns 8*w4 .. 8*w4+7
-                                            const float4 xa = xq[2 * w4], xb = xq[2 * w4 + 1];
-                                            float v[8];
-                                            e2m1x8_to_float(cw[w4], v);
-                                            t = fmaf(v[0], xa.x, t); t = fmaf(v[1], xa.y, t);
-                                            t = fmaf(v[2], xa.z, t); t = fmaf(v[3], xa.w, t);
-                                            t = fmaf(v[4], xb.x, t); t = fmaf(v[5], xb.y, t);
-                                            t = fmaf(v[6], xb.z, t); t = fmaf(v[7], xb.w, t);
-                                        }
-                                        acc[m][q] += t * ssc;
+                                    for (int j = 0; j < 2; ++j) {
+                                        const uint32_t x0 = j ? xb[b].z : xb[b].x, x1 = j ? xb[b].w : xb[b].y;
+                                        mma_16816(c, e2m1x2_h2(wa[b] >> (16 * j)), e2m1x2_h2(wb[b] >> (16 * j)),
+                                                  e2m1x2_h2(wa[b] >> (16 * j + 8)), e2m1x2_h2(wb[b] >> (16 * j + 8)), x0, x1);
                                     }
+                                    // E8M0 scales reach 2^127: the token factors come off first (exact
+                                    // powers of two), so no partial sum leaves the range of the result
+                                    const float da = e8m0_float((sa >> (8 * b)) & 0xffu), db = e8m0_float((sb2 >> (8 * b)) & 0xffu);
+                                    acc[0] = fmaf(da, c[0] * s0, acc[0]);
+                                    acc[1] = fmaf(da, c[1] * s1, acc[1]);
+                                    acc[2] = fmaf(db, c[2] * s0, acc[2]);
+                                    acc[3] = fmaf(db, c[3] * s1, acc[3]);
                                 }
                             } else {
-                                const uint8_t* qp[NMAT];
-                                float dsc[NMAT];
-    #pragma unroll
-                                for (int m = 0; m < NMAT; ++m) {
-                                    const uint8_t* pc = ring + (size_t)s * kGvStage + (size_t)(m * kps + kk) * f.nrow * L.rb + roff;
-                                    qp[m] = pc + (size_t)hh * nr * 32 + (size_t)rr * 32;
-                                    dsc[m] = __half2float(*(const __half*)(pc + (size_t)nr * kTileK + rr * 4 + hh * 2));
-                                }
-                                // two chunks of 16 columns, in an order that alternates between groups of
-                                // four lanes (conflict-free 16-byte loads): dequantise (exact q*d), then the
-                                // dot with each token; the order is fixed per row, so runs agree bit for bit
-    #pragma unroll
-                                for (int ci = 0; ci < 2; ++ci) {
-                                    const int c2 = ci ^ first;
-                                    uint64_t w2[NMAT][8];
-    #pragma unroll
-                                    for (int m = 0; m < NMAT; ++m) {
-                                        const uint64_t dd = ptx::f2pack(dsc[m], dsc[m]);
-                                        const uint64_t nd = ptx::f2pack(-32896.0f * dsc[m], -32896.0f * dsc[m]);
-                                        const uint4 qv = *(const uint4*)(qp[m] + c2 * 16);
-                                        const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
-    #pragma unroll
-                                        for (int i = 0; i < 8; ++i) {
-                                            const uint32_t wd = qw[i >> 1];
-                                            const int b0 = (2 * i) & 3;
-                                            w2[m][i] = ptx::fma2(ptx::f2pack(magic_byte(wd, b0), magic_byte(wd, b0 + 1)), dd, nd);
-                                        }
+                                // block b: 8 bytes at 32 b nr + 32 row + 8 tq (columns 32b + 8tq .. 32b + 8tq + 7)
+                                const uint8_t* qa = pc + (size_t)rra * 32 + 8 * tq;
+                                const uint2 ua[2] = {*(const uint2*)qa, *(const uint2*)(qa + (size_t)nr * 32)};
+                                const uint2 ub[2] = {*(const uint2*)(qa + 256), *(const uint2*)(qa + (size_t)nr * 32 + 256)};
+                                const uint32_t da2 = *(const uint32_t*)(pc + (size_t)nr * kTileK + rra * 4);
+                                const uint32_t db2 = *(const uint32_t*)(pc + (size_t)nr * kTileK + (rra + 8) * 4);
+#pragma unroll
+                                for (int b = 0; b < 2; ++b) {
+                                    float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                                    for (int j = 0; j < 2; ++j) {
+                                        const uint32_t wa = j ? ua[b].y : ua[b].x, wb = j ? ub[b].y : ub[b].x;
+                                        const uint32_t x0 = j ? xb[b].z : xb[b].x, x1 = j ? xb[b].w : xb[b].y;
+                                        mma_16816(c, q8_h2(wa, 0x7170u), q8_h2(wb, 0x7170u), q8_h2(wa, 0x7372u),
+                                                  q8_h2(wb, 0x7372u), x0, x1);
                                     }
-    #pragma unroll
-                                    for (int q = 0; q < kGvNT; ++q) {
-                                        if (q >= nt) break;
-                                        const ulonglong2* xv = (const ulonglong2*)(xk + (size_t)q * cols + c2 * 16);
-                                        uint64_t t0[NMAT], t1[NMAT];
-    #pragma unroll
-                                        for (int m = 0; m < NMAT; ++m) t0[m] = t1[m] = 0ull;
-    #pragma unroll
-                                        for (int v8 = 0; v8 < 4; ++v8) {
-                                            const ulonglong2 u = xv[v8];
-    #pragma unroll
-                                            for (int m = 0; m < NMAT; ++m) {
-                                                t0[m] = ptx::fma2(w2[m][2 * v8], u.x, t0[m]);
-                                                t1[m] = ptx::fma2(w2[m][2 * v8 + 1], u.y, t1[m]);
-                                            }
-                                        }
-    #pragma unroll
-                                        for (int m = 0; m < NMAT; ++m) acc[m][q] += f2sum(t0[m]) + f2sum(t1[m]);
-                                    }
+                                    const float da = __half2float(__ushort_as_half((unsigned short)(da2 >> (16 * b))));
+                                    const float db = __half2float(__ushort_as_half((unsigned short)(db2 >> (16 * b))));
+                                    acc[0] = fmaf(da, c[0], acc[0]);
+                                    acc[1] = fmaf(da, c[1], acc[1]);
+                                    acc[2] = fmaf(db, c[2], acc[2]);
+                                    acc[3] = fmaf(db, c[3], acc[3]);
                                 }
                             }
                         }
@@ -627,22 +694,34 @@ gemv_kernel(const GemvArgs a) {
                     __syncwarp();
                     if (lane == 0) ptx::mbar_arrive(&empty[s]);
                 }
+                // Q8_0: undo the window's token scaling (exact powers of two) into the
+                // totals (fp16 block scales keep the scaled sums far inside the float range)
+                if (WT == MOE_MXFP4) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) tot[i] += acc[i];
+                } else {
+                    tot[0] = fmaf(acc[0], s0, tot[0]);
+                    tot[1] = fmaf(acc[1], s1, tot[1]);
+                    tot[2] = fmaf(acc[2], s0, tot[2]);
+                    tot[3] = fmaf(acc[3], s1, tot[3]);
+                }
+                // a failed wait is acted on at the next barrier, which every consumer reaches
             }
-            // slice partial sums, then each (row, token) adds its slices in slice order
+            // per-warp totals, then each (row, token) adds its k-step residues in order
 #pragma unroll
-            for (int m = 0; m < NMAT; ++m)
-#pragma unroll
-                for (int q = 0; q < kGvNT; ++q) red[(ct * kGvNT + q) * NMAT + m] = acc[m][q];
+            for (int i = 0; i < 4; ++i) red[((kr * P + pr) * 32 + lane) * 4 + i] = tot[i];
             if (!consumers_and(ok && !*abort_flag)) return;  // uniform
             for (int idx = ct; idx < rsub * nt; idx += kGvConsumers) {
                 const int r = idx % rsub, q = idx / rsub;
                 const int n = f.mt * kTileM + f.r0 + r;
                 if (r >= f.nrow || n >= L.n_out) continue;
+                const int rgi = r >> 4, r16 = r & 15;
+                const int ln = (r16 & 7) * 4 + (q >> 1), ii = (r16 >> 3) * 2 + (q & 1);
                 float v[NMAT];
 #pragma unroll
                 for (int m = 0; m < NMAT; ++m) {
                     float t = 0.f;
-                    for (int s2 = 0; s2 < nsig; ++s2) t += red[((s2 * rsub + r) * kGvNT + q) * NMAT + m];
+                    for (int k2 = 0; k2 < W; ++k2) t += red[((k2 * P + m * nrg + rgi) * 32 + ln) * 4 + ii];
                     v[m] = t;
                 }
                 const int sl = slot_of(g * kGvNT + q);

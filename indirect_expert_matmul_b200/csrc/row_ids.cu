@@ -18,6 +18,7 @@ namespace moe {
 
 constexpr int kRowIdThreads = 1024;
 constexpr int kRowIdWarps = kRowIdThreads / 32;
+constexpr int kBatch = 8;  // 32-slot steps whose ids a warp loads at once
 
 // Exclusive block-wide prefix sum of one value per thread (1024 threads).
 __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_sums, int* total) {
@@ -71,19 +72,27 @@ row_ids_kernel(const int32_t* __restrict__ ids, int S, int k, int E, int mode, i
     const int c1 = min(S, c0 + L);
     const unsigned lt_mask = (1u << lane) - 1u;
 
-    // pass 1: per-chunk histogram
+    // pass 1: per-chunk histogram (the ids of kBatch 32-slot steps are loaded
+    // together, so their load latencies overlap)
     if (warp < n_chunks) {
         int* row = off + (size_t)warp * E;
         int my_bad = 0;
-        for (int base = c0; base < c1; base += 32) {
-            int i = base + lane;
-            int e = -1;
-            if (i < c1) {
-                e = __ldg(ids + i);
-                if (e < 0 || e >= E) { my_bad = 1; e = -1; }
+        for (int b0 = c0; b0 < c1; b0 += 32 * kBatch) {
+            int ev[kBatch];
+#pragma unroll
+            for (int j = 0; j < kBatch; ++j) {
+                const int i = b0 + 32 * j + lane;
+                ev[j] = i < c1 ? __ldg(ids + i) : -1;
             }
-            unsigned m = __match_any_sync(0xffffffffu, e);
-            if (e >= 0 && (m & lt_mask) == 0) row[e] += __popc(m);
+#pragma unroll
+            for (int j = 0; j < kBatch; ++j) {
+                const int i = b0 + 32 * j + lane;
+                int e = ev[j];
+                if (i < c1 && (e < 0 || e >= E)) { my_bad = 1; e = -1; }
+                unsigned m = __match_any_sync(0xffffffffu, e);
+                if (e >= 0 && (m & lt_mask) == 0) row[e] += __popc(m);
+                __syncwarp();
+            }
         }
         if (__any_sync(0xffffffffu, my_bad) && lane == 0) bad = 1;
     }
@@ -145,23 +154,32 @@ row_ids_kernel(const int32_t* __restrict__ ids, int S, int k, int E, int mode, i
     for (int i = tid; i < n_chunks * E; i += blockDim.x) off[i] += cnt[i % E];
     __syncthreads();
 
-    // pass 3: stable placement
+    // pass 3: stable placement (ids loaded kBatch steps at a time, as in pass 1)
     if (warp < n_chunks) {
         int* row = off + (size_t)warp * E;
-        for (int base = c0; base < c1; base += 32) {
-            int i = base + lane;
-            int e = (i < c1) ? __ldg(ids + i) : -1;
-            unsigned m = __match_any_sync(0xffffffffu, e);
-            int p = 0;
-            if (e >= 0) p = row[e] + __popc(m & lt_mask);
-            __syncwarp();
-            if (e >= 0) {
-                ids_dst[p] = i;
-                ids_src1[p] = (mode == MOE_BROADCAST) ? i / k : i;
-                if (slot_prow) slot_prow[i] = p + pad_delta[e];
-                if ((m & lt_mask) == 0) row[e] += __popc(m);
+        for (int b0 = c0; b0 < c1; b0 += 32 * kBatch) {
+            int ev[kBatch];
+#pragma unroll
+            for (int j = 0; j < kBatch; ++j) {
+                const int i = b0 + 32 * j + lane;
+                ev[j] = i < c1 ? __ldg(ids + i) : -1;
             }
-            __syncwarp();
+#pragma unroll
+            for (int j = 0; j < kBatch; ++j) {
+                const int i = b0 + 32 * j + lane;
+                const int e = ev[j];
+                unsigned m = __match_any_sync(0xffffffffu, e);
+                int p = 0;
+                if (e >= 0) p = row[e] + __popc(m & lt_mask);
+                __syncwarp();
+                if (e >= 0) {
+                    ids_dst[p] = i;
+                    ids_src1[p] = (mode == MOE_BROADCAST) ? i / k : i;
+                    if (slot_prow) slot_prow[i] = p + pad_delta[e];
+                    if ((m & lt_mask) == 0) row[e] += __popc(m);
+                }
+                __syncwarp();
+            }
         }
     }
 }

@@ -39,7 +39,7 @@ def test_expired_wait_reports_timeout_and_the_device_recovers(stage):
     assert st == moe.ERR_TIMEOUT
     site = int(ws[12:16].view(torch.int32).item())  # header word 3
     assert site >> 30 == 1, hex(site)
-    assert 0 <= (site >> 20) & 0x3ff < 9  # a warp of the 288-thread mat-vec CTA
+    assert 0 <= (site >> 20) & 0x3ff < 17  # a warp of the 544-thread mat-vec CTA
     # the device answers, and the same call on a re-initialised workspace is correct
     torch.cuda.synchronize()
     assert lib.moe_workspace_init(ws.data_ptr(), None) == moe.OK
