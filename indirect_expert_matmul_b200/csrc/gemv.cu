@@ -32,6 +32,8 @@
 // dst[t][s]), or dual gate/up with a SwiGLU epilogue writing bf16 h[t][s].
 #include <atomic>
 
+#include <cudaTypedefs.h>
+
 #include "common.cuh"
 #include "gemv_args.cuh"
 #include "moe_testing.h"
@@ -221,11 +223,10 @@ struct Routing {
 };
 
 // Warp-level distinct-expert scan for up to 64 slots (every lane of the warp).
-__device__ __forceinline__ void routing_fast(Routing& R, const int32_t* ids, int S, int E, int* status) {
+// v0, v1: the ids of slots lane and lane + 32 (loaded by the caller; -1 past S).
+__device__ __forceinline__ void routing_fast(Routing& R, int v0, int v1, int S, int E, int* status) {
     const int lane = threadIdx.x & 31;
     const uint32_t lt = (1u << lane) - 1u;
-    int v0 = lane < S ? __ldg(ids + lane) : -1;
-    int v1 = lane + 32 < S ? __ldg(ids + lane + 32) : -1;
     const bool bad = (lane < S && (v0 < 0 || v0 >= E)) || (lane + 32 < S && (v1 < 0 || v1 >= E));
     if (__any_sync(0xffffffffu, bad) && lane == 0) set_status(status, MOE_ERR_BAD_ID);
     if (v0 >= E) v0 = -1;
@@ -361,7 +362,7 @@ struct GvItem {
 // One CTA of 544 threads an SM.
 template <int DUAL, int XB, int WT>
 __global__ void __launch_bounds__(kGvThreads, 1)
-gemv_kernel(const GemvArgs a) {
+gemv_kernel(const __grid_constant__ GemvArgs a) {
     extern __shared__ __align__(128) uint8_t sm[];
     constexpr int NMAT = DUAL + 1;
     int* status = a.hdr + kHdrStatus;
@@ -390,12 +391,18 @@ gemv_kernel(const GemvArgs a) {
     if (a.pdl_trigger) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     // a sticky error stops the launch; one read, shared, so that the exit is
     // uniform (the other launch of the FFN may write the word meanwhile)
+    // (the ids of a small call are loaded first, so that both loads are in flight together)
+    int id0 = -1, id1 = -1;
+    if (S <= kGvFast) {
+        id0 = lane < S ? __ldg(a.ids + lane) : -1;
+        id1 = lane + 32 < S ? __ldg(a.ids + lane + 32) : -1;
+    }
     if (tid == 0) *st_copy = read_status(status);
     __syncthreads();
     if (*st_copy != 0) return;
 
     Routing R;
-    if (S <= kGvFast) routing_fast(R, a.ids, S, a.n_experts, status);
+    if (S <= kGvFast) routing_fast(R, id0, id1, S, a.n_experts, status);
     else routing_slow(R, a.ids, S, a.n_experts, (int*)(sm + lay.tab), status);
 
     // A field of a side, read from the parameter space where it is used (taking
@@ -404,6 +411,10 @@ gemv_kernel(const GemvArgs a) {
 #define GV_SIDE(sh, field) ((sh) ? a.shared.field : a.routed.field)
     const int n_sh = a.has_shared ? a.shared.subs : 0;
     const int n_items = n_sh + R.n * a.routed.subs;
+    // a contiguous range of items a CTA: consecutive items of one expert share
+    // their tokens, so the activation window staged for one serves the next
+    const int it_begin = (int)(((int64_t)blockIdx.x * n_items) / gridDim.x);
+    const int it_end = (int)(((int64_t)(blockIdx.x + 1) * n_items) / gridDim.x);
     // items: the shared expert's sub-tiles first, then each distinct routed expert's
     auto item_of = [&](int it) {  // warp-collective in fast mode
         GvItem f;
@@ -438,7 +449,7 @@ gemv_kernel(const GemvArgs a) {
         // of each matrix: NMAT * kps copies of nrow * 68 bytes.
         uint32_t sc = 0;
         bool ok = true;
-        for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+        for (int it = it_begin; it < it_end && ok; ++it) {
             const GvItem f = item_of(it);
             if (f.nrow == 0) continue;
             int nsl = f.nsl;
@@ -463,15 +474,29 @@ gemv_kernel(const GemvArgs a) {
                     }
                     const int nk = KT - k0 < kps ? KT - k0 : kps;
                     const bool stall = (int)blockIdx.x == a.stall_cta && (int)sc == a.stall_stage;  // test only
-                    if (lane == 0 && !stall) {
-                        ptx::mbar_arrive_expect_tx(&full[s], (uint32_t)(NMAT * nk) * piece);
+                    uint8_t* st_base = ring + (size_t)s * kGvStage;
+                    if (GV_SIDE(f.side, tma)) {
+                        // one tensor copy a matrix: kps k-steps of the sub-tile's lines (a
+                        // last stage past KT reads zeros there and still lands kps pieces)
+                        if (lane == 0 && !stall) {
+                            ptx::mbar_arrive_expect_tx(&full[s], (uint32_t)(NMAT * kps) * piece);
+                            const int line0 = (f.r0 / kSubRows) * 17, tile = f.e * L.mt_count + f.mt;
 #pragma unroll
-                        for (int m = 0; m < NMAT; ++m)
-                            for (int kk = 0; kk < nk; ++kk)
-                                ptx::bulk_g2s(ring + (size_t)s * kGvStage + (size_t)(m * kps + kk) * piece,
-                                              (m ? W1 : W0) + L.block(f.e, f.mt, k0 + kk) +
-                                                  (size_t)f.r0 * L.rb,
-                                              piece, &full[s]);
+                            for (int m = 0; m < NMAT; ++m)
+                                ptx::tma_load_4d(st_base + (size_t)m * kps * piece,
+                                                 f.side ? &a.shared.tm[m] : &a.routed.tm[m], 0, line0, k0, tile,
+                                                 &full[s]);
+                        }
+                    } else {
+                        // one bulk copy a (matrix, k-step), issued by as many lanes
+                        if (lane == 0 && !stall) ptx::mbar_arrive_expect_tx(&full[s], (uint32_t)(NMAT * nk) * piece);
+                        __syncwarp();
+                        if (lane < NMAT * nk && !stall) {
+                            const int m = lane / nk, kk = lane - m * nk;
+                            ptx::bulk_g2s(st_base + (size_t)(m * kps + kk) * piece,
+                                          (m ? W1 : W0) + L.block(f.e, f.mt, k0 + kk) + (size_t)f.r0 * L.rb, piece,
+                                          &full[s]);
+                        }
                     }
                     __syncwarp();
                 }
@@ -508,7 +533,8 @@ gemv_kernel(const GemvArgs a) {
     uint32_t sc = 0;
     bool waited_primary = !a.pdl_secondary;
 
-    for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
+    int staged_side = -1, staged_e = -1;  // the item whose tokens the window holds (one group, one window)
+    for (int it = it_begin; it < it_end; ++it) {
         const GvItem f = item_of(it);
         if (f.nrow == 0) continue;
         const WLayout L = GV_SIDE(f.side, L);
@@ -546,85 +572,91 @@ gemv_kernel(const GemvArgs a) {
             const int nt = nsl - g * kGvNT < kGvNT ? nsl - g * kGvNT : kGvNT;
             float tot[4] = {0.f, 0.f, 0.f, 0.f};  // rows rra, rra+8 x tokens 2tq, 2tq+1
             bool ok = true;
+            // the window still holds this item's tokens (the previous item was the same
+            // expert, in one token group and one window): no restaging
+            const bool one = G == 1 && KT <= kGvXSteps;
+            const bool reuse = one && staged_side == f.side && staged_e == f.e;
             for (int w0 = 0; w0 < KT; w0 += kGvXSteps) {
                 const int nw = KT - w0 < kGvXSteps ? KT - w0 : kGvXSteps;
-                ok = consumers_and(ok && !*abort_flag);  // the previous window is no longer read
-                if (!ok) break;
-                if (!waited_primary) {
-                    asm volatile("griddepcontrol.wait;" ::: "memory");
-                    waited_primary = true;
-                }
-                // stage the nt tokens' activations of this window: each token's largest
-                // magnitude first, then the values times the power of two that puts it in
-                // [2^14, 2^15), rounded to fp16 (exact for 16-bit inputs in range)
-                const int cols = nw * kTileK, col0 = w0 * kTileK;
-                constexpr int VE = 16 / XB;  // elements per 16-byte vector
-                const int vpr = cols / VE;   // vectors per token row
-                const void* xg = GV_SIDE(f.side, x);
-                const int xt = GV_SIDE(f.side, x_type);
-                // every vector of the window is loaded once, into registers (at most 8
-                // tokens x 2048 columns: RV vectors a thread), then converted from there
-                constexpr int RV = XB == 4 ? 8 : 4;
-                uint4 v[RV];
-                int qv[RV];
-#pragma unroll
-                for (int r = 0; r < RV; ++r) {
-                    const int idx = ct + r * kGvConsumers;
-                    qv[r] = -1;
-                    v[r] = make_uint4(0u, 0u, 0u, 0u);
-                    if (idx < nt * vpr) {
-                        const int q = idx / vpr, cc = (idx - q * vpr) * VE, col = col0 + cc;
-                        const int sl = slot_of(g * kGvNT + q);
-                        const int row = f.side == 1 ? sl : (a.routed.x_per_slot ? sl : sl / a.k);
-                        qv[r] = q;
-                        if (col < L.n_in)
-                            v[r] = __ldg((const uint4*)((const uint8_t*)xg + ((size_t)row * L.n_in + col) * XB));
+                if (!reuse) {
+                    ok = consumers_and(ok && !*abort_flag);  // the previous window is no longer read
+                    if (!ok) break;
+                    if (!waited_primary) {
+                        asm volatile("griddepcontrol.wait;" ::: "memory");
+                        waited_primary = true;
                     }
-                }
-                auto unpack = [&](const uint4& u, float (&e)[8]) {
-                    if (XB == 4) {
-                        e[0] = __uint_as_float(u.x); e[1] = __uint_as_float(u.y);
-                        e[2] = __uint_as_float(u.z); e[3] = __uint_as_float(u.w);
-                    } else {
-                        const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-                        for (int b = 0; b < 4; ++b) {
-                            e[2 * b] = ld_x16(uw[b] & 0xffffu, xt);
-                            e[2 * b + 1] = ld_x16(uw[b] >> 16, xt);
+                    // stage the nt tokens' activations of this window: each token's largest
+                    // magnitude first, then the values times the power of two that puts it in
+                    // [2^14, 2^15), rounded to fp16 (exact for 16-bit inputs in range)
+                    const int cols = nw * kTileK, col0 = w0 * kTileK;
+                    constexpr int VE = 16 / XB;  // elements per 16-byte vector
+                    const int vpr = cols / VE;   // vectors per token row
+                    const void* xg = GV_SIDE(f.side, x);
+                    const int xt = GV_SIDE(f.side, x_type);
+                    // every vector of the window is loaded once, into registers (at most 8
+                    // tokens x 2048 columns: RV vectors a thread), then converted from there
+                    constexpr int RV = XB == 4 ? 8 : 4;
+                    uint4 v[RV];
+                    int qv[RV];
+    #pragma unroll
+                    for (int r = 0; r < RV; ++r) {
+                        const int idx = ct + r * kGvConsumers;
+                        qv[r] = -1;
+                        v[r] = make_uint4(0u, 0u, 0u, 0u);
+                        if (idx < nt * vpr) {
+                            const int q = idx / vpr, cc = (idx - q * vpr) * VE, col = col0 + cc;
+                            const int sl = slot_of(g * kGvNT + q);
+                            const int row = f.side == 1 ? sl : (a.routed.x_per_slot ? sl : sl / a.k);
+                            qv[r] = q;
+                            if (col < L.n_in)
+                                v[r] = __ldg((const uint4*)((const uint8_t*)xg + ((size_t)row * L.n_in + col) * XB));
                         }
                     }
-                };
-#pragma unroll
-                for (int r = 0; r < RV; ++r) {
-                    if (qv[r] < 0) continue;
-                    float e[8];
-                    unpack(v[r], e);
-                    float mx = 0.f;
-#pragma unroll
-                    for (int i = 0; i < VE; ++i) mx = fmaxf(mx, fabsf(e[i]));
-                    if (mx > 0.f) atomicMax(&xmax[qv[r]], __float_as_int(mx));
-                }
-                consumers_sync();
-#pragma unroll
-                for (int r = 0; r < RV; ++r) {
-                    if (qv[r] < 0) continue;
-                    const int q = qv[r], idx = ct + r * kGvConsumers;
-                    float e[8];
-                    unpack(v[r], e);
-                    const float sinv = ldexpf(1.0f, -scale_exp(__int_as_float(xmax[q])));
-                    uint32_t hv[4];
-#pragma unroll
-                    for (int i = 0; i < VE / 2; ++i) {
-                        const __half2 hh = __floats2half2_rn(e[2 * i] * sinv, e[2 * i + 1] * sinv);
-                        hv[i] = *(const uint32_t*)&hh;
+                    auto unpack = [&](const uint4& u, float (&e)[8]) {
+                        if (XB == 4) {
+                            e[0] = __uint_as_float(u.x); e[1] = __uint_as_float(u.y);
+                            e[2] = __uint_as_float(u.z); e[3] = __uint_as_float(u.w);
+                        } else {
+                            const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
+    #pragma unroll
+                            for (int b = 0; b < 4; ++b) {
+                                e[2 * b] = ld_x16(uw[b] & 0xffffu, xt);
+                                e[2 * b + 1] = ld_x16(uw[b] >> 16, xt);
+                            }
+                        }
+                    };
+    #pragma unroll
+                    for (int r = 0; r < RV; ++r) {
+                        if (qv[r] < 0) continue;
+                        float e[8];
+                        unpack(v[r], e);
+                        float mx = 0.f;
+    #pragma unroll
+                        for (int i = 0; i < VE; ++i) mx = fmaxf(mx, fabsf(e[i]));
+                        if (mx > 0.f) atomicMax(&xmax[qv[r]], __float_as_int(mx));
                     }
-                    uint8_t* dstx = sxb + (size_t)q * kGvXRow + (size_t)(idx - q * vpr) * VE * 2;
-                    if (XB == 4) *(uint2*)dstx = make_uint2(hv[0], hv[1]);
-                    else *(uint4*)dstx = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+                    consumers_sync();
+    #pragma unroll
+                    for (int r = 0; r < RV; ++r) {
+                        if (qv[r] < 0) continue;
+                        const int q = qv[r], idx = ct + r * kGvConsumers;
+                        float e[8];
+                        unpack(v[r], e);
+                        const float sinv = ldexpf(1.0f, -scale_exp(__int_as_float(xmax[q])));
+                        uint32_t hv[4];
+    #pragma unroll
+                        for (int i = 0; i < VE / 2; ++i) {
+                            const __half2 hh = __floats2half2_rn(e[2 * i] * sinv, e[2 * i + 1] * sinv);
+                            hv[i] = *(const uint32_t*)&hh;
+                        }
+                        uint8_t* dstx = sxb + (size_t)q * kGvXRow + (size_t)(idx - q * vpr) * VE * 2;
+                        if (XB == 4) *(uint2*)dstx = make_uint2(hv[0], hv[1]);
+                        else *(uint4*)dstx = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+                    }
+                    if (ct < kGvNT) xsc[ct] = ldexpf(1.0f, scale_exp(__int_as_float(xmax[ct])));
+                    consumers_sync();
+                    if (ct < kGvNT) xmax[ct] = 0;  // next written after the next window's first barrier
                 }
-                if (ct < kGvNT) xsc[ct] = ldexpf(1.0f, scale_exp(__int_as_float(xmax[ct])));
-                consumers_sync();
-                if (ct < kGvNT) xmax[ct] = 0;  // next written after the next window's first barrier
                 const float s0 = xsc[2 * tq], s1 = xsc[2 * tq + 1];  // tokens 2tq, 2tq + 1
                 float acc[4] = {0.f, 0.f, 0.f, 0.f};
                 const uint8_t* xrow = sxb + (size_t)gq * kGvXRow + 16 * tq;  // token gq, columns 8tq..
@@ -707,6 +739,8 @@ gemv_kernel(const GemvArgs a) {
                 }
                 // a failed wait is acted on at the next barrier, which every consumer reaches
             }
+            staged_side = one ? f.side : -1;
+            staged_e = f.e;
             // per-warp totals, then each (row, token) adds its k-step residues in order
 #pragma unroll
             for (int i = 0; i < 4; ++i) red[((kr * P + pr) * 32 + lane) * 4 + i] = tot[i];
@@ -801,6 +835,50 @@ static int gv_sm_count() {
     return n > 0 ? n : 148;
 }
 
+// cuTensorMapEncodeTiled from the driver, fetched once through the runtime.
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::atomic<int> tried{0};
+    if (!fn && !tried.exchange(1)) {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = (PFN_cuTensorMapEncodeTiled_v12000)f;
+    }
+    return fn;
+}
+
+// Tensor maps of a side's weight matrices over the repacked layout seen as
+// [expert x row tile][k-step][line][inner bytes] (uint8): a k-step block of a
+// 128-row tile is 68 lines of inner = 32 rb / 17 bytes (128 for Q8_0, 64 for
+// MXFP4), a 32-row sub-block 17 of them.  The box is a sub-tile's lines for
+// kps k-steps of one tile.  Only when every row tile is full (one stride per
+// dimension); otherwise the side keeps the per-k-step bulk copies.
+static void plan_tensor_maps(GemvSide& sd, int n_experts, int nmat) {
+    sd.tma = 0;
+    const WLayout& L = sd.L;
+    if (L.n_out_pad % kTileM != 0) return;
+    const uint8_t* W[2] = {sd.W0, sd.W1};
+    for (int m = 0; m < nmat; ++m)
+        if (!W[m] || ((uintptr_t)W[m] & 15)) return;
+    auto enc = tensor_map_encoder();
+    if (!enc) return;
+    const cuuint64_t inner = (cuuint64_t)L.rb * kSubRows / 17, blk = (cuuint64_t)kTileM * L.rb;
+    cuuint64_t dims[4] = {inner, blk / inner, (cuuint64_t)L.kt_count, (cuuint64_t)n_experts * L.mt_count};
+    cuuint64_t strides[3] = {inner, blk, blk * (cuuint64_t)L.kt_count};
+    cuuint32_t box[4] = {(cuuint32_t)inner, (cuuint32_t)(17 * (sd.rsub / kSubRows)), (cuuint32_t)sd.kps, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    for (int m = 0; m < nmat; ++m) {
+        if (enc(&sd.tm[m], CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<uint8_t*>(W[m]), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return;
+    }
+    sd.tma = 1;
+}
+
 // test-only stall (moe_testing_stall): CTA, stage, wait limit in microseconds
 static std::atomic<int> g_stall_cta{-1}, g_stall_stage{0}, g_stall_wait_us{0};
 
@@ -833,6 +911,8 @@ moe_status launch_gemv(const GemvArgs& in, cudaStream_t stream) {
     a.routed.subs = a.routed.L.mt_count * (kTileM / a.routed.rsub);
     a.routed.kps = stage_ksteps(a.routed.L, a.routed.rsub, nmat);
     if (a.wait_limit <= 0) a.wait_limit = kGvWaitLimit;
+    plan_tensor_maps(a.routed, a.n_experts, nmat);
+    if (a.has_shared) plan_tensor_maps(a.shared, 1, nmat);
 
     const uint32_t fixed = gv_lay(0, S, a.n_experts).total;
     int ns = (int)((kGvSmemBudget - fixed - 2 * 8 * 8) / kGvStage);

@@ -1,5 +1,7 @@
 // Argument block of the expert mat-vec kernel (gemv.cu).
 #pragma once
+#include <cuda.h>
+
 #include "common.cuh"
 
 namespace moe {
@@ -20,6 +22,11 @@ struct GemvSide {
     int rsub;           // rows per work item: 32, 64 or 128
     int subs;           // work items per expert (row sub-tiles, counting empty ones of a tail tile)
     int kps;            // k-steps per ring stage
+    // tensor maps of W0 / W1 over [tile][k-step][line][inner bytes] (filled by
+    // launch_gemv when every row tile is full): one copy fetches a stage's
+    // k-steps of a sub-tile; tma = 0: one bulk copy per k-step instead
+    CUtensorMap tm[2];
+    int tma;
 };
 
 struct GemvArgs {

@@ -102,6 +102,17 @@ __device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
+// One box of a 4-D tensor map (coordinates innermost first) into dst, completing
+// its bytes on bar.  No multicast: the box lands in this CTA's shared memory.
+__device__ __forceinline__ void tma_load_4d(void* dst, const void* tmap, int c0, int c1, int c2, int c3,
+                                            uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_u32(dst)),
+        "l"(tmap), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
+        : "memory");
+}
+
 // Four rows (row0..row3) of a 2-D tensor map, one box wide starting at column
 // col, into consecutive box-sized slots at dst (tile::gather4).
 __device__ __forceinline__ void tma_gather4(void* dst, const void* tmap, int col, int r0, int r1, int r2, int r3,
