@@ -44,7 +44,7 @@ namespace moe {
 constexpr int kGvConsumers = 512;
 constexpr int kGvThreads = 32 + kGvConsumers;  // warp 0: producer
 constexpr uint32_t kGvStage = 512 * kRowBytes;  // 34816 bytes: 512 (row, k-step) pieces of Q8_0
-constexpr uint32_t kGvSmemBudget = 216 * 1024;
+constexpr uint32_t kGvSmemBudget = 224 * 1024;
 constexpr long long kGvWaitLimit = 1ll << 32;   // ~2 s
 constexpr int kGvFast = 64;                     // slots up to which the experts come from warp ballots
 constexpr int kGvXSteps = 32;                   // k-steps of the activation window (2048 columns)
@@ -62,7 +62,7 @@ __host__ __device__ inline GvLay gv_lay(int ns, int S, int n_experts) {
     uint32_t o = 0;
     m.ring = o; o += (uint32_t)ns * kGvStage;
     m.x = o; o += kGvXBytes;
-    m.red = o; o += kGvRedBytes;
+    m.red = o; o += 2 * kGvRedBytes;  // two buffers: an item writes one while the last is still read
     m.tab = o;
     if (S > kGvFast) o += (uint32_t)(((n_experts + 31) / 32) * 2 + 2 + 2 * (S + 1) + 2 * S) * 4u;
     o = (o + 15u) & ~15u;
@@ -236,10 +236,11 @@ __device__ __forceinline__ void routing_fast(Routing& R, int v0, int v1, int S, 
     const uint32_t m0 = __match_any_sync(0xffffffffu, v0), m1 = __match_any_sync(0xffffffffu, v1);
     bool f0 = v0 >= 0 && (m0 & lt) == 0u;
     bool f1 = v1 >= 0 && (m1 & lt) == 0u;
-    for (int i = 0; i < 32; ++i) {  // an expert of the second half seen in the first is not new
-        const int o = __shfl_sync(0xffffffffu, v0, i);
-        if (o == v1) f1 = false;
-    }
+    if (S > 32)  // an expert of the second half seen in the first is not new
+        for (int i = 0; i < 32; ++i) {
+            const int o = __shfl_sync(0xffffffffu, v0, i);
+            if (o == v1) f1 = false;
+        }
     R.v0 = v0;
     R.v1 = v1;
     R.fb0 = __ballot_sync(0xffffffffu, f0);
@@ -468,7 +469,9 @@ gemv_kernel(const __grid_constant__ GemvArgs a) {
             for (int g = 0; g < G && ok; ++g)
                 for (int k0 = 0; k0 < KT; k0 += kps, ++sc) {
                     const int s = (int)(sc % (uint32_t)a.ns);
-                    if (!gv_warp_wait(&empty[s], ((sc / a.ns) & 1u) ^ 1u, status, abort_flag, a.wait_limit)) {
+                    // (the first ns stages are fresh: nothing to wait for)
+                    if (sc >= (uint32_t)a.ns &&
+                        !gv_warp_wait(&empty[s], ((sc / a.ns) & 1u) ^ 1u, status, abort_flag, a.wait_limit)) {
                         ok = false;
                         break;
                     }
@@ -530,7 +533,7 @@ gemv_kernel(const __grid_constant__ GemvArgs a) {
     int* xmax = (int*)(sm + lay.x + kGvNT * kGvXRow);  // [kGvNT]: max |x| of the window (float bits)
     float* xsc = (float*)(xmax + kGvNT);               // [kGvNT]: the factor that undoes the scaling
     if (ct < kGvNT) xmax[ct] = 0;             // ordered before first use by the window barrier
-    uint32_t sc = 0;
+    uint32_t sc = 0, rbuf = 0;
     bool waited_primary = !a.pdl_secondary;
 
     int staged_side = -1, staged_e = -1;  // the item whose tokens the window holds (one group, one window)
@@ -742,8 +745,10 @@ gemv_kernel(const __grid_constant__ GemvArgs a) {
             staged_side = one ? f.side : -1;
             staged_e = f.e;
             // per-warp totals, then each (row, token) adds its k-step residues in order
+            float* rd = red + (rbuf & 1u) * (kGvRedBytes / 4);  // alternate buffers: no barrier after the reads
+            ++rbuf;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) red[((kr * P + pr) * 32 + lane) * 4 + i] = tot[i];
+            for (int i = 0; i < 4; ++i) rd[((kr * P + pr) * 32 + lane) * 4 + i] = tot[i];
             if (!consumers_and(ok && !*abort_flag)) return;  // uniform
             for (int idx = ct; idx < rsub * nt; idx += kGvConsumers) {
                 const int r = idx % rsub, q = idx / rsub;
@@ -755,7 +760,7 @@ gemv_kernel(const __grid_constant__ GemvArgs a) {
 #pragma unroll
                 for (int m = 0; m < NMAT; ++m) {
                     float t = 0.f;
-                    for (int k2 = 0; k2 < W; ++k2) t += red[((k2 * P + m * nrg + rgi) * 32 + ln) * 4 + ii];
+                    for (int k2 = 0; k2 < W; ++k2) t += rd[((k2 * P + m * nrg + rgi) * 32 + ln) * 4 + ii];
                     v[m] = t;
                 }
                 const int sl = slot_of(g * kGvNT + q);
@@ -766,7 +771,8 @@ gemv_kernel(const __grid_constant__ GemvArgs a) {
                     GV_SIDE(f.side, out)[(int64_t)sl * L.n_out + n] = v[0];
                 }
             }
-            consumers_sync();  // red is free again
+            // (the buffer just read is written again two groups later, after the next
+            // group's barrier, which every consumer reaches only after these reads)
         }
     }
 #undef GV_SIDE
