@@ -13,6 +13,7 @@
 // The result is unique (ascending (t, s) inside each expert), independent of
 // scheduling, and uses no global atomics.
 #include "common.cuh"
+#include "warp_match.cuh"
 
 namespace moe {
 
@@ -71,6 +72,7 @@ row_ids_kernel(const int32_t* __restrict__ ids, int S, int k, int E, int mode, i
     const int c0 = warp * L;
     const int c1 = min(S, c0 + L);
     const unsigned lt_mask = (1u << lane) - 1u;
+    const int nb = E > 1 ? 32 - __clz(E - 1) : 1;  // bits of the largest id
 
     // pass 1: per-chunk histogram (the ids of kBatch 32-slot steps are loaded
     // together, so their load latencies overlap)
@@ -89,7 +91,7 @@ row_ids_kernel(const int32_t* __restrict__ ids, int S, int k, int E, int mode, i
                 const int i = b0 + 32 * j + lane;
                 int e = ev[j];
                 if (i < c1 && (e < 0 || e >= E)) { my_bad = 1; e = -1; }
-                unsigned m = __match_any_sync(0xffffffffu, e);
+                unsigned m = match_by_ballots(e, nb);
                 if (e >= 0 && (m & lt_mask) == 0) row[e] += __popc(m);
                 __syncwarp();
             }
@@ -168,7 +170,7 @@ row_ids_kernel(const int32_t* __restrict__ ids, int S, int k, int E, int mode, i
             for (int j = 0; j < kBatch; ++j) {
                 const int i = b0 + 32 * j + lane;
                 const int e = ev[j];
-                unsigned m = __match_any_sync(0xffffffffu, e);
+                unsigned m = match_by_ballots(e, nb);
                 int p = 0;
                 if (e >= 0) p = row[e] + __popc(m & lt_mask);
                 __syncwarp();
