@@ -452,11 +452,16 @@ gemv_kernel(const __grid_constant__ GemvArgs a) {
         }
         const int rsub = f.side ? a.shared.rsub : a.routed.rsub;
         const WLayout L = f.side ? a.shared.L : a.routed.L;
-        const int per_tile = kTileM / rsub;
-        f.mt = u / per_tile;
-        f.r0 = (u - f.mt * per_tile) * rsub;
-        const int rows = L.rows(f.mt);
-        f.nrow = rows - f.r0 < rsub ? rows - f.r0 : rsub;
+        if (rsub > kTileM) {  // a pair of full tiles
+            f.mt = 2 * u;
+            f.r0 = 0;
+        } else {
+            const int per_tile = kTileM / rsub;
+            f.mt = u / per_tile;
+            f.r0 = (u - f.mt * per_tile) * rsub;
+        }
+        const int rows = L.n_out_pad - (f.mt * kTileM + f.r0);  // rows from the item's first to the end
+        f.nrow = rows < rsub ? rows : rsub;
         if (f.nrow < 0) f.nrow = 0;
         return f;
     };
@@ -582,12 +587,16 @@ gemv_kernel(const __grid_constant__ GemvArgs a) {
         const int pr = cw % P, kr = cw / P;
         const int mw = pr / nrg, rg = pr - mw * nrg;
         const bool live = 16 * rg < f.nrow;
-        // the row group inside the stage piece: sub-block (r0 + 16 rg) / 32 of the tile
-        const int sbk = (f.r0 + 16 * rg) / kSubRows;
-        const int nr = sub_rows(L.rows(f.mt), sbk);
-        const uint32_t roff = (uint32_t)((16 * rg / kSubRows) * L.sub_bytes());
-        const int rra = (16 * rg) % kSubRows + gq;  // rows rra and rra + 8 of the sub-block
-        const uint32_t piece = (uint32_t)f.nrow * L.rb;
+        // the row group's tile (a 256-row item spans two) and row inside it; a
+        // k-step of a stage holds one piece per matrix, or per tile of a pair
+        const int tt = (16 * rg) / kTileM, rin = (16 * rg) % kTileM;
+        const int pm = NMAT == 2 ? mw : tt;
+        // the row group inside its piece: sub-block (r0 + rin) / 32 of the tile
+        const int sbk = (f.r0 + rin) / kSubRows;
+        const int nr = sub_rows(L.rows(f.mt + tt), sbk);
+        const uint32_t roff = (uint32_t)((rin / kSubRows) * L.sub_bytes());
+        const int rra = rin % kSubRows + gq;  // rows rra and rra + 8 of the sub-block
+        const uint32_t piece = (uint32_t)(f.nrow < kTileM ? f.nrow : kTileM) * L.rb;
         const int G = (nsl + kGvNT - 1) / kGvNT;
         for (int g = 0; g < G; ++g) {
             const int nt = nsl - g * kGvNT < kGvNT ? nsl - g * kGvNT : kGvNT;
@@ -690,7 +699,7 @@ gemv_kernel(const __grid_constant__ GemvArgs a) {
                     }
                     if (live) {
                         for (int kk = kr; kk < nk; kk += W) {
-                            const uint8_t* pc = ring + (size_t)s * kGvStage + (size_t)(mw * kps + kk) * piece + roff;
+                            const uint8_t* pc = ring + (size_t)s * kGvStage + (size_t)(pm * kps + kk) * piece + roff;
                             const uint8_t* xk = xrow + (size_t)(k0 - w0 + kk) * kTileK * 2;
                             const uint4 xb[2] = {*(const uint4*)xk, *(const uint4*)(xk + 64)};
                             if (WT == MOE_MXFP4) {
@@ -796,15 +805,28 @@ gemv_kernel(const __grid_constant__ GemvArgs a) {
 #undef GV_SIDE
 }
 
-// Rows per item of the routed side: the largest of 128, 64, 32 whose items
-// (over at most `experts` experts, plus the shared side's) come to at least
-// 0.9 of the SMs, else 32.
-static int pick_rsub(const WLayout& L, int64_t experts, int64_t other_items, int sms) {
-    for (int r : {128, 64}) {
-        const int64_t items = experts * L.mt_count * (kTileM / r) + other_items;
-        if (items * 10 >= (int64_t)sms * 9) return r;
+// Rows per item of the routed side: 256 (a pair of full tiles, single-matrix
+// sides only), 128, 64 or 32.  A CTA streams a contiguous range of items and
+// the launch ends with its fullest CTA: ceil(items / SMs) items, each costing
+// its bytes plus a fixed cost (decode, activation window, reduction) worth
+// about 64 KB of stream.  The height with the least such cost wins (the
+// larger one on a tie); `experts` is an upper bound on the distinct experts.
+static int pick_rsub(const WLayout& L, int nmat, int64_t experts, int64_t other_items, int sms, bool pairs) {
+    constexpr int64_t kItemCost = 64 * 1024;
+    int best = 32;
+    int64_t best_cost = -1;
+    for (int r : {256, 128, 64, 32}) {
+        if (r > kTileM && !pairs) continue;
+        const int64_t per_expert = r > kTileM ? L.mt_count / 2 : (int64_t)L.mt_count * (kTileM / r);
+        const int64_t items = experts * per_expert + other_items;
+        const int64_t per_cta = (items + sms - 1) / sms;
+        const int64_t cost = per_cta * ((int64_t)r * L.kt_count * L.rb * nmat + kItemCost);
+        if (best_cost < 0 || cost < best_cost) {
+            best = r;
+            best_cost = cost;
+        }
     }
-    return 32;
+    return best;
 }
 
 // k-steps per ring stage: as many as fill kGvStage bytes with the sub-tile's
@@ -892,7 +914,10 @@ static void plan_tensor_maps(GemvSide& sd, int n_experts, int nmat) {
     const cuuint64_t inner = (cuuint64_t)L.rb * kSubRows / 17, blk = (cuuint64_t)kTileM * L.rb;
     cuuint64_t dims[4] = {inner, blk / inner, (cuuint64_t)L.kt_count, (cuuint64_t)n_experts * L.mt_count};
     cuuint64_t strides[3] = {inner, blk, blk * (cuuint64_t)L.kt_count};
-    cuuint32_t box[4] = {(cuuint32_t)inner, (cuuint32_t)(17 * (sd.rsub / kSubRows)), (cuuint32_t)sd.kps, 1};
+    // a 256-row item: the full lines of two consecutive tiles
+    const int rt = sd.rsub < kTileM ? sd.rsub : kTileM;
+    cuuint32_t box[4] = {(cuuint32_t)inner, (cuuint32_t)(17 * (rt / kSubRows)), (cuuint32_t)sd.kps,
+                         (cuuint32_t)(sd.rsub / rt)};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     for (int m = 0; m < nmat; ++m) {
         if (enc(&sd.tm[m], CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<uint8_t*>(W[m]), dims, strides, box, estr,
@@ -931,11 +956,18 @@ moe_status launch_gemv(const GemvArgs& in, cudaStream_t stream) {
         a.shared.kps = stage_ksteps(a.shared.L, a.shared.rsub, nmat);
         sh_items = a.shared.subs;
     }
-    a.routed.rsub = pick_rsub(a.routed.L, a.max_distinct, sh_items, sms);
-    a.routed.subs = a.routed.L.mt_count * (kTileM / a.routed.rsub);
-    a.routed.kps = stage_ksteps(a.routed.L, a.routed.rsub, nmat);
+    // tile pairs: one matrix, every tile full and an even count of them, the
+    // copies by tensor map (the only copy path that fetches two tiles at once)
+    const bool pairs = nmat == 1 && a.routed.L.n_out_pad % (2 * kTileM) == 0;
+    auto plan_routed = [&](int rsub) {
+        a.routed.rsub = rsub;
+        a.routed.subs = rsub > kTileM ? a.routed.L.mt_count / 2 : a.routed.L.mt_count * (kTileM / rsub);
+        a.routed.kps = stage_ksteps(a.routed.L, rsub, nmat);
+        plan_tensor_maps(a.routed, a.n_experts, nmat);
+    };
+    plan_routed(pick_rsub(a.routed.L, nmat, a.max_distinct, sh_items, sms, pairs));
+    if (a.routed.rsub > kTileM && !a.routed.tma) plan_routed(kTileM);
     if (a.wait_limit <= 0) a.wait_limit = kGvWaitLimit;
-    plan_tensor_maps(a.routed, a.n_experts, nmat);
     if (a.has_shared) plan_tensor_maps(a.shared, 1, nmat);
 
     const uint32_t fixed = gv_lay(0, S, a.n_experts).total;
