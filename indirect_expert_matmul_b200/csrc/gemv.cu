@@ -771,6 +771,23 @@ gemv_kernel(const __grid_constant__ GemvArgs a) {
             }
             staged_side = one ? f.side : -1;
             staged_e = f.e;
+            if (NMAT == 1 && W == 1) {
+                // every k-step of the row group was this warp's: its totals are the
+                // results, stored without a reduction or a barrier (a failed wait is
+                // acted on at the next window's barrier, or ends with the range)
+                if (ok && live) {
+                    const int sl0 = 2 * tq < nt ? slot_of(g * kGvNT + 2 * tq) : 0;
+                    const int sl1 = 2 * tq + 1 < nt ? slot_of(g * kGvNT + 2 * tq + 1) : 0;
+#pragma unroll
+                    for (int ii = 0; ii < 4; ++ii) {
+                        const int r = 16 * rg + gq + 8 * (ii >> 1), q = 2 * tq + (ii & 1);
+                        const int n = f.mt * kTileM + f.r0 + r;
+                        if (r < f.nrow && n < L.n_out && q < nt)
+                            GV_SIDE(f.side, out)[(int64_t)((ii & 1) ? sl1 : sl0) * L.n_out + n] = tot[ii];
+                    }
+                }
+                continue;
+            }
             // per-warp totals, then each (row, token) adds its k-step residues in order
             float* rd = red + (rbuf & 1u) * (kGvRedBytes / 4);  // alternate buffers: no barrier after the reads
             ++rbuf;
