@@ -471,7 +471,9 @@ gemv_kernel(const __grid_constant__ GemvArgs a) {
         // Every lane runs the loop (the item decode is warp-collective); lane 0
         // issues the copies.  A stage holds kps k-steps of the sub-tile's rows
         // of each matrix: NMAT * kps copies of nrow * 68 bytes.
-        uint32_t sc = 0;
+        // stage counter, its ring slot and the slot's phase (advanced together:
+        // a division by the runtime ring depth per stage costs every warp)
+        uint32_t sc = 0, slot = 0, ph = 0;
         bool ok = true;
         for (int it = it_begin; it < it_end && ok; ++it) {
             const GvItem f = item_of(it);
@@ -491,10 +493,10 @@ gemv_kernel(const __grid_constant__ GemvArgs a) {
             const uint32_t piece = (uint32_t)f.nrow * L.rb;
             for (int g = 0; g < G && ok; ++g)
                 for (int k0 = 0; k0 < KT; k0 += kps, ++sc) {
-                    const int s = (int)(sc % (uint32_t)a.ns);
+                    const int s = (int)slot;
                     // (the first ns stages are fresh: nothing to wait for)
                     if (sc >= (uint32_t)a.ns &&
-                        !gv_warp_wait(&empty[s], ((sc / a.ns) & 1u) ^ 1u, status, abort_flag, a.wait_limit)) {
+                        !gv_warp_wait(&empty[s], ph ^ 1u, status, abort_flag, a.wait_limit)) {
                         ok = false;
                         break;
                     }
@@ -525,6 +527,10 @@ gemv_kernel(const __grid_constant__ GemvArgs a) {
                         }
                     }
                     __syncwarp();
+                    if (++slot == (uint32_t)a.ns) {
+                        slot = 0;
+                        ph ^= 1u;
+                    }
                 }
         }
         // every copy issued lands before the CTA can exit (bounded; a stage the
@@ -556,7 +562,7 @@ gemv_kernel(const __grid_constant__ GemvArgs a) {
     int* xmax = (int*)(sm + lay.x + kGvNT * kGvXRow);  // [kGvNT]: max |x| of the window (float bits)
     float* xsc = (float*)(xmax + kGvNT);               // [kGvNT]: the factor that undoes the scaling
     if (ct < kGvNT) xmax[ct] = 0;             // ordered before first use by the window barrier
-    uint32_t sc = 0, rbuf = 0;
+    uint32_t slot = 0, ph = 0, rbuf = 0;  // ring slot and its phase, advanced per stage
     bool waited_primary = !a.pdl_secondary;
 
     int staged_side = -1, staged_e = -1;  // the item whose tokens the window holds (one group, one window)
@@ -690,10 +696,15 @@ gemv_kernel(const __grid_constant__ GemvArgs a) {
                 const float s0 = xsc[2 * tq], s1 = xsc[2 * tq + 1];  // tokens 2tq, 2tq + 1
                 float acc[4] = {0.f, 0.f, 0.f, 0.f};
                 const uint8_t* xrow = sxb + (size_t)gq * kGvXRow + 16 * tq;  // token gq, columns 8tq..
-                for (int k0 = w0; k0 < w0 + nw; k0 += kps, ++sc) {
+                for (int k0 = w0; k0 < w0 + nw; k0 += kps) {
                     const int nk = KT - k0 < kps ? KT - k0 : kps;
-                    const int s = (int)(sc % (uint32_t)a.ns);
-                    if (!gv_warp_wait(&full[s], (sc / a.ns) & 1u, status, abort_flag, a.wait_limit)) {
+                    const int s = (int)slot;
+                    const uint32_t par = ph;
+                    if (++slot == (uint32_t)a.ns) {
+                        slot = 0;
+                        ph ^= 1u;
+                    }
+                    if (!gv_warp_wait(&full[s], par, status, abort_flag, a.wait_limit)) {
                         ok = false;
                         break;
                     }
