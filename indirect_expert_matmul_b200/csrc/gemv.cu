@@ -8,13 +8,14 @@
 //  - the down launch is a programmatic dependent of gate/up: its CTAs start as
 //    gate/up's leave the SMs, their producers stream the down weights at once
 //    and only their consumers wait for gate/up's h;
-//  - a work item is (routed expert, row sub-tile of 32, 64 or 128 rows) or
-//    (shared expert, row sub-tile), always over the whole K, so no item needs
-//    another's partial sums; the sub-tile height is chosen per launch so that
-//    the items cover the SMs;
-//  - one producer warp streams 34 KB stages (the sub-tile's rows for several
-//    k-steps of each matrix: one bulk copy per k-step and matrix, the rows of
-//    a sub-tile being contiguous in the repacked layout) through a ring,
+//  - a work item is (routed expert, row sub-tile of 32, 64 or 128 rows, or a
+//    pair of full 128-row tiles for a single matrix) or (shared expert, row
+//    sub-tile), always over the whole K, so no item needs another's partial
+//    sums; the height is chosen per launch from an estimate of the fullest
+//    CTA's stream (its items' bytes plus a fixed cost per item);
+//  - one producer warp streams 34 KB stages (the item's rows for several
+//    k-steps of each matrix: one tensor copy per matrix, or one bulk copy per
+//    k-step and matrix where a tensor map does not apply) through a ring,
 //    running ahead across items;
 //  - 16 consumer warps on the tensor cores (mma.sync m16n8k16, fp16 in, fp32
 //    out): A = 16 weight rows of quantised values, exact in fp16; B = up to 8
@@ -22,7 +23,9 @@
 //    range; each 32-column block's product is multiplied by its block scales
 //    in fp32.  A warp owns one (matrix, 16-row group) and every W-th k-step;
 //    the warps of a group are added in a fixed order, so results do not
-//    depend on timing.
+//    depend on timing (with W = 1 on a single matrix the warp stores its
+//    totals itself).  The consumers are bound by instruction issue, so the
+//    per-stage bookkeeping is kept to additions and compares.
 // The distinct routed experts come from ids directly: for up to 64 slots every
 // warp finds them with ballots in its own registers (no block-wide pass before
 // the first copy); for more slots a block-wide pass builds tables in shared
@@ -78,7 +81,10 @@ __device__ __forceinline__ bool gv_wait(uint64_t* bar, uint32_t parity, int* sta
                                         long long limit) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
-    while (!ptx::mbar_try_wait_sleep(bar, parity, 20000)) {
+    // a short sleep between polls: the consumers are issue-bound, and a warp
+    // that polls takes issue slots from the warps on its sub-partition
+    while (!ptx::mbar_try_wait(bar, parity)) {
+        __nanosleep(128);
         if (*abort_flag) return false;
         if (clock64() - t0 > limit) {
             *abort_flag = 1;
