@@ -223,14 +223,17 @@ MOE_API moe_status moe_ffn_w(moe_wtype w_type, const void *Wg, const void *Wu, c
  * Scratch is one static device array in the library (256-byte status header +
  * 256 KB routed hidden activations + 256 KB shared hidden activations, about
  * 512 KB per device); no call allocates or frees memory.
- *   - Only the status header must start at zero: each call clears it with an
- *     asynchronous memset on `stream` before its kernels.  The hidden
+ *   - A call is two kernel launches on `stream` (gate/up, then down), with no
+ *     memset or copy: the status header is zero when the library is loaded,
+ *     and every call leaves it zero - the last CTA of the down launch to
+ *     finish copies the status word out and clears the header.  The hidden
  *     activations need no initial value (the gate/up kernel writes every
- *     element the down kernel reads).
+ *     element the down kernel reads).  If the down launch cannot be enqueued,
+ *     the call enqueues a memset of the header before returning the error.
  *   - status_out (device int, may be NULL): receives the call's device status
- *     (MOE_OK, MOE_ERR_BAD_ID, MOE_ERR_TIMEOUT) by an asynchronous
- *     device-to-device copy at the end of the call; with NULL, device-side
- *     errors are not observable.
+ *     (MOE_OK, MOE_ERR_BAD_ID, MOE_ERR_TIMEOUT), written by that last CTA (for
+ *     n_tokens == 0, by an asynchronous memset to MOE_OK); with NULL,
+ *     device-side errors are not observable.
  *   - All calls on one device share the one scratch array: calls that may
  *     overlap in time (other streams, other host threads) race on it and give
  *     undefined results.  Order them on one stream or serialise them.

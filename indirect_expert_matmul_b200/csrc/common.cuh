@@ -114,6 +114,7 @@ constexpr int kHdrStatus = 0;
 constexpr int kHdrActive = 1;
 constexpr int kHdrTiles = 2;   // total column tiles of the grouped GEMM
 constexpr int kHdrWaitSite = 3;  // first expired wait: 1<<30 | warp<<20 | shared address of its barrier
+constexpr int kHdrDone = 4;      // CTAs of a finalising mat-vec launch that have finished
 constexpr int kGemmBN = 192;   // column (token) tile of the grouped GEMM
 
 // ---------------------------------------------------------------- profiling

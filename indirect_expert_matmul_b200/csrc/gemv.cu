@@ -384,10 +384,9 @@ struct GvItem {
     int nsl;     // slots (routed) or tokens (shared)
 };
 
-// One CTA of 544 threads an SM.
+// The work of one CTA of 544 threads (a return ends the thread's part only).
 template <int DUAL, int XB, int WT>
-__global__ void __launch_bounds__(kGvThreads, 1)
-gemv_kernel(const __grid_constant__ GemvArgs a) {
+__device__ __forceinline__ void gemv_body(const GemvArgs& a) {
     extern __shared__ __align__(128) uint8_t sm[];
     constexpr int NMAT = DUAL + 1;
     int* status = a.hdr + kHdrStatus;
@@ -837,6 +836,36 @@ gemv_kernel(const __grid_constant__ GemvArgs a) {
         }
     }
 #undef GV_SIDE
+}
+
+// The call's status, once every CTA of the finalising launch has finished: the
+// last CTA to finish copies the status word to status_out and clears the
+// header words the launches use, so that the next call starts from zero with
+// no memset or copy of its own (thread 0 of each CTA).
+__device__ __forceinline__ void gemv_finalize(const GemvArgs& a) {
+    // the primary launch's status writes are visible past this wait (a no-op
+    // for a launch that is not a programmatic dependent)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    __threadfence();  // this CTA's writes before its count
+    int* hdr = a.hdr;
+    if (atomicAdd(hdr + kHdrDone, 1) != (int)gridDim.x - 1) return;
+    __threadfence();  // every other CTA's writes before the read
+    const int st = read_status(hdr + kHdrStatus);
+    if (a.status_out) *a.status_out = st;
+    hdr[kHdrStatus] = 0;
+    hdr[kHdrWaitSite] = 0;
+    hdr[kHdrDone] = 0;
+}
+
+// One CTA of 544 threads an SM.
+template <int DUAL, int XB, int WT>
+__global__ void __launch_bounds__(kGvThreads, 1)
+gemv_kernel(const __grid_constant__ GemvArgs a) {
+    gemv_body<DUAL, XB, WT>(a);
+    if (a.finalize) {
+        __syncthreads();
+        if (threadIdx.x == 0) gemv_finalize(a);
+    }
 }
 
 // Rows per item of the routed side: 256 (a pair of full tiles, single-matrix

@@ -40,6 +40,8 @@ struct GemvArgs {
     int pdl_wait;        // may start before the previous kernel of the stream ends: wait first
     int pdl_trigger;     // has a programmatic dependent: let it start once ids are valid
     int pdl_secondary;   // programmatic dependent: consumers wait before reading activations
+    int finalize;        // the last CTA to finish copies the status to status_out and clears the header
+    int* status_out;     // finalize: receives the status word (may be null)
     int* hdr;
     long long wait_limit;  // cycles a bounded wait may take (0: the default, ~2 s)
     int stall_cta, stall_stage;  // test-only: this CTA's producer skips this ring stage (-1: none)

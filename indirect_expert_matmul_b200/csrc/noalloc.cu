@@ -84,9 +84,15 @@ extern "C" moe_status moe_ffn_decode_noalloc(const void* Wg, const void* Wu, con
     int* hdr = (int*)scratch;
     __nv_bfloat16* h = (__nv_bfloat16*)(scratch + kNaHdrBytes);
     __nv_bfloat16* h_sh = (__nv_bfloat16*)(scratch + kNaHdrBytes + kNaHBytes);
-    if (cudaMemsetAsync(hdr, 0, kNaHdrBytes, s) != cudaSuccess) return MOE_ERR_CUDA;
-
-    if (n_tokens > 0) {
+    // The header is zero when the library loads and every call leaves it zero:
+    // the down launch's last CTA copies the status to status_out and clears
+    // it.  So a call is two launches, gate/up a programmatic dependent of
+    // whatever ran before it on the stream.
+    if (n_tokens == 0) {
+        if (status_out && cudaMemsetAsync(status_out, 0, sizeof(int), s) != cudaSuccess) return MOE_ERR_CUDA;
+        return MOE_OK;
+    }
+    {
         const int64_t S = n_tokens * k;
         GemvArgs a = {};
         a.has_shared = has_shared;
@@ -104,7 +110,8 @@ extern "C" moe_status moe_ffn_decode_noalloc(const void* Wg, const void* Wu, con
         a.routed.x_type = x_type;
         a.routed.h = h;
         gemv_plan_side(a.routed, 1);
-        a.pdl_trigger = 1;  // the down launch may start once ids are valid (after the header memset)
+        a.pdl_wait = 1;     // may start during the previous kernel's tail; reads nothing before its wait
+        a.pdl_trigger = 1;  // the down launch may start once ids are valid
         if (has_shared) {
             a.shared.W0 = (const uint8_t*)Sg;
             a.shared.W1 = (const uint8_t*)Su;
@@ -126,6 +133,8 @@ extern "C" moe_status moe_ffn_decode_noalloc(const void* Wg, const void* Wu, con
         b.hdr = hdr;
         b.dual = 0;
         b.pdl_secondary = 1;
+        b.finalize = 1;
+        b.status_out = status_out;
         b.routed.W0 = (const uint8_t*)Wd;
         b.routed.L = WLayout(n_embd, n_ff);
         b.routed.x = h;
@@ -142,10 +151,11 @@ extern "C" moe_status moe_ffn_decode_noalloc(const void* Wg, const void* Wu, con
             gemv_plan_side(b.shared, 0);
         }
         st = launch_gemv(b, s);
-        if (st) return st;
+        if (st) {
+            // gate/up may have written the header: leave it zero for the next call
+            cudaMemsetAsync(hdr, 0, kNaHdrBytes, s);
+            return st;
+        }
     }
-    if (status_out &&
-        cudaMemcpyAsync(status_out, hdr + kHdrStatus, sizeof(int), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
-        return MOE_ERR_CUDA;
     return MOE_OK;
 }
