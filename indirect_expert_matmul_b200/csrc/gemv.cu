@@ -593,21 +593,25 @@ __device__ __forceinline__ void gemv_body(const GemvArgs& a) {
             if (f.side == 1) return q;
             return R.fast ? nth_bit(mk0, mk1, q) : R.slots[R.off[jrow] + q];
         };
-        // this warp's (matrix, row group) pair and k-step residue
-        const int nrg = rsub / 16, P = nrg * NMAT, W = (kGvConsumers / 32) / P;
-        const int pr = cw % P, kr = cw / P;
-        const int mw = pr / nrg, rg = pr - mw * nrg;
-        const bool live = 16 * rg < f.nrow;
+        // this warp's row group and k-step residue.  One matrix: 16 rows, the
+        // fragment's rows 0-7 and 8-15 being rows rg16 + 0..7 and + 8..15.  Gate/up:
+        // 8 rows of both matrices, the fragment's rows 0-7 from gate and 8-15 from
+        // up, so that one thread holds both halves of its SwiGLU.
+        const int GR = NMAT == 2 ? 8 : 16;  // rows of a group
+        const int nrg = rsub / GR, P = nrg, W = (kGvConsumers / 32) / P;
+        const int rg = cw % P, kr = cw / P;
+        const bool live = GR * rg < f.nrow;
         // the row group's tile (a 256-row item spans two) and row inside it; a
         // k-step of a stage holds one piece per matrix, or per tile of a pair
-        const int tt = (16 * rg) / kTileM, rin = (16 * rg) % kTileM;
-        const int pm = NMAT == 2 ? mw : tt;
+        const int tt = (GR * rg) / kTileM, rin = (GR * rg) % kTileM;
         // the row group inside its piece: sub-block (r0 + rin) / 32 of the tile
         const int sbk = (f.r0 + rin) / kSubRows;
         const int nr = sub_rows(L.rows(f.mt + tt), sbk);
         const uint32_t roff = (uint32_t)((rin / kSubRows) * L.sub_bytes());
-        const int rra = rin % kSubRows + gq;  // rows rra and rra + 8 of the sub-block
+        const int rra = rin % kSubRows + gq;  // the fragment's row gq: row rra of the sub-block
         const uint32_t piece = (uint32_t)(f.nrow < kTileM ? f.nrow : kTileM) * L.rb;
+        // the fragment's rows 8-15: the up piece's row rra (gate/up), or row rra + 8
+        const uint32_t offb = NMAT == 2 ? (uint32_t)kps * piece : 8u * 32u;
         const int G = (nsl + kGvNT - 1) / kGvNT;
         for (int g = 0; g < G; ++g) {
             const int nt = nsl - g * kGvNT < kGvNT ? nsl - g * kGvNT : kGvNT;
@@ -715,16 +719,17 @@ __device__ __forceinline__ void gemv_body(const GemvArgs& a) {
                     }
                     if (live) {
                         for (int kk = kr; kk < nk; kk += W) {
-                            const uint8_t* pc = ring + (size_t)s * kGvStage + (size_t)(pm * kps + kk) * piece + roff;
+                            const uint8_t* pc = ring + (size_t)s * kGvStage + (size_t)(tt * kps + kk) * piece + roff;
                             const uint8_t* xk = xrow + (size_t)(k0 - w0 + kk) * kTileK * 2;
                             const uint4 xb[2] = {*(const uint4*)xk, *(const uint4*)(xk + 64)};
                             if (WT == MOE_MXFP4) {
                                 // block b: bytes 16b + 4tq .. of the row (columns 32b + 8tq .. 32b + 8tq + 7)
                                 const uint8_t* ca = pc + (size_t)rra * 32 + 4 * tq;
                                 const uint32_t wa[2] = {*(const uint32_t*)ca, *(const uint32_t*)(ca + 16)};
-                                const uint32_t wb[2] = {*(const uint32_t*)(ca + 256), *(const uint32_t*)(ca + 256 + 16)};
-                                const uint32_t sa = *(const uint16_t*)(pc + (size_t)nr * 32 + rra * 2);
-                                const uint32_t sb2 = *(const uint16_t*)(pc + (size_t)nr * 32 + (rra + 8) * 2);
+                                const uint32_t wb[2] = {*(const uint32_t*)(ca + offb), *(const uint32_t*)(ca + offb + 16)};
+                                const uint8_t* sp = pc + (size_t)nr * 32 + rra * 2;
+                                const uint32_t sa = *(const uint16_t*)sp;
+                                const uint32_t sb2 = *(const uint16_t*)(sp + (NMAT == 2 ? offb : 16u));
 #pragma unroll
                                 for (int b = 0; b < 2; ++b) {
                                     float c[4] = {0.f, 0.f, 0.f, 0.f};
@@ -746,9 +751,10 @@ __device__ __forceinline__ void gemv_body(const GemvArgs& a) {
                                 // block b: 8 bytes at 32 b nr + 32 row + 8 tq (columns 32b + 8tq .. 32b + 8tq + 7)
                                 const uint8_t* qa = pc + (size_t)rra * 32 + 8 * tq;
                                 const uint2 ua[2] = {*(const uint2*)qa, *(const uint2*)(qa + (size_t)nr * 32)};
-                                const uint2 ub[2] = {*(const uint2*)(qa + 256), *(const uint2*)(qa + (size_t)nr * 32 + 256)};
-                                const uint32_t da2 = *(const uint32_t*)(pc + (size_t)nr * kTileK + rra * 4);
-                                const uint32_t db2 = *(const uint32_t*)(pc + (size_t)nr * kTileK + (rra + 8) * 4);
+                                const uint2 ub[2] = {*(const uint2*)(qa + offb), *(const uint2*)(qa + (size_t)nr * 32 + offb)};
+                                const uint8_t* sp = pc + (size_t)nr * kTileK + rra * 4;
+                                const uint32_t da2 = *(const uint32_t*)sp;
+                                const uint32_t db2 = *(const uint32_t*)(sp + (NMAT == 2 ? offb : 32u));
 #pragma unroll
                                 for (int b = 0; b < 2; ++b) {
                                     float c[4] = {0.f, 0.f, 0.f, 0.f};
@@ -787,19 +793,30 @@ __device__ __forceinline__ void gemv_body(const GemvArgs& a) {
             }
             staged_side = one ? f.side : -1;
             staged_e = f.e;
-            if (NMAT == 1 && W == 1) {
+            if (W == 1) {
                 // every k-step of the row group was this warp's: its totals are the
                 // results, stored without a reduction or a barrier (a failed wait is
                 // acted on at the next window's barrier, or ends with the range)
                 if (ok && live) {
                     const int sl0 = 2 * tq < nt ? slot_of(g * kGvNT + 2 * tq) : 0;
                     const int sl1 = 2 * tq + 1 < nt ? slot_of(g * kGvNT + 2 * tq + 1) : 0;
+                    if (DUAL) {  // tot[0..1]: gate, tot[2..3]: up, row GR rg + gq, tokens 2tq, 2tq + 1
+                        const int r = GR * rg + gq, n = f.mt * kTileM + f.r0 + r;
 #pragma unroll
-                    for (int ii = 0; ii < 4; ++ii) {
-                        const int r = 16 * rg + gq + 8 * (ii >> 1), q = 2 * tq + (ii & 1);
-                        const int n = f.mt * kTileM + f.r0 + r;
-                        if (r < f.nrow && n < L.n_out && q < nt)
-                            GV_SIDE(f.side, out)[(int64_t)((ii & 1) ? sl1 : sl0) * L.n_out + n] = tot[ii];
+                        for (int i = 0; i < 2; ++i) {
+                            const float gt = tot[i], up = tot[2 + i];
+                            if (r < f.nrow && n < L.n_out && 2 * tq + i < nt)
+                                GV_SIDE(f.side, h)[(int64_t)(i ? sl1 : sl0) * L.n_out + n] =
+                                    __float2bfloat16_rn(gt / (1.0f + expf(-gt)) * up);
+                        }
+                    } else {
+#pragma unroll
+                        for (int ii = 0; ii < 4; ++ii) {
+                            const int r = GR * rg + gq + 8 * (ii >> 1), q = 2 * tq + (ii & 1);
+                            const int n = f.mt * kTileM + f.r0 + r;
+                            if (r < f.nrow && n < L.n_out && q < nt)
+                                GV_SIDE(f.side, out)[(int64_t)((ii & 1) ? sl1 : sl0) * L.n_out + n] = tot[ii];
+                        }
                     }
                 }
                 continue;
@@ -808,19 +825,23 @@ __device__ __forceinline__ void gemv_body(const GemvArgs& a) {
             float* rd = red + (rbuf & 1u) * (kGvRedBytes / 4);  // alternate buffers: no barrier after the reads
             ++rbuf;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) rd[((kr * P + pr) * 32 + lane) * 4 + i] = tot[i];
+            for (int i = 0; i < 4; ++i) rd[((kr * P + rg) * 32 + lane) * 4 + i] = tot[i];
             if (!consumers_and(ok && !*abort_flag)) return;  // uniform
             for (int idx = ct; idx < rsub * nt; idx += kGvConsumers) {
                 const int r = idx % rsub, q = idx / rsub;
                 const int n = f.mt * kTileM + f.r0 + r;
                 if (r >= f.nrow || n >= L.n_out) continue;
-                const int rgi = r >> 4, r16 = r & 15;
-                const int ln = (r16 & 7) * 4 + (q >> 1), ii = (r16 >> 3) * 2 + (q & 1);
+                // (row, token) in the fragments of group r / GR: lane (r mod 8) * 4 + q / 2,
+                // entry q mod 2 of the matrix's half (gate/up: gate 0-1, up 2-3; one
+                // matrix: rows r mod 16 < 8 in 0-1, the others in 2-3)
+                const int rgi = r / GR, rr = r % GR;
+                const int ln = (rr & 7) * 4 + (q >> 1);
                 float v[NMAT];
 #pragma unroll
                 for (int m = 0; m < NMAT; ++m) {
+                    const int ii = (NMAT == 2 ? 2 * m : (rr >> 3) * 2) + (q & 1);
                     float t = 0.f;
-                    for (int k2 = 0; k2 < W; ++k2) t += rd[((k2 * P + m * nrg + rgi) * 32 + ln) * 4 + ii];
+                    for (int k2 = 0; k2 < W; ++k2) t += rd[((k2 * P + rgi) * 32 + ln) * 4 + ii];
                     v[m] = t;
                 }
                 const int sl = slot_of(g * kGvNT + q);
