@@ -137,6 +137,25 @@ def test_decode_ffn_with_shared_expert(path, T):
     check_close(dsh, ref_sh, tol_sh, f"decode T={T} shared")
 
 
+@pytest.mark.parametrize("n_out", [1024, 1000, 384])
+@pytest.mark.parametrize("mode", ["broadcast", "per_slot"])
+def test_matvec_row_tile_pairs(n_out, mode):
+    """The mat-vec path with many distinct experts over several row tiles: a
+    single-matrix launch takes items of two full 128-row tiles (one tensor copy
+    for both, every k-step of a row group in one warp) when the padded n_out is
+    a multiple of 256 - 1024, and 1000 with the last pair ragged - and 128-row
+    items otherwise (384, three tiles)."""
+    E, k, T, n_in = 64, 8, 8, 256
+    W = workloads.q8_0_weights(E, n_out, n_in, 23, 5)
+    ids = workloads.routing("uniform", T, E, k, 23)
+    rows = T if mode == "broadcast" else T * k
+    x = workloads.activations(rows, n_in, "bf16", 23, 6)
+    ref, tol = oracle.mul_mat_id(W, x, "bf16", ids, mode)
+    with paths(1):
+        dst = moe.mul_mat_id(prep(W), E, n_out, n_in, to_dev_x(x, "bf16"), torch.from_numpy(ids).cuda(), mode)
+    check_close(dst, ref, tol, f"mat-vec row tile pairs n_out={n_out} {mode}")
+
+
 @pytest.mark.parametrize("path", PATHS)
 def test_f32_activations_ffn(path):
     """fp32 x goes through fp16 operands for gate/up; bf16 h for down."""
