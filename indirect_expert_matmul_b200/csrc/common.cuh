@@ -79,9 +79,14 @@ __host__ __device__ __forceinline__ int sub_rows(int rows, int sb) {
 inline int64_t tiled_rows(int64_t S, int n_groups) {
     return S + 8 * (S < n_groups ? S : n_groups) + 32;
 }
+// The row-id pass over several CTAs (up to kRidMaxCtas, for up to kRidMaxE
+// experts) keeps its per-CTA counts, first positions and per-expert padding
+// offsets in the workspace: 2 * kRidMaxCtas * E + E words.
+constexpr int kRidMaxCtas = 64;
+constexpr int kRidMaxE = 1024;
 struct WsLayout {
     int64_t S, rows_pad, rows_pad_sh;
-    size_t hdr, src1, dst, sprow, bounds, active, tiles, pad, h, h_sh, xt, xt_sh, xs, xs_sh, total;
+    size_t hdr, rid, src1, dst, sprow, bounds, active, tiles, pad, h, h_sh, xt, xt_sh, xs, xs_sh, total;
     static size_t up(size_t v) { return (v + 255) / 256 * 256; }
     WsLayout(int64_t n_tokens, int k, int n_experts, int n_in, int n_hidden, int n_hidden_sh, int x_type) {
         (void)x_type;
@@ -97,6 +102,7 @@ struct WsLayout {
         dst = o; o += up(S * 4);
         sprow = o; o += up(S * 4);  // tiled row of each slot t*k+s
         bounds = o; o += up((size_t)(n_experts + 1) * 4);
+        rid = o; o += n_experts <= kRidMaxE ? up(((size_t)2 * kRidMaxCtas * n_experts + n_experts) * 4) : 0;
         active = o; o += up((size_t)(n_experts + 1) * 4);
         tiles = o; o += up((size_t)(n_experts + 1) * 4);
         pad = o; o += up((size_t)(n_experts + 1) * 4);
