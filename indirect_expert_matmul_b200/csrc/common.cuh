@@ -125,7 +125,7 @@ constexpr int kGemmBN = 192;   // column (token) tile of the grouped GEMM
 
 // ---------------------------------------------------------------- profiling
 void prof_begin(cudaStream_t s);                     // start of an operator call
-void prof_mark(cudaStream_t s, const char* stage);   // after the launch of `stage`
+void prof_mark(cudaStream_t s, const char* stage, int launches = 1);  // after the launch(es) of `stage`
 
 // ------------------------------------------------------------------ dequant
 // u = q + 128 as a byte; f = as_float(0x47000000 | u << 8) = 32768 + u exactly.

@@ -9,7 +9,7 @@ namespace moe {
 moe_status launch_row_ids(const int32_t* ids, int64_t S, int k, int E, int mode, int32_t* ids_src1,
                           int32_t* ids_dst, int32_t* bounds, int32_t* active, int32_t* ntile_prefix,
                           int32_t* pad_start, int32_t* slot_prow, int bn, int* hdr, int32_t* rid_scratch,
-                          cudaStream_t stream);
+                          cudaStream_t stream, int* launches = nullptr);
 moe_status launch_prepare(int wtype, const void* src, int E, int n_out, int n_in, void* dst, cudaStream_t stream);
 }  // namespace moe
 
@@ -110,11 +110,12 @@ moe_status moe_row_ids(const int32_t* ids, int64_t n_tokens, int k, int n_expert
     WsLayout W(n_tokens, k, n_experts, 0, 0, 0, MOE_BF16);
     char* ws = (char*)workspace;
     prof_begin((cudaStream_t)stream);
+    int n_rid = 1;  // launches of the row-id pass
     st = launch_row_ids(ids, n_tokens * k, k, n_experts, mode, ids_src1, ids_dst, expert_bounds,
                         (int32_t*)(ws + W.active), (int32_t*)(ws + W.tiles), (int32_t*)(ws + W.pad),
                         (int32_t*)(ws + W.sprow), kGemmBN, (int*)(ws + W.hdr),
-                        n_experts <= kRidMaxE ? (int32_t*)(ws + W.rid) : nullptr, (cudaStream_t)stream);
-    prof_mark((cudaStream_t)stream, "row_ids");
+                        n_experts <= kRidMaxE ? (int32_t*)(ws + W.rid) : nullptr, (cudaStream_t)stream, &n_rid);
+    prof_mark((cudaStream_t)stream, "row_ids", n_rid);
     return st;
 }
 
@@ -169,11 +170,12 @@ moe_status moe_mul_mat_id_w(moe_wtype w_type, const void* W_prepared, int n_expe
         prof_mark(s, "gemv");
         return st;
     }
+    int n_rid = 1;  // launches of the row-id pass
     st = launch_row_ids(ids, S, k, n_experts, mode, src1, dstr, bounds, active, tiles, (int32_t*)(ws + W.pad),
                         (int32_t*)(ws + W.sprow), kGemmBN, hdr,
-                        n_experts <= kRidMaxE ? (int32_t*)(ws + W.rid) : nullptr, s);
+                        n_experts <= kRidMaxE ? (int32_t*)(ws + W.rid) : nullptr, s, &n_rid);
     if (st) return st;
-    prof_mark(s, "row_ids");
+    prof_mark(s, "row_ids", n_rid);
     GemmMulMatId g = {};
     g.wtype = w_type;
     g.W = (const uint8_t*)W_prepared;
@@ -302,11 +304,12 @@ moe_status moe_ffn_w(moe_wtype w_type, const void* Wg, const void* Wu, const voi
         prof_mark(s, "gemv_down");
         return st;
     }
+    int n_rid = 1;  // launches of the row-id pass
     st = launch_row_ids(ids, S, k, n_experts, MOE_BROADCAST, src1, dstr, bounds, active, tiles,
                         (int32_t*)(ws + W.pad), (int32_t*)(ws + W.sprow), kGemmBN, hdr,
-                        n_experts <= kRidMaxE ? (int32_t*)(ws + W.rid) : nullptr, s);
+                        n_experts <= kRidMaxE ? (int32_t*)(ws + W.rid) : nullptr, s, &n_rid);
     if (st) return st;
-    prof_mark(s, "row_ids");
+    prof_mark(s, "row_ids", n_rid);
     GemmFfn g = {};
     g.wtype = w_type;
     g.Wg = (const uint8_t*)Wg;

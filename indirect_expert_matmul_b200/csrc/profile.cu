@@ -13,6 +13,7 @@ constexpr int kMaxEvents = 4096;
 struct Rec {
     cudaEvent_t ev;
     const char* name;  // null = start of a call
+    int launches;      // kernels launched since the previous record
 };
 bool g_enabled = false;
 int g_count = 0;
@@ -21,7 +22,7 @@ cudaEvent_t g_pool[kMaxEvents];
 int g_pool_n = 0;
 std::mutex g_mu;
 
-void record(cudaStream_t s, const char* name) {
+void record(cudaStream_t s, const char* name, int launches) {
     std::lock_guard<std::mutex> lk(g_mu);
     if (!g_enabled || g_count >= kMaxEvents) return;
     if (g_count >= g_pool_n) {
@@ -30,12 +31,12 @@ void record(cudaStream_t s, const char* name) {
     }
     cudaEvent_t e = g_pool[g_count];
     if (cudaEventRecord(e, s) != cudaSuccess) return;
-    g_recs[g_count++] = Rec{e, name};
+    g_recs[g_count++] = Rec{e, name, launches};
 }
 }  // namespace
 
-void prof_begin(cudaStream_t s) { if (g_enabled) record(s, nullptr); }
-void prof_mark(cudaStream_t s, const char* stage) { if (g_enabled) record(s, stage); }
+void prof_begin(cudaStream_t s) { if (g_enabled) record(s, nullptr, 0); }
+void prof_mark(cudaStream_t s, const char* stage, int launches) { if (g_enabled) record(s, stage, launches); }
 
 }  // namespace moe
 
@@ -66,7 +67,7 @@ int moe_profile_read(const char** names, int* launches, double* total_ms, int ma
             total_ms[n] = 0.0;
             ++n;
         }
-        launches[j] += 1;
+        launches[j] += g_recs[i].launches;
         total_ms[j] += ms;
     }
     return n;

@@ -323,10 +323,12 @@ static size_t row_ids_smem(int n_chunks, int E) { return ((size_t)n_chunks + 2) 
 moe_status launch_row_ids(const int32_t* ids, int64_t S, int k, int E, int mode, int32_t* ids_src1,
                           int32_t* ids_dst, int32_t* bounds, int32_t* active, int32_t* ntile_prefix,
                           int32_t* pad_start, int32_t* slot_prow, int bn, int* hdr, int32_t* rid_scratch,
-                          cudaStream_t stream) {
+                          cudaStream_t stream, int* launches) {
     // G CTAs of 32 chunks: about 2048 slots a CTA
     const int64_t G = S / 2048 < kRidMaxCtas ? S / 2048 : kRidMaxCtas;
+    if (launches) *launches = 1;
     if (rid_scratch && E <= kRidMaxE && G >= 2) {
+        if (launches) *launches = 3;
         const size_t smem = (size_t)kRowIdWarps * E * sizeof(int);
         static int attr_dev_g = -1;
         int dev = 0;
