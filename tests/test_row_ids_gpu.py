@@ -118,3 +118,29 @@ def test_repeatable_ten_runs():
         again = gpu_tables(ids, wl.n_experts, "broadcast")
         for x, y in zip(ref, again):
             assert np.array_equal(x, y)
+
+
+@pytest.mark.parametrize("E", [1024, 1025])
+def test_many_ctas_at_the_expert_limit(E):
+    # 8192 x 8 slots: the pass runs over 32 CTAs up to 1024 experts (32 chunk rows
+    # of E counters in shared memory), and in one CTA past that
+    rng = np.random.default_rng(7)
+    ids = rng.integers(0, E, size=(8192, 8)).astype(np.int32)
+    assert_tables_equal(ids, E, "per_slot")
+
+
+def test_many_ctas_one_heavy_expert():
+    # every slot but a few on expert 3: one column of per-CTA counts carries all
+    rng = np.random.default_rng(8)
+    ids = np.full((4096, 8), 3, dtype=np.int32)
+    ids[rng.integers(0, 4096, 50), rng.integers(0, 8, 50)] = 200
+    assert_tables_equal(ids, 256, "broadcast")
+
+
+def test_many_ctas_bad_id_reports_status():
+    ids = np.zeros((4096, 8), dtype=np.int32)
+    ids[3000, 5] = 256  # outside [0, 256), counted by the CTA that owns slot 24005
+    t = torch.from_numpy(ids).cuda()
+    ws = moe.workspace(4096, 8, 256, 0)
+    moe.row_ids(t, 256, "broadcast", ws=ws)
+    assert moe.get_status(ws) == moe.ERR_BAD_ID
