@@ -73,6 +73,28 @@ def test_noalloc_reports_bad_id():
     assert int(status.item()) == moe.ERR_BAD_ID
 
 
+def test_noalloc_header_clears_itself_after_an_error():
+    # the down launch's last CTA copies the status out and zeroes the header, so
+    # a good call right after a failing one reports MOE_OK and computes exactly
+    wl = workloads.WORKLOADS["decode"]
+    Wg, Wu, Wd, _, x, ids = _inputs(wl, 4)
+    dWg, dWu, dWd, xd = prep(Wg), prep(Wu), prep(Wd), to_dev_x(x, "bf16")
+    bad = ids.copy()
+    bad[1, 2] = -1
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    moe.ffn_decode_noalloc(dWg, dWu, dWd, wl.n_experts, wl.n_in, wl.n_out, xd, torch.from_numpy(bad).cuda(),
+                           status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == moe.ERR_BAD_ID
+    dst, _ = moe.ffn_decode_noalloc(dWg, dWu, dWd, wl.n_experts, wl.n_in, wl.n_out, xd, torch.from_numpy(ids).cuda(),
+                                    status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == moe.OK
+    exact, tol = oracle.ffn(Wg, Wu, Wd, x, "bf16", ids)
+    got = dst.cpu().numpy().reshape(4 * wl.k, wl.n_in).astype(np.float64)
+    assert np.all(np.abs(got - exact) <= tol)
+
+
 def test_noalloc_refuses_sizes_past_its_scratch():
     wl = workloads.WORKLOADS["decode"]
     Wg, Wu, Wd, _, x, ids = _inputs(wl, 1)
