@@ -35,11 +35,11 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 # describes only the kernel sources it was measured on; when any of them changes
 # the bench reports null.
 GATE_UP_TRAFFIC = {
-    "bytes_per_launch": 8 * (1107833856 + 16241920),
+    "bytes_per_launch": 8 * (1133592320 + 16340992),
     "sources_sha256": {
         "gemm.cu": "c539fc93caa5560ca55fdfced7c924b60da2624bd4c500c4b9e681a1b7f3ff8c",
         "gemm_api.cuh": "dd7bf3b03c707a7676aafa55f8e79562e44196a9042c9cbac6d70b1f1cb10cfb",
-        "common.cuh": "a2bf4588757d7ed956e2aed19c2c845a652de7f12b8779a5c349cd66dd606530",
+        "common.cuh": "79d6480bd268349c0de107f1d8d81c039fdfe2f08bf55125faebb8ecc9e51fcf",
         "ptx.cuh": "97cfc9fdc310cea2e8c0da15d23992e95fd628c6bc2c31e12b73afb34926ba82",
     },
 }
