@@ -13,7 +13,7 @@
 // The result is unique (ascending (t, s) inside each expert), independent of
 // scheduling, and uses no global atomics.
 //
-// Larger calls (at least two CTAs' worth of slots, at most kRidMaxE experts)
+// Larger calls (at least 16384 slots, at most kRidMaxE experts)
 // spread the same three passes over G CTAs of 32 chunks each, in three
 // launches: per-CTA counts; one CTA's prefix over CTAs and experts (the
 // tables, each CTA's first position per expert); each CTA counting its chunks
@@ -324,10 +324,11 @@ moe_status launch_row_ids(const int32_t* ids, int64_t S, int k, int E, int mode,
                           int32_t* ids_dst, int32_t* bounds, int32_t* active, int32_t* ntile_prefix,
                           int32_t* pad_start, int32_t* slot_prow, int bn, int* hdr, int32_t* rid_scratch,
                           cudaStream_t stream, int* launches) {
-    // G CTAs of 32 chunks: about 2048 slots a CTA
+    // G CTAs of 32 chunks: about 2048 slots a CTA, from 8 CTAs on (below that
+    // one CTA's pass costs less than two more launches)
     const int64_t G = S / 2048 < kRidMaxCtas ? S / 2048 : kRidMaxCtas;
     if (launches) *launches = 1;
-    if (rid_scratch && E <= kRidMaxE && G >= 2) {
+    if (rid_scratch && E <= kRidMaxE && G >= 8) {
         if (launches) *launches = 3;
         const size_t smem = (size_t)kRowIdWarps * E * sizeof(int);
         static int attr_dev_g = -1;
