@@ -267,15 +267,20 @@ rid_scan_kernel(int E, int G, int bn, int32_t* __restrict__ scratch, int32_t* __
     __shared__ int warp_sums[32];
     __shared__ int totals[4];
     if (read_status(hdr + kHdrStatus) != 0) return;
-    int32_t* cta_cnt = scratch;
-    int32_t* cta_first = scratch + (size_t)G * E;
+    const int32_t* __restrict__ cta_cnt = scratch;
+    int32_t* __restrict__ cta_first = scratch + (size_t)G * E;
     int32_t* pad_delta = scratch + (size_t)2 * G * E;
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         int run = 0;
-        for (int g = 0; g < G; ++g) {
-            const int v = cta_cnt[(size_t)g * E + e];
-            cta_first[(size_t)g * E + e] = run;
-            run += v;
+        for (int g0 = 0; g0 < G; g0 += 8) {  // eight loads in flight, then their prefix
+            int v[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v[j] = g0 + j < G ? cta_cnt[(size_t)(g0 + j) * E + e] : 0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                if (g0 + j < G) cta_first[(size_t)(g0 + j) * E + e] = run;
+                run += v[j];
+            }
         }
         cnt[e] = run;
     }
