@@ -300,7 +300,7 @@ MOE_API moe_status moe_combine(const float *dst, const float *weights, const flo
 
 /* ------------------------------------------------------------------ tuning */
 
-/* Token count at or below which the mat-vec path is used (default 8); the
+/* Token count at or below which the mat-vec path is used (default 24); the
  * analogue of ggml's mmq_id threshold ([PR283] section 2.1, ggml-cuda.cu#L2944).
  * The mat-vec path takes n_tokens*k <= 1024; larger calls use the GEMM. */
 MOE_API void moe_set_gemv_threshold(int n_tokens);
