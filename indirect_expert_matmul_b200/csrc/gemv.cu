@@ -893,10 +893,11 @@ gemv_kernel(const __grid_constant__ GemvArgs a) {
 // sides only), 128, 64 or 32.  A CTA streams a contiguous range of items and
 // the launch ends with its fullest CTA: ceil(items / SMs) items, each costing
 // its bytes plus a fixed cost (decode, activation window, reduction) worth
-// about 64 KB of stream.  The height with the least such cost wins (the
-// larger one on a tie); `experts` is an upper bound on the distinct experts.
+// about 96 KB of stream (~2 us at one SM's share of HBM).  The height with the
+// least such cost wins (the larger one on a tie); `experts` estimates the
+// distinct experts.
 static int pick_rsub(const WLayout& L, int nmat, int64_t experts, int64_t other_items, int sms, bool pairs) {
-    constexpr int64_t kItemCost = 64 * 1024;
+    constexpr int64_t kItemCost = 96 * 1024;
     int best = 32;
     int64_t best_cost = -1;
     for (int r : {256, 128, 64, 32}) {
@@ -1049,7 +1050,13 @@ moe_status launch_gemv(const GemvArgs& in, cudaStream_t stream) {
         a.routed.kps = stage_ksteps(a.routed.L, rsub, nmat);
         plan_tensor_maps(a.routed, a.n_experts, nmat);
     };
-    plan_routed(pick_rsub(a.routed.L, nmat, a.max_distinct, sh_items, sms, pairs));
+    // distinct experts expected of S slots drawn uniformly from E, E (1 - (1 - 1/E)^S),
+    // at most max_distinct (the bound that sizes the grid)
+    const double e_f = (double)a.n_experts;
+    int64_t experts = (int64_t)(e_f * (1.0 - pow(1.0 - 1.0 / e_f, (double)S)) + 0.5);
+    if (experts > a.max_distinct) experts = a.max_distinct;
+    if (experts < 1) experts = 1;
+    plan_routed(pick_rsub(a.routed.L, nmat, experts, sh_items, sms, pairs));
     if (a.routed.rsub > kTileM && !a.routed.tma) plan_routed(kTileM);
     if (a.wait_limit <= 0) a.wait_limit = kGvWaitLimit;
     if (a.has_shared) plan_tensor_maps(a.shared, 1, nmat);
