@@ -11,21 +11,34 @@
 // exactly one CTA with one fixed reduction order: the result is bit-identical
 // from run to run.
 //
-// Both operands come from shared memory (128-byte-swizzled, K-major); the two
-// fp32 accumulators live in tensor memory.  Warp roles (768 threads):
+// The dequantised weights (A) live in tensor memory, beside the two fp32
+// accumulators; the activations (B) come from shared memory (128-byte-swizzled,
+// K-major).  Shared-memory bandwidth (128 bytes a clock per SM, shared by the
+// tensor core's operand reads and every copy and load) is what bounds a k-step
+// when A too is staged there: A written and read back costs 64 KB a k-step on
+// top of the raw weights and activations.  Warp roles (640 threads):
 //   warp 0      weight producer: L2 prefetch and 1-D bulk copies of the
 //               repacked int8+scale blocks of both A sources.
 //   warp 1      TMEM allocation and the single thread issuing tcgen05.mma
-//               (M=128, N=16..192, K=16 per instruction).  Its sub-partition
-//               runs no arithmetic: work there stretches every k-step.
+//               (M=128, N=16..192, K=16 per instruction, A from tensor memory).
+//               It touches no shared memory between k-steps: any shared-memory
+//               access by the issuing thread (an mbarrier wait, even one that
+//               passes, or a plain load) waits for its MMAs in flight to drain,
+//               ~250 cycles a k-step, more than half the MMA time of a
+//               96-column tile.
+//   warp 3      the MMA warp's waits: the accumulators free at a tile's start,
+//               then each k-step's A and B stages; it meets warp 1 at a named
+//               barrier whose AND carries "ready" (false: abort).
 //   warp 2      activation producer: one bulk copy per k-step of the
 //               pre-swizzled, tile-major activation rows.
-//   warps 3-23 but 5, 9, 13, 17, 21 (16 warps on sub-partitions 0, 2, 3):
+//   warps 4-19  four per tensor-memory lane quarter (warp % 4):
 //               dequantisation, int8 q + fp16 d -> q*d rounded once to the
-//               operand type, stored in the layout the tensor core reads.
-//   warps 4-19  epilogue, four per tensor-memory lane quarter (warp % 4):
-//               tcgen05.ld of the accumulators; SwiGLU of the gate/up pair to
-//               bf16 h, or fp32 rows scattered to dst by ids_dst.
+//               operand type, one row of one matrix a thread on alternate
+//               k-steps, converted in registers before the stage is free and
+//               then stored into tensor memory (a warp may only write its own
+//               lane quarter); and the epilogue: tcgen05.ld of the
+//               accumulators, SwiGLU of the gate/up pair to bf16 h, or fp32
+//               rows scattered to dst by ids_dst.
 // All waits are bounded; an expired wait sets MOE_ERR_TIMEOUT in the status
 // word and every role leaves its loop.
 #include "common.cuh"
@@ -34,18 +47,14 @@
 
 namespace moe {
 
-constexpr int kGemmThreads = 768;
+constexpr int kGemmThreads = 640;
 constexpr int kWarpProdA = 0;   // weight blocks: L2 prefetch + bulk copies
 constexpr int kWarpMma = 1;     // TMEM allocation + tcgen05.mma issue
 constexpr int kWarpProdB = 2;   // activation tiles: bulk copies
-constexpr int kWorkWarp0 = 4;   // warps 4-19: epilogue, four per lane quarter
+constexpr int kWarpWait = 3;    // the MMA warp's mbarrier waits
+constexpr uint32_t kBarIssue = 8;  // named barrier: warp 3 hands each k-step to warp 1 (64 threads)
+constexpr int kWorkWarp0 = 4;   // warps 4-19: dequantisation and epilogue, four per lane quarter
 constexpr int kWorkWarps = 16;
-constexpr int kDeqWarps = 16;   // warps 3-23 off the MMA warp's sub-partition: dequantisation
-// Dequantisation warp index 0..15 of warp w, or -1 (the MMA warp's sub-partition, w % 4 == 1,
-// is left to tcgen05.mma issue: arithmetic there stretches every k-step).
-__host__ __device__ constexpr int deq_index(int w) {
-    return (w < 3 || w > 23 || (w & 3) == 1) ? -1 : (w - 3) - ((w - 3 + 2) >> 2);
-}
 static_assert(kGemmBN <= 3 * 64, "a worker holds the output rows of three 16-column chunks");
 constexpr uint32_t kBTileBytes = kGemmBN * kTileK * 2; // 24 KB
 constexpr uint32_t kRawBytes = kTileM * kRowBytes;     // 8704
@@ -53,10 +62,13 @@ constexpr int kSmemGroups = 256;                       // schedule tables kept i
 constexpr int kPrefetchSteps = 8;                      // weight k-steps prefetched into L2 ahead of use
 constexpr long long kWaitLimitCycles = 1ll << 32;      // ~2 s
 constexpr uint32_t kSleepNs = 20000;                   // upper bound of one hardware wait
-// Tensor memory (512 columns): two fp32 accumulators of kGemmBN columns.
+// Tensor memory (512 columns): two fp32 accumulators of kGemmBN columns, then
+// kMA stages of the dequantised A operands, each two 128 x 64 matrices of
+// 16-bit values (32 columns a matrix: lane = row, two K values a column).
 constexpr uint32_t kAccCols = kGemmBN;
-constexpr int kMA = 2;   // dequantised A stages in shared memory: two 128 x 64 matrices, SW128 K-major
-constexpr uint32_t kATileBytes = kTileM * kTileK * 2;  // 16 KB per matrix
+constexpr int kMA = 2;
+constexpr uint32_t kACol0 = 2 * kAccCols;
+static_assert(kACol0 + kMA * 64 <= 512, "accumulators and A stages fill tensor memory");
 constexpr int kRS = 4;   // raw weight stages (int8 + scales of both matrices)
 constexpr int kMB = 3;   // activation (B) stages
 // Dequantisation warps take alternate k-steps by parity: with an even number
@@ -66,8 +78,7 @@ static_assert(kRS % 2 == 0 && kMA % 2 == 0, "ring stages are owned by one k-step
 
 struct Cfg {
     static constexpr uint32_t b_off = 0;
-    static constexpr uint32_t a_off = b_off + kMB * kBTileBytes;
-    static constexpr uint32_t raw_off = a_off + kMA * 2 * kATileBytes;
+    static constexpr uint32_t raw_off = b_off + kMB * kBTileBytes;
     static constexpr uint32_t bar_off = raw_off + kRS * 2 * kRawBytes;
     static constexpr int n_bars = 2 * kRS + 2 * kMA + 2 * kMB + 2;
     static constexpr uint32_t misc_off = bar_off + n_bars * 8;
@@ -193,13 +204,12 @@ __device__ __forceinline__ uint32_t pack2x(uint64_t v) {
 // one 128-row tile (SwiGLU epilogue into h); DUAL=0 two consecutive 128-row
 // tiles of one matrix (fp32 scatter to dst).  BF16: operand type bf16 (1) or
 // fp16 (0), which must equal p.bf16.
-// 16 quantised bytes (16 consecutive K values of one row) -> two 16-byte
-// chunks of operand values, exact: q*d rounded once to the operand type.
+// 16 quantised bytes (16 consecutive K values of one row) -> 8 packed pairs of
+// operand values in K order, exact: q*d rounded once to the operand type.
 // d2: the row's fp16 scale in both halves (fp16 route); dsc: the same as fp32.
 template <int BF16>
-__device__ __forceinline__ void dequant16_sts(uint4 x, uint32_t d2, float dsc, uint32_t dst0, uint32_t dst1) {
+__device__ __forceinline__ void dequant16(uint4 x, uint32_t d2, float dsc, uint32_t* pk) {
     const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-    uint32_t pk[8];
     if (BF16) {
         const uint64_t dd = ptx::f2pack(dsc, dsc);
         const uint64_t nd = ptx::f2pack(-32896.0f * dsc, -32896.0f * dsc);
@@ -223,8 +233,6 @@ __device__ __forceinline__ void dequant16_sts(uint4 x, uint32_t d2, float dsc, u
             pk[2 * j + 1] = *(const uint32_t*)&vhi;
         }
     }
-    ptx::sts128(dst0, make_uint4(pk[0], pk[1], pk[2], pk[3]));
-    ptx::sts128(dst1, make_uint4(pk[4], pk[5], pk[6], pk[7]));
 }
 
 // E8M0 scale byte -> 2^(x - 127) as a float (x = 0: 2^-127; x = 255: NaN).
@@ -233,10 +241,10 @@ __device__ __forceinline__ float e8m0_scale(uint32_t x) {
 }
 
 // 8 MXFP4 codes (one 32-bit word, code i in bits 4i..4i+3; consecutive
-// columns) -> one 16-byte chunk of bf16 operand values, exact: the pair
+// columns) -> 4 packed pairs of bf16 operand values, exact: the pair
 // conversion to f16 is exact (two significant bits), the power-of-two scale
 // is exact in float, and the product has at most two significant bits.
-__device__ __forceinline__ void dequant_mx8_sts(uint32_t w, float s, uint32_t dst) {
+__device__ __forceinline__ void dequant_mx8(uint32_t w, float s, uint32_t* pk) {
     uint32_t h[4];
     asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
         "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
@@ -246,14 +254,12 @@ __device__ __forceinline__ void dequant_mx8_sts(uint32_t w, float s, uint32_t ds
         "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
         : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
         : "r"(w));
-    uint32_t pk[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const __half2 v = *(const __half2*)&h[i];
         const __nv_bfloat162 b = __floats2bfloat162_rn(__low2float(v) * s, __high2float(v) * s);
         pk[i] = *(const uint32_t*)&b;
     }
-    ptx::sts128(dst, make_uint4(pk[0], pk[1], pk[2], pk[3]));
 }
 
 // WT: weight type of the A operand (MOE_Q8_0, or MOE_MXFP4 with BF16 = 1).
@@ -270,7 +276,6 @@ grouped_gemm_kernel(const GemmParams p) {
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_dyn + 1023) & ~(uintptr_t)1023);
     uint8_t* sB = smem + Cfg::b_off;
     uint8_t* sRaw = smem + Cfg::raw_off;
-    const uint32_t a_sa = ptx::smem_u32(smem + Cfg::a_off);
     const uint32_t raw_sa = ptx::smem_u32(sRaw);
     uint64_t* bars = (uint64_t*)(smem + Cfg::bar_off);
     uint64_t* raw_full = bars;
@@ -306,10 +311,10 @@ grouped_gemm_kernel(const GemmParams p) {
     if (tid == 0) {
         for (int i = 0; i < kRS; ++i) {
             ptx::mbar_init(&raw_full[i], 1);
-            ptx::mbar_init(&raw_empty[i], kDeqWarps / 2);
+            ptx::mbar_init(&raw_empty[i], kWorkWarps / 2);
         }
         for (int i = 0; i < kMA; ++i) {
-            ptx::mbar_init(&a_full[i], kDeqWarps / 2);
+            ptx::mbar_init(&a_full[i], kWorkWarps / 2);
             ptx::mbar_init(&a_empty[i], 1);
         }
         for (int i = 0; i < kMB; ++i) {
@@ -425,64 +430,80 @@ grouped_gemm_kernel(const GemmParams p) {
         }
     } else if (warp == kWarpMma) {
         // ----------------------------------------------------------------- MMA
-        // A and B from shared memory; the two accumulators' instructions
-        // interleave so neither chain waits on itself.
-        if (lane == 0) {
-            int as = 0, bs = 0;
-            uint32_t aph = 0, bph = 0, use = 0;
-            bool ok = true;
-            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-                const Tile tl = decode_tile(t, MU, p, s_prefix, s_bounds, s_pad);
-                const int n16 = (tl.n + 15) & ~15;
-                const bool has1 = DUAL || (2 * tl.mt + 1 < MT);
-                ok = wait_bar(tmem_empty, (use & 1) ^ 1, abort_flag, status);
+        // A from tensor memory, B from shared memory; the two accumulators'
+        // instructions interleave, sharing each B descriptor.  The whole warp
+        // runs the loop (the named barrier takes whole warps); lane 0 issues.
+        int as = 0, bs = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            const Tile tl = decode_tile(t, MU, p, s_prefix, s_bounds, s_pad);
+            const int n16 = (tl.n + 15) & ~15;
+            const bool has1 = DUAL || (2 * tl.mt + 1 < MT);
+            const uint32_t d0 = tmem_base, d1 = tmem_base + kAccCols;
+            const uint32_t idesc = ptx::idesc_f16(BF16, n16, 128);
+            for (int kt = 0; kt < KT; ++kt) {
+                // warp 3 has seen this k-step's stages (and at kt = 0 the accumulators) ready
+                ok = ptx::bar_red_and(kBarIssue, 64, true);
                 if (!ok) break;
                 ptx::tc_fence_after();
-                const uint32_t d0 = tmem_base, d1 = tmem_base + kAccCols;
-                const uint32_t idesc = ptx::idesc_f16(BF16, n16, 128);
-                for (int kt = 0; kt < KT; ++kt) {
-                    ok = wait_bar(&a_full[as], aph, abort_flag, status) &&
-                         wait_bar(&b_full[bs], bph, abort_flag, status);
-                    if (!ok) break;
-                    ptx::tc_fence_after();
-                    const uint32_t a0 = a_sa + (uint32_t)as * 2u * kATileBytes;
+                if (lane == 0) {
+                    const uint32_t a0 = tmem_base + kACol0 + (uint32_t)as * 64u;  // 8 columns per K=16 slice
                     const uint32_t b = ptx::smem_u32(sB + bs * kBTileBytes);
 #pragma unroll
                     for (int kk = 0; kk < kTileK / 16; ++kk) {
                         const uint32_t acc = (kt | kk) != 0;
                         const uint64_t bd = ptx::desc_k_sw128(b + kk * 32);
-                        ptx::mma_f16_ss(d0, ptx::desc_k_sw128(a0 + kk * 32), bd, idesc, acc);
-                        if (has1) ptx::mma_f16_ss(d1, ptx::desc_k_sw128(a0 + kATileBytes + kk * 32), bd, idesc, acc);
+                        ptx::mma_f16_ts(d0, a0 + kk * 8, bd, idesc, acc);
+                        if (has1) ptx::mma_f16_ts(d1, a0 + 32 + kk * 8, bd, idesc, acc);
                     }
                     ptx::mma_commit(&a_empty[as]);
                     ptx::mma_commit(&b_empty[bs]);
-                    if (++as == kMA) { as = 0; aph ^= 1; }
-                    if (++bs == kMB) { bs = 0; bph ^= 1; }
                 }
-                if (!ok) break;
-                ptx::mma_commit(tmem_full);
-                use += 1;
+                __syncwarp();
+                if (++as == kMA) as = 0;
+                if (++bs == kMB) bs = 0;
             }
+            if (!ok) break;
+            if (lane == 0) ptx::mma_commit(tmem_full);
+            __syncwarp();
         }
-        __syncwarp();
-    } else if (deq_index(warp) >= 0 || (warp >= kWorkWarp0 && warp < kWorkWarp0 + kWorkWarps)) {
+    } else if (warp == kWarpWait) {
+        // ------------------------------------------------- the MMA warp's waits
+        // The same k-step sequence as warp 1: wait (bounded) for what the k-step
+        // needs, then meet warp 1 at the named barrier with the outcome.  Both
+        // warps pass the barrier equally often: a failed wait is handed over,
+        // and both leave their loops after it.
+        int as = 0, bs = 0;
+        uint32_t aph = 0, bph = 0, use = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            for (int kt = 0; kt < KT; ++kt) {
+                bool ready = true;
+                if (kt == 0) ready = warp_wait(tmem_empty, (use & 1) ^ 1, abort_flag, status);
+                ready = ready && warp_wait(&a_full[as], aph, abort_flag, status) &&
+                        warp_wait(&b_full[bs], bph, abort_flag, status);
+                ok = ptx::bar_red_and(kBarIssue, 64, ready);
+                if (!ok) break;
+                if (++as == kMA) { as = 0; aph ^= 1; }
+                if (++bs == kMB) { bs = 0; bph ^= 1; }
+            }
+            use += 1;
+        }
+    } else if (warp >= kWorkWarp0 && warp < kWorkWarp0 + kWorkWarps) {
         // ------------------------------------- dequantisation and epilogue warps
-        // Dequantisation (16 warps on sub-partitions 0, 2, 3, two groups of eight
-        // taking alternate k-steps): each warp converts 32 rows of one source,
-        // all 64 columns, exactly (q*d rounded once to the operand type) into the
-        // SW128 K-major A stage in shared memory.  Epilogue (warps 4-19, four per
-        // tensor-memory lane quarter warp % 4): at the end of a tile each drains a
-        // quarter of the 16-column chunks of its lanes; warps 5, 9, 13, 17 do only
-        // this.
-        const int di = deq_index(warp);
-        const bool epi = warp >= kWorkWarp0 && warp < kWorkWarp0 + kWorkWarps;
-        const int wq = warp & 3, wj = (warp - kWorkWarp0) >> 2;  // epilogue lane quarter, chunk phase
-        const int kpar = di >> 3, mat = (di >> 2) & 1;
-        const int r = 32 * (di & 3) + lane;
+        // Four per tensor-memory lane quarter wq = warp % 4.  Dequantisation:
+        // thread `lane` converts row 32 wq + lane of matrix `mat`, all 64
+        // columns, in the k-steps of parity kpar, exactly (q*d rounded once to
+        // the operand type), into registers as soon as the raw stage lands, and
+        // stores them into the A stage of tensor memory once the MMAs of two
+        // k-steps back have released it.  Epilogue: at the end of a tile each
+        // drains a quarter of the 16-column chunks of its lanes.
+        const int wq = warp & 3, wj = (warp - kWorkWarp0) >> 2;  // lane quarter; (parity, matrix) and chunk phase
+        const int kpar = wj & 1, mat = wj >> 1;
+        const int r = 32 * wq + lane;       // the thread's row of the tile: its tensor-memory lane
         const int first = (lane >> 2) & 1;  // alternate read order: conflict-free 16-byte loads
         const uint32_t lanes = (uint32_t)(32 * wq) << 16;
-        const uint32_t a_row = (uint32_t)mat * kATileBytes + (uint32_t)(r >> 3) * 1024u + (uint32_t)(r & 7) * 128u;
-        const uint32_t rx = (uint32_t)(r & 7);
+        const uint32_t a_dst = tmem_base + lanes + kACol0 + (uint32_t)mat * 32u;
         int rs = 0, as = 0;
         uint32_t rph = 0, aph = 0, use = 0;
         bool ok = true;
@@ -496,94 +517,94 @@ grouped_gemm_kernel(const GemmParams p) {
                 const int col = (4 * q + wj) * 16 + (lane & 15);
                 orow[q] = -1;
                 oscale[q] = 1.0f;
-                if (epi && col < tl.n) {
+                if (col < tl.n) {
                     if (!DUAL) orow[q] = p.dst_rows ? __ldg(p.dst_rows + tl.p0 + col) : tl.p0 + col;
                     if (p.col_scale) oscale[q] = __ldg(p.col_scale + tl.p0pad + col);
                 }
             }
-            if (di >= 0) {
-                int nr;
-                {
-                    const uint8_t* dummy;
-                    int mt;
-                    source(tl, mat, dummy, nr, mt);
-                }
-                for (int kt = 0; kt < KT; ++kt) {
-                    if ((as & 1) == kpar) {  // the k-step count's parity, continued across tiles
-                        ok = warp_wait(&raw_full[rs], rph, abort_flag, status) &&
-                             warp_wait(&a_empty[as], aph ^ 1, abort_flag, status);
-                        if (!ok) break;
-                        if (nr > 0 && WT == MOE_MXFP4) {
-                            // this warp's rows are sub-block di & 3 (nsr rows): 32 code bytes a row at
-                            // sub + lane*32 (two 16-byte halves, read in alternating order), then two
-                            // scale bytes a row at sub + nsr*32 + lane*2
+            int nr;
+            {
+                const uint8_t* dummy;
+                int mt;
+                source(tl, mat, dummy, nr, mt);
+            }
+            for (int kt = 0; kt < KT; ++kt) {
+                if ((as & 1) == kpar) {  // the k-step count's parity, continued across tiles
+                    ok = warp_wait(&raw_full[rs], rph, abort_flag, status);
+                    if (!ok) break;
+                    // the row's 64 operand values, packed in pairs in K order (padding rows: 0)
+                    uint32_t pk[32];
+                    if (nr > 0 && WT == MOE_MXFP4) {
+                        // sub-block wq (nsr rows): 32 code bytes a row at sub + lane*32 (two 16-byte
+                        // halves, read in alternating order), then two scale bytes a row at
+                        // sub + nsr*32 + lane*2
+                        uint4 h0 = make_uint4(0u, 0u, 0u, 0u), h1 = h0;
+                        uint32_t xs = 0x7f7fu;  // padding rows: codes 0, scale 1
+                        if (r < nr) {
                             const uint32_t raw = raw_sa + (uint32_t)(rs * 2 + mat) * kRawBytes;
-                            const uint32_t dst = a_sa + (uint32_t)as * 2u * kATileBytes + a_row;
-                            uint4 h0 = make_uint4(0u, 0u, 0u, 0u), h1 = h0;
-                            uint32_t xs = 0x7f7fu;  // padding rows: codes 0, scale 1
-                            if (r < nr) {
-                                const int nsr = sub_rows(nr, di & 3);
-                                const uint32_t sub = raw + (uint32_t)(di & 3) * (uint32_t)L.sub_bytes();
-                                const uint32_t q = sub + (uint32_t)lane * 32u;
-                                const uint4 ca = ptx::lds128(q + first * 16), cb = ptx::lds128(q + (first ^ 1) * 16);
-                                h0 = first ? cb : ca;
-                                h1 = first ? ca : cb;
-                                xs = ptx::lds16(sub + (uint32_t)nsr * 32u + (uint32_t)lane * 2u);
-                            }
-                            const float s0 = e8m0_scale(xs & 0xffu), s1 = e8m0_scale(xs >> 8);
-                            const uint32_t w0[4] = {h0.x, h0.y, h0.z, h0.w}, w1[4] = {h1.x, h1.y, h1.z, h1.w};
+                            const int nsr = sub_rows(nr, wq);
+                            const uint32_t sub = raw + (uint32_t)wq * (uint32_t)L.sub_bytes();
+                            const uint32_t q = sub + (uint32_t)lane * 32u;
+                            const uint4 ca = ptx::lds128(q + first * 16), cb = ptx::lds128(q + (first ^ 1) * 16);
+                            h0 = first ? cb : ca;
+                            h1 = first ? ca : cb;
+                            xs = ptx::lds16(sub + (uint32_t)nsr * 32u + (uint32_t)lane * 2u);
+                        }
+                        const float s0 = e8m0_scale(xs & 0xffu), s1 = e8m0_scale(xs >> 8);
+                        const uint32_t w0[4] = {h0.x, h0.y, h0.z, h0.w}, w1[4] = {h1.x, h1.y, h1.z, h1.w};
 #pragma unroll
-                            for (int i = 0; i < 4; ++i) {  // word i of half h holds operand chunk 4h + i
-                                dequant_mx8_sts(w0[i], s0, dst + ((((uint32_t)i) ^ rx) << 4));
-                                dequant_mx8_sts(w1[i], s1, dst + (((4u + (uint32_t)i) ^ rx) << 4));
-                            }
-                            ptx::fence_proxy_async_smem();  // generic writes -> tensor-core reads
-                        } else if (nr > 0) {
+                        for (int i = 0; i < 4; ++i) {  // word i of half h holds values 32h + 8i .. 32h + 8i + 7
+                            dequant_mx8(w0[i], s0, pk + 4 * i);
+                            dequant_mx8(w1[i], s1, pk + 16 + 4 * i);
+                        }
+                    } else if (nr > 0) {
+                        uint4 x[4];
+                        uint32_t sc = 0u;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) x[i] = make_uint4(0x80808080u, 0x80808080u, 0x80808080u, 0x80808080u);
+                        if (r < nr) {
+                            // sub-block wq (nsr rows); block h, 16-byte chunk c at sub + h*nsr*32 +
+                            // lane*32 + c*16; lanes alternate the chunk order so that the 16-byte
+                            // loads are conflict-free
                             const uint32_t raw = raw_sa + (uint32_t)(rs * 2 + mat) * kRawBytes;
-                            const uint32_t dst = a_sa + (uint32_t)as * 2u * kATileBytes + a_row;
-                            uint4 x[4];
-                            uint32_t sc = 0u;
-#pragma unroll
-                            for (int i = 0; i < 4; ++i) x[i] = make_uint4(0x80808080u, 0x80808080u, 0x80808080u, 0x80808080u);
-                            if (r < nr) {
-                                // this warp's rows are sub-block di & 3 (nsr rows); half h, 16-byte chunk
-                                // c at sub + h*nsr*32 + lane*32 + c*16; lanes alternate the chunk order so
-                                // that the 16-byte loads are conflict-free
-                                const int nsr = sub_rows(nr, di & 3);
-                                const uint32_t sub = raw + (uint32_t)(di & 3) * (uint32_t)L.sub_bytes();
-                                const uint32_t q = sub + (uint32_t)lane * 32u;
-                                const uint32_t h1 = (uint32_t)nsr * 32u;
-                                x[0] = ptx::lds128(q + first * 16);
-                                x[1] = ptx::lds128(q + (first ^ 1) * 16);
-                                x[2] = ptx::lds128(q + h1 + first * 16);
-                                x[3] = ptx::lds128(q + h1 + (first ^ 1) * 16);
-                                sc = ptx::lds32(sub + (uint32_t)nsr * kTileK + (uint32_t)lane * 4u);
-                            }
-                            uint32_t d0, d1;
-                            asm("prmt.b32 %0, %1, %1, 0x1010;" : "=r"(d0) : "r"(sc));
-                            asm("prmt.b32 %0, %1, %1, 0x3232;" : "=r"(d1) : "r"(sc));
-                            const float f0 = BF16 ? __half2float(__ushort_as_half((unsigned short)(sc & 0xffffu))) : 0.f;
-                            const float f1 = BF16 ? __half2float(__ushort_as_half((unsigned short)(sc >> 16))) : 0.f;
-                            // raw chunk c of half h holds operand chunks 4h + 2c and 4h + 2c + 1 of the row
-                            const uint32_t c0 = (uint32_t)first * 2u, c1 = (uint32_t)(first ^ 1) * 2u;
-                            dequant16_sts<BF16>(x[0], d0, f0, dst + (((c0 + 0u) ^ rx) << 4), dst + (((c0 + 1u) ^ rx) << 4));
-                            dequant16_sts<BF16>(x[1], d0, f0, dst + (((c1 + 0u) ^ rx) << 4), dst + (((c1 + 1u) ^ rx) << 4));
-                            dequant16_sts<BF16>(x[2], d1, f1, dst + (((4u + c0) ^ rx) << 4), dst + (((5u + c0) ^ rx) << 4));
-                            dequant16_sts<BF16>(x[3], d1, f1, dst + (((4u + c1) ^ rx) << 4), dst + (((5u + c1) ^ rx) << 4));
-                            ptx::fence_proxy_async_smem();  // generic writes -> tensor-core reads
+                            const int nsr = sub_rows(nr, wq);
+                            const uint32_t sub = raw + (uint32_t)wq * (uint32_t)L.sub_bytes();
+                            const uint32_t q = sub + (uint32_t)lane * 32u;
+                            const uint32_t h1 = (uint32_t)nsr * 32u;
+                            x[0] = ptx::lds128(q + first * 16);
+                            x[1] = ptx::lds128(q + (first ^ 1) * 16);
+                            x[2] = ptx::lds128(q + h1 + first * 16);
+                            x[3] = ptx::lds128(q + h1 + (first ^ 1) * 16);
+                            sc = ptx::lds32(sub + (uint32_t)nsr * kTileK + (uint32_t)lane * 4u);
                         }
-                        __syncwarp();
-                        if (lane == 0) {
-                            ptx::mbar_arrive(&raw_empty[rs]);
-                            ptx::mbar_arrive(&a_full[as]);
-                        }
+                        uint32_t d0, d1;
+                        asm("prmt.b32 %0, %1, %1, 0x1010;" : "=r"(d0) : "r"(sc));
+                        asm("prmt.b32 %0, %1, %1, 0x3232;" : "=r"(d1) : "r"(sc));
+                        const float f0 = BF16 ? __half2float(__ushort_as_half((unsigned short)(sc & 0xffffu))) : 0.f;
+                        const float f1 = BF16 ? __half2float(__ushort_as_half((unsigned short)(sc >> 16))) : 0.f;
+                        // chunk c of block h: K values 32h + 16c .. 32h + 16c + 15
+                        dequant16<BF16>(first ? x[1] : x[0], d0, f0, pk + 0);
+                        dequant16<BF16>(first ? x[0] : x[1], d0, f0, pk + 8);
+                        dequant16<BF16>(first ? x[3] : x[2], d1, f1, pk + 16);
+                        dequant16<BF16>(first ? x[2] : x[3], d1, f1, pk + 24);
                     }
-                    if (++rs == kRS) { rs = 0; rph ^= 1; }
-                    if (++as == kMA) { as = 0; aph ^= 1; }
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(&raw_empty[rs]);  // its loads have been consumed
+                    ok = warp_wait(&a_empty[as], aph ^ 1, abort_flag, status);
+                    if (!ok) break;
+                    if (nr > 0) {
+                        ptx::tc_fence_after();
+                        ptx::tmem_st_32x32b_x32(a_dst + (uint32_t)as * 64u, pk);
+                        ptx::tmem_st_wait();
+                        ptx::tc_fence_before();
+                    }
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(&a_full[as]);
                 }
+                if (++rs == kRS) { rs = 0; rph ^= 1; }
+                if (++as == kMA) { as = 0; aph ^= 1; }
             }
             if (!ok) break;
-            if (!epi) continue;
             // ---- epilogue of this tile
             if (!warp_wait(tmem_full, use & 1, abort_flag, status)) break;
             use += 1;
