@@ -26,7 +26,16 @@ extern "C" {
  * waits for data that never comes; its wait expires, the status word gets
  * MOE_ERR_TIMEOUT and header word 3 the expired wait's site (1<<30 | warp<<20
  * | shared-memory offset of its barrier); every role of the CTA leaves its loop
- * and the launch ends.  Not thread-safe; not for production use.
+ * and the launch ends.
+ *
+ * The same stall applies to the grouped GEMM (moe_ffn / moe_mul_mat_id above
+ * the mat-vec threshold): the activation producer of CTA `cta` does not issue
+ * the copy of its k-step number `stage` (counted from 0 across its tiles), and
+ * every bounded wait of those launches gives up after `wait_us` microseconds.
+ * The warp that waits for the MMA warp's operands then gives up, hands the
+ * failure to the MMA warp through their named barrier, and the launch ends the
+ * same way (status MOE_ERR_TIMEOUT, the site in header word 3).  Not
+ * thread-safe; not for production use.
  */
 MOE_API void moe_testing_stall(int cta, int stage, int wait_us);
 

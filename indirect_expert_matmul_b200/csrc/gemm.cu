@@ -80,7 +80,7 @@ struct Cfg {
     static constexpr uint32_t b_off = 0;
     static constexpr uint32_t raw_off = b_off + kMB * kBTileBytes;
     static constexpr uint32_t bar_off = raw_off + kRS * 2 * kRawBytes;
-    static constexpr int n_bars = 2 * kRS + 2 * kMA + 2 * kMB + 2;
+    static constexpr int n_bars = 2 * kRS + 2 * kMA + 2 * kMB + 3;
     static constexpr uint32_t misc_off = bar_off + n_bars * 8;
     static constexpr uint32_t smem_bytes = misc_off + 64 + 1024;  // + alignment slack
 };
@@ -105,6 +105,8 @@ struct GemmParams {
     int bf16;                   // operand type: 1 bf16, 0 fp16
     int wtype;                  // A operand: MOE_Q8_0, or MOE_MXFP4 (bf16 operands)
     const float* col_scale;     // per tiled row of B (a tile column): factor the accumulator takes (null: 1)
+    long long wait_limit;       // cycles a wait may take before the launch gives up (MOE_ERR_TIMEOUT)
+    int stall_cta, stall_stage; // test only: that CTA's activation copy of that k-step is never issued (-1: off)
 };
 
 struct Tile {
@@ -144,13 +146,14 @@ __device__ __forceinline__ Tile decode_tile(int t, int mt_count, const GemmParam
 // Bounded wait by one lane; false when the kernel is aborting.  The lane
 // sleeps in hardware between polls (suspend-time hint), so waiting roles do
 // not take issue slots from the dequantisation warps.
-__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status) {
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status,
+                                         long long limit) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {
         if (ptx::mbar_try_wait_sleep(bar, parity, kSleepNs)) return true;
         if (*abort_flag) return false;
-        if (clock64() - t0 > kWaitLimitCycles) {
+        if (clock64() - t0 > limit) {
             *abort_flag = 1;
             const int site = (1 << 30) | ((int)(threadIdx.x >> 5) << 20) | (int)(ptx::smem_u32(bar) & 0xfffffu);
             atomicCAS(status + (kHdrWaitSite - kHdrStatus), 0, site);
@@ -161,14 +164,15 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
 }
 
 // lane 0 waits, the warp learns the outcome
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status) {
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status,
+                                          long long limit) {
     // every lane polls (no lane-0 branch); lanes that see different phases simply poll again
     if (ptx::mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {
         if (ptx::mbar_try_wait_sleep(bar, parity, kSleepNs)) return true;
         if (*abort_flag) return false;
-        if (clock64() - t0 > kWaitLimitCycles) {
+        if (clock64() - t0 > limit) {
             if ((threadIdx.x & 31) == 0) {
                 *abort_flag = 1;
                 const int site = (1 << 30) | ((int)(threadIdx.x >> 5) << 20) | (int)(ptx::smem_u32(bar) & 0xfffffu);
@@ -286,6 +290,7 @@ grouped_gemm_kernel(const GemmParams p) {
     uint64_t* b_empty = b_full + kMB;
     uint64_t* tmem_full = b_empty + kMB;
     uint64_t* tmem_empty = tmem_full + 1;
+    uint64_t* mma_drained = tmem_empty + 1;
     uint32_t* tmem_base_sh = (uint32_t*)(smem + Cfg::misc_off);
     volatile int* abort_flag = (volatile int*)(smem + Cfg::misc_off + 4);
     int* status = p.hdr + kHdrStatus;
@@ -323,6 +328,7 @@ grouped_gemm_kernel(const GemmParams p) {
         }
         ptx::mbar_init(tmem_full, 1);
         ptx::mbar_init(tmem_empty, kWorkWarps);
+        ptx::mbar_init(mma_drained, 1);
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
@@ -383,7 +389,7 @@ grouped_gemm_kernel(const GemmParams p) {
                 }
                 for (int kt = 0; kt < KT; ++kt) {
                     prefetch_one();
-                    ok = wait_bar(&raw_empty[rs], rph ^ 1, abort_flag, status);
+                    ok = wait_bar(&raw_empty[rs], rph ^ 1, abort_flag, status, p.wait_limit);
                     if (!ok) break;
                     ptx::mbar_arrive_expect_tx(&raw_full[rs], nb[0] + nb[1]);
                     for (int i = 0; i < 2; ++i)
@@ -398,7 +404,7 @@ grouped_gemm_kernel(const GemmParams p) {
             // let every copy issued land before the CTA can exit (bounded)
             volatile int never = 0;
             for (int s = 0; s < kRS; ++s)
-                if (used >> s & 1) wait_bar(&raw_full[s], (par >> s) & 1, &never, status);
+                if (used >> s & 1) wait_bar(&raw_full[s], (par >> s) & 1, &never, status, p.wait_limit);
         }
     } else if (warp == kWarpProdB) {
         // ------------------------------------------------ activation producer
@@ -410,23 +416,26 @@ grouped_gemm_kernel(const GemmParams p) {
             uint32_t used = 0, par = 0;
             bool ok = true;
             const size_t plane = (size_t)p.b_rows * 128u;
+            int q = 0;  // k-steps of this CTA so far
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
                 const Tile tl = decode_tile(t, MU, p, s_prefix, s_bounds, s_pad);
                 const uint32_t bytes = (uint32_t)((tl.n + 15) & ~15) * 128u;
                 const uint8_t* src = p.B + (size_t)tl.p0pad * 128u;
-                for (int kt = 0; kt < KT; ++kt) {
-                    ok = wait_bar(&b_empty[bs], bph ^ 1, abort_flag, status);
+                for (int kt = 0; kt < KT; ++kt, ++q) {
+                    ok = wait_bar(&b_empty[bs], bph ^ 1, abort_flag, status, p.wait_limit);
                     if (!ok) break;
-                    ptx::mbar_arrive_expect_tx(&b_full[bs], bytes);
-                    ptx::bulk_g2s(sB + bs * kBTileBytes, src + kt * plane, bytes, &b_full[bs]);
-                    used |= 1u << bs;
-                    par = (par & ~(1u << bs)) | (bph << bs);
+                    if (!((int)blockIdx.x == p.stall_cta && q == p.stall_stage)) {  // (test-only stall)
+                        ptx::mbar_arrive_expect_tx(&b_full[bs], bytes);
+                        ptx::bulk_g2s(sB + bs * kBTileBytes, src + kt * plane, bytes, &b_full[bs]);
+                        used |= 1u << bs;
+                        par = (par & ~(1u << bs)) | (bph << bs);
+                    }
                     if (++bs == kMB) { bs = 0; bph ^= 1; }
                 }
             }
             volatile int never = 0;
             for (int s = 0; s < kMB; ++s)
-                if (used >> s & 1) wait_bar(&b_full[s], (par >> s) & 1, &never, status);
+                if (used >> s & 1) wait_bar(&b_full[s], (par >> s) & 1, &never, status, p.wait_limit);
         }
     } else if (warp == kWarpMma) {
         // ----------------------------------------------------------------- MMA
@@ -467,6 +476,14 @@ grouped_gemm_kernel(const GemmParams p) {
             if (lane == 0) ptx::mma_commit(tmem_full);
             __syncwarp();
         }
+        // every MMA issued has completed before the CTA can release tensor memory
+        // (after an abort no epilogue waited for them); bounded like every wait
+        if (lane == 0) {
+            ptx::mma_commit(mma_drained);
+            volatile int never = 0;
+            wait_bar(mma_drained, 0, &never, status, p.wait_limit);
+        }
+        __syncwarp();
     } else if (warp == kWarpWait) {
         // ------------------------------------------------- the MMA warp's waits
         // The same k-step sequence as warp 1: wait (bounded) for what the k-step
@@ -479,9 +496,9 @@ grouped_gemm_kernel(const GemmParams p) {
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
             for (int kt = 0; kt < KT; ++kt) {
                 bool ready = true;
-                if (kt == 0) ready = warp_wait(tmem_empty, (use & 1) ^ 1, abort_flag, status);
-                ready = ready && warp_wait(&a_full[as], aph, abort_flag, status) &&
-                        warp_wait(&b_full[bs], bph, abort_flag, status);
+                if (kt == 0) ready = warp_wait(tmem_empty, (use & 1) ^ 1, abort_flag, status, p.wait_limit);
+                ready = ready && warp_wait(&a_full[as], aph, abort_flag, status, p.wait_limit) &&
+                        warp_wait(&b_full[bs], bph, abort_flag, status, p.wait_limit);
                 ok = ptx::bar_red_and(kBarIssue, 64, ready);
                 if (!ok) break;
                 if (++as == kMA) { as = 0; aph ^= 1; }
@@ -530,7 +547,7 @@ grouped_gemm_kernel(const GemmParams p) {
             }
             for (int kt = 0; kt < KT; ++kt) {
                 if ((as & 1) == kpar) {  // the k-step count's parity, continued across tiles
-                    ok = warp_wait(&raw_full[rs], rph, abort_flag, status);
+                    ok = warp_wait(&raw_full[rs], rph, abort_flag, status, p.wait_limit);
                     if (!ok) break;
                     // the row's 64 operand values, packed in pairs in K order (padding rows: 0)
                     uint32_t pk[32];
@@ -590,7 +607,7 @@ grouped_gemm_kernel(const GemmParams p) {
                     }
                     __syncwarp();
                     if (lane == 0) ptx::mbar_arrive(&raw_empty[rs]);  // its loads have been consumed
-                    ok = warp_wait(&a_empty[as], aph ^ 1, abort_flag, status);
+                    ok = warp_wait(&a_empty[as], aph ^ 1, abort_flag, status, p.wait_limit);
                     if (!ok) break;
                     if (nr > 0) {
                         ptx::tc_fence_after();
@@ -606,7 +623,7 @@ grouped_gemm_kernel(const GemmParams p) {
             }
             if (!ok) break;
             // ---- epilogue of this tile
-            if (!warp_wait(tmem_full, use & 1, abort_flag, status)) break;
+            if (!warp_wait(tmem_full, use & 1, abort_flag, status, p.wait_limit)) break;
             use += 1;
             ptx::tc_fence_after();
             if (DUAL) {
@@ -837,8 +854,18 @@ static int sm_count() {
     return n > 0 ? n : 148;
 }
 
+// The test-only stall set by moe_testing_stall (csrc/gemv.cu): CTA, k-step and
+// the wait limit in cycles; false when none is set.
+bool testing_stall_state(int* cta, int* stage, long long* limit_cycles);
+
 template <int DUAL, int BF16, int WT>
-static moe_status launch_grouped(const GemmParams& p, int grid, cudaStream_t stream) {
+static moe_status launch_grouped(const GemmParams& in, int grid, cudaStream_t stream) {
+    GemmParams p = in;
+    p.wait_limit = kWaitLimitCycles;
+    p.stall_cta = -1;
+    p.stall_stage = 0;
+    long long limit = 0;
+    if (testing_stall_state(&p.stall_cta, &p.stall_stage, &limit)) p.wait_limit = limit;
     static int attr_dev = -1;
     int dev = 0;
     cudaGetDevice(&dev);

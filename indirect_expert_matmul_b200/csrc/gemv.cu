@@ -1016,16 +1016,29 @@ static void plan_tensor_maps(GemvSide& sd, int n_experts, int nmat) {
 // test-only stall (moe_testing_stall): CTA, stage, wait limit in microseconds
 static std::atomic<int> g_stall_cta{-1}, g_stall_stage{0}, g_stall_wait_us{0};
 
+static long long stall_limit_cycles() {
+    int dev = 0, khz = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&khz, cudaDevAttrClockRate, dev);
+    return (long long)g_stall_wait_us.load() * (khz > 0 ? khz : 2000000) / 1000;
+}
+
+// The stall as the grouped GEMM uses it: that CTA's activation copy of that
+// k-step (counted over the CTA's tiles) is never issued.
+bool testing_stall_state(int* cta, int* stage, long long* limit_cycles) {
+    const int c = g_stall_cta.load();
+    if (c < 0) return false;
+    *cta = c;
+    *stage = g_stall_stage.load();
+    *limit_cycles = stall_limit_cycles();
+    return true;
+}
+
 moe_status launch_gemv(const GemvArgs& in, cudaStream_t stream) {
     GemvArgs a = in;
     a.stall_cta = g_stall_cta.load();
     a.stall_stage = g_stall_stage.load();
-    if (a.stall_cta >= 0) {
-        int dev = 0, khz = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&khz, cudaDevAttrClockRate, dev);
-        a.wait_limit = (long long)g_stall_wait_us.load() * (khz > 0 ? khz : 2000000) / 1000;
-    }
+    if (a.stall_cta >= 0) a.wait_limit = stall_limit_cycles();
     const int S = a.n_tokens * a.k;
     if (S > kGvMaxSlots || (a.wtype != MOE_Q8_0 && a.wtype != MOE_MXFP4)) return MOE_ERR_UNSUPPORTED;
     const bool f32 = a.routed.x_type == MOE_F32 || (a.has_shared && a.shared.x_type == MOE_F32);
